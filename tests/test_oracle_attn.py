@@ -1,0 +1,147 @@
+"""Pins for the oracle's tree-masked attention over the FP8 paged cache.
+
+(1) a chain-shaped tree equals causal attention (torch SDPA, fp64, explicit
+    causal mask) over context + tree tokens;
+(2) a tree equals running each root-to-node path as its own chain;
+(3) one node with no context returns its own V;
+(4) identical keys give the mean of the visible V;
+(5) pure-Python brute force at L=3, D=4, T=4;
+(6) a random permutation of the physical pool (with the page table) changes
+    nothing; bytes outside the visible positions change nothing.
+"""
+import math
+
+import numpy as np
+import torch
+
+from nvfp4_skinny_gemm_b200 import inputs
+
+
+def _dense(cache, Hkv, D, P):
+    """Dequantised dense K, V [L+T, Hkv, D] (torch float8 view x scale)."""
+    total = cache.ctx_len + cache.T
+    kp = torch.from_numpy(cache.k_pool.copy()).view(torch.float8_e4m3fn).double().numpy()
+    vp = torch.from_numpy(cache.v_pool.copy()).view(torch.float8_e4m3fn).double().numpy()
+    K = np.zeros((total, Hkv, D))
+    V = np.zeros((total, Hkv, D))
+    for p in range(total):
+        pg = cache.page_table[p // P]
+        K[p] = kp[pg, :, p % P, :] * cache.k_scale[:, None]
+        V[p] = vp[pg, :, :, p % P] * cache.v_scale[:, None]
+    return K, V
+
+
+def _run(oracle, q, cache, parent):
+    return oracle.tree_attn(q, cache.k_pool, cache.v_pool, cache.page_table, cache.ctx_len, parent,
+                            cache.k_scale, cache.v_scale)
+
+
+def test_chain_equals_causal_sdpa(oracle):
+    T, Hq, Hkv, D, P, L = 5, 6, 2, 16, 8, 21
+    cache = inputs.kv_cache(100, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=3)
+    q = inputs.query_bf16(100, T, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, inputs.chain_parent(T))
+    K, V = _dense(cache, Hkv, D, P)
+    grp = Hq // Hkv
+    qt = torch.from_numpy(q.astype(np.float64)).permute(1, 0, 2)                 # [Hq, T, D]
+    kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(grp, 0)          # [Hq, L+T, D]
+    vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(grp, 0)
+    mask = torch.tensor([[p <= L + i for p in range(L + T)] for i in range(T)])
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)
+    assert np.allclose(out, ref.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_tree_equals_per_path_chains(oracle):
+    T, Hq, Hkv, D, P, L = 16, 4, 2, 8, 16, 37
+    cache = inputs.kv_cache(101, L, T=T, Hkv=Hkv, D=D, P=P)
+    parent = inputs.tree_parent(101, T)
+    q = inputs.query_bf16(101, T, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, parent)
+    total = L + T
+    for i in range(T):
+        path = sorted(oracle.ancestors(parent, i))                  # root .. i
+        d = len(path)
+        # a fresh cache: same context pages, the path's tree slots in order
+        n_log = (L + d + P - 1) // P
+        kp = np.zeros((n_log, Hkv, P, D), np.uint8)
+        vp = np.zeros((n_log, Hkv, D, P), np.uint8)
+        for p in range(L + d):
+            src = p if p < L else L + path[p - L]
+            spg, sslot = cache.page_table[src // P], src % P
+            kp[p // P, :, p % P, :] = cache.k_pool[spg, :, sslot, :]
+            vp[p // P, :, :, p % P] = cache.v_pool[spg, :, :, sslot]
+        sub = oracle.tree_attn(q[path], kp, vp, np.arange(n_log, dtype=np.int32), L,
+                               inputs.chain_parent(d), cache.k_scale, cache.v_scale)
+        assert np.allclose(sub[-1], out[i], rtol=1e-12, atol=1e-14), i
+    assert total == L + T
+
+
+def test_single_node_no_context_returns_v0(oracle):
+    Hq, Hkv, D, P = 2, 1, 8, 4
+    cache = inputs.kv_cache(102, 0, T=1, Hkv=Hkv, D=D, P=P)
+    cache.k_scale[:] = 0.5
+    cache.v_scale[:] = 0.25
+    q = inputs.query_bf16(102, 1, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, np.array([-1], np.int32))
+    _, V = _dense(cache, Hkv, D, P)
+    for h in range(Hq):
+        assert np.array_equal(out[0, h], V[0, 0])
+
+
+def test_identical_keys_give_mean_of_visible_v(oracle):
+    T, Hq, Hkv, D, P, L = 6, 2, 1, 8, 8, 13
+    cache = inputs.kv_cache(103, L, T=T, Hkv=Hkv, D=D, P=P)
+    for p in range(L + T):
+        cache.k_pool[cache.page_table[p // P], 0, p % P, :] = 0x30   # same key everywhere
+    parent = np.array([-1, 0, 0, 1, 2, 3], np.int32)
+    q = inputs.query_bf16(103, T, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, parent)
+    _, V = _dense(cache, Hkv, D, P)
+    for i in range(T):
+        vis = list(range(L)) + [L + j for j in oracle.ancestors(parent, i)]
+        want = V[vis, 0].mean(axis=0)
+        for h in range(Hq):
+            assert np.allclose(out[i, h], want, rtol=1e-12, atol=1e-14)
+
+
+def test_bruteforce_tiny(oracle):
+    T, Hq, Hkv, D, P, L = 4, 2, 1, 4, 2, 3
+    cache = inputs.kv_cache(104, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=2)
+    parent = np.array([-1, 0, 0, 2], np.int32)
+    q = inputs.query_bf16(104, T, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, parent)
+    K, V = _dense(cache, Hkv, D, P)
+    anc = {0: [0], 1: [0, 1], 2: [0, 2], 3: [0, 2, 3]}
+    for i in range(T):
+        for h in range(Hq):
+            pos = [0, 1, 2] + [L + j for j in anc[i]]
+            s = [sum(float(q[i, h, d]) * K[p, 0, d] for d in range(D)) / math.sqrt(D) for p in pos]
+            m = max(s)
+            w = [math.exp(x - m) for x in s]
+            o = [sum(w[j] * V[p, 0, d] for j, p in enumerate(pos)) / sum(w) for d in range(D)]
+            assert np.allclose(out[i, h], o, rtol=1e-12, atol=1e-14)
+
+
+def test_page_permutation_and_unseen_bytes_do_not_matter(oracle):
+    T, Hq, Hkv, D, P, L = 16, 6, 2, 16, 8, 45
+    cache = inputs.kv_cache(105, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=5)
+    parent = inputs.tree_parent(105, T)
+    q = inputs.query_bf16(105, T, Hq, D).float().numpy()
+    out = _run(oracle, q, cache, parent)
+    rng = np.random.default_rng(9)
+    perm = rng.permutation(cache.k_pool.shape[0])        # new physical id of old page j = perm[j]
+    kp = np.empty_like(cache.k_pool); vp = np.empty_like(cache.v_pool)
+    kp[perm] = cache.k_pool; vp[perm] = cache.v_pool
+    out2 = oracle.tree_attn(q, kp, vp, perm[cache.page_table].astype(np.int32), L, parent,
+                            cache.k_scale, cache.v_scale)
+    assert np.array_equal(out, out2)
+    # scribble over every byte that no node may see
+    used = {(cache.page_table[p // P], p % P) for p in range(L + T)}
+    kp3, vp3 = cache.k_pool.copy(), cache.v_pool.copy()
+    for pg in range(kp3.shape[0]):
+        for slot in range(P):
+            if (pg, slot) not in used:
+                kp3[pg, :, slot, :] = 0x7E
+                vp3[pg, :, :, slot] = 0x7E
+    out3 = oracle.tree_attn(q, kp3, vp3, cache.page_table, L, parent, cache.k_scale, cache.v_scale)
+    assert np.array_equal(out, out3)
