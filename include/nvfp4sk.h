@@ -1,0 +1,228 @@
+/*
+ * nvfp4sk.h -- C ABI of libnvfp4sk, the B200 (sm_100a) kernels of the
+ * tree-MTP verification forward step of a 27B-class dense LLM:
+ *   W4A4 NVFP4 linear layers at M = 1..16 query tokens (LM head included),
+ *   tree-masked attention of the draft nodes over an FP8 paged KV cache,
+ *   and the page gather that restores a cached prompt prefix.
+ *
+ * The operations are those of "TensorRT Edge-LLM Completes the MLPerf Edge
+ * Agentic Benchmark 6.4x Faster on Jetson AGX Thor" (spbcomputers.ru,
+ * mechatronicstore.cl and ai4snews copies of the NVIDIA post):
+ *   - section "NVFP4 and FP8: smaller weights, faster decoding": low-batch
+ *     decode is DRAM-bandwidth bound; weights AND activations are NVFP4,
+ *     the LM head included; the KV cache is FP8;
+ *   - section "KV-cache reuse between agent steps": the runtime finds reused
+ *     prompt prefixes and restores their cached attention KV pages;
+ *   - section "Tree multi-token prediction": candidates are organised into a
+ *     16-node tree (8 draft steps, top-2 per depth) and verified in ONE
+ *     forward pass of the target model.
+ * Codec definitions: E2M1 per OCP Microscaling Formats (MX) v1.0, E4M3 per
+ * OCP 8-bit Floating Point Specification (OFP8, "fn" variant, max 448).
+ *
+ * Conventions for every call
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory unless
+ *     stated otherwise; the library allocates nothing per call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t) and return before
+ *     the GPU work ends.  Host-side argument checks return an error code and
+ *     launch nothing.  Device-side problems (a page id out of range, a wait
+ *     that ran out) never trap: the kernel skips the access, records the
+ *     problem in a device error word and returns; nvfp4sk_get_device_status()
+ *     reports and clears it.
+ *   - A "workspace" is caller-owned device scratch of at least the size the
+ *     matching *_workspace_bytes() query returns.  It must be zero-filled once
+ *     when it is first allocated; every successful call leaves it ready for
+ *     the next call.  Calls that share one workspace must be stream-ordered.
+ *   - Scalars such as tensor scales are device pointers, so no call syncs.
+ *   - Error codes are negative; nvfp4sk_last_error() gives a message for the
+ *     last failing call of the calling thread.
+ */
+#ifndef NVFP4SK_H
+#define NVFP4SK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NVFP4SK_API __attribute__((visibility("default")))
+#else
+#define NVFP4SK_API
+#endif
+
+typedef struct CUstream_st *nvfp4sk_stream_t; /* same type as cudaStream_t */
+typedef int nvfp4sk_status;
+
+#define NVFP4SK_OK 0
+#define NVFP4SK_ERR_INVALID_ARG (-1)       /* null pointer, bad dtype, bad tree     */
+#define NVFP4SK_ERR_UNSUPPORTED_SHAPE (-2) /* shape outside what the kernels cover  */
+#define NVFP4SK_ERR_MISALIGNED (-3)        /* pointer/stride not 16-byte aligned    */
+#define NVFP4SK_ERR_WORKSPACE (-4)         /* workspace missing or too small        */
+#define NVFP4SK_ERR_CUDA (-5)              /* a CUDA runtime/driver call failed     */
+#define NVFP4SK_ERR_TIMEOUT (-6)           /* a device wait ran out (device status) */
+#define NVFP4SK_ERR_OUT_OF_RANGE (-7)      /* a device bounds check failed          */
+#define NVFP4SK_ERR_DEVICE (-8)            /* current device is not sm_100          */
+
+enum { NVFP4SK_BF16 = 0, NVFP4SK_FP32 = 1 };
+
+/* ------------------------------------------------------------------------
+ * nvfp4_quantize_act -- NVFP4 quantisation of an activation (or weight)
+ * tensor (section "NVFP4 and FP8": NVFP4 for weights and activations).
+ *
+ * x: rows x K elements of type x_dtype (NVFP4SK_BF16 or NVFP4SK_FP32), row
+ *    stride ld_x elements.  K % 16 == 0, ld_x >= K, x 16-byte aligned and
+ *    ld_x * element size a multiple of 16 bytes.
+ * g_in: device fp32 tensor scale, or NULL for the dynamic per-tensor scale
+ *    g = fp32(amax(|x|) / 2688) (g = 1 when x is all zero).
+ * Per 16-element block b of a row: r = fp32(amax_b / 6), t = fp32(r / g),
+ *    scale = E4M3(t) (round-to-nearest-even, saturating at 448),
+ *    s = fp32(value(scale) * g), code_k = s == 0 ? +0 : E2M1(fp32(x_k / s))
+ *    (round-to-nearest-even, saturating at 6, sign kept).
+ * codes:  u8 [rows][K/2], two codes per byte, even k in the low nibble.
+ * scales: u8 [rows][K/16] E4M3 (canonical row-major layout).
+ * g_out:  device fp32, receives g (may equal g_in).
+ * ws: workspace of nvfp4_quantize_workspace_bytes(rows, K) bytes.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K);
+NVFP4SK_API nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int64_t K, int64_t ld_x,
+                                  const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
+                                  void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_prepare_weight_scales -- one-time rearrangement of a weight's
+ * canonical E4M3 block scales [N][K/16] into the tile order that
+ * nvfp4_linear streams into tensor memory.  Offline step for the NVFP4
+ * weights of section "NVFP4 and FP8" (calibrated once, then served).
+ * prepared: u8 buffer of nvfp4_prepared_scale_bytes(N, K) bytes (opaque).
+ * K % 64 == 0.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K);
+NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, int64_t N, int64_t K, uint8_t *prepared,
+                                           nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_linear -- the W4A4 NVFP4 linear layer of the verify step at
+ * M = 1..16 tokens, LM head included (section "NVFP4 and FP8": low-batch
+ * decode is DRAM-bandwidth bound; weights, activations and the LM head are
+ * NVFP4).  Y[m][n] = bf16( g_a*g_w * sum_b s_a[m,b] s_w[n,b] sum_{k in b}
+ * a[m,k] w[n,k]  (+ residual[m][n]) ), fp32 accumulation on tcgen05
+ * block-scaled tensor cores, split-K across all SMs.
+ *
+ * a_codes [M][K/2], a_scales [M][K/16] (canonical), g_a: from
+ *   nvfp4_quantize_act.  1 <= M <= 16.
+ * w_codes [N][K/2]; w_scales_prepared from nvfp4_prepare_weight_scales; g_w.
+ * K % 64 == 0, N >= 1, all code/scale pointers 16-byte aligned.
+ * residual: NULL or bf16 [M][ldy] added before rounding (may alias y).
+ * y: bf16 [M][ldy], ldy >= N, ldy even.
+ * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes (zero-filled once).
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, int64_t M,
+                            const uint8_t *w_codes, const uint8_t *w_scales_prepared, const float *g_w,
+                            int64_t N, int64_t K, const void *residual, void *y, int64_t ldy, void *ws,
+                            size_t ws_bytes, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * tree_attn_fp8kv -- attention of the T tree nodes over the FP8 paged KV
+ * cache with the ancestor mask (section "Tree multi-token prediction": the
+ * target model verifies all candidates of the tree in one forward pass;
+ * section "NVFP4 and FP8": FP8 KV cache).
+ *
+ * q: bf16, node i head hq at q[i*ld_q + hq*D + d] (ld_q >= Hq*D, even).
+ * Cache (one layer): k_pool u8 [n_pool_pages][Hkv][page_size][D]
+ *   (token-major pages); v_pool u8 [n_pool_pages][Hkv][D][page_size]
+ *   (dimension-major pages).  Position p lives in page page_table[p /
+ *   page_size], slot p % page_size.  Context positions are 0..ctx_len-1; the
+ *   tree nodes' own K/V are at ctx_len + i (node i).
+ * page_table: i32 [ceil((ctx_len+T)/page_size)] physical page ids.
+ * parent: i32 [T], parent[0] == -1, 0 <= parent[i] < i (topological order).
+ * k_scale, v_scale: fp32 [Hkv]; K = value(code) * k_scale[h] (same for V).
+ * Node i, head hq (KV head h = hq / (Hq/Hkv)) attends to every context
+ *   position and to the tree positions of {i} and its ancestors:
+ *   out = softmax_p(sm_scale * q . K_p) . V_p, bf16 [T][Hq][D] (dense).
+ * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 8.
+ * ws: tree_attn_workspace_bytes(...) bytes.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
+NVFP4SK_API nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D,
+                               const uint8_t *k_pool, const uint8_t *v_pool, int64_t n_pool_pages,
+                               int page_size, const int32_t *page_table, int64_t ctx_len,
+                               const int32_t *parent, const float *k_scale, const float *v_scale,
+                               float sm_scale, void *out, void *ws, size_t ws_bytes,
+                               nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * kv_page_restore -- restore cached KV pages of a reused prompt prefix into
+ * the live page pool (section "KV-cache reuse between agent steps": the
+ * runtime restores the cached attention KV pages; ~96% of prompt tokens
+ * came from the hot cache).  dst page dst_ids[i] <- src page src_ids[i],
+ * page_bytes each, i = 0..n-1, as one gather-copy kernel.
+ * src_ids, dst_ids: device i32 [n]; ids outside [0, n_src_pages) /
+ * [0, n_dst_pages) are skipped and flagged (NVFP4SK_ERR_OUT_OF_RANGE in the
+ * device status).  page_bytes % 16 == 0, pools 16-byte aligned.  dst ids
+ * should be distinct (duplicates race).
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_t *src_ids, uint8_t *dst_pool,
+                               const int32_t *dst_ids, int64_t n, int64_t page_bytes, int64_t n_src_pages,
+                               int64_t n_dst_pages, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Layer glue of the 64-layer verify step (not on the pages; fused where the
+ * next op is an NVFP4 linear so that activations are quantised in the same
+ * kernel that produces them).
+ * ---------------------------------------------------------------------- */
+/* y = x / sqrt(mean(x^2) + eps) * w rounded to bf16, then NVFP4-quantised
+ * exactly as nvfp4_quantize_act (dynamic g).  x bf16 [rows][n] (row stride
+ * n), w bf16 [n].  rows <= 16, n % 16 == 0, n <= 8192. */
+NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows, int64_t n,
+                                      uint8_t *codes, uint8_t *scales, float *g_out, void *ws,
+                                      size_t ws_bytes, nvfp4sk_stream_t stream);
+/* h = silu(gu[:, :F]) * gu[:, F:] rounded to bf16, then NVFP4-quantised
+ * (dynamic g).  gu bf16 [rows][2F].  rows <= 16, F % 16 == 0, F <= 32768. */
+NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes,
+                                     uint8_t *scales, float *g_out, void *ws, size_t ws_bytes,
+                                     nvfp4sk_stream_t stream);
+/* Append T new tokens' K and V (bf16, token i head h at k_new[i*ld_new +
+ * h*D + d]) to the cache at positions ctx_len .. ctx_len+T-1 as
+ * E4M3(fp32(x / scale[h])) (round-to-nearest-even, saturating); the FP8 KV
+ * cache write of section "NVFP4 and FP8".  Layouts as tree_attn_fp8kv. */
+NVFP4SK_API nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_new, int T, int Hkv, int D,
+                             uint8_t *k_pool, uint8_t *v_pool, int64_t n_pool_pages, int page_size,
+                             const int32_t *page_table, int64_t ctx_len, const float *k_scale,
+                             const float *v_scale, nvfp4sk_stream_t stream);
+/* idx[r] = argmax_j x[r*ld + j] over bf16 values, lowest index on ties. */
+NVFP4SK_API size_t argmax_workspace_bytes(int64_t rows, int64_t n);
+NVFP4SK_API nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t ld, int32_t *idx, void *ws,
+                                size_t ws_bytes, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status, options, diagnostics
+ * ---------------------------------------------------------------------- */
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns NVFP4SK_OK, NVFP4SK_ERR_TIMEOUT or NVFP4SK_ERR_OUT_OF_RANGE;
+ * *site (if non-NULL) receives the id of the last failing check. */
+NVFP4SK_API nvfp4sk_status nvfp4sk_get_device_status(nvfp4sk_stream_t stream, int *site);
+NVFP4SK_API const char *nvfp4sk_last_error(void);
+NVFP4SK_API int nvfp4sk_version(void);
+
+enum {
+    NVFP4SK_OPT_PDL = 0,          /* 1: launch with programmatic dependent launch (default 1) */
+    NVFP4SK_OPT_TIMEOUT_NS = 1,   /* per-wait limit of device spin-waits (default 1e9)        */
+    NVFP4SK_OPT_ATTN_SPLITS = 2,  /* 0: automatic; else KV splits per KV head                 */
+    NVFP4SK_OPT_LINEAR_CTAS = 3   /* 0: one CTA per SM; else the split-K grid size            */
+};
+NVFP4SK_API nvfp4sk_status nvfp4sk_set_option(int option, int64_t value);
+NVFP4SK_API int64_t nvfp4sk_get_option(int option);
+
+/* Diagnostic: element-wise device conversion of fp32 values with the same
+ * instructions the quantisers use: e2m1[i] = E2M1 code (low nibble), e4m3[i]
+ * = E4M3 code (RNE, satfinite).  Either output may be NULL. */
+NVFP4SK_API nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, uint8_t *e4m3,
+                                    nvfp4sk_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4SK_H */

@@ -1,0 +1,564 @@
+// nvfp4sk.cu -- C ABI of libnvfp4sk (declared in include/nvfp4sk.h): host-side
+// argument checks, tensor-map encoding, launch configuration and the device
+// status word.  All kernels live in the *.cuh files included below (one
+// translation unit, so that the device error word is a single variable).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "glue.cuh"
+#include "linear.cuh"
+#include "quant.cuh"
+#include "restore.cuh"
+
+using namespace nvfp4sk;
+
+namespace {
+
+thread_local std::string t_last_error;
+int g_opt_pdl = 1;
+int64_t g_opt_timeout_ns = 1000000000ll;
+int g_opt_attn_splits = 0;
+int g_opt_linear_ctas = 0;
+
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(NVFP4SK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DevInfo {
+    int sms = 0;
+    int major = 0, minor = 0;
+    bool ready = false;
+};
+constexpr int MAX_DEV = 64;
+DevInfo g_dev[MAX_DEV];
+std::mutex g_mu;
+
+template <typename K> cudaError_t set_smem(K kern, size_t bytes)
+{
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+template <typename K> cudaError_t allow_big_cluster(K kern)
+{
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
+// Per device: query the SM count, check sm_100, set kernel attributes once.
+int device_info(DevInfo **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= MAX_DEV) return fail(NVFP4SK_ERR_DEVICE, "device id %d out of range", dev);
+    DevInfo &d = g_dev[dev];
+    if (!d.ready) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!d.ready) {
+            if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+                return cuda_fail(e, "cudaDeviceGetAttribute");
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+            if (d.major != 10 || d.minor != 0)
+                return fail(NVFP4SK_ERR_DEVICE, "libnvfp4sk is built for sm_100a; device %d is sm_%d%d", dev,
+                            d.major, d.minor);
+            cudaError_t es[] = {
+                set_smem(nvfp4_linear_kernel, LIN_SMEM_BYTES),
+                set_smem(tree_attn_split_kernel, ATT_SMEM_BYTES),
+                set_smem(kv_page_restore_kernel, RST_SMEM_BUDGET + 1024),
+                allow_big_cluster(quant_fused_kernel<__nv_bfloat16, 0>),
+                allow_big_cluster(quant_fused_kernel<float, 0>),
+                allow_big_cluster(quant_fused_kernel<__nv_bfloat16, 1>),
+                allow_big_cluster(rmsnorm_quant_kernel),
+            };
+            for (cudaError_t x : es)
+                if (x != cudaSuccess) return cuda_fail(x, "cudaFuncSetAttribute");
+            unsigned long long t = (unsigned long long)g_opt_timeout_ns;
+            if ((e = cudaMemcpyToSymbol(g_timeout_ns, &t, sizeof t)) != cudaSuccess)
+                return cuda_fail(e, "cudaMemcpyToSymbol(timeout)");
+            d.ready = true;
+        }
+    }
+    *out = &d;
+    return NVFP4SK_OK;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
+                   Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (g_opt_pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (cluster > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = cluster;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+int launched(cudaError_t e, const char *what)
+{
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return NVFP4SK_OK;
+}
+
+// ---- tensor maps (driver entry point fetched through the runtime) ---------
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled_t encode_fn()
+{
+    static PFN_encodeTiled_t fn = []() -> PFN_encodeTiled_t {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_encodeTiled_t>(p);
+    }();
+    return fn;
+}
+
+// 2-D byte tensor [rows][inner] with row stride `stride`, box [box_rows][box_inner]
+int make_map_u8(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t stride, uint32_t box_inner,
+                uint32_t box_rows, CUtensorMapSwizzle swz)
+{
+    PFN_encodeTiled_t fn = encode_fn();
+    if (!fn) return fail(NVFP4SK_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {stride};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4SK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return NVFP4SK_OK;
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---- sizes shared by the workspace queries and the calls -------------------
+int linear_grid(const DevInfo &d, int64_t U)
+{
+    int64_t G = g_opt_linear_ctas > 0 ? g_opt_linear_ctas : d.sms;
+    return (int)std::min<int64_t>(G, U);
+}
+size_t linear_ws(int64_t G, int64_t NT) { return up256((size_t)G * 2 * 16 * 128 * 4) + up256((size_t)NT * 4 * 4); }
+
+int attn_splits(const DevInfo &d, int Hkv, int64_t n_log)
+{
+    int64_t S = g_opt_attn_splits > 0 ? g_opt_attn_splits : std::max<int64_t>(1, d.sms / std::max(1, Hkv));
+    return (int)std::max<int64_t>(1, std::min<int64_t>(S, n_log));
+}
+size_t attn_ws(int Hkv, int S, int group)
+{
+    const size_t rows = (size_t)Hkv * S * group * 16;
+    return up256(rows * ATT_D * 4) + up256(rows * 2 * 4);
+}
+
+int argmax_chunks(int64_t n) { return (int)std::max<int64_t>(1, std::min<int64_t>(64, n / 4096)); }
+
+}  // namespace
+
+// ============================================================================
+extern "C" {
+
+int nvfp4sk_version(void) { return 100; }
+const char *nvfp4sk_last_error(void) { return t_last_error.c_str(); }
+
+nvfp4sk_status nvfp4sk_set_option(int option, int64_t value)
+{
+    switch (option) {
+    case NVFP4SK_OPT_PDL: g_opt_pdl = value ? 1 : 0; return NVFP4SK_OK;
+    case NVFP4SK_OPT_TIMEOUT_NS: {
+        if (value <= 0) return fail(NVFP4SK_ERR_INVALID_ARG, "timeout must be positive");
+        g_opt_timeout_ns = value;
+        unsigned long long t = (unsigned long long)value;
+        cudaError_t e = cudaMemcpyToSymbol(g_timeout_ns, &t, sizeof t);
+        return e == cudaSuccess ? NVFP4SK_OK : cuda_fail(e, "cudaMemcpyToSymbol(timeout)");
+    }
+    case NVFP4SK_OPT_ATTN_SPLITS: g_opt_attn_splits = (int)std::max<int64_t>(0, value); return NVFP4SK_OK;
+    case NVFP4SK_OPT_LINEAR_CTAS: g_opt_linear_ctas = (int)std::max<int64_t>(0, value); return NVFP4SK_OK;
+    default: return fail(NVFP4SK_ERR_INVALID_ARG, "unknown option %d", option);
+    }
+}
+
+int64_t nvfp4sk_get_option(int option)
+{
+    switch (option) {
+    case NVFP4SK_OPT_PDL: return g_opt_pdl;
+    case NVFP4SK_OPT_TIMEOUT_NS: return g_opt_timeout_ns;
+    case NVFP4SK_OPT_ATTN_SPLITS: return g_opt_attn_splits;
+    case NVFP4SK_OPT_LINEAR_CTAS: return g_opt_linear_ctas;
+    default: return -1;
+    }
+}
+
+nvfp4sk_status nvfp4sk_get_device_status(nvfp4sk_stream_t stream, int *site)
+{
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int err = 0, where = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&err, g_err, sizeof err)) != cudaSuccess) return cuda_fail(e, "read status");
+    cudaMemcpyFromSymbol(&where, g_err_site, sizeof where);
+    cudaMemcpyToSymbol(g_err, &zero, sizeof zero);
+    cudaMemcpyToSymbol(g_err_site, &zero, sizeof zero);
+    if (site) *site = (int)where;
+    if (err & ERRBIT_TIMEOUT) return fail(NVFP4SK_ERR_TIMEOUT, "device wait ran out (site %u)", where);
+    if (err & ERRBIT_RANGE) return fail(NVFP4SK_ERR_OUT_OF_RANGE, "device bounds check failed (site %u)", where);
+    return NVFP4SK_OK;
+}
+
+// ---------------------------------------------------------------- quantise
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K)
+{
+    (void)rows; (void)K;
+    return QBIG_MAX_PARTIALS * sizeof(float);
+}
+
+nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int64_t K, int64_t ld_x,
+                                  const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out, void *ws,
+                                  size_t ws_bytes, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!x || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (x_dtype != NVFP4SK_BF16 && x_dtype != NVFP4SK_FP32) return fail(NVFP4SK_ERR_INVALID_ARG, "bad dtype");
+    if (rows < 1 || K < 16 || K % 16 != 0 || ld_x < K)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need rows >= 1, K %% 16 == 0, ld_x >= K");
+    const int64_t esz = x_dtype == NVFP4SK_BF16 ? 2 : 4;
+    if (!al16(x) || (ld_x * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(codes) & 7u) != 0)
+        return fail(NVFP4SK_ERR_MISALIGNED, "x and its row stride must be 16-byte aligned, codes 8-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t nblk = rows * (K / 16);
+    if (nblk <= QSMALL_MAX_BLOCKS) {
+        const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
+        cudaError_t e = x_dtype == NVFP4SK_BF16
+                            ? launch(quant_fused_kernel<__nv_bfloat16, 0>, dim3(cs), dim3(QTHREADS), 0, st, cs,
+                                     (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, codes, scales, g_out)
+                            : launch(quant_fused_kernel<float, 0>, dim3(cs), dim3(QTHREADS), 0, st, cs,
+                                     (const float *)x, rows, K, ld_x, g_in, codes, scales, g_out);
+        return launched(e, "quant_fused_kernel");
+    }
+    if (!g_in && (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(rows, K)))
+        return fail(NVFP4SK_ERR_WORKSPACE, "workspace too small");
+    const int grid = (int)std::min<int64_t>(std::min<int64_t>(QBIG_MAX_PARTIALS, 4 * d->sms),
+                                            cdiv(nblk, QBIG_THREADS));
+    float *partial = (float *)ws;
+    cudaError_t e = cudaSuccess;
+    if (!g_in) {
+        e = x_dtype == NVFP4SK_BF16
+                ? launch(amax_partial_kernel<__nv_bfloat16>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1,
+                         (const __nv_bfloat16 *)x, rows, K, ld_x, partial)
+                : launch(amax_partial_kernel<float>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1, (const float *)x,
+                         rows, K, ld_x, partial);
+        if (e != cudaSuccess) return cuda_fail(e, "amax_partial_kernel");
+    }
+    e = x_dtype == NVFP4SK_BF16
+            ? launch(quant_blocks_kernel<__nv_bfloat16>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1,
+                     (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, (const float *)partial, grid, codes, scales,
+                     g_out)
+            : launch(quant_blocks_kernel<float>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1, (const float *)x, rows,
+                     K, ld_x, g_in, (const float *)partial, grid, codes, scales, g_out);
+    return launched(e, "quant_blocks_kernel");
+}
+
+size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K) { return (size_t)cdiv(N, 128) * cdiv(K, 256) * 2048; }
+
+nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, int64_t N, int64_t K, uint8_t *prepared,
+                                           nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!scales || !prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (N < 1 || K < 64 || K % 64 != 0) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need N >= 1, K %% 64 == 0");
+    const int64_t total = (int64_t)nvfp4_prepared_scale_bytes(N, K);
+    const int grid = (int)std::min<int64_t>(cdiv(total, 256), 8 * d->sms);
+    return launched(launch(prepare_scales_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, scales, N, K,
+                           cdiv(K, 256), prepared, total),
+                    "prepare_scales_kernel");
+}
+
+// ---------------------------------------------------------------- linear
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    (void)M;
+    DevInfo *d;
+    if (device_info(&d)) return 0;
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 256);
+    const int64_t G = std::max<int64_t>(d->sms, g_opt_linear_ctas);
+    return linear_ws(std::min<int64_t>(G, NT * KT), NT);
+}
+
+nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, int64_t M,
+                            const uint8_t *w_codes, const uint8_t *w_scales_prepared, const float *g_w, int64_t N,
+                            int64_t K, const void *residual, void *y, int64_t ldy, void *ws, size_t ws_bytes,
+                            nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!a_codes || !a_scales || !g_a || !w_codes || !w_scales_prepared || !g_w || !y)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (M < 1 || M > 16 || N < 1 || K < 64 || K % 64 != 0 || ldy < N || N > (int64_t)1 << 30 || K > (int64_t)1 << 24)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, N >= 1, K %% 64 == 0, ldy >= N");
+    if (!al16(a_codes) || !al16(a_scales) || !al16(w_codes) || !al16(w_scales_prepared))
+        return fail(NVFP4SK_ERR_MISALIGNED, "code and scale pointers must be 16-byte aligned");
+    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 256), U = NT * KT;
+    const int G = linear_grid(*d, U);
+    const size_t need = linear_ws(G, NT);
+    if (!ws || ws_bytes < need || !al16(ws))
+        return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
+    CUtensorMap tw, ta;
+    if (int rc = make_map_u8(&tw, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    if (int rc = make_map_u8(&ta, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128, 16,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    LinearParams p;
+    p.w_sf = w_scales_prepared;
+    p.a_scales = a_scales;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.residual = (const __nv_bfloat16 *)residual;
+    p.y = (__nv_bfloat16 *)y;
+    p.partial = (float *)ws;
+    p.counters = (int *)((uint8_t *)ws + up256((size_t)G * 2 * 16 * 128 * 4));
+    p.ldy = ldy;
+    p.U = U;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.NT = (int)NT;
+    p.KT = (int)KT;
+    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, (cudaStream_t)stream,
+                           1, tw, ta, p),
+                    "nvfp4_linear_kernel");
+}
+
+// ---------------------------------------------------------------- attention
+size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len)
+{
+    (void)D;
+    DevInfo *d;
+    if (device_info(&d) || Hkv <= 0 || page_size <= 0 || Hq % Hkv) return 0;
+    const int64_t n_log = cdiv(ctx_len + T, page_size);
+    return attn_ws(Hkv, attn_splits(*d, Hkv, n_log), Hq / Hkv);
+}
+
+nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D, const uint8_t *k_pool,
+                               const uint8_t *v_pool, int64_t n_pool_pages, int page_size,
+                               const int32_t *page_table, int64_t ctx_len, const int32_t *parent,
+                               const float *k_scale, const float *v_scale, float sm_scale, void *out, void *ws,
+                               size_t ws_bytes, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!q || !k_pool || !v_pool || !page_table || !parent || !k_scale || !v_scale || !out)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 8 ||
+        ctx_len < 0 || n_pool_pages < 1 || ld_q < (int64_t)Hq * D || n_pool_pages * Hkv * ATT_P > INT32_MAX)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 8, ld_q >= Hq*D");
+    if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool))
+        return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes) and the pools must be 16-byte aligned");
+    const int64_t n_log = cdiv(ctx_len + T, ATT_P);
+    const int group = Hq / Hkv;
+    const int S = attn_splits(*d, Hkv, n_log);
+    const size_t need = attn_ws(Hkv, S, group);
+    if (!ws || ws_bytes < need || !al16(ws))
+        return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
+    CUtensorMap tk;
+    if (int rc = make_map_u8(&tk, k_pool, ATT_D, (uint64_t)n_pool_pages * Hkv * ATT_P, ATT_D, ATT_D, ATT_P,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    AttnParams p;
+    p.q = (const __nv_bfloat16 *)q;
+    p.ld_q = ld_q;
+    p.v_pool = v_pool;
+    p.page_table = page_table;
+    p.parent = parent;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.part_o = (float *)ws;
+    p.part_ml = (float *)((uint8_t *)ws + up256((size_t)Hkv * S * group * 16 * ATT_D * 4));
+    p.out = (__nv_bfloat16 *)out;
+    p.ctx_len = ctx_len;
+    p.n_pool_pages = n_pool_pages;
+    p.sm_scale = sm_scale;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.group = group;
+    p.S = S;
+    p.n_log_pages = (int)n_log;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, Hkv), dim3((group + 1) * 32), ATT_SMEM_BYTES, st, 1, tk, p);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_attn_split_kernel");
+    return launched(launch(tree_attn_combine_kernel, dim3(T, Hq), dim3(ATT_D), 0, st, 1, p),
+                    "tree_attn_combine_kernel");
+}
+
+// ---------------------------------------------------------------- restore
+nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_t *src_ids, uint8_t *dst_pool,
+                               const int32_t *dst_ids, int64_t n, int64_t page_bytes, int64_t n_src_pages,
+                               int64_t n_dst_pages, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (n == 0) return NVFP4SK_OK;
+    if (!src_pool || !src_ids || !dst_pool || !dst_ids) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (n < 0 || page_bytes < 16 || page_bytes % 16 != 0 || n_src_pages < 1 || n_dst_pages < 1)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need n >= 0, page_bytes %% 16 == 0");
+    if (!al16(src_pool) || !al16(dst_pool)) return fail(NVFP4SK_ERR_MISALIGNED, "pools must be 16-byte aligned");
+    RestoreParams p;
+    p.src = src_pool;
+    p.src_ids = src_ids;
+    p.dst = dst_pool;
+    p.dst_ids = dst_ids;
+    p.page_bytes = page_bytes;
+    p.n_src_pages = n_src_pages;
+    p.n_dst_pages = n_dst_pages;
+    p.chunk = (uint32_t)std::min<int64_t>(page_bytes, 32768);
+    p.chunks_per_page = (int)cdiv(page_bytes, p.chunk);
+    p.n_items = n * p.chunks_per_page;
+    p.stages = (int)std::max<uint32_t>(2, std::min<uint32_t>(RST_MAX_STAGES, RST_SMEM_BUDGET / p.chunk));
+    const size_t smem = (size_t)p.stages * p.chunk + 128 + 8 * RST_MAX_STAGES + 64;
+    const int grid = (int)std::min<int64_t>(p.n_items, d->sms);
+    return launched(launch(kv_page_restore_kernel, dim3(grid), dim3(RST_THREADS), smem, (cudaStream_t)stream, 1, p),
+                    "kv_page_restore_kernel");
+}
+
+// ---------------------------------------------------------------- glue
+nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows, int64_t n,
+                                      uint8_t *codes, uint8_t *scales, float *g_out, void *ws, size_t ws_bytes,
+                                      nvfp4sk_stream_t stream)
+{
+    (void)ws; (void)ws_bytes;
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!x || !w || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 16 || n < 16 || n % 16 != 0 || n > (int64_t)RTHREADS * RNB * 16)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, n %% 16 == 0, n <= 8192");
+    if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u))
+        return fail(NVFP4SK_ERR_MISALIGNED, "x, w must be 16-byte aligned, codes 8-byte aligned");
+    const int cs = rows <= 8 ? 8 : 16;
+    return launched(launch(rmsnorm_quant_kernel, dim3(cs), dim3(RTHREADS), 0, (cudaStream_t)stream, cs,
+                           (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, rows, n, codes, scales, g_out),
+                    "rmsnorm_quant_kernel");
+}
+
+nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes, uint8_t *scales,
+                                     float *g_out, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
+{
+    (void)ws; (void)ws_bytes;
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!gu || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 16 || F < 16 || F % 16 != 0 || rows * (F / 16) > QSMALL_MAX_BLOCKS)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, F %% 16 == 0, rows*F <= 524288");
+    if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u))
+        return fail(NVFP4SK_ERR_MISALIGNED, "gu must be 16-byte aligned, codes 8-byte aligned");
+    const int64_t nblk = rows * (F / 16);
+    const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
+    return launched(launch(quant_fused_kernel<__nv_bfloat16, 1>, dim3(cs), dim3(QTHREADS), 0, (cudaStream_t)stream,
+                           cs, (const __nv_bfloat16 *)gu, rows, F, 2 * F, (const float *)nullptr, codes, scales,
+                           g_out),
+                    "swiglu_quant_kernel");
+}
+
+nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_new, int T, int Hkv, int D,
+                             uint8_t *k_pool, uint8_t *v_pool, int64_t n_pool_pages, int page_size,
+                             const int32_t *page_table, int64_t ctx_len, const float *k_scale, const float *v_scale,
+                             nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!k_new || !v_new || !k_pool || !v_pool || !page_table || !k_scale || !v_scale)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (T < 1 || Hkv < 1 || D < 1 || page_size < 1 || ctx_len < 0 || ld_new < (int64_t)Hkv * D || n_pool_pages < 1)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "bad shape");
+    return launched(launch(kv_append_kernel, dim3(T, Hkv), dim3(128), 0, (cudaStream_t)stream, 1,
+                           (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new, ld_new, Hkv, D, k_pool,
+                           v_pool, n_pool_pages, page_size, page_table, ctx_len, k_scale, v_scale),
+                    "kv_append_kernel");
+}
+
+size_t argmax_workspace_bytes(int64_t rows, int64_t n)
+{
+    const int nch = argmax_chunks(n);
+    return up256((size_t)rows * nch * 4) * 2 + up256((size_t)rows * 4);
+}
+
+nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t ld, int32_t *idx, void *ws,
+                                size_t ws_bytes, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!x || !idx) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 65535 || n < 1 || n > INT32_MAX || ld < n)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "bad shape");
+    const size_t need = argmax_workspace_bytes(rows, n);
+    if (!ws || ws_bytes < need) return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    const int nch = argmax_chunks(n);
+    uint8_t *b = (uint8_t *)ws;
+    float *pv = (float *)b;
+    int32_t *pi = (int32_t *)(b + up256((size_t)rows * nch * 4));
+    int32_t *cnt = (int32_t *)(b + 2 * up256((size_t)rows * nch * 4));
+    return launched(launch(argmax_rows_kernel, dim3(nch, rows), dim3(AMX_THREADS), 0, (cudaStream_t)stream, 1,
+                           (const __nv_bfloat16 *)x, n, ld, idx, pv, pi, cnt),
+                    "argmax_rows_kernel");
+}
+
+nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, uint8_t *e4m3,
+                                    nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!x || n < 0) return fail(NVFP4SK_ERR_INVALID_ARG, "bad arguments");
+    if (n == 0) return NVFP4SK_OK;
+    const int grid = (int)std::min<int64_t>(cdiv(n, 256), 16 * d->sms);
+    return launched(launch(debug_encode_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, x, n, e2m1, e4m3),
+                    "debug_encode_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,364 @@
+// quant.cuh -- NVFP4 quantisation kernels (E2M1 codes, one E4M3 scale per 16
+// elements, fp32 tensor scale amax/2688), bit-exact to the fp32 recipe:
+//   r = fp32(amax_b / 6), t = fp32(r / g), scale = E4M3_rne_sat(t),
+//   s = fp32(value(scale) * g), code = s == 0 ? +0 : E2M1_rne_sat(fp32(x / s)).
+// Division and multiplication use the IEEE round-to-nearest intrinsics so the
+// compiler cannot contract or approximate them.
+#pragma once
+#include "common.cuh"
+
+namespace nvfp4sk {
+
+constexpr int QCL_MAX = 16;            // max CTAs per cluster of the fused path
+constexpr int QTHREADS = 512;          // threads per CTA of the fused path
+constexpr int QNB = 4;                 // max 16-blocks per thread of the fused path
+constexpr int64_t QSMALL_MAX_BLOCKS = (int64_t)QCL_MAX * QTHREADS * QNB;
+constexpr int RTHREADS = 256;          // threads per CTA of the fused RMSNorm path
+constexpr int RNB = 2;                 // 16-blocks per thread of a row (n <= 8192)
+
+__device__ __forceinline__ float tensor_scale_from_amax(float amax)
+{
+    return amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// Quantise one 16-element block held in registers; returns the scale code
+// and writes the 8 code bytes (two per byte, even element in the low nibble).
+__device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float g, uint2 &packed)
+{
+    float amax_b = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[k]));
+    const float r = __fdiv_rn(amax_b, 6.0f);
+    const float t = __fdiv_rn(r, g);
+    const uint32_t sc = cvt_e4m3x2(t, 0.f) & 0xFFu;
+    const float s = __fmul_rn(e4m3_to_float(sc), g);
+    uint32_t w0 = 0, w1 = 0;
+    if (s != 0.f) {
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+            uint32_t b0 = cvt_e2m1x2(__fdiv_rn(v[k], s), __fdiv_rn(v[k + 1], s));
+            w0 |= b0 << (k * 4);
+        }
+#pragma unroll
+        for (int k = 8; k < 16; k += 2) {
+            uint32_t b1 = cvt_e2m1x2(__fdiv_rn(v[k], s), __fdiv_rn(v[k + 1], s));
+            w1 |= b1 << ((k - 8) * 4);
+        }
+    }
+    packed = make_uint2(w0, w1);
+    return sc;
+}
+
+// ---- element loaders ------------------------------------------------------
+template <typename T> __device__ __forceinline__ void load16(const T *p, float (&v)[16]);
+
+template <> __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[16])
+{
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+    uint4 a = q[0], b = q[1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+template <> __device__ __forceinline__ void load16<float>(const float *p, float (&v)[16])
+{
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float4 f = q[i];
+        v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+    }
+}
+
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// SwiGLU block: h_k = bf16(silu(g_k) * u_k), silu(x) = x / (1 + e^-x)
+__device__ __forceinline__ void load16_swiglu(const __nv_bfloat16 *gp, const __nv_bfloat16 *up, float (&v)[16])
+{
+    float g[16], u[16];
+    load16<__nv_bfloat16>(gp, g);
+    load16<__nv_bfloat16>(up, u);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float sg = __fdiv_rn(g[k], 1.0f + expf(-g[k]));
+        v[k] = round_bf16(sg * u[k]);
+    }
+}
+
+// ---- cluster-wide amax via distributed shared memory ----------------------
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_cluster_f32(const float *local, uint32_t rank)
+{
+    uint32_t a = smem_u32(local), ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+// Block-wide max into s_red[0]; all threads get the result.
+__device__ __forceinline__ float block_max(float v, float *s_red)
+{
+    v = warp_max(v);
+    if (lane_id() == 0) s_red[warp_id()] = v;
+    __syncthreads();
+    if (warp_id() == 0) {
+        float w = lane_id() < (blockDim.x >> 5) ? s_red[lane_id()] : 0.f;
+        w = warp_max(w);
+        if (lane_id() == 0) s_red[32] = w;
+    }
+    __syncthreads();
+    return s_red[32];
+}
+
+__device__ __forceinline__ float block_sum(float v, float *s_red)
+{
+    v = warp_sum(v);
+    __syncthreads();
+    if (lane_id() == 0) s_red[warp_id()] = v;
+    __syncthreads();
+    if (warp_id() == 0) {
+        float w = lane_id() < (blockDim.x >> 5) ? s_red[lane_id()] : 0.f;
+        w = warp_sum(w);
+        if (lane_id() == 0) s_red[32] = w;
+    }
+    __syncthreads();
+    return s_red[32];
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Every CTA of the cluster contributes its local amax; returns the global g.
+__device__ __forceinline__ float cluster_tensor_scale(float local_amax, float *s_red, float *s_cta_amax)
+{
+    float a = block_max(local_amax, s_red);
+    if (threadIdx.x == 0) *s_cta_amax = a;
+    cluster_sync_all();
+    float amax = 0.f;
+    const uint32_t n = cluster_size();
+    for (uint32_t r = 0; r < n; ++r) amax = fmaxf(amax, ld_cluster_f32(s_cta_amax, r));
+    return tensor_scale_from_amax(amax);
+}
+
+// Fused single-launch quantiser for small tensors.  Blocks are spread over
+// the CTAs of one cluster (8 or 16, chosen at launch); values stay in
+// registers between the amax reduction and the encode.  MODE 0: plain x
+// (type T), MODE 1: SwiGLU of a [rows][2K] bf16 input.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(QTHREADS, 1)
+    quant_fused_kernel(const T *__restrict__ x, int64_t rows, int64_t K, int64_t ld_x,
+                       const float *__restrict__ g_in, uint8_t *__restrict__ codes,
+                       uint8_t *__restrict__ scales, float *__restrict__ g_out)
+{
+    __shared__ float s_red[33];
+    __shared__ float s_cta_amax;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t kb = K / 16;
+    const int64_t nblk = rows * kb;
+    const uint32_t ncta = cluster_size();
+    const int64_t per_cta = (nblk + ncta - 1) / ncta;
+    const uint32_t rank = cluster_rank();
+    const int64_t b0 = (int64_t)rank * per_cta;
+    const int64_t b1 = min(nblk, b0 + per_cta);
+    float v[QNB][16];
+    float local = 0.f;
+#pragma unroll
+    for (int j = 0; j < QNB; ++j) {
+        const int64_t b = b0 + threadIdx.x + (int64_t)j * blockDim.x;
+        if (b < b1) {
+            const int64_t r = b / kb, c = b % kb;
+            if (MODE == 0) load16<T>(x + r * ld_x + c * 16, v[j]);
+            else load16_swiglu(reinterpret_cast<const __nv_bfloat16 *>(x) + r * ld_x + c * 16,
+                               reinterpret_cast<const __nv_bfloat16 *>(x) + r * ld_x + K + c * 16, v[j]);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) local = fmaxf(local, fabsf(v[j][k]));
+        }
+    }
+    float g;
+    if (g_in) {
+        g = *g_in;
+        cluster_sync_all();
+    } else {
+        g = cluster_tensor_scale(local, s_red, &s_cta_amax);
+    }
+    if (rank == 0 && threadIdx.x == 0) *g_out = g;
+#pragma unroll
+    for (int j = 0; j < QNB; ++j) {
+        const int64_t b = b0 + threadIdx.x + (int64_t)j * blockDim.x;
+        if (b < b1) {
+            const int64_t r = b / kb, c = b % kb;
+            uint2 pk;
+            const uint32_t sc = quant_block16(v[j], g, pk);
+            *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
+            scales[r * kb + c] = (uint8_t)sc;
+        }
+    }
+    cluster_sync_all();   // keep this CTA's shared memory alive until peers have read it
+}
+
+// Fused RMSNorm + quantise: row r is handled by CTA r of the cluster (one
+// cluster of >= rows CTAs); each thread owns up to RNB 16-blocks of its row.
+__global__ void __launch_bounds__(RTHREADS, 1)
+    rmsnorm_quant_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
+                         int64_t rows, int64_t n, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                         float *__restrict__ g_out)
+{
+    __shared__ float s_red[33];
+    __shared__ float s_cta_amax;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t r = cluster_rank();
+    const int64_t kb = n / 16;
+    float v[RNB][16];
+    float ss = 0.f, local = 0.f;
+#pragma unroll
+    for (int j = 0; j < RNB; ++j) {
+        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
+        if (r < rows && c < kb) {
+            load16<__nv_bfloat16>(x + r * n + c * 16, v[j]);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) ss += v[j][k] * v[j][k];
+        }
+    }
+    const float tot = block_sum(ss, s_red);
+    const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
+#pragma unroll
+    for (int j = 0; j < RNB; ++j) {
+        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
+        if (r < rows && c < kb) {
+            float wv[16];
+            load16<__nv_bfloat16>(w + c * 16, wv);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                v[j][k] = round_bf16(__fmul_rn(__fmul_rn(v[j][k], inv), wv[k]));
+                local = fmaxf(local, fabsf(v[j][k]));
+            }
+        }
+    }
+    const float g = cluster_tensor_scale(local, s_red, &s_cta_amax);
+    if (r == 0 && threadIdx.x == 0) *g_out = g;
+#pragma unroll
+    for (int j = 0; j < RNB; ++j) {
+        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
+        if (r < rows && c < kb) {
+            uint2 pk;
+            const uint32_t sc = quant_block16(v[j], g, pk);
+            *reinterpret_cast<uint2 *>(codes + r * (n / 2) + c * 8) = pk;
+            scales[r * kb + c] = (uint8_t)sc;
+        }
+    }
+    cluster_sync_all();
+}
+
+// ---- large tensors: amax partials, then encode ----------------------------
+constexpr int QBIG_THREADS = 256;
+constexpr int QBIG_MAX_PARTIALS = 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(QBIG_THREADS) amax_partial_kernel(const T *__restrict__ x, int64_t rows,
+                                                                     int64_t K, int64_t ld_x,
+                                                                     float *__restrict__ partial)
+{
+    __shared__ float s_red[33];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t kb = K / 16, nblk = rows * kb;
+    float local = 0.f;
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblk;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        float v[16];
+        load16<T>(x + (b / kb) * ld_x + (b % kb) * 16, v);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) local = fmaxf(local, fabsf(v[k]));
+    }
+    const float a = block_max(local, s_red);
+    if (threadIdx.x == 0) partial[blockIdx.x] = a;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(QBIG_THREADS) quant_blocks_kernel(const T *__restrict__ x, int64_t rows,
+                                                                     int64_t K, int64_t ld_x,
+                                                                     const float *__restrict__ g_in,
+                                                                     const float *__restrict__ partial,
+                                                                     int n_partial, uint8_t *__restrict__ codes,
+                                                                     uint8_t *__restrict__ scales,
+                                                                     float *__restrict__ g_out)
+{
+    __shared__ float s_red[33];
+    pdl_wait();
+    pdl_launch_dependents();
+    float g;
+    if (g_in) {
+        g = *g_in;
+    } else {
+        float a = 0.f;
+        for (int i = threadIdx.x; i < n_partial; i += blockDim.x) a = fmaxf(a, __ldcg(partial + i));
+        g = tensor_scale_from_amax(block_max(a, s_red));
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const int64_t kb = K / 16, nblk = rows * kb;
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblk;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = b / kb, c = b % kb;
+        float v[16];
+        load16<T>(x + r * ld_x + c * 16, v);
+        uint2 pk;
+        const uint32_t sc = quant_block16(v, g, pk);
+        *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
+        scales[r * kb + c] = (uint8_t)sc;
+    }
+}
+
+// ---- weight scale-factor rearrangement -------------------------------------
+// prepared[t][kt][j][l][c*4 + kb] = scales[t*128 + l + 32c][kt*16 + 4j + kb]
+// (zero outside the matrix): for every 128-row x 256-column weight tile, four
+// 512-byte chunks, one per 64-wide MMA step, each the 32 x 16-byte image that
+// tcgen05.cp 32x128b.warpx4 replicates into the scale-factor columns.
+__global__ void prepare_scales_kernel(const uint8_t *__restrict__ scales, int64_t N, int64_t K, int64_t KT,
+                                      uint8_t *__restrict__ out, int64_t total)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t kb = K / 16;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t byte = i & 15, l = (i >> 4) & 31, j = (i >> 9) & 3, tile = i >> 11;
+        const int64_t kt = tile % KT, t = tile / KT;
+        const int64_t c = byte >> 2, kbi = byte & 3;
+        const int64_t row = t * 128 + l + 32 * c, col = kt * 16 + 4 * j + kbi;
+        out[i] = (row < N && col < kb) ? scales[row * kb + col] : 0;
+    }
+}
+
+// ---- diagnostics: element-wise conversions ---------------------------------
+__global__ void debug_encode_kernel(const float *__restrict__ x, int64_t n, uint8_t *__restrict__ e2m1,
+                                    uint8_t *__restrict__ e4m3)
+{
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = x[i];
+        if (e2m1) e2m1[i] = (uint8_t)(cvt_e2m1x2(v, 0.f) & 0xFu);
+        if (e4m3) e4m3[i] = (uint8_t)(cvt_e4m3x2(v, 0.f) & 0xFFu);
+    }
+}
+
+}  // namespace nvfp4sk

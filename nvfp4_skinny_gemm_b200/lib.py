@@ -1,0 +1,245 @@
+"""ctypes binding of libnvfp4sk (C ABI in include/nvfp4sk.h).
+
+Argument marshalling only: every step runs in the CUDA library.  Functions
+take torch CUDA tensors (or None), pass their device pointers and the current
+CUDA stream, and raise NvFp4Error on a non-zero status.  If the shared library
+is missing, the first call raises -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB_PATH = os.path.join(HERE, "libnvfp4sk.so")
+HEADER = os.path.join(ROOT, "include", "nvfp4sk.h")
+
+BF16, FP32 = 0, 1
+OPT_PDL, OPT_TIMEOUT_NS, OPT_ATTN_SPLITS, OPT_LINEAR_CTAS = 0, 1, 2, 3
+STATUS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED_SHAPE", -3: "MISALIGNED", -4: "WORKSPACE",
+          -5: "CUDA", -6: "TIMEOUT", -7: "OUT_OF_RANGE", -8: "DEVICE"}
+
+
+class NvFp4Error(RuntimeError):
+    def __init__(self, fn, code, msg):
+        super().__init__(f"{fn}: {STATUS.get(code, code)} ({code}): {msg}")
+        self.code = code
+
+
+_lib = None
+_vp, _i64, _int, _sz, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+
+_SIGS = {
+    "nvfp4_quantize_workspace_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_prepared_scale_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_prepare_weight_scales": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "nvfp4_linear": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
+    "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
+                               _vp, _f32, _vp, _vp, _sz, _vp]),
+    "kv_page_restore": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
+    "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "kv_append_fp8": (_int, [_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp, _vp]),
+    "argmax_workspace_bytes": (_sz, [_i64, _i64]),
+    "argmax_rows_bf16": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "nvfp4sk_get_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
+    "nvfp4sk_last_error": (ctypes.c_char_p, []),
+    "nvfp4sk_version": (_int, []),
+    "nvfp4sk_set_option": (_int, [_int, _i64]),
+    "nvfp4sk_get_option": (_i64, [_int]),
+    "nvfp4sk_debug_encode": (_int, [_vp, _i64, _vp, _vp, _vp]),
+}
+
+
+def header_symbols():
+    """Names of the functions include/nvfp4sk.h declares."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^NVFP4SK_API [^(]*?\b([a-z_0-9]+)\(", txt, re.M)))
+
+
+def load(path: str = LIB_PATH):
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"libnvfp4sk.so not found at {path}; build it with "
+                               "`python -m nvfp4_skinny_gemm_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    assert t.is_cuda, "device tensor expected"
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
+
+
+def _check(name, rc):
+    if rc != 0:
+        raise NvFp4Error(name, rc, load().nvfp4sk_last_error().decode())
+
+
+def _call(name, *args):
+    _check(name, getattr(load(), name)(*args))
+
+
+class Workspace:
+    """Zero-filled device scratch that grows on demand (kept zeroed by the calls)."""
+
+    def __init__(self, device=None):
+        self.buf = None
+        self.device = device
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws, nbytes):
+    if ws is None:
+        dev = torch.cuda.current_device()
+        ws = _default_ws.setdefault(dev, Workspace(f"cuda:{dev}"))
+    buf = ws.get(nbytes)
+    return buf.data_ptr(), buf.numel()
+
+
+# ------------------------------------------------------------------ calls
+def set_option(opt, value):
+    _call("nvfp4sk_set_option", opt, int(value))
+
+
+def get_option(opt):
+    return load().nvfp4sk_get_option(opt)
+
+
+def device_status(stream=None):
+    """(status code, site): synchronises the stream, reads and clears the error word."""
+    site = _int(0)
+    rc = load().nvfp4sk_get_device_status(_stream(stream), ctypes.byref(site))
+    return rc, site.value
+
+
+def quantize(x: torch.Tensor, g_in: torch.Tensor | None = None, out=None, ws=None, stream=None):
+    """NVFP4-quantise x [rows, K] (bf16 or fp32, row stride x.stride(0)).
+
+    Returns (codes u8 [rows, K/2], scales u8 [rows, K/16], g f32 [1])."""
+    rows, K = x.shape
+    assert x.stride(1) == 1
+    dt = BF16 if x.dtype == torch.bfloat16 else FP32
+    if out is None:
+        out = (torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device),
+               torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device),
+               torch.empty(1, dtype=torch.float32, device=x.device))
+    codes, scales, g = out
+    wp, wn = _ws(ws, load().nvfp4_quantize_workspace_bytes(rows, K))
+    _call("nvfp4_quantize_act", x.data_ptr(), dt, rows, K, x.stride(0), _p(g_in), codes.data_ptr(),
+          scales.data_ptr(), g.data_ptr(), wp, wn, _stream(stream))
+    return codes, scales, g
+
+
+def prepare_weight_scales(scales: torch.Tensor, N: int, K: int, stream=None):
+    out = torch.empty(load().nvfp4_prepared_scale_bytes(N, K), dtype=torch.uint8, device=scales.device)
+    _call("nvfp4_prepare_weight_scales", scales.data_ptr(), N, K, out.data_ptr(), _stream(stream))
+    return out
+
+
+def linear(a_codes, a_scales, g_a, w_codes, w_prep, g_w, N, K, y=None, residual=None, ws=None, stream=None):
+    """Y [M, N] bf16 = NVFP4 linear (+ residual)."""
+    M = a_codes.shape[0]
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a_codes.device)
+    wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K))
+    _call("nvfp4_linear", a_codes.data_ptr(), a_scales.data_ptr(), g_a.data_ptr(), M, w_codes.data_ptr(),
+          w_prep.data_ptr(), g_w.data_ptr(), N, K, _p(residual), y.data_ptr(), y.stride(0), wp, wn,
+          _stream(stream))
+    return y
+
+
+def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None, out=None,
+              ld_q=None, T=None, Hq=None, ws=None, stream=None):
+    """q bf16 [T, Hq, D] (or a strided [T, >= Hq*D] view with ld_q); pools u8
+    [pages, Hkv, P, D] / [pages, Hkv, D, P]; returns bf16 [T, Hq, D]."""
+    n_pages, Hkv, P, D = k_pool.shape
+    if T is None:
+        T, Hq = q.shape[0], q.shape[1]
+    if ld_q is None:
+        ld_q = q.stride(0)
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=q.device)
+    wp, wn = _ws(ws, load().tree_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)))
+    _call("tree_attn_fp8kv", q.data_ptr(), ld_q, T, Hq, Hkv, D, k_pool.data_ptr(), v_pool.data_ptr(), n_pages, P,
+          page_table.data_ptr(), int(ctx_len), parent.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
+          float(sm_scale), out.data_ptr(), wp, wn, _stream(stream))
+    return out
+
+
+def kv_page_restore(src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, stream=None):
+    n = src_ids.numel() if n is None else n
+    _call("kv_page_restore", src_pool.data_ptr(), src_ids.data_ptr(), dst_pool.data_ptr(), dst_ids.data_ptr(), n,
+          page_bytes, src_pool.numel() // page_bytes, dst_pool.numel() // page_bytes, _stream(stream))
+
+
+def rmsnorm_quantize(x, w, eps, out, stream=None):
+    rows, n = x.shape
+    codes, scales, g = out
+    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, codes.data_ptr(),
+          scales.data_ptr(), g.data_ptr(), None, 0, _stream(stream))
+    return out
+
+
+def swiglu_quantize(gu, out, stream=None):
+    rows, F2 = gu.shape
+    codes, scales, g = out
+    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, codes.data_ptr(), scales.data_ptr(),
+          g.data_ptr(), None, 0, _stream(stream))
+    return out
+
+
+def kv_append(k_new, v_new, ld_new, T, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, stream=None):
+    n_pages, Hkv, P, D = k_pool.shape
+    _call("kv_append_fp8", k_new.data_ptr() if hasattr(k_new, "data_ptr") else k_new,
+          v_new.data_ptr() if hasattr(v_new, "data_ptr") else v_new, ld_new, T, Hkv, D, k_pool.data_ptr(),
+          v_pool.data_ptr(), n_pages, P, page_table.data_ptr(), int(ctx_len), k_scale.data_ptr(),
+          v_scale.data_ptr(), _stream(stream))
+
+
+def argmax(x, idx=None, ws=None, stream=None):
+    rows, n = x.shape
+    if idx is None:
+        idx = torch.empty(rows, dtype=torch.int32, device=x.device)
+    wp, wn = _ws(ws, load().argmax_workspace_bytes(rows, n))
+    _call("argmax_rows_bf16", x.data_ptr(), rows, n, x.stride(0), idx.data_ptr(), wp, wn, _stream(stream))
+    return idx
+
+
+def debug_encode(x: torch.Tensor, stream=None):
+    n = x.numel()
+    e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _call("nvfp4sk_debug_encode", x.data_ptr(), n, e2.data_ptr(), e4.data_ptr(), _stream(stream))
+    return e2, e4

@@ -1,0 +1,146 @@
+"""GPU parity of the tree-masked attention over the FP8 paged cache.
+
+Bar: max |o_gpu - o| <= 2e-3 on bf16 outputs at the 23,552-token workload.
+Small cases, whose outputs are O(1) rather than O(0.01), additionally allow
+the bf16 output rounding and the two-term E4M3 operand error:
+|o_gpu - o| <= 2e-3 + 2^-8 |o|.  Also: page-pool permutation gives
+bit-identical outputs, the split count changes results only within the
+probability-quantisation error, and bad page ids / parents are flagged in the
+device status without any out-of-bounds access."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import ATTN_ABS_TOL, cuda, host, to_dev
+from nvfp4_skinny_gemm_b200 import inputs
+from nvfp4_skinny_gemm_b200 import lib as nv
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev_cache(cache):
+    return (to_dev(cache.k_pool), to_dev(cache.v_pool), to_dev(cache.page_table), to_dev(cache.k_scale),
+            to_dev(cache.v_scale))
+
+
+def _run_gpu(q, cache, parent, dev=None):
+    kp, vp, pt, ks, vs = dev if dev is not None else _dev_cache(cache)
+    out = nv.tree_attn(to_dev(q), kp, vp, pt, cache.ctx_len, to_dev(parent), ks, vs)
+    return host(out)
+
+
+def _tree(kind, T, seed):
+    if kind == "chain":
+        return inputs.chain_parent(T)
+    if kind == "star":
+        p = np.zeros(T, np.int32)
+        p[0] = -1
+        return p
+    return inputs.tree_parent(seed, T)
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,L,kind", [
+    (16, 24, 4, 0, "tree"), (16, 24, 4, 37, "tree"), (16, 24, 4, 1000, "tree"), (1, 24, 4, 100, "chain"),
+    (5, 8, 2, 200, "chain"), (16, 6, 1, 64, "star"), (16, 24, 4, 4096, "tree"), (9, 16, 2, 127, "tree"),
+])
+def test_attention_small(oracle, T, Hq, Hkv, L, kind):
+    cuda()
+    seed = 70 + L % 50 + T
+    cache = inputs.kv_cache(seed, L, T=T, Hkv=Hkv, extra_pages=3)
+    parent = _tree(kind, T, seed)
+    q = inputs.query_bf16(seed, T, Hq)
+    got = _run_gpu(q, cache, parent)
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, L, parent,
+                            cache.k_scale, cache.v_scale)
+    err = np.abs(got - want)
+    bound = ATTN_ABS_TOL + 2.0 ** -8 * np.abs(want)
+    assert np.all(err <= bound), f"max err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
+
+
+def test_attention_full_context(oracle):
+    """The 23,552-token workload: 16-node tree, 24 query / 4 KV heads, FP8 pages."""
+    cuda()
+    L = inputs.CTX_MAX
+    cache = inputs.kv_cache(3, L)
+    parent = inputs.tree_parent(3)
+    q = inputs.query_bf16(3)
+    got = _run_gpu(q, cache, parent)
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, L, parent,
+                            cache.k_scale, cache.v_scale)
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    print(f"config3: max abs err {err.max():.3e}, rel-Frobenius {rel:.3e}, max |o| {np.abs(want).max():.3e}")
+    assert err.max() <= ATTN_ABS_TOL
+    assert rel <= 2e-2
+
+
+def test_page_permutation_bit_identical():
+    cuda()
+    L, T = 3000, 16
+    cache = inputs.kv_cache(75, L, extra_pages=20)
+    parent = inputs.tree_parent(75)
+    q = inputs.query_bf16(75)
+    a = _run_gpu(q, cache, parent)
+    perm = np.random.default_rng(76).permutation(cache.k_pool.shape[0])
+    kp = np.empty_like(cache.k_pool); vp = np.empty_like(cache.v_pool)
+    kp[perm] = cache.k_pool; vp[perm] = cache.v_pool
+    cache.k_pool, cache.v_pool = kp, vp
+    cache.page_table = perm[cache.page_table].astype(np.int32)
+    b = _run_gpu(q, cache, parent)
+    assert np.array_equal(a, b)
+
+
+def test_split_count_invariance():
+    cuda()
+    L = 8192
+    cache = inputs.kv_cache(77, L)
+    parent = inputs.tree_parent(77)
+    q = inputs.query_bf16(77)
+    dev = _dev_cache(cache)
+    outs = []
+    try:
+        for S in (1, 3, 37, 129):
+            nv.set_option(nv.OPT_ATTN_SPLITS, S)
+            outs.append(_run_gpu(q, cache, parent, dev))
+    finally:
+        nv.set_option(nv.OPT_ATTN_SPLITS, 0)
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 5e-4
+
+
+def test_strided_query_view(oracle):
+    """q read in place from a [T, 4096] QKV output (ld_q = 4096)."""
+    cuda()
+    L, T, Hq = 500, 16, 24
+    cache = inputs.kv_cache(78, L)
+    parent = inputs.tree_parent(78)
+    qkv = inputs.bf16_normal(78, 1, (T, 4096))
+    kp, vp, pt, ks, vs = _dev_cache(cache)
+    qd = to_dev(qkv)
+    out = nv.tree_attn(qd, kp, vp, pt, L, to_dev(parent), ks, vs, ld_q=4096, T=T, Hq=Hq)
+    q = qkv[:, :Hq * 128].reshape(T, Hq, 128)
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, L, parent,
+                            cache.k_scale, cache.v_scale)
+    err = np.abs(host(out) - want)
+    assert np.all(err <= ATTN_ABS_TOL + 2.0 ** -8 * np.abs(want))
+
+
+def test_bad_page_id_and_parent_are_flagged():
+    cuda()
+    L = 300
+    cache = inputs.kv_cache(79, L)
+    parent = inputs.tree_parent(79)
+    q = inputs.query_bf16(79)
+    nv.device_status()                       # clear
+    kp, vp, pt, ks, vs = _dev_cache(cache)
+    pt_bad = pt.clone()
+    pt_bad[2] = kp.shape[0] + 5               # page id beyond the pool
+    nv.tree_attn(to_dev(q), kp, vp, pt_bad, L, to_dev(parent), ks, vs)
+    rc, site = nv.device_status()
+    assert rc == -7, (rc, site)
+    bad_parent = parent.copy()
+    bad_parent[4] = 40
+    nv.tree_attn(to_dev(q), kp, vp, pt, L, to_dev(bad_parent), ks, vs)
+    rc, site = nv.device_status()
+    assert rc == -7 and site == 305, (rc, site)
+    assert nv.device_status()[0] == 0
