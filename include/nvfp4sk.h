@@ -29,9 +29,13 @@
  *     problem in a device error word and returns; nvfp4sk_get_device_status()
  *     reports and clears it.
  *   - A "workspace" is caller-owned device scratch of at least the size the
- *     matching *_workspace_bytes() query returns.  It must be zero-filled once
- *     when it is first allocated; every successful call leaves it ready for
- *     the next call.  Calls that share one workspace must be stream-ordered.
+ *     matching *_workspace_bytes() query returns.  The nvfp4_linear and
+ *     argmax_rows_bf16 workspaces start with arrival counters that must read
+ *     zero when a call starts: zero-fill such a workspace once when it is
+ *     allocated and do not lend it to another kind of call (tree_attn_fp8kv
+ *     and nvfp4_quantize_act leave partial results in theirs); every
+ *     successful call leaves its counters zero again.  Calls that share one
+ *     workspace must be stream-ordered.
  *   - Scalars such as tensor scales are device pointers, so no call syncs.
  *   - Error codes are negative; nvfp4sk_last_error() gives a message for the
  *     last failing call of the calling thread.
@@ -113,7 +117,7 @@ NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, in
  * a_codes [M][K/2], a_scales [M][K/16] (canonical), g_a: from
  *   nvfp4_quantize_act.  1 <= M <= 16.
  * w_codes [N][K/2]; w_scales_prepared from nvfp4_prepare_weight_scales; g_w.
- * K % 64 == 0, N >= 1, all code/scale pointers 16-byte aligned.
+ * K % 64 == 0, 1 <= N <= 524288, all code/scale pointers 16-byte aligned.
  * residual: NULL or bf16 [M][ldy] added before rounding (may alias y).
  * y: bf16 [M][ldy], ldy >= N, ldy even.
  * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes (zero-filled once).

@@ -182,7 +182,12 @@ int linear_grid(const DevInfo &d, int64_t U)
     int64_t G = g_opt_linear_ctas > 0 ? g_opt_linear_ctas : d.sms;
     return (int)std::min<int64_t>(G, U);
 }
-size_t linear_ws(int64_t G, int64_t NT) { return up256((size_t)G * 2 * 16 * 128 * 4) + up256((size_t)NT * 4 * 4); }
+// Linear workspace: arrival counters int32 [NT][4] at offset 0 (fixed
+// capacity, so that calls of any shape agree on where they live), then the
+// split-K partial tiles fp32 [G][2][16][128].
+constexpr int64_t LIN_MAX_NT = 4096;
+constexpr size_t LIN_COUNTER_BYTES = LIN_MAX_NT * 4 * 4;
+size_t linear_ws(int64_t G, int64_t NT) { (void)NT; return LIN_COUNTER_BYTES + up256((size_t)G * 2 * 16 * 128 * 4); }
 
 int attn_splits(const DevInfo &d, int Hkv, int64_t n_log)
 {
@@ -338,8 +343,8 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, con
     if (int rc = device_info(&d)) return rc;
     if (!a_codes || !a_scales || !g_a || !w_codes || !w_scales_prepared || !g_w || !y)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (M < 1 || M > 16 || N < 1 || K < 64 || K % 64 != 0 || ldy < N || N > (int64_t)1 << 30 || K > (int64_t)1 << 24)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, N >= 1, K %% 64 == 0, ldy >= N");
+    if (M < 1 || M > 16 || N < 1 || N > LIN_MAX_NT * 128 || K < 64 || K % 64 != 0 || ldy < N || K > (int64_t)1 << 24)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, 1 <= N <= 524288, K %% 64 == 0, ldy >= N");
     if (!al16(a_codes) || !al16(a_scales) || !al16(w_codes) || !al16(w_scales_prepared))
         return fail(NVFP4SK_ERR_MISALIGNED, "code and scale pointers must be 16-byte aligned");
     const int64_t NT = cdiv(N, 128), KT = cdiv(K, 256), U = NT * KT;
@@ -361,8 +366,8 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, con
     p.g_w = g_w;
     p.residual = (const __nv_bfloat16 *)residual;
     p.y = (__nv_bfloat16 *)y;
-    p.partial = (float *)ws;
-    p.counters = (int *)((uint8_t *)ws + up256((size_t)G * 2 * 16 * 128 * 4));
+    p.counters = (int *)ws;
+    p.partial = (float *)((uint8_t *)ws + LIN_COUNTER_BYTES);
     p.ldy = ldy;
     p.U = U;
     p.M = (int)M;
@@ -523,10 +528,14 @@ nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_ne
                     "kv_append_kernel");
 }
 
+// Argmax workspace: arrival counters int32 [rows] at offset 0 (fixed
+// capacity), then per-chunk values fp32 [rows][nch] and indices i32 [rows][nch].
+constexpr int64_t AMX_MAX_ROWS = 4096;
+constexpr size_t AMX_COUNTER_BYTES = AMX_MAX_ROWS * 4;
 size_t argmax_workspace_bytes(int64_t rows, int64_t n)
 {
     const int nch = argmax_chunks(n);
-    return up256((size_t)rows * nch * 4) * 2 + up256((size_t)rows * 4);
+    return AMX_COUNTER_BYTES + up256((size_t)rows * nch * 4) * 2;
 }
 
 nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t ld, int32_t *idx, void *ws,
@@ -535,15 +544,15 @@ nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t 
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
     if (!x || !idx) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (rows < 1 || rows > 65535 || n < 1 || n > INT32_MAX || ld < n)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "bad shape");
+    if (rows < 1 || rows > AMX_MAX_ROWS || n < 1 || n > INT32_MAX || ld < n)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 4096, ld >= n");
     const size_t need = argmax_workspace_bytes(rows, n);
     if (!ws || ws_bytes < need) return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes", need);
     const int nch = argmax_chunks(n);
     uint8_t *b = (uint8_t *)ws;
-    float *pv = (float *)b;
-    int32_t *pi = (int32_t *)(b + up256((size_t)rows * nch * 4));
-    int32_t *cnt = (int32_t *)(b + 2 * up256((size_t)rows * nch * 4));
+    int32_t *cnt = (int32_t *)b;
+    float *pv = (float *)(b + AMX_COUNTER_BYTES);
+    int32_t *pi = (int32_t *)(b + AMX_COUNTER_BYTES + up256((size_t)rows * nch * 4));
     return launched(launch(argmax_rows_kernel, dim3(nch, rows), dim3(AMX_THREADS), 0, (cudaStream_t)stream, 1,
                            (const __nv_bfloat16 *)x, n, ld, idx, pv, pi, cnt),
                     "argmax_rows_kernel");

@@ -118,10 +118,13 @@ class Workspace:
 _default_ws = {}
 
 
-def _ws(ws, nbytes):
+def _ws(ws, nbytes, kind):
+    """Workspace pointer and size; by default one zero-filled buffer per
+    (device, op kind): the linear and argmax workspaces hold arrival counters
+    that must read zero at call start, which another op's partials would break."""
     if ws is None:
         dev = torch.cuda.current_device()
-        ws = _default_ws.setdefault(dev, Workspace(f"cuda:{dev}"))
+        ws = _default_ws.setdefault((dev, kind), Workspace(f"cuda:{dev}"))
     buf = ws.get(nbytes)
     return buf.data_ptr(), buf.numel()
 
@@ -154,7 +157,7 @@ def quantize(x: torch.Tensor, g_in: torch.Tensor | None = None, out=None, ws=Non
                torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device),
                torch.empty(1, dtype=torch.float32, device=x.device))
     codes, scales, g = out
-    wp, wn = _ws(ws, load().nvfp4_quantize_workspace_bytes(rows, K))
+    wp, wn = _ws(ws, load().nvfp4_quantize_workspace_bytes(rows, K), "quantize")
     _call("nvfp4_quantize_act", x.data_ptr(), dt, rows, K, x.stride(0), _p(g_in), codes.data_ptr(),
           scales.data_ptr(), g.data_ptr(), wp, wn, _stream(stream))
     return codes, scales, g
@@ -171,7 +174,7 @@ def linear(a_codes, a_scales, g_a, w_codes, w_prep, g_w, N, K, y=None, residual=
     M = a_codes.shape[0]
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a_codes.device)
-    wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K))
+    wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K), "linear")
     _call("nvfp4_linear", a_codes.data_ptr(), a_scales.data_ptr(), g_a.data_ptr(), M, w_codes.data_ptr(),
           w_prep.data_ptr(), g_w.data_ptr(), N, K, _p(residual), y.data_ptr(), y.stride(0), wp, wn,
           _stream(stream))
@@ -191,7 +194,7 @@ def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, 
         sm_scale = D ** -0.5
     if out is None:
         out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=q.device)
-    wp, wn = _ws(ws, load().tree_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)))
+    wp, wn = _ws(ws, load().tree_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)), "attn")
     _call("tree_attn_fp8kv", q.data_ptr(), ld_q, T, Hq, Hkv, D, k_pool.data_ptr(), v_pool.data_ptr(), n_pages, P,
           page_table.data_ptr(), int(ctx_len), parent.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
           float(sm_scale), out.data_ptr(), wp, wn, _stream(stream))
@@ -232,7 +235,7 @@ def argmax(x, idx=None, ws=None, stream=None):
     rows, n = x.shape
     if idx is None:
         idx = torch.empty(rows, dtype=torch.int32, device=x.device)
-    wp, wn = _ws(ws, load().argmax_workspace_bytes(rows, n))
+    wp, wn = _ws(ws, load().argmax_workspace_bytes(rows, n), "argmax")
     _call("argmax_rows_bf16", x.data_ptr(), rows, n, x.stride(0), idx.data_ptr(), wp, wn, _stream(stream))
     return idx
 
