@@ -1,0 +1,429 @@
+"""Benchmark: the 64-layer tree-MTP verify step (27B-class dense model, NVFP4
+W4A4 linears incl. the LM head, FP8 paged KV cache, 16-node tree, 23,552
+cached tokens, kv_page_restore of the reused 96% prefix) on one B200 per rank.
+
+One step = restore of the prefix pages + 64 layers + LM head + argmax, captured
+as one CUDA graph.  `value` is verify steps/s over all ranks (replicas: each
+rank verifies its own tree), timed on the device with CUDA events around K
+graph replays, max over ranks.  `e2e` adds, per step, the host->device copy of
+the step's inputs (16 hidden rows + parent array, pinned) and the
+device->host read of the 16 argmax ids.  Weights (11.4 GB) far exceed L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HBM GB/s (% of B200 peak) for NVFP4 linear + tree attn at M=16; verify steps/s"
+UNIT = "verify steps/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ctx", type=int, default=23552)
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", default=None,
+                    choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "attn", "restore", "quantize"],
+                    help="run one kernel on a small case (for ncu captures) instead of the step")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.distributed.get_backend() == "nccl" else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    """nvidia-smi sampling (200 ms) during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", uuid], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ peaks / traffic
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("linear.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "nvfp4_skinny_gemm_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per linear launch of the step, from the committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "nvfp4_linear_verify_step.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"traffic_bytes_per_step_of_linears:\s*([0-9.eE+]+)\s+source:\s*([0-9a-f]+)", txt)
+    if m and m.group(2) == kernel_source_hash():
+        return float(m.group(1))
+    return None
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+def oracle_sample(ctx, layers, seconds_hint=15.0):
+    """Time the CPU oracle on a bounded sample of one verify step and
+    extrapolate to a whole step.  Returns (steps/s, threads, description)."""
+    import oracle
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    T = I.TREE_NODES
+    rng = np.random.default_rng(7)
+    est = {}
+    t_lin = 0.0
+    ns = 1024
+    for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items()):
+        w = I.weight_fp32(4, t, N, K, sub=0)
+        wc, ws, gw = oracle.quantize(w)
+        del w
+        a = I.activation_bf16(4, 100 + t, T, K, 0.01).float().numpy()
+        t0 = time.perf_counter()
+        ac, asc, ga = oracle.quantize(a)
+        im, inn = rng.integers(0, T, ns), rng.integers(0, N, ns)
+        oracle.linear_sampled(ac, asc, ga, wc, ws, gw, im, inn)
+        dt = time.perf_counter() - t0
+        t_lin += dt * (T * N) / ns
+        est[name] = dt * (T * N) / ns
+    cache = I.kv_cache(4, ctx, T=T, Hkv=1)
+    q = I.query_bf16(4, T, 6).float().numpy()
+    parent = I.tree_parent(4)
+    t0 = time.perf_counter()
+    oracle.tree_attn(q, cache.k_pool, cache.v_pool, cache.page_table, ctx, parent, cache.k_scale, cache.v_scale)
+    t_att = (time.perf_counter() - t0) * I.N_KV_HEADS
+    pb, n_pages = 32768, 256
+    src = np.random.default_rng(1).integers(0, 256, n_pages * pb, dtype=np.uint8)
+    dst = np.zeros_like(src)
+    ids = np.arange(n_pages, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.kv_page_restore(src, ids, dst, ids, pb)
+    n_restore = layers * 2 * math.ceil(round(0.96 * ctx) / 64)
+    t_rst = (time.perf_counter() - t0) * n_restore / n_pages
+    w = I.weight_fp32(4, 9, 4096, I.HIDDEN)
+    wc, ws, gw = oracle.quantize(w)
+    a = I.activation_bf16(4, 200, T, I.HIDDEN).float().numpy()
+    t0 = time.perf_counter()
+    ac, asc, ga = oracle.quantize(a)
+    im, inn = rng.integers(0, T, ns), rng.integers(0, 4096, ns)
+    oracle.linear_sampled(ac, asc, ga, wc, ws, gw, im, inn)
+    t_head = (time.perf_counter() - t0) * T * I.VOCAB / ns
+    step = layers * (t_lin + t_att) + t_head + t_rst
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = (f"oracle (fp64 C, OpenMP) on one layer's linears ({ns} sampled outputs each of 16xN), "
+            f"attention of 1 of 4 KV heads at ctx {ctx}, restore of {n_pages} of {n_restore} pages, "
+            f"LM head {ns} sampled logits; extrapolated to {layers} layers + LM head + restore "
+            f"({step:.1f} s per step)")
+    return 1.0 / step, threads, desc
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        pass
+    vals, desc, threads = [], "", 1
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        v, threads, desc = oracle_sample(args.ctx, args.layers)
+        vals.append(v)
+        if time.perf_counter() - t0 > 240:
+            break
+    v = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": len(vals), "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"64-layer 27B-class verify step, 16-node tree, ctx {args.ctx} FP8 paged KV, "
+                                   f"NVFP4 W4A4 linears + LM head, kv_page_restore of 96% prefix",
+                       "layers": args.layers, "ctx": args.ctx, "tree_nodes": 16, "parallelism": "replicas"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    from nvfp4_skinny_gemm_b200.step import VerifyModel
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    model = VerifyModel(n_layers=args.layers, ctx_len=args.ctx, weights="device", device=dev)
+    h0 = I.bf16_normal(4, 300, (I.TREE_NODES, I.HIDDEN)).pin_memory()
+    par0 = torch.from_numpy(I.tree_parent(4)).pin_memory()
+    ids_host = torch.empty(I.TREE_NODES, dtype=torch.int32).pin_memory()
+    stream = torch.cuda.Stream(device=dev)
+
+    def load_inputs():
+        model.h.copy_(h0, non_blocking=True)
+        model.parent.copy_(par0, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        load_inputs()
+        model.step()                                       # eager: allocates workspaces
+        torch.cuda.synchronize()
+        rc, site = nv.device_status(stream)
+        assert rc == 0, f"device status {rc} at site {site}"
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            model.step()
+        lin_graph = torch.cuda.CUDAGraph()                 # the dominant kernel alone, same launches
+        with torch.cuda.graph(lin_graph, stream=stream):
+            for lay in model.layers:
+                model._linear(model.q_h, lay["qkv"], model.qkv)
+                model._linear(model.q_a, lay["o"], model.h, residual=model.h)
+                model._linear(model.q_h, lay["gate_up"], model.gu)
+                model._linear(model.q_f, lay["down"], model.h, residual=model.h)
+            model._linear(model.q_h, model.lm_head, model.logits)
+        load_inputs()
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+
+        # ---- device-timed step
+        barrier(world)
+        torch.cuda.synchronize()
+        clocks = Clocks(dev)
+        time.sleep(0.3)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        t_dev = max_over_ranks(ev0.elapsed_time(ev1) * 1e-3, world)
+        rc, site = nv.device_status(stream)
+        assert rc == 0, f"device status {rc} at site {site}"
+
+        # ---- dominant kernel: all linear launches of one step, back to back
+        reps = max(3, min(20, args.steps))
+        for _ in range(2):
+            lin_graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            lin_graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_lin = e0.elapsed_time(e1) * 1e-3 / reps
+        n_lin = 4 * model.n_layers + 1
+
+        # ---- end to end: pinned host inputs in, argmax ids out, every step
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            load_inputs()
+            graph.replay()
+            ids_host.copy_(model.ids, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
+
+    peak, peak_kind = measured_peak()
+    lin_bytes = model.linear_bytes()
+    achieved = lin_bytes / t_lin / 1e9
+    traffic = recorded_traffic()
+    step_bytes = model.step_bytes()
+    value = world * args.steps / t_dev
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate); fp8 e4m3 KV",
+        "data": "synthetic",
+        "config": {"workload": f"64-layer 27B-class verify step, 16-node tree, ctx {args.ctx} FP8 paged KV, "
+                               f"NVFP4 W4A4 linears + LM head, kv_page_restore of 96% prefix",
+                   "layers": args.layers, "ctx": args.ctx, "tree_nodes": 16, "hidden": I.HIDDEN,
+                   "weights_gb": round(sum(l.nbytes for lay in model.layers for l in lay.values()) / 1e9
+                                       + model.lm_head.nbytes / 1e9, 3),
+                   "l2": "inputs larger than L2 (11.4 GB of weights streamed per step)",
+                   "parallelism": f"replicas x{world}"},
+        "step_pct_of_peak": round(100 * step_bytes / (t_dev / args.steps) / 1e9 / peak, 1),
+        "roofline": {"kernel": "nvfp4_linear_kernel (all 257 linear launches of one step, back to back)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_step": lin_bytes, "launches": n_lin,
+                     "us_per_step_of_linears": round(t_lin * 1e6, 1),
+                     "traffic": traffic},
+        "clocks": clk,
+        "e2e": {"value": world * args.steps / t_e2e, "unit": UNIT,
+                "h2d_bytes_per_step": h0.numel() * 2 + par0.numel() * 4,
+                "d2h_bytes_per_step": ids_host.numel() * 4},
+        "gpu_launches": model.launches_per_step() * args.steps,
+    }
+    line["step_hbm_gbs"] = round(step_bytes / (t_dev / args.steps) / 1e9, 1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, desc = oracle_sample(args.ctx, args.layers)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph, lin_graph
+
+
+# ------------------------------------------------------------------ single-kernel cases
+def run_kernel_case(args):
+    """A few launches of one kernel on a small case (a few GB at most): the
+    command that ncu captures for the per-kernel profiles."""
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    case = args.kernel_case
+    if case.startswith("linear"):
+        K, N = {"linear_lmhead": (I.HIDDEN, I.VOCAB), "linear_gate_up": I.LAYER_LINEARS["gate_up"],
+                "linear_qkv": I.LAYER_LINEARS["qkv"]}[case]
+        ncopy = max(1, math.ceil(400e6 / (N * K * 9 // 16)))     # rotate copies: > L2 per sweep
+        ws = []
+        for _ in range(ncopy):
+            c = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+            sc = torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g)
+            ws.append((nv.prepare_weight(c, sc, N, K), torch.full((1,), 0.01, device=dev)))
+            del c, sc
+        a = torch.randn(16, K, device=dev, generator=g).to(torch.bfloat16)
+        act = nv.act_buffer(K)
+        _, _, ga = nv.quantize(a, act=act)
+        y = torch.empty(16, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: nv.linear(act, ga, 16, ws[i % ncopy][0], ws[i % ncopy][1], N, K, y=y)
+        nbytes = N * K * 9 // 16
+    elif case == "attn":
+        cache = I.kv_cache(3, I.CTX_MAX)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+        kp, vp, pt, ks, vs = t(cache.k_pool), t(cache.v_pool), t(cache.page_table), t(cache.k_scale), t(cache.v_scale)
+        par, q = t(I.tree_parent(3)), I.query_bf16(3).to(dev)
+        out = torch.empty(16, 24, 128, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: nv.tree_attn(q, kp, vp, pt, I.CTX_MAX, par, ks, vs, out=out)
+        nbytes = (I.CTX_MAX + 16) * 4 * 128 * 2
+    elif case == "restore":
+        pb, n = 32768, 354 * 128
+        src = torch.empty((n + 64) * pb, dtype=torch.uint8, device=dev)
+        dst = torch.empty((n + 64) * pb, dtype=torch.uint8, device=dev)
+        sid = torch.randperm(n + 64, device=dev, generator=g)[:n].to(torch.int32)
+        did = torch.randperm(n + 64, device=dev, generator=g)[:n].to(torch.int32)
+        fn = lambda i: nv.kv_page_restore(src, sid, dst, did, pb)
+        nbytes = 2 * n * pb
+    else:
+        x = torch.randn(16, I.FFN, device=dev, generator=g).to(torch.bfloat16)
+        fn = lambda i: nv.quantize(x)
+        nbytes = x.numel() * 2
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(3):
+        fn(i + 3)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) * 1e-3 / 3
+    print(json.dumps({"kernel_case": case, "us_per_call_incl_launch": round(t * 1e6, 2),
+                      "algorithmic_bytes": nbytes, "status": nv.device_status()[0]}), flush=True)
+
+
+def main():
+    args = parse()
+    if args.kernel_case:
+        torch.cuda.set_device(0)
+        run_kernel_case(args)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -79,32 +79,45 @@ enum { NVFP4SK_BF16 = 0, NVFP4SK_FP32 = 1 };
  *    stride ld_x elements.  K % 16 == 0, ld_x >= K, x 16-byte aligned and
  *    ld_x * element size a multiple of 16 bytes.
  * g_in: device fp32 tensor scale, or NULL for the dynamic per-tensor scale
- *    g = fp32(amax(|x|) / 2688) (g = 1 when x is all zero).
+ *    g = fp32(amax(|x|) / 2688) (g = 1 when x is all zero).  g must be > 0.
  * Per 16-element block b of a row: r = fp32(amax_b / 6), t = fp32(r / g),
  *    scale = E4M3(t) (round-to-nearest-even, saturating at 448),
  *    s = fp32(value(scale) * g), code_k = s == 0 ? +0 : E2M1(fp32(x_k / s))
  *    (round-to-nearest-even, saturating at 6, sign kept).
- * codes:  u8 [rows][K/2], two codes per byte, even k in the low nibble.
- * scales: u8 [rows][K/16] E4M3 (canonical row-major layout).
- * g_out:  device fp32, receives g (may equal g_in).
+ * Outputs (codes + scales, and/or act_prepared):
+ *   codes:  u8 [rows][K/2], two codes per byte, even k in the low nibble.
+ *   scales: u8 [rows][K/16] E4M3 (canonical row-major layout).
+ *   g_out:  device fp32, receives g (may equal g_in).
+ *   act_prepared: NULL, or the same codes and scales in the tile image that
+ *     nvfp4_linear streams (nvfp4_prepared_act_bytes(K) bytes, 16-byte
+ *     aligned, zero-filled once at allocation; needs rows <= 16, K % 64 == 0).
  * ws: workspace of nvfp4_quantize_workspace_bytes(rows, K) bytes.
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K);
+NVFP4SK_API size_t nvfp4_prepared_act_bytes(int64_t K);
 NVFP4SK_API nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int64_t K, int64_t ld_x,
-                                  const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
-                                  void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
+                                              const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
+                                              uint8_t *act_prepared, void *ws, size_t ws_bytes,
+                                              nvfp4sk_stream_t stream);
+
+/* Re-layout of canonical NVFP4 activation codes [rows][K/2] and scales
+ * [rows][K/16] (e.g. quantised elsewhere) into act_prepared, byte-identical to
+ * what nvfp4_quantize_act writes there.  rows <= 16, K % 64 == 0. */
+NVFP4SK_API nvfp4sk_status nvfp4_prepare_act(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,
+                                             uint8_t *act_prepared, nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * nvfp4_prepare_weight_scales -- one-time rearrangement of a weight's
- * canonical E4M3 block scales [N][K/16] into the tile order that
- * nvfp4_linear streams into tensor memory.  Offline step for the NVFP4
- * weights of section "NVFP4 and FP8" (calibrated once, then served).
- * prepared: u8 buffer of nvfp4_prepared_scale_bytes(N, K) bytes (opaque).
- * K % 64 == 0.
+ * nvfp4_prepare_weight -- one-time rearrangement of an NVFP4 weight (codes
+ * [N][K/2], canonical E4M3 scales [N][K/16]) into the tile image that
+ * nvfp4_linear streams: per 128-row x 512-K unit, 32 KB of 128-byte-swizzled
+ * codes followed by 4 KB of tensor-memory scale images, contiguous.  Offline
+ * step for the NVFP4 weights of section "NVFP4 and FP8" (calibrated once,
+ * then served).  prepared: nvfp4_prepared_weight_bytes(N, K) bytes, 16-byte
+ * aligned (opaque).  K % 64 == 0; rows/columns beyond N/K are zero-padded.
  * ---------------------------------------------------------------------- */
-NVFP4SK_API size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K);
-NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, int64_t N, int64_t K, uint8_t *prepared,
-                                           nvfp4sk_stream_t stream);
+NVFP4SK_API size_t nvfp4_prepared_weight_bytes(int64_t N, int64_t K);
+NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K,
+                                                uint8_t *prepared, nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * nvfp4_linear -- the W4A4 NVFP4 linear layer of the verify step at
@@ -114,19 +127,19 @@ NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, in
  * a[m,k] w[n,k]  (+ residual[m][n]) ), fp32 accumulation on tcgen05
  * block-scaled tensor cores, split-K across all SMs.
  *
- * a_codes [M][K/2], a_scales [M][K/16] (canonical), g_a: from
- *   nvfp4_quantize_act.  1 <= M <= 16.
- * w_codes [N][K/2]; w_scales_prepared from nvfp4_prepare_weight_scales; g_w.
- * K % 64 == 0, 1 <= N <= 524288, all code/scale pointers 16-byte aligned.
+ * a_prepared, g_a: activation from nvfp4_quantize_act (act_prepared) or the
+ *   fused quantisers; 1 <= M <= 16 rows.
+ * w_prepared, g_w: weight from nvfp4_prepare_weight (+ its tensor scale).
+ * K % 64 == 0, 1 <= N <= 524288; prepared operands 16-byte aligned.
  * residual: NULL or bf16 [M][ldy] added before rounding (may alias y).
- * y: bf16 [M][ldy], ldy >= N, ldy even.
- * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes (zero-filled once).
+ * y: bf16 [M][ldy], ldy >= N.
+ * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes (see workspace rule).
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
-NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, int64_t M,
-                            const uint8_t *w_codes, const uint8_t *w_scales_prepared, const float *g_w,
-                            int64_t N, int64_t K, const void *residual, void *y, int64_t ldy, void *ws,
-                            size_t ws_bytes, nvfp4sk_stream_t stream);
+NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t M,
+                                        const uint8_t *w_prepared, const float *g_w, int64_t N, int64_t K,
+                                        const void *residual, void *y, int64_t ldy, void *ws, size_t ws_bytes,
+                                        nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * tree_attn_fp8kv -- attention of the T tree nodes over the FP8 paged KV
@@ -146,7 +159,7 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a
  * Node i, head hq (KV head h = hq / (Hq/Hkv)) attends to every context
  *   position and to the tree positions of {i} and its ancestors:
  *   out = softmax_p(sm_scale * q . K_p) . V_p, bf16 [T][Hq][D] (dense).
- * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 8.
+ * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 7.
  * ws: tree_attn_workspace_bytes(...) bytes.
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
@@ -178,16 +191,18 @@ NVFP4SK_API nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_
  * kernel that produces them).
  * ---------------------------------------------------------------------- */
 /* y = x / sqrt(mean(x^2) + eps) * w rounded to bf16, then NVFP4-quantised
- * exactly as nvfp4_quantize_act (dynamic g).  x bf16 [rows][n] (row stride
- * n), w bf16 [n].  rows <= 16, n % 16 == 0, n <= 8192. */
-NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows, int64_t n,
-                                      uint8_t *codes, uint8_t *scales, float *g_out, void *ws,
-                                      size_t ws_bytes, nvfp4sk_stream_t stream);
+ * exactly as nvfp4_quantize_act (dynamic g), with the same outputs.  x bf16
+ * [rows][n] (row stride n), w bf16 [n].  rows <= 16, n % 64 == 0, n <= 8192. */
+NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows,
+                                                  int64_t n, uint8_t *codes, uint8_t *scales, float *g_out,
+                                                  uint8_t *act_prepared, void *ws, size_t ws_bytes,
+                                                  nvfp4sk_stream_t stream);
 /* h = silu(gu[:, :F]) * gu[:, F:] rounded to bf16, then NVFP4-quantised
- * (dynamic g).  gu bf16 [rows][2F].  rows <= 16, F % 16 == 0, F <= 32768. */
+ * (dynamic g), same outputs.  gu bf16 [rows][2F].  rows <= 16, F % 64 == 0,
+ * rows * F <= 524288. */
 NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes,
-                                     uint8_t *scales, float *g_out, void *ws, size_t ws_bytes,
-                                     nvfp4sk_stream_t stream);
+                                                 uint8_t *scales, float *g_out, uint8_t *act_prepared, void *ws,
+                                                 size_t ws_bytes, nvfp4sk_stream_t stream);
 /* Append T new tokens' K and V (bf16, token i head h at k_new[i*ld_new +
  * h*D + d]) to the cache at positions ctx_len .. ctx_len+T-1 as
  * E4M3(fp32(x / scale[h])) (round-to-nearest-even, saturating); the FP8 KV

@@ -50,7 +50,7 @@ struct AttnParams {
 
 __device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -90,7 +90,7 @@ __device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint32_t &hi2, 
     lo2 = l & 0xFFFFu;
 }
 
-__global__ void __launch_bounds__(9 * 32, 1)
+__global__ void __launch_bounds__(8 * 32, 1)
     tree_attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const AttnParams p)
 {
     extern __shared__ uint8_t att_smem_raw[];
@@ -245,17 +245,24 @@ __global__ void __launch_bounds__(9 * 32, 1)
             const int64_t pos0 = (int64_t)(pg0 + i) * ATT_P;
             float sacc[8][4];
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-                const int tok = 16 * (g >> 1) + 8 * (nt >> 2) + 4 * ((nt & 3) >> 1) + 2 * (nt & 1) + (g & 1);
+            for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            // k-steps outermost so that consecutive MMAs update different n-tiles
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(kt + tok * 128 + (((2 * c + u) ^ (tok & 7)) << 4));
-                    mma_e4m3_16832(sacc[nt], qa_hi[2 * u], w.x, w.y);
-                    mma_e4m3_16832(sacc[nt], qa_lo[2 * u], w.x, w.y);
-                    mma_e4m3_16832(sacc[nt], qa_hi[2 * u + 1], w.z, w.w);
-                    mma_e4m3_16832(sacc[nt], qa_lo[2 * u + 1], w.z, w.w);
+            for (int u = 0; u < 2; ++u) {
+                uint4 kw[8];
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    const int tok = 16 * (g >> 1) + 8 * (nt >> 2) + 4 * ((nt & 3) >> 1) + 2 * (nt & 1) + (g & 1);
+                    kw[nt] = *reinterpret_cast<const uint4 *>(kt + tok * 128 + (((2 * c + u) ^ (tok & 7)) << 4));
                 }
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_hi[2 * u], kw[nt].x, kw[nt].y);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_hi[2 * u + 1], kw[nt].z, kw[nt].w);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_lo[2 * u], kw[nt].x, kw[nt].y);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_lo[2 * u + 1], kw[nt].z, kw[nt].w);
             }
             // scale, mask, row max
             const bool tail = pos0 + ATT_P > L;
@@ -314,15 +321,25 @@ __global__ void __launch_bounds__(9 * 32, 1)
             }
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) l_run[rr] = l_run[rr] * alpha[rr] + psum[rr];
+            // four dimension tiles at a time: their MMAs are independent
 #pragma unroll
-            for (int nd = 0; nd < 16; ++nd) {
-                O[nd][0] *= alpha[0]; O[nd][1] *= alpha[0];
-                O[nd][2] *= alpha[1]; O[nd][3] *= alpha[1];
-                const uint4 x = *reinterpret_cast<const uint4 *>(vt + (8 * nd + g) * ATT_P + 16 * c);
-                mma_e4m3_16832(O[nd], pa_hi[0], x.x, x.y);
-                mma_e4m3_16832(O[nd], pa_lo[0], x.x, x.y);
-                mma_e4m3_16832(O[nd], pa_hi[1], x.z, x.w);
-                mma_e4m3_16832(O[nd], pa_lo[1], x.z, x.w);
+            for (int nd0 = 0; nd0 < 16; nd0 += 4) {
+                uint4 x[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int nd = nd0 + k;
+                    O[nd][0] *= alpha[0]; O[nd][1] *= alpha[0];
+                    O[nd][2] *= alpha[1]; O[nd][3] *= alpha[1];
+                    x[k] = *reinterpret_cast<const uint4 *>(vt + (8 * nd + g) * ATT_P + 16 * c);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_hi[0], x[k].x, x[k].y);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_hi[1], x[k].z, x[k].w);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_lo[0], x[k].x, x[k].y);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_lo[1], x[k].z, x[k].w);
             }
         }
         __syncwarp();

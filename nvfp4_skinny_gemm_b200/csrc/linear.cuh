@@ -7,18 +7,29 @@
 //   M = 128 weight rows, N = 16 tokens, K = 64 per instruction,
 //   fp32 accumulator in tensor memory, UE4M3 scales (one per 16 K) in TMEM.
 //
-// Work unit = one 128-row x 256-K weight tile (16 KB codes + 2 KB scales).
-// The NT x KT units are cut into G = min(#SMs, units) contiguous ranges
-// (stream-K split-K): every CTA streams the same number of weight bytes.
-// A tile whose K range is split over several CTAs is reduced by the CTA that
-// finishes it last (per-tile arrival counter); partial sums are added in
-// contributor order, so results do not depend on timing.
+// Operands arrive pre-tiled in exactly the shared-memory image the MMA reads
+// (128-byte swizzled E2M1 rows, scale factors as the 32 x 16-byte blocks that
+// tcgen05.cp replicates into tensor memory):
+//   weight unit (tile t of 128 rows, chunk c of 512 K):  36 KB contiguous
+//     [2 x 16 KB codes (one per 256-K swizzle atom) | 8 x 512 B scale images]
+//   activation chunk c: 8 KB contiguous
+//     [2 x 2 KB codes (16 rows) | 8 x 512 B scale images]
+// so one pipeline stage is two bulk copies (cp.async.bulk) and nothing else.
+// (A single issuing thread sustains ~7 TB/s over the GPU with >= 32 KB
+// requests; small per-tile requests and generic shared-memory writes were
+// what limited the earlier 2-D tensor-map version to ~3.4 TB/s.)
+//
+// Work unit = one weight unit.  The NT x KC units are cut into
+// G = min(#SMs, units) contiguous ranges (stream-K split-K), so every CTA
+// streams the same number of weight bytes.  A tile whose K range is split
+// over several CTAs is reduced by the CTA that finishes it last (per-tile,
+// per-sub-partition arrival counter); partial sums are added in contributor
+// order, so results do not depend on timing.
 //
 // Warp roles (192 threads, one CTA per SM):
-//   warp 0   TMA producer: weight tile (2-D tensor map, 128B swizzle) and
-//            prepared weight scales (1-D bulk copy) for the first stages are
-//            issued before griddepcontrol.wait (they never depend on the
-//            previous kernel); activation tile + activation scales after it.
+//   warp 0   producer: weight units of the first stages are requested before
+//            griddepcontrol.wait (weights never depend on the previous
+//            kernel); activation chunks after it.
 //   warp 1   allocates TMEM; lane 0 copies scales smem->TMEM (tcgen05.cp) and
 //            issues the MMAs, releasing stages with tcgen05.commit.
 //   warps 2-5 epilogue: tcgen05.ld of the 128x16 accumulator, scale by
@@ -28,17 +39,24 @@
 
 namespace nvfp4sk {
 
-constexpr int LIN_STAGES = 8;
+constexpr int LIN_STAGES = 4;
 constexpr int LIN_THREADS = 192;
-constexpr uint32_t LIN_W_BYTES = 128 * 128;   // 128 rows x 256 E2M1
-constexpr uint32_t LIN_A_BYTES = 16 * 128;    // 16 rows x 256 E2M1
-constexpr uint32_t LIN_SF_BYTES = 2048;       // 4 x (32 x 16 B)
-constexpr uint32_t LIN_STAGE_BYTES = LIN_W_BYTES + LIN_A_BYTES + 2 * LIN_SF_BYTES;   // 22528
-constexpr uint32_t LIN_TX_BYTES = LIN_W_BYTES + LIN_A_BYTES + LIN_SF_BYTES;
-constexpr uint32_t LIN_SMEM_BYTES = LIN_STAGES * LIN_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t LIN_TMEM_COLS = 128;
-// TMEM column map: acc[b] at 16*b, SFA[r] at 32 + 16*r, SFB[r] at 64 + 16*r
-constexpr uint32_t TM_ACC = 0, TM_SFA = 32, TM_SFB = 64;
+constexpr int LIN_KC = 512;                       // K elements per unit / chunk
+constexpr int LIN_KSTEPS = LIN_KC / 64;           // MMA steps per unit
+constexpr uint32_t LIN_W_ATOM = 128 * 128;        // 128 rows x 256 E2M1, swizzled
+constexpr uint32_t LIN_A_ATOM = 16 * 128;         // 16 rows x 256 E2M1, swizzled
+constexpr uint32_t LIN_SF_IMG = 512;              // 32 lines x 16 B
+constexpr uint32_t LIN_W_UNIT = 2 * LIN_W_ATOM + LIN_KSTEPS * LIN_SF_IMG;    // 36864
+constexpr uint32_t LIN_A_UNIT = 2 * LIN_A_ATOM + LIN_KSTEPS * LIN_SF_IMG;    // 8192
+constexpr uint32_t LIN_STAGE_BYTES = LIN_W_UNIT + LIN_A_UNIT;                // 45056 = 44 * 1024
+constexpr uint32_t LIN_OFF_BAR = LIN_STAGES * LIN_STAGE_BYTES;
+constexpr uint32_t LIN_SMEM_BYTES = LIN_OFF_BAR + 256 + 1024;
+constexpr uint32_t LIN_TMEM_COLS = 256;
+// TMEM columns: acc[b] at 16*b (16 fp32 columns = 16 tokens); weight scales
+// SFA[r] at 32 + 32*r and activation scales SFB[r] at 96 + 32*r, 4 columns
+// per MMA step.  Scale-factor column addresses handed to the MMA stay
+// multiples of 4.
+constexpr uint32_t TM_ACC = 0, TM_SFA = 32, TM_SFB = 96;
 
 // Instruction descriptor (kind::mxf4nvf4): A/B format E2M1 (1) in bits 7-9 and
 // 10-12, K-major A and B, N>>3 in bits 17-22, scale format UE4M3 (0) in
@@ -49,29 +67,28 @@ constexpr uint32_t lin_idesc(uint32_t M, uint32_t N)
 }
 
 struct LinearParams {
-    const uint8_t *w_sf;           // prepared weight scales [NT][KT][2048]
-    const uint8_t *a_scales;       // [M][K/16]
+    const uint8_t *w;              // prepared weight units [NT][KC][36864]
+    const uint8_t *a;              // prepared activation chunks [KC][8192]
     const float *g_a;
     const float *g_w;
     const __nv_bfloat16 *residual; // nullable, [M][ldy]
     __nv_bfloat16 *y;              // [M][ldy]
-    float *partial;                // [G][2][16][128]
+    float *partial;                // [G][2][128 rows][16 tokens]
     int *counters;                 // [NT][4] (one per TMEM sub-partition)
     int64_t ldy;
-    int64_t U;                     // NT * KT
-    int M, N, K, NT, KT;
+    int64_t U;                     // NT * KC
+    int M, N, NT, KC;
 };
 
 __device__ __forceinline__ int64_t lin_start(int64_t c, int64_t U, int64_t G) { return c * U / G; }
 __device__ __forceinline__ int64_t lin_cta_of(int64_t u, int64_t U, int64_t G) { return ((u + 1) * G + U - 1) / U - 1; }
 
 __global__ void __launch_bounds__(LIN_THREADS, 1)
-    nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
-                        const LinearParams p)
+    nvfp4_linear_kernel(const LinearParams p)
 {
     extern __shared__ uint8_t lin_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lin_smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + LIN_STAGES * LIN_STAGE_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + LIN_OFF_BAR);
     uint64_t *empty = full + LIN_STAGES;
     uint64_t *accf = empty + LIN_STAGES;
     uint64_t *acce = accf + 2;
@@ -81,13 +98,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 
     const uint32_t warp = warp_id(), lane = lane_id();
     const int64_t G = gridDim.x, c = blockIdx.x, U = p.U;
-    const int KT = p.KT;
+    const int KC = p.KC;
     const int64_t u0 = lin_start(c, U, G), u1 = lin_start(c + 1, U, G);
     const int64_t n_units = u1 - u0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < LIN_STAGES; ++s) {
-            mbar_init(&full[s], 2);
+            mbar_init(&full[s], 2);          // weight-unit arrive.expect_tx + activation arrive.expect_tx
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -102,14 +119,6 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         tmem_alloc(tmem_holder, LIN_TMEM_COLS);
         tmem_relinquish();
     }
-    // zero the activation scale-factor images once; only column 0 of lines
-    // 0..M-1 is rewritten per stage
-    for (uint32_t i = threadIdx.x; i < LIN_STAGES * (LIN_SF_BYTES / 16); i += blockDim.x) {
-        const uint32_t s = i / (LIN_SF_BYTES / 16), o = i % (LIN_SF_BYTES / 16);
-        *reinterpret_cast<uint4 *>(smem + s * LIN_STAGE_BYTES + LIN_W_BYTES + LIN_A_BYTES + LIN_SF_BYTES + o * 16) =
-            make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -118,62 +127,40 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        const uint64_t pol_w = policy_evict_first();
-        const uint64_t pol_a = policy_evict_last();
-        const int64_t n_pre = n_units < LIN_STAGES ? n_units : LIN_STAGES;
-        auto unit_tile = [&](int64_t i, int &t, int &kt) {
-            const int64_t u = u0 + i;
-            t = (int)(u / KT);
-            kt = (int)(u % KT);
-        };
-        auto issue_w = [&](int64_t i) {
-            int t, kt;
-            unit_tile(i, t, kt);
-            uint8_t *st = smem + (i % LIN_STAGES) * LIN_STAGE_BYTES;
-            mbar_arrive_expect_tx(&full[i % LIN_STAGES], LIN_TX_BYTES);
-            tma_load_2d_hint(st, &tm_w, &full[i % LIN_STAGES], kt * 128, t * 128, pol_w);
-            bulk_load_hint(st + LIN_W_BYTES + LIN_A_BYTES, p.w_sf + ((int64_t)t * KT + kt) * LIN_SF_BYTES,
-                           LIN_SF_BYTES, &full[i % LIN_STAGES], pol_w);
-        };
-        auto issue_a = [&](int64_t i) {
-            int t, kt;
-            unit_tile(i, t, kt);
-            uint8_t *st = smem + (i % LIN_STAGES) * LIN_STAGE_BYTES;
-            if (lane == 0) tma_load_2d_hint(st + LIN_W_BYTES, &tm_a, &full[i % LIN_STAGES], kt * 128, 0, pol_a);
-            // activation scales: line m, column 0 of chunk j <- scales[m][kt*16 + 4j .. +3]
-            const int kb = p.K / 16;
-            if ((int)lane < p.M) {
-                uint8_t *sfb = st + LIN_W_BYTES + LIN_A_BYTES + LIN_SF_BYTES;
-                const uint8_t *src = p.a_scales + (int64_t)lane * kb;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int col = kt * 16 + 4 * j;
-                    const uint32_t w = col < kb ? *reinterpret_cast<const uint32_t *>(src + col) : 0u;
-                    *reinterpret_cast<uint32_t *>(sfb + j * 512 + lane * 16) = w;
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full[i % LIN_STAGES]);
-        };
-        if (lane == 0)
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            const int64_t n_pre = n_units < LIN_STAGES ? n_units : LIN_STAGES;
+            auto issue_w = [&](int64_t i) {
+                const int s = (int)(i % LIN_STAGES);
+                mbar_arrive_expect_tx(&full[s], LIN_W_UNIT);
+                bulk_load_hint(smem + s * LIN_STAGE_BYTES, p.w + (u0 + i) * (int64_t)LIN_W_UNIT, LIN_W_UNIT,
+                               &full[s], pol_w);
+            };
+            auto issue_a = [&](int64_t i) {
+                const int s = (int)(i % LIN_STAGES);
+                const int64_t kc = (u0 + i) % KC;
+                mbar_arrive_expect_tx(&full[s], LIN_A_UNIT);
+                bulk_load_hint(smem + s * LIN_STAGE_BYTES + LIN_W_UNIT, p.a + kc * (int64_t)LIN_A_UNIT, LIN_A_UNIT,
+                               &full[s], pol_a);
+            };
             for (int64_t i = 0; i < n_pre; ++i) issue_w(i);
-        pdl_wait();
-        for (int64_t i = 0; i < n_pre; ++i) issue_a(i);
-        int64_t issued = n_pre;
-        for (int64_t i = n_pre; i < n_units; ++i) {
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&empty[i % LIN_STAGES], (uint32_t)(((i / LIN_STAGES) & 1) ^ 1), 101, s_abort);
-            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            if (lane == 0) issue_w(i);
-            issue_a(i);
-            issued = i + 1;
-        }
-        if (*s_abort && lane == 0) {
-            // let every copy still in flight land before the CTA exits
-            for (int64_t i = issued > LIN_STAGES ? issued - LIN_STAGES : 0; i < issued; ++i)
-                mbar_wait(&full[i % LIN_STAGES], (uint32_t)((i / LIN_STAGES) & 1), 102);
+            pdl_wait();
+            for (int64_t i = 0; i < n_pre; ++i) issue_a(i);
+            int64_t issued = n_pre;
+            for (int64_t i = n_pre; i < n_units; ++i) {
+                if (!mbar_wait(&empty[i % LIN_STAGES], (uint32_t)(((i / LIN_STAGES) & 1) ^ 1), 101, s_abort)) break;
+                issue_w(i);
+                issue_a(i);
+                issued = i + 1;
+            }
+            if (*s_abort) {
+                // let every copy still in flight land before the CTA exits
+                for (int64_t i = issued > LIN_STAGES ? issued - LIN_STAGES : 0; i < issued; ++i)
+                    mbar_wait(&full[i % LIN_STAGES], (uint32_t)((i / LIN_STAGES) & 1), 102);
+            }
+        } else {
+            pdl_wait();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -182,39 +169,39 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             int64_t i = 0, seg = 0;
             bool ok = true;
             for (int64_t u = u0; u < u1 && ok; ++seg) {
-                const int64_t ka = u % KT;
-                const int64_t kb = (ka + (u1 - u)) < KT ? ka + (u1 - u) : KT;
+                const int64_t ka = u % KC;
+                const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
                 const uint32_t b = (uint32_t)(seg & 1);
                 if (!mbar_wait(&acce[b], (uint32_t)(((seg >> 1) & 1) ^ 1), 103, s_abort)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + TM_ACC + 16 * b;
-                for (int64_t kt = ka; kt < kb; ++kt, ++i) {
+                for (int64_t kc = ka; kc < kend; ++kc, ++i) {
                     const int s = (int)(i % LIN_STAGES);
                     if (!mbar_wait(&full[s], (uint32_t)((i / LIN_STAGES) & 1), 104, s_abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t r = (uint32_t)(i & 1);
-                    const uint32_t st = smem_u32(smem + s * LIN_STAGE_BYTES);
-                    const uint32_t sfa_t = tmem_base + TM_SFA + 16 * r, sfb_t = tmem_base + TM_SFB + 16 * r;
+                    const uint32_t w_s = smem_u32(smem + s * LIN_STAGE_BYTES);
+                    const uint32_t a_s = w_s + LIN_W_UNIT;
+                    const uint32_t sfa_s = w_s + 2 * LIN_W_ATOM, sfb_s = a_s + 2 * LIN_A_ATOM;
+                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * r, sfb_t = tmem_base + TM_SFB + 32 * r;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
-                                               smem_desc(st + LIN_W_BYTES + LIN_A_BYTES + 512 * j, 512, 128, SWZ_NONE));
-                        tmem_cp_32x128b_warpx4(sfb_t + 4 * j,
-                                               smem_desc(st + LIN_W_BYTES + LIN_A_BYTES + LIN_SF_BYTES + 512 * j, 512,
-                                                         128, SWZ_NONE));
+                    for (int j = 0; j < LIN_KSTEPS; ++j) {
+                        tmem_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
+                        tmem_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
                     }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint64_t adesc = smem_desc(st + 32 * j, 16, 1024, SWZ_128B);
-                        const uint64_t bdesc = smem_desc(st + LIN_W_BYTES + 32 * j, 16, 1024, SWZ_128B);
+                    for (int j = 0; j < LIN_KSTEPS; ++j) {
+                        const uint32_t atom = (uint32_t)(j >> 2), ko = 32u * (uint32_t)(j & 3);
+                        const uint64_t adesc = smem_desc(w_s + atom * LIN_W_ATOM + ko, 16, 1024, SWZ_128B);
+                        const uint64_t bdesc = smem_desc(a_s + atom * LIN_A_ATOM + ko, 16, 1024, SWZ_128B);
                         mma_mxf4nvf4(d_tmem, adesc, bdesc, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
-                                     (kt > ka || j > 0) ? 1u : 0u);
+                                     (kc > ka || j > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
                 if (!ok) break;
                 tc_commit(&accf[b]);
-                u += kb - ka;
+                u += kend - ka;
             }
             if (!ok) {
                 // drain: wait for every MMA issued so far before TMEM is freed
@@ -230,11 +217,11 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         const int row = (int)(32 * q + lane);         // weight row within the tile
         const float gs = __fmul_rn(*p.g_a, *p.g_w);
         const int M = p.M;
-        const int64_t first_tile_of_me = u0 / KT;
+        const int64_t first_tile_of_me = u0 / KC;
         int64_t seg = 0;
         for (int64_t u = u0; u < u1; ++seg) {
-            const int64_t t = u / KT, ka = u % KT;
-            const int64_t kb = (ka + (u1 - u)) < KT ? ka + (u1 - u) : KT;
+            const int64_t t = u / KC, ka = u % KC;
+            const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
             const uint32_t b = (uint32_t)(seg & 1);
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&accf[b], (uint32_t)((seg >> 1) & 1), 106, s_abort);
@@ -248,7 +235,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[b]);
             const int64_t n = t * 128 + row;
-            if (ka == 0 && kb == KT) {
+            if (ka == 0 && kend == KC) {
                 if (n < p.N) {
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
@@ -261,15 +248,18 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 }
             } else {
                 // split-K fix-up, per warp: each warp owns rows 32q..32q+31 of the
-                // tile and its own arrival counter, so no cross-warp barrier is needed
+                // tile and its own arrival counter, so no cross-warp barrier is needed.
+                // Partial slots are [128 rows][16 tokens] fp32: a lane's 16 values
+                // are 64 contiguous bytes (four 16-byte stores / loads).
                 const int slot = (t == first_tile_of_me) ? 0 : 1;
-                float *P = p.partial + ((c * 2 + slot) * 16) * 128;
+                float4 *P = reinterpret_cast<float4 *>(p.partial + ((c * 2 + slot) * 128 + row) * 16);
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    if (m < M) __stcg(P + m * 128 + row, __uint_as_float(r[m]));
+                for (int v = 0; v < 4; ++v)
+                    __stcg(P + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                              __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                 __threadfence();
                 __syncwarp();
-                const int64_t first = lin_cta_of(t * KT, U, G), last = lin_cta_of(t * KT + KT - 1, U, G);
+                const int64_t first = lin_cta_of(t * KC, U, G), last = lin_cta_of(t * KC + KC - 1, U, G);
                 int is_last = 0;
                 if (lane == 0) is_last = (atomicAdd(p.counters + t * 4 + q, 1) == (int)(last - first)) ? 1 : 0;
                 is_last = __shfl_sync(0xFFFFFFFFu, is_last, 0);
@@ -278,12 +268,31 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     float acc[16];
 #pragma unroll
                     for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-                    for (int64_t cc = first; cc <= last; ++cc) {
-                        const int sl = ((lin_start(cc, U, G) / KT) == t) ? 0 : 1;
-                        const float *Q = p.partial + ((cc * 2 + sl) * 16) * 128;
+                    // contributors in order; up to 8 of them loaded before summing
+                    for (int64_t c0 = first; c0 <= last; c0 += 8) {
+                        float4 part[8][4];
 #pragma unroll
-                        for (int m = 0; m < 16; ++m)
-                            if (m < M) acc[m] = __fadd_rn(acc[m], __ldcg(Q + m * 128 + row));
+                        for (int k = 0; k < 8; ++k) {
+                            const int64_t cc = c0 + k;
+                            if (cc <= last) {
+                                const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
+                                const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) part[k][v] = __ldcg(Q + v);
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (c0 + k <= last) {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    acc[4 * v] = __fadd_rn(acc[4 * v], part[k][v].x);
+                                    acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], part[k][v].y);
+                                    acc[4 * v + 2] = __fadd_rn(acc[4 * v + 2], part[k][v].z);
+                                    acc[4 * v + 3] = __fadd_rn(acc[4 * v + 3], part[k][v].w);
+                                }
+                            }
+                        }
                     }
                     if (n < p.N) {
 #pragma unroll
@@ -298,7 +307,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     if (lane == 0) p.counters[t * 4 + q] = 0;
                 }
             }
-            u += kb - ka;
+            u += kend - ka;
         }
     }
 
@@ -307,6 +316,46 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, LIN_TMEM_COLS);
+    }
+}
+
+// ---- operand preparation ----------------------------------------------------
+// Offset, inside a 128-byte-swizzled image (rows of 128 B, base 1024-aligned),
+// of byte b of row r: the 16-byte chunk index is XORed with r % 8 (the layout
+// a 128-byte-swizzle TMA load would produce and the MMA descriptor expects).
+__host__ __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t b)
+{
+    return r * 128u + ((((b >> 4) ^ (r & 7u)) << 4) | (b & 15u));
+}
+
+// Weight units: for tile t, chunk c:
+//   atom a, row r, byte b   <- codes[t*128 + r][c*256 + a*128 + b]
+//   scale image j, line l, byte 4*cc + kb <- scales[t*128 + l + 32*cc][c*32 + 4*j + kb]
+// zero outside the matrix.
+__global__ void prepare_weight_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                      int64_t N, int64_t K, int64_t KC, uint8_t *__restrict__ out, int64_t total)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t kbytes = K / 2, kb = K / 16;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t unit = i / LIN_W_UNIT, o = i % LIN_W_UNIT;
+        const int64_t t = unit / KC, cidx = unit % KC;
+        uint8_t v = 0;
+        if (o < 2 * LIN_W_ATOM) {
+            const uint32_t a = (uint32_t)(o / LIN_W_ATOM), o2 = (uint32_t)(o % LIN_W_ATOM);
+            const uint32_t r = o2 / 128u, pos = o2 % 128u;
+            const uint32_t b = (((pos >> 4) ^ (r & 7u)) << 4) | (pos & 15u);     // inverse of swz128
+            const int64_t row = t * 128 + r, col = cidx * 256 + a * 128 + b;
+            if (row < N && col < kbytes) v = codes[row * kbytes + col];
+        } else {
+            const uint32_t o2 = (uint32_t)(o - 2 * LIN_W_ATOM);
+            const uint32_t j = o2 / 512u, l = (o2 % 512u) / 16u, cc = (o2 % 16u) / 4u, kbi = o2 % 4u;
+            const int64_t row = t * 128 + l + 32 * cc, blk = cidx * 32 + 4 * j + kbi;
+            if (row < N && blk < kb) v = scales[row * kb + blk];
+        }
+        out[i] = v;
     }
 }
 

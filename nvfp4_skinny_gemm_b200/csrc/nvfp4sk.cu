@@ -260,28 +260,36 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t K)
     return QBIG_MAX_PARTIALS * sizeof(float);
 }
 
+size_t nvfp4_prepared_act_bytes(int64_t K) { return (size_t)cdiv(K, LIN_KC) * LIN_A_UNIT; }
+
 nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int64_t K, int64_t ld_x,
-                                  const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out, void *ws,
-                                  size_t ws_bytes, nvfp4sk_stream_t stream)
+                                  const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
+                                  uint8_t *act_prepared, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
-    if (!x || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (!x || !g_out || (!act_prepared && (!codes || !scales)))
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer (need codes+scales and/or act_prepared)");
     if (x_dtype != NVFP4SK_BF16 && x_dtype != NVFP4SK_FP32) return fail(NVFP4SK_ERR_INVALID_ARG, "bad dtype");
     if (rows < 1 || K < 16 || K % 16 != 0 || ld_x < K)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need rows >= 1, K %% 16 == 0, ld_x >= K");
+    if (act_prepared && (rows > 16 || K % 64 != 0))
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "the prepared activation needs rows <= 16 and K %% 64 == 0");
     const int64_t esz = x_dtype == NVFP4SK_BF16 ? 2 : 4;
-    if (!al16(x) || (ld_x * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(codes) & 7u) != 0)
-        return fail(NVFP4SK_ERR_MISALIGNED, "x and its row stride must be 16-byte aligned, codes 8-byte aligned");
+    if (!al16(x) || (ld_x * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(codes) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(act_prepared) & 15u) != 0)
+        return fail(NVFP4SK_ERR_MISALIGNED,
+                    "x, its row stride and act_prepared must be 16-byte aligned, codes 8-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t nblk = rows * (K / 16);
     if (nblk <= QSMALL_MAX_BLOCKS) {
         const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
         cudaError_t e = x_dtype == NVFP4SK_BF16
                             ? launch(quant_fused_kernel<__nv_bfloat16, 0>, dim3(cs), dim3(QTHREADS), 0, st, cs,
-                                     (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, codes, scales, g_out)
+                                     (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, codes, scales, g_out,
+                                     act_prepared)
                             : launch(quant_fused_kernel<float, 0>, dim3(cs), dim3(QTHREADS), 0, st, cs,
-                                     (const float *)x, rows, K, ld_x, g_in, codes, scales, g_out);
+                                     (const float *)x, rows, K, ld_x, g_in, codes, scales, g_out, act_prepared);
         return launched(e, "quant_fused_kernel");
     }
     if (!g_in && (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(rows, K)))
@@ -301,26 +309,44 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
     e = x_dtype == NVFP4SK_BF16
             ? launch(quant_blocks_kernel<__nv_bfloat16>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1,
                      (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, (const float *)partial, grid, codes, scales,
-                     g_out)
+                     g_out, act_prepared)
             : launch(quant_blocks_kernel<float>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1, (const float *)x, rows,
-                     K, ld_x, g_in, (const float *)partial, grid, codes, scales, g_out);
+                     K, ld_x, g_in, (const float *)partial, grid, codes, scales, g_out, act_prepared);
     return launched(e, "quant_blocks_kernel");
 }
 
-size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K) { return (size_t)cdiv(N, 128) * cdiv(K, 256) * 2048; }
-
-nvfp4sk_status nvfp4_prepare_weight_scales(const uint8_t *scales, int64_t N, int64_t K, uint8_t *prepared,
-                                           nvfp4sk_stream_t stream)
+nvfp4sk_status nvfp4_prepare_act(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,
+                                 uint8_t *act_prepared, nvfp4sk_stream_t stream)
 {
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
-    if (!scales || !prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (!codes || !scales || !act_prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 16 || K < 64 || K % 64 != 0)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, K %% 64 == 0");
+    if ((reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
+        return fail(NVFP4SK_ERR_MISALIGNED, "codes 8-byte aligned, act_prepared 16-byte aligned");
+    const int64_t nblk = rows * (K / 16);
+    const int grid = (int)std::min<int64_t>(cdiv(nblk, 256), 4 * d->sms);
+    return launched(launch(prepare_act_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, codes, scales, rows,
+                           K, act_prepared),
+                    "prepare_act_kernel");
+}
+
+size_t nvfp4_prepared_weight_bytes(int64_t N, int64_t K) { return (size_t)cdiv(N, 128) * cdiv(K, LIN_KC) * LIN_W_UNIT; }
+
+nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K,
+                                    uint8_t *prepared, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!codes || !scales || !prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (N < 1 || K < 64 || K % 64 != 0) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need N >= 1, K %% 64 == 0");
-    const int64_t total = (int64_t)nvfp4_prepared_scale_bytes(N, K);
-    const int grid = (int)std::min<int64_t>(cdiv(total, 256), 8 * d->sms);
-    return launched(launch(prepare_scales_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, scales, N, K,
-                           cdiv(K, 256), prepared, total),
-                    "prepare_scales_kernel");
+    if (!al16(prepared)) return fail(NVFP4SK_ERR_MISALIGNED, "prepared buffer must be 16-byte aligned");
+    const int64_t total = (int64_t)nvfp4_prepared_weight_bytes(N, K);
+    const int grid = (int)std::min<int64_t>(cdiv(total, 256), 16 * d->sms);
+    return launched(launch(prepare_weight_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, codes, scales, N,
+                           K, cdiv(K, LIN_KC), prepared, total),
+                    "prepare_weight_kernel");
 }
 
 // ---------------------------------------------------------------- linear
@@ -329,39 +355,30 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K)
     (void)M;
     DevInfo *d;
     if (device_info(&d)) return 0;
-    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 256);
+    const int64_t NT = cdiv(N, 128), KC = cdiv(K, LIN_KC);
     const int64_t G = std::max<int64_t>(d->sms, g_opt_linear_ctas);
-    return linear_ws(std::min<int64_t>(G, NT * KT), NT);
+    return linear_ws(std::min<int64_t>(G, NT * KC), NT);
 }
 
-nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, int64_t M,
-                            const uint8_t *w_codes, const uint8_t *w_scales_prepared, const float *g_w, int64_t N,
-                            int64_t K, const void *residual, void *y, int64_t ldy, void *ws, size_t ws_bytes,
-                            nvfp4sk_stream_t stream)
+nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t M, const uint8_t *w_prepared,
+                            const float *g_w, int64_t N, int64_t K, const void *residual, void *y, int64_t ldy,
+                            void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
-    if (!a_codes || !a_scales || !g_a || !w_codes || !w_scales_prepared || !g_w || !y)
-        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (M < 1 || M > 16 || N < 1 || N > LIN_MAX_NT * 128 || K < 64 || K % 64 != 0 || ldy < N || K > (int64_t)1 << 24)
+    if (!a_prepared || !g_a || !w_prepared || !g_w || !y) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (M < 1 || M > 16 || N < 1 || N > LIN_MAX_NT * 128 || K < 64 || K % 64 != 0 || ldy < N)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, 1 <= N <= 524288, K %% 64 == 0, ldy >= N");
-    if (!al16(a_codes) || !al16(a_scales) || !al16(w_codes) || !al16(w_scales_prepared))
-        return fail(NVFP4SK_ERR_MISALIGNED, "code and scale pointers must be 16-byte aligned");
-    const int64_t NT = cdiv(N, 128), KT = cdiv(K, 256), U = NT * KT;
+    if (!al16(a_prepared) || !al16(w_prepared))
+        return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands must be 16-byte aligned");
+    const int64_t NT = cdiv(N, 128), KC = cdiv(K, LIN_KC), U = NT * KC;
     const int G = linear_grid(*d, U);
     const size_t need = linear_ws(G, NT);
     if (!ws || ws_bytes < need || !al16(ws))
         return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
-    CUtensorMap tw, ta;
-    if (int rc = make_map_u8(&tw, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128, 128,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
-        return rc;
-    if (int rc = make_map_u8(&ta, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128, 16,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
-        return rc;
     LinearParams p;
-    p.w_sf = w_scales_prepared;
-    p.a_scales = a_scales;
+    p.w = w_prepared;
+    p.a = a_prepared;
     p.g_a = g_a;
     p.g_w = g_w;
     p.residual = (const __nv_bfloat16 *)residual;
@@ -372,11 +389,10 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_codes, const uint8_t *a_scales, con
     p.U = U;
     p.M = (int)M;
     p.N = (int)N;
-    p.K = (int)K;
     p.NT = (int)NT;
-    p.KT = (int)KT;
-    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, (cudaStream_t)stream,
-                           1, tw, ta, p),
+    p.KC = (int)KC;
+    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, (cudaStream_t)stream, 1,
+                           p),
                     "nvfp4_linear_kernel");
 }
 
@@ -400,10 +416,10 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     if (int rc = device_info(&d)) return rc;
     if (!q || !k_pool || !v_pool || !page_table || !parent || !k_scale || !v_scale || !out)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 8 ||
+    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 7 ||
         ctx_len < 0 || n_pool_pages < 1 || ld_q < (int64_t)Hq * D || n_pool_pages * Hkv * ATT_P > INT32_MAX)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
-                    "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 8, ld_q >= Hq*D");
+                    "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 7, ld_q >= Hq*D");
     if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool))
         return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes) and the pools must be 16-byte aligned");
     const int64_t n_log = cdiv(ctx_len + T, ATT_P);
@@ -475,39 +491,44 @@ nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_t *src_ids, 
 
 // ---------------------------------------------------------------- glue
 nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows, int64_t n,
-                                      uint8_t *codes, uint8_t *scales, float *g_out, void *ws, size_t ws_bytes,
-                                      nvfp4sk_stream_t stream)
+                                      uint8_t *codes, uint8_t *scales, float *g_out, uint8_t *act_prepared, void *ws,
+                                      size_t ws_bytes, nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
-    if (!x || !w || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (rows < 1 || rows > 16 || n < 16 || n % 16 != 0 || n > (int64_t)RTHREADS * RNB * 16)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, n %% 16 == 0, n <= 8192");
-    if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u))
-        return fail(NVFP4SK_ERR_MISALIGNED, "x, w must be 16-byte aligned, codes 8-byte aligned");
+    if (!x || !w || !g_out || (!act_prepared && (!codes || !scales)))
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 16 || n < 64 || n % 64 != 0 || n > (int64_t)RTHREADS * RNB * 16)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, n %% 64 == 0, n <= 8192");
+    if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
+        (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
+        return fail(NVFP4SK_ERR_MISALIGNED, "x, w, act_prepared must be 16-byte aligned, codes 8-byte aligned");
     const int cs = rows <= 8 ? 8 : 16;
     return launched(launch(rmsnorm_quant_kernel, dim3(cs), dim3(RTHREADS), 0, (cudaStream_t)stream, cs,
-                           (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, rows, n, codes, scales, g_out),
+                           (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, rows, n, codes, scales, g_out,
+                           act_prepared),
                     "rmsnorm_quant_kernel");
 }
 
 nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes, uint8_t *scales,
-                                     float *g_out, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
+                                     float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
+                                     nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
-    if (!gu || !codes || !scales || !g_out) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (rows < 1 || rows > 16 || F < 16 || F % 16 != 0 || rows * (F / 16) > QSMALL_MAX_BLOCKS)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, F %% 16 == 0, rows*F <= 524288");
-    if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u))
-        return fail(NVFP4SK_ERR_MISALIGNED, "gu must be 16-byte aligned, codes 8-byte aligned");
+    if (!gu || !g_out || (!act_prepared && (!codes || !scales)))
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || rows > 16 || F < 64 || F % 64 != 0 || rows * (F / 16) > QSMALL_MAX_BLOCKS)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, F %% 64 == 0, rows*F <= 524288");
+    if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
+        return fail(NVFP4SK_ERR_MISALIGNED, "gu, act_prepared must be 16-byte aligned, codes 8-byte aligned");
     const int64_t nblk = rows * (F / 16);
     const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
     return launched(launch(quant_fused_kernel<__nv_bfloat16, 1>, dim3(cs), dim3(QTHREADS), 0, (cudaStream_t)stream,
                            cs, (const __nv_bfloat16 *)gu, rows, F, 2 * F, (const float *)nullptr, codes, scales,
-                           g_out),
+                           g_out, act_prepared),
                     "swiglu_quant_kernel");
 }
 

@@ -6,6 +6,7 @@
 // compiler cannot contract or approximate them.
 #pragma once
 #include "common.cuh"
+#include "linear.cuh"
 
 namespace nvfp4sk {
 
@@ -47,6 +48,27 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float g,
     }
     packed = make_uint2(w0, w1);
     return sc;
+}
+
+// Store one quantised 16-block (row r < 16, block index blk along K) into the
+// prepared activation image read by nvfp4_linear: chunk c = blk / 32 holds
+// [2 x 2 KB 128-byte-swizzled code atoms | 8 x 512 B scale images], scale
+// image j = MMA step (64 K), line r, byte (blk % 4).  Bytes that are never
+// written (rows >= M, unused image bytes) stay as the caller zero-filled them.
+__device__ __forceinline__ void store_prepared(uint8_t *act, int64_t r, int64_t blk, uint2 pk, uint32_t sc)
+{
+    const uint32_t bi = (uint32_t)(blk % 32);
+    uint8_t *base = act + (blk / 32) * (int64_t)LIN_A_UNIT;
+    *reinterpret_cast<uint2 *>(base + (bi / 16) * LIN_A_ATOM + swz128((uint32_t)r, (bi % 16) * 8)) = pk;
+    base[2 * LIN_A_ATOM + (bi / 4) * LIN_SF_IMG + r * 16 + (bi % 4)] = (uint8_t)sc;
+}
+
+__device__ __forceinline__ void store_block(uint8_t *codes, uint8_t *scales, uint8_t *act, int64_t r, int64_t c,
+                                            int64_t K, uint2 pk, uint32_t sc)
+{
+    if (codes) *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
+    if (scales) scales[r * (K / 16) + c] = (uint8_t)sc;
+    if (act) store_prepared(act, r, c, pk, sc);
 }
 
 // ---- element loaders ------------------------------------------------------
@@ -167,7 +189,7 @@ template <typename T, int MODE>
 __global__ void __launch_bounds__(QTHREADS, 1)
     quant_fused_kernel(const T *__restrict__ x, int64_t rows, int64_t K, int64_t ld_x,
                        const float *__restrict__ g_in, uint8_t *__restrict__ codes,
-                       uint8_t *__restrict__ scales, float *__restrict__ g_out)
+                       uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
 {
     __shared__ float s_red[33];
     __shared__ float s_cta_amax;
@@ -209,8 +231,7 @@ __global__ void __launch_bounds__(QTHREADS, 1)
             const int64_t r = b / kb, c = b % kb;
             uint2 pk;
             const uint32_t sc = quant_block16(v[j], g, pk);
-            *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
-            scales[r * kb + c] = (uint8_t)sc;
+            store_block(codes, scales, act, r, c, K, pk, sc);
         }
     }
     cluster_sync_all();   // keep this CTA's shared memory alive until peers have read it
@@ -221,7 +242,7 @@ __global__ void __launch_bounds__(QTHREADS, 1)
 __global__ void __launch_bounds__(RTHREADS, 1)
     rmsnorm_quant_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
                          int64_t rows, int64_t n, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                         float *__restrict__ g_out)
+                         float *__restrict__ g_out, uint8_t *__restrict__ act)
 {
     __shared__ float s_red[33];
     __shared__ float s_cta_amax;
@@ -263,8 +284,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         if (r < rows && c < kb) {
             uint2 pk;
             const uint32_t sc = quant_block16(v[j], g, pk);
-            *reinterpret_cast<uint2 *>(codes + r * (n / 2) + c * 8) = pk;
-            scales[r * kb + c] = (uint8_t)sc;
+            store_block(codes, scales, act, r, c, n, pk, sc);
         }
     }
     cluster_sync_all();
@@ -302,7 +322,8 @@ __global__ void __launch_bounds__(QBIG_THREADS) quant_blocks_kernel(const T *__r
                                                                      const float *__restrict__ partial,
                                                                      int n_partial, uint8_t *__restrict__ codes,
                                                                      uint8_t *__restrict__ scales,
-                                                                     float *__restrict__ g_out)
+                                                                     float *__restrict__ g_out,
+                                                                     uint8_t *__restrict__ act)
 {
     __shared__ float s_red[33];
     pdl_wait();
@@ -324,29 +345,21 @@ __global__ void __launch_bounds__(QBIG_THREADS) quant_blocks_kernel(const T *__r
         load16<T>(x + r * ld_x + c * 16, v);
         uint2 pk;
         const uint32_t sc = quant_block16(v, g, pk);
-        *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
-        scales[r * kb + c] = (uint8_t)sc;
+        store_block(codes, scales, act, r, c, K, pk, sc);
     }
 }
 
-// ---- weight scale-factor rearrangement -------------------------------------
-// prepared[t][kt][j][l][c*4 + kb] = scales[t*128 + l + 32c][kt*16 + 4j + kb]
-// (zero outside the matrix): for every 128-row x 256-column weight tile, four
-// 512-byte chunks, one per 64-wide MMA step, each the 32 x 16-byte image that
-// tcgen05.cp 32x128b.warpx4 replicates into the scale-factor columns.
-__global__ void prepare_scales_kernel(const uint8_t *__restrict__ scales, int64_t N, int64_t K, int64_t KT,
-                                      uint8_t *__restrict__ out, int64_t total)
+// ---- canonical activation -> prepared tile image ---------------------------
+__global__ void prepare_act_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                                   int64_t rows, int64_t K, uint8_t *__restrict__ act)
 {
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t kb = K / 16;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t byte = i & 15, l = (i >> 4) & 31, j = (i >> 9) & 3, tile = i >> 11;
-        const int64_t kt = tile % KT, t = tile / KT;
-        const int64_t c = byte >> 2, kbi = byte & 3;
-        const int64_t row = t * 128 + l + 32 * c, col = kt * 16 + 4 * j + kbi;
-        out[i] = (row < N && col < kb) ? scales[row * kb + col] : 0;
+    const int64_t kb = K / 16, nblk = rows * kb;
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblk; b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = b / kb, c = b % kb;
+        const uint2 pk = *reinterpret_cast<const uint2 *>(codes + r * (K / 2) + c * 8);
+        store_prepared(act, r, c, pk, scales[r * kb + c]);
     }
 }
 

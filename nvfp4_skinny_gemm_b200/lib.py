@@ -35,17 +35,19 @@ _vp, _i64, _int, _sz, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctyp
 
 _SIGS = {
     "nvfp4_quantize_workspace_bytes": (_sz, [_i64, _i64]),
-    "nvfp4_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "nvfp4_prepared_scale_bytes": (_sz, [_i64, _i64]),
-    "nvfp4_prepare_weight_scales": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "nvfp4_prepared_act_bytes": (_sz, [_i64]),
+    "nvfp4_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_prepare_act": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
+    "nvfp4_prepared_weight_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_prepare_weight": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
-    "nvfp4_linear": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "nvfp4_linear": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
     "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
     "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
                                _vp, _f32, _vp, _vp, _sz, _vp]),
     "kv_page_restore": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
-    "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kv_append_fp8": (_int, [_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp, _vp]),
     "argmax_workspace_bytes": (_sz, [_i64, _i64]),
     "argmax_rows_bf16": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
@@ -145,39 +147,53 @@ def device_status(stream=None):
     return rc, site.value
 
 
-def quantize(x: torch.Tensor, g_in: torch.Tensor | None = None, out=None, ws=None, stream=None):
+def act_buffer(K: int, device=None) -> torch.Tensor:
+    """Zero-filled prepared-activation buffer for K input features."""
+    return torch.zeros(load().nvfp4_prepared_act_bytes(K), dtype=torch.uint8, device=device or "cuda")
+
+
+def quantize(x: torch.Tensor, g_in: torch.Tensor | None = None, out=None, act: torch.Tensor | None = None,
+             canonical: bool = True, ws=None, stream=None):
     """NVFP4-quantise x [rows, K] (bf16 or fp32, row stride x.stride(0)).
 
-    Returns (codes u8 [rows, K/2], scales u8 [rows, K/16], g f32 [1])."""
+    Returns (codes u8 [rows, K/2], scales u8 [rows, K/16], g f32 [1]); with
+    act (a buffer from act_buffer) the prepared tile image is written too;
+    canonical=False skips the canonical outputs (codes/scales are None)."""
     rows, K = x.shape
     assert x.stride(1) == 1
     dt = BF16 if x.dtype == torch.bfloat16 else FP32
     if out is None:
-        out = (torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device),
-               torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device),
+        out = (torch.empty(rows, K // 2, dtype=torch.uint8, device=x.device) if canonical else None,
+               torch.empty(rows, K // 16, dtype=torch.uint8, device=x.device) if canonical else None,
                torch.empty(1, dtype=torch.float32, device=x.device))
     codes, scales, g = out
     wp, wn = _ws(ws, load().nvfp4_quantize_workspace_bytes(rows, K), "quantize")
-    _call("nvfp4_quantize_act", x.data_ptr(), dt, rows, K, x.stride(0), _p(g_in), codes.data_ptr(),
-          scales.data_ptr(), g.data_ptr(), wp, wn, _stream(stream))
+    _call("nvfp4_quantize_act", x.data_ptr(), dt, rows, K, x.stride(0), _p(g_in), _p(codes), _p(scales),
+          g.data_ptr(), _p(act), wp, wn, _stream(stream))
     return codes, scales, g
 
 
-def prepare_weight_scales(scales: torch.Tensor, N: int, K: int, stream=None):
-    out = torch.empty(load().nvfp4_prepared_scale_bytes(N, K), dtype=torch.uint8, device=scales.device)
-    _call("nvfp4_prepare_weight_scales", scales.data_ptr(), N, K, out.data_ptr(), _stream(stream))
+def prepare_act(codes: torch.Tensor, scales: torch.Tensor, K: int, act=None, stream=None):
+    rows = codes.shape[0]
+    if act is None:
+        act = act_buffer(K, codes.device)
+    _call("nvfp4_prepare_act", codes.data_ptr(), scales.data_ptr(), rows, K, act.data_ptr(), _stream(stream))
+    return act
+
+
+def prepare_weight(codes: torch.Tensor, scales: torch.Tensor, N: int, K: int, stream=None):
+    out = torch.empty(load().nvfp4_prepared_weight_bytes(N, K), dtype=torch.uint8, device=codes.device)
+    _call("nvfp4_prepare_weight", codes.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(stream))
     return out
 
 
-def linear(a_codes, a_scales, g_a, w_codes, w_prep, g_w, N, K, y=None, residual=None, ws=None, stream=None):
-    """Y [M, N] bf16 = NVFP4 linear (+ residual)."""
-    M = a_codes.shape[0]
+def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, stream=None):
+    """Y [M, N] bf16 = NVFP4 linear (+ residual) on prepared operands."""
     if y is None:
-        y = torch.empty(M, N, dtype=torch.bfloat16, device=a_codes.device)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a_act.device)
     wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K), "linear")
-    _call("nvfp4_linear", a_codes.data_ptr(), a_scales.data_ptr(), g_a.data_ptr(), M, w_codes.data_ptr(),
-          w_prep.data_ptr(), g_w.data_ptr(), N, K, _p(residual), y.data_ptr(), y.stride(0), wp, wn,
-          _stream(stream))
+    _call("nvfp4_linear", a_act.data_ptr(), g_a.data_ptr(), M, w_prep.data_ptr(), g_w.data_ptr(), N, K,
+          _p(residual), y.data_ptr(), y.stride(0), wp, wn, _stream(stream))
     return y
 
 
@@ -207,19 +223,20 @@ def kv_page_restore(src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, st
           page_bytes, src_pool.numel() // page_bytes, dst_pool.numel() // page_bytes, _stream(stream))
 
 
-def rmsnorm_quantize(x, w, eps, out, stream=None):
+def rmsnorm_quantize(x, w, eps, out, act=None, stream=None):
+    """out = (codes or None, scales or None, g); act: prepared buffer or None."""
     rows, n = x.shape
     codes, scales, g = out
-    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, codes.data_ptr(),
-          scales.data_ptr(), g.data_ptr(), None, 0, _stream(stream))
+    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, _p(codes), _p(scales),
+          g.data_ptr(), _p(act), None, 0, _stream(stream))
     return out
 
 
-def swiglu_quantize(gu, out, stream=None):
+def swiglu_quantize(gu, out, act=None, stream=None):
     rows, F2 = gu.shape
     codes, scales, g = out
-    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, codes.data_ptr(), scales.data_ptr(),
-          g.data_ptr(), None, 0, _stream(stream))
+    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, _p(codes), _p(scales), g.data_ptr(), _p(act),
+          None, 0, _stream(stream))
     return out
 
 

@@ -1,0 +1,219 @@
+"""The tree-MTP verification forward step of a 27B-class dense model, composed
+from the library's C-ABI calls (nothing here computes; every op is a kernel).
+
+Per layer (pre-norm decoder block, 16 tree nodes = 16 rows):
+    RMSNorm + NVFP4 quantise -> QKV linear -> FP8 KV append of the 16 nodes
+    -> tree attention over the paged FP8 cache -> quantise -> O linear
+    (+ residual, in place) -> RMSNorm + quantise -> gate+up linear
+    -> SwiGLU + quantise -> down linear (+ residual, in place).
+After the last layer: RMSNorm + quantise -> LM head -> per-node argmax.
+Before the layers, kv_page_restore copies the reused prompt prefix (96% of
+the context) from the prefix cache into the live pool ("KV-cache reuse
+between agent steps"); the 16-node tree is verified in one forward pass
+("Tree multi-token prediction"); weights, activations and the LM head are
+NVFP4 and the cache is FP8 ("NVFP4 and FP8").
+
+All buffers are allocated once, so a step can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from . import inputs as I
+from . import lib as nv
+
+PAGE_BYTES = I.N_KV_HEADS * I.PAGE * I.HEAD_DIM      # one (layer, K|V, page) plane: 32 KB
+
+
+class Linear:
+    """NVFP4 weight in the linear kernel's tile image (codes + scales) and its
+    fp32 tensor scale g."""
+
+    def __init__(self, prep, g, N, K):
+        self.prep, self.g, self.N, self.K = prep, g, N, K
+
+    @property
+    def nbytes(self):
+        """Algorithmic weight bytes (codes + E4M3 block scales)."""
+        return self.N * self.K // 2 + self.N * self.K // 16
+
+    @staticmethod
+    def from_fp32(w: torch.Tensor):
+        N, K = w.shape
+        codes, scales, g = nv.quantize(w)
+        prep = nv.prepare_weight(codes, scales, N, K)
+        del codes, scales
+        return Linear(prep, g, N, K)
+
+
+class Act:
+    """A quantised activation: prepared tile image + tensor scale."""
+
+    def __init__(self, K, dev):
+        self.K = K
+        self.buf = nv.act_buffer(K, dev)
+        self.g = torch.empty(1, dtype=torch.float32, device=dev)
+
+    @property
+    def out(self):
+        return (None, None, self.g)
+
+
+class VerifyModel:
+    """64-layer NVFP4 model + paged FP8 KV cache + prefix cache, on one GPU.
+
+    weights="device": N(0, 0.02) weights drawn on the GPU (torch generator,
+    seeded per layer) -- same distribution as the host generator, used for
+    timing; weights="host": the seeded numpy generator of `inputs` (layer l,
+    tensor t -> inputs.weight_fp32(4, t, N, K, sub=l)), which the oracle
+    reproduces."""
+
+    def __init__(self, n_layers=I.N_LAYERS, ctx_len=I.CTX_MAX, T=I.TREE_NODES, weights="device",
+                 prefix_frac=0.96, device="cuda", lm_head=True, seed=42):
+        self.dev = torch.device(device)
+        self.n_layers, self.L, self.T = n_layers, ctx_len, T
+        self.eps = 1e-6
+        H, F, Hq, Hkv, D, P = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM, I.PAGE
+        self.layers = []
+        gen = torch.Generator(device=self.dev)
+        for l in range(n_layers):
+            lay = {}
+            for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items()):
+                if weights == "host":
+                    w = torch.from_numpy(I.weight_fp32(4, t, N, K, sub=l)).to(self.dev)
+                else:
+                    gen.manual_seed(seed * 1000003 + l * 17 + t)
+                    w = torch.randn(N, K, generator=gen, device=self.dev, dtype=torch.float32).mul_(I.W_STD)
+                lay[name] = Linear.from_fp32(w)
+                del w
+            self.layers.append(lay)
+        self.norm_w = torch.ones(2 * n_layers + 1, H, dtype=torch.bfloat16, device=self.dev)
+        self.lm_head = None
+        if lm_head:
+            if weights == "host":
+                w = torch.from_numpy(I.weight_fp32(4, 9, I.VOCAB, H)).to(self.dev)
+            else:
+                gen.manual_seed(seed * 1000003 + 999)
+                w = torch.randn(I.VOCAB, H, generator=gen, device=self.dev).mul_(I.W_STD)
+            self.lm_head = Linear.from_fp32(w)
+            del w
+        torch.cuda.empty_cache()
+
+        # paged FP8 cache: planes (layer, K|V) x pool pages x 32 KB
+        self.n_log = math.ceil((ctx_len + T) / P)
+        self.n_pool = self.n_log + 8
+        g = I.rng(4, 500)
+        self.page_table_h = g.permutation(self.n_pool)[:self.n_log].astype(np.int32)
+        self.page_table = torch.from_numpy(self.page_table_h).to(self.dev)
+        self.kv = self._random_fp8((n_layers, 2, self.n_pool, PAGE_BYTES), 4, 501)
+        self.k_scale = torch.full((n_layers, Hkv), 0.02, dtype=torch.float32, device=self.dev)
+        self.v_scale = torch.full((n_layers, Hkv), 0.02, dtype=torch.float32, device=self.dev)
+        # prefix cache (hot cache of the previous agent turn) and restore ids
+        self.prefix_tokens = int(round(prefix_frac * ctx_len))
+        self.n_prefix_pages = math.ceil(self.prefix_tokens / P)
+        self.n_src = self.n_prefix_pages + 16
+        self.src = self._random_fp8((n_layers, 2, self.n_src, PAGE_BYTES), 4, 502)
+        src_pages = g.permutation(self.n_src)[:self.n_prefix_pages]
+        planes = np.arange(n_layers * 2)[:, None]
+        self.src_ids = torch.from_numpy((planes * self.n_src + src_pages[None, :]).ravel().astype(np.int32)).to(self.dev)
+        self.dst_ids = torch.from_numpy(
+            (planes * self.n_pool + self.page_table_h[None, :self.n_prefix_pages]).ravel().astype(np.int32)).to(self.dev)
+
+        # activations (static buffers)
+        self.h = torch.empty(T, H, dtype=torch.bfloat16, device=self.dev)
+        self.parent = torch.empty(T, dtype=torch.int32, device=self.dev)
+        self.qkv = torch.empty(T, (Hq + 2 * Hkv) * D, dtype=torch.bfloat16, device=self.dev)
+        self.attn = torch.empty(T, Hq * D, dtype=torch.bfloat16, device=self.dev)
+        self.gu = torch.empty(T, 2 * F, dtype=torch.bfloat16, device=self.dev)
+        self.q_h = Act(H, self.dev)
+        self.q_a = Act(Hq * D, self.dev)
+        self.q_f = Act(F, self.dev)
+        self.logits = torch.empty(T, I.VOCAB, dtype=torch.bfloat16, device=self.dev)
+        self.ids = torch.empty(T, dtype=torch.int32, device=self.dev)
+
+    def _random_fp8(self, shape, *seed):
+        """Random finite E4M3 bytes (never the NaN codes 0x7F / 0xFF)."""
+        gen = torch.Generator(device=self.dev)
+        gen.manual_seed(int(np.random.default_rng([42, *seed]).integers(1 << 62)))
+        x = torch.randint(0, 0x7E, shape, dtype=torch.uint8, device=self.dev, generator=gen)
+        sign = torch.randint(0, 2, shape, dtype=torch.uint8, device=self.dev, generator=gen)
+        return x | (sign << 7)
+
+    # ------------------------------------------------------------------ pools
+    def k_pool(self, l):
+        return self.kv[l, 0].view(self.n_pool, I.N_KV_HEADS, I.PAGE, I.HEAD_DIM)
+
+    def v_pool(self, l):
+        return self.kv[l, 1].view(self.n_pool, I.N_KV_HEADS, I.HEAD_DIM, I.PAGE)
+
+    # ------------------------------------------------------------------ ops
+    def restore(self):
+        nv.kv_page_restore(self.src.view(-1), self.src_ids, self.kv.view(-1), self.dst_ids, PAGE_BYTES)
+
+    def layer(self, l):
+        lay, T = self.layers[l], self.T
+        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l], self.eps, self.q_h.out, act=self.q_h.buf)
+        self._linear(self.q_h, lay["qkv"], self.qkv)
+        qd = I.N_Q_HEADS * I.HEAD_DIM
+        kd = I.N_KV_HEADS * I.HEAD_DIM
+        nv.kv_append(self.qkv[:, qd:], self.qkv[:, qd + kd:], self.qkv.stride(0), T, self.k_pool(l),
+                     self.v_pool(l), self.page_table, self.L, self.k_scale[l], self.v_scale[l])
+        nv.tree_attn(self.qkv, self.k_pool(l), self.v_pool(l), self.page_table, self.L, self.parent,
+                     self.k_scale[l], self.v_scale[l], out=self.attn, ld_q=self.qkv.stride(0), T=T,
+                     Hq=I.N_Q_HEADS)
+        nv.quantize(self.attn, out=self.q_a.out, act=self.q_a.buf, canonical=False)
+        self._linear(self.q_a, lay["o"], self.h, residual=self.h)
+        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l + 1], self.eps, self.q_h.out, act=self.q_h.buf)
+        self._linear(self.q_h, lay["gate_up"], self.gu)
+        nv.swiglu_quantize(self.gu, self.q_f.out, act=self.q_f.buf)
+        self._linear(self.q_f, lay["down"], self.h, residual=self.h)
+
+    def head(self):
+        nv.rmsnorm_quantize(self.h, self.norm_w[-1], self.eps, self.q_h.out, act=self.q_h.buf)
+        self._linear(self.q_h, self.lm_head, self.logits)
+        nv.argmax(self.logits, self.ids)
+
+    def _linear(self, q, lin, y, residual=None):
+        nv.linear(q.buf, q.g, self.T, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
+
+    def step(self, restore=True):
+        """One verify step on the current self.h / self.parent; result in self.ids."""
+        if restore:
+            self.restore()
+        for l in range(self.n_layers):
+            self.layer(l)
+        if self.lm_head is not None:
+            self.head()
+
+    LAUNCHES_PER_LAYER = 11          # norm-q, qkv, kv-append, attn split+combine, q, o, norm-q, gate_up, swiglu-q, down
+    LAUNCHES_HEAD = 3                # norm-q, lm head, argmax
+
+    def launches_per_step(self, restore=True):
+        return (1 if restore else 0) + self.n_layers * self.LAUNCHES_PER_LAYER + \
+            (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
+
+    # ------------------------------------------------------------------ bytes
+    def linear_bytes(self):
+        """Algorithmic HBM bytes of all linear launches in one step: weight codes
+        + scales, activation codes + scales, bf16 outputs (+ residual reads)."""
+        T, tot = self.T, 0
+        for lay in self.layers:
+            for name, lin in lay.items():
+                tot += lin.nbytes + T * lin.K * 9 // 16 + T * lin.N * 2 * (2 if name in ("o", "down") else 1)
+        if self.lm_head is not None:
+            lin = self.lm_head
+            tot += lin.nbytes + T * lin.K * 9 // 16 + T * lin.N * 2
+        return tot
+
+    def attn_bytes(self):
+        """K + V bytes read per step (context + tree slots, all layers)."""
+        return self.n_layers * 2 * (self.L + self.T) * I.N_KV_HEADS * I.HEAD_DIM
+
+    def restore_bytes(self):
+        return 2 * self.src_ids.numel() * PAGE_BYTES          # read + write
+
+    def step_bytes(self, restore=True):
+        return self.linear_bytes() + self.attn_bytes() + (self.restore_bytes() if restore else 0)

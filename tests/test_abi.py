@@ -33,11 +33,14 @@ def test_version_and_options_without_gpu():
     assert b"unknown option" in L.nvfp4sk_last_error()
 
 
-def test_prepared_scale_bytes():
+def test_prepared_sizes():
     L = lib.load()
-    assert L.nvfp4_prepared_scale_bytes(128, 256) == 2048
-    assert L.nvfp4_prepared_scale_bytes(129, 320) == 2 * 2 * 2048
-    assert L.nvfp4_prepared_scale_bytes(151936, 5120) == 1187 * 20 * 2048
+    unit = 2 * 128 * 128 + 8 * 512              # 128 rows x 512 K: codes + scale images
+    assert L.nvfp4_prepared_weight_bytes(128, 512) == unit
+    assert L.nvfp4_prepared_weight_bytes(129, 576) == 2 * 2 * unit
+    assert L.nvfp4_prepared_weight_bytes(151936, 5120) == 1187 * 10 * unit
+    assert L.nvfp4_prepared_act_bytes(5120) == 10 * (2 * 16 * 128 + 8 * 512)
+    assert L.nvfp4_prepared_act_bytes(17408) == 34 * 8192
 
 
 def test_header_is_plain_c():

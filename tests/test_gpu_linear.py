@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 def _gpu_operands(codes, scales, g, N, K):
     c, s = to_dev(codes), to_dev(scales)
-    return c, s, to_dev(np.array([g], np.float32)), nv.prepare_weight_scales(s, N, K)
+    return c, s, to_dev(np.array([g], np.float32)), nv.prepare_weight(c, s, N, K)
 
 
 @pytest.mark.parametrize("mode", ["unit_scales", "row_scales", "kblock_scales", "token_scales", "random"])
@@ -45,8 +45,9 @@ def test_scale_layout_structures(oracle, mode):
         wsc[:] = rng.integers(0x30, 0x41, (N, K // 16))
     gA, gW = 1.0, 0.5
     a_c, a_s, a_g = to_dev(ac), to_dev(asc), to_dev(np.array([gA], np.float32))
+    a_p = nv.prepare_act(a_c, a_s, K)
     w_c, _, w_g, w_p = _gpu_operands(wc, wsc, gW, N, K)
-    y = host(nv.linear(a_c, a_s, a_g, w_c, w_p, w_g, N, K))
+    y = host(nv.linear(a_p, a_g, M, w_p, w_g, N, K))
     want = oracle.linear(ac, asc, gA, wc, wsc, gW)
     err = rel_fro(y, bf16_round(want))
     assert err <= REL_FRO_TOL, f"{mode}: rel err {err:.3e}"
@@ -58,19 +59,21 @@ def _case(oracle, M, N, K, outliers, seed, full=True, n_samples=8192):
     owc, ows, ogw = oracle.quantize(w)
     oac, oas, oga = oracle.quantize(a.float().numpy())
     wc, ws, gw = nv.quantize(to_dev(w))
-    ac, asc, ga = nv.quantize(to_dev(a))
+    act = nv.act_buffer(K)
+    ac, asc, ga = nv.quantize(to_dev(a), act=act)
     assert np.array_equal(wc.cpu().numpy(), owc) and np.array_equal(ws.cpu().numpy(), ows)
     assert np.array_equal(ac.cpu().numpy(), oac) and np.array_equal(asc.cpu().numpy(), oas)
-    wp = nv.prepare_weight_scales(ws, N, K)
-    y = nv.linear(ac, asc, ga, wc, wp, gw, N, K)
+    wp = nv.prepare_weight(wc, ws, N, K)
+    y = nv.linear(act, ga, M, wp, gw, N, K)
+    ops = (act, ga, M, wp, gw)
     if full:
         want = oracle.linear(oac, oas, oga, owc, ows, ogw)
-        return host(y), want, (ac, asc, ga, wc, wp, gw)
+        return host(y), want, ops
     rng = np.random.default_rng(seed)
     im = rng.integers(0, M, n_samples)
     inn = rng.integers(0, N, n_samples)
     want = oracle.linear_sampled(oac, oas, oga, owc, ows, ogw, im, inn)
-    return host(y)[im, inn], want, (ac, asc, ga, wc, wp, gw)
+    return host(y)[im, inn], want, ops
 
 
 @pytest.mark.parametrize("name,M,N,K,outl", [
@@ -102,14 +105,18 @@ def test_rows_independent_and_deterministic(oracle):
     w = inputs.weight_fp32(60, 1, N, K)
     a = inputs.activation_bf16(60, 2, M, K, 0.01)
     wc, ws, gw = nv.quantize(to_dev(w))
-    wp = nv.prepare_weight_scales(ws, N, K)
+    wp = nv.prepare_weight(wc, ws, N, K)
     gin = to_dev(np.array([0.01], np.float32))
-    ac, asc, ga = nv.quantize(to_dev(a), g_in=gin)
-    y16 = nv.linear(ac, asc, ga, wc, wp, gw, N, K).clone()
-    y16b = nv.linear(ac, asc, ga, wc, wp, gw, N, K).clone()
+    ad = to_dev(a)
+    act = nv.act_buffer(K)
+    _, _, ga = nv.quantize(ad, g_in=gin, act=act)
+    y16 = nv.linear(act, ga, M, wp, gw, N, K).clone()
+    y16b = nv.linear(act, ga, M, wp, gw, N, K).clone()
     assert torch.equal(y16, y16b)
     for m in (0, 9, 15):
-        y1 = nv.linear(ac[m:m + 1].contiguous(), asc[m:m + 1].contiguous(), ga, wc, wp, gw, N, K)
+        act1 = nv.act_buffer(K)
+        _, _, g1 = nv.quantize(ad[m:m + 1], g_in=gin, act=act1)
+        y1 = nv.linear(act1, g1, 1, wp, gw, N, K)
         assert torch.equal(y1[0], y16[m]), m
 
 
@@ -118,12 +125,12 @@ def test_linear_split_grid_invariance(oracle):
     cuda()
     M, N, K = 16, 1024, 5120
     _, _, ops = _case(oracle, M, N, K, 0.01, seed=61, full=False, n_samples=16)
-    ac, asc, ga, wc, wp, gw = ops
-    ref = host(nv.linear(ac, asc, ga, wc, wp, gw, N, K))
+    act, ga, M, wp, gw = ops
+    ref = host(nv.linear(act, ga, M, wp, gw, N, K))
     try:
         for G in (1, 7, 33, 160):
             nv.set_option(nv.OPT_LINEAR_CTAS, G)
-            y = host(nv.linear(ac, asc, ga, wc, wp, gw, N, K))
+            y = host(nv.linear(act, ga, M, wp, gw, N, K))
             assert rel_fro(y, ref) < 1e-5, G
     finally:
         nv.set_option(nv.OPT_LINEAR_CTAS, 0)
@@ -133,10 +140,10 @@ def test_residual_epilogue(oracle):
     cuda()
     M, N, K = 16, 640, 1024
     y, want, ops = _case(oracle, M, N, K, 0.0, seed=62)
-    ac, asc, ga, wc, wp, gw = ops
+    act, ga, M, wp, gw = ops
     res = inputs.bf16_normal(62, 5, (M, N))
     out = to_dev(res).clone()
-    nv.linear(ac, asc, ga, wc, wp, gw, N, K, y=out, residual=out)     # in place
+    nv.linear(act, ga, M, wp, gw, N, K, y=out, residual=out)     # in place
     err = rel_fro(host(out), bf16_round(want + res.double().numpy()))
     assert err <= REL_FRO_TOL
 
@@ -156,9 +163,11 @@ def test_lm_head_argmax(oracle, M):
     del w
     assert np.array_equal(ws.cpu().numpy(), ows)
     assert np.array_equal(wc.cpu().numpy(), owc)
-    ac, asc, ga = nv.quantize(to_dev(a))
-    wp = nv.prepare_weight_scales(ws, N, K)
-    y = nv.linear(ac, asc, ga, wc, wp, gw, N, K)
+    act = nv.act_buffer(K)
+    _, _, ga = nv.quantize(to_dev(a), act=act)
+    wp = nv.prepare_weight(wc, ws, N, K)
+    del wc, ws
+    y = nv.linear(act, ga, M, wp, gw, N, K)
     idx = nv.argmax(y).cpu().numpy()
     yh = host(y)
     want = oracle.linear(oac, oas, oga, owc, ows, ogw)
@@ -175,14 +184,40 @@ def test_lm_head_argmax(oracle, M):
 
 def test_linear_rejects_bad_arguments():
     cuda()
-    z = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    z = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
     g = torch.ones(1, device="cuda")
-    with pytest.raises(nv.NvFp4Error) as e:
-        nv.load().nvfp4_linear and nv._call("nvfp4_linear", z.data_ptr(), z.data_ptr(), g.data_ptr(), 17,
-                                            z.data_ptr(), z.data_ptr(), g.data_ptr(), 8, 64, None,
-                                            z.data_ptr(), 8, z.data_ptr(), 64, 0)
+    with pytest.raises(nv.NvFp4Error) as e:          # M > 16
+        nv._call("nvfp4_linear", z.data_ptr(), g.data_ptr(), 17, z.data_ptr(), g.data_ptr(), 8, 64, None,
+                 z.data_ptr(), 8, z.data_ptr(), 1 << 16, 0)
     assert e.value.code == -2
-    with pytest.raises(nv.NvFp4Error) as e:
-        nv._call("nvfp4_linear", z.data_ptr() + 1, z.data_ptr(), g.data_ptr(), 1, z.data_ptr(), z.data_ptr(),
-                 g.data_ptr(), 8, 64, None, z.data_ptr(), 8, z.data_ptr(), 64, 0)
+    with pytest.raises(nv.NvFp4Error) as e:          # misaligned prepared activation
+        nv._call("nvfp4_linear", z.data_ptr() + 1, g.data_ptr(), 1, z.data_ptr(), g.data_ptr(), 8, 64, None,
+                 z.data_ptr(), 8, z.data_ptr(), 1 << 16, 0)
     assert e.value.code == -3
+    with pytest.raises(nv.NvFp4Error) as e:          # workspace too small
+        nv._call("nvfp4_linear", z.data_ptr(), g.data_ptr(), 1, z.data_ptr(), g.data_ptr(), 8, 64, None,
+                 z.data_ptr(), 8, z.data_ptr(), 16, 0)
+    assert e.value.code == -4
+
+
+@pytest.mark.parametrize("M,K", [(16, 5120), (3, 576), (1, 64)])
+def test_prepared_activation_layout(M, K):
+    """quantize(act=...) writes exactly the re-layout of its canonical outputs,
+    which follows the documented tile image; untouched bytes stay zero."""
+    cuda()
+    a = inputs.activation_bf16(63, 0, M, K, 0.01)
+    act = nv.act_buffer(K)
+    codes, scales, g = nv.quantize(to_dev(a), act=act)
+    act2 = nv.prepare_act(codes, scales, K)
+    assert torch.equal(act, act2)
+    c, sc = codes.cpu().numpy(), scales.cpu().numpy()
+    want = np.zeros(act.numel(), np.uint8)
+    for m in range(M):
+        for blk in range(K // 16):
+            cidx, bi = blk // 32, blk % 32
+            base = cidx * 8192
+            b = (bi % 16) * 8
+            off = base + (bi // 16) * 2048 + m * 128 + ((((b >> 4) ^ (m & 7)) << 4) | (b & 15))
+            want[off:off + 8] = c[m, blk * 8:blk * 8 + 8]
+            want[base + 4096 + (bi // 4) * 512 + m * 16 + bi % 4] = sc[m, blk]
+    assert np.array_equal(act.cpu().numpy(), want)

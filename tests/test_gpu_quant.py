@@ -104,21 +104,34 @@ def test_rejects_bad_shapes():
     assert e.value.code == -2
 
 
-def test_prepare_scales_layout():
+def test_prepare_weight_layout():
+    """Prepared weight units: per (128-row tile, 512-K chunk), two 128-byte-
+    swizzled 16 KB code atoms then eight 512-byte scale images (line l, byte
+    4c + kb = scale of row l + 32c, block 4j + kb); zero-padded."""
     cuda()
     rng = np.random.default_rng(34)
-    for N, K in [(128, 256), (200, 320), (384, 5120)]:
+    for N, K in [(128, 512), (200, 576), (300, 1024)]:
+        codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
         sc = rng.integers(0, 0x7F, (N, K // 16), dtype=np.uint8)
-        prep = nv.prepare_weight_scales(to_dev(sc), N, K).cpu().numpy()
-        NT, KT = -(-N // 128), -(-K // 256)
-        want = np.zeros((NT, KT, 4, 32, 4, 4), np.uint8)     # [t][kt][j][l][c][kb]
+        prep = nv.prepare_weight(to_dev(codes), to_dev(sc), N, K).cpu().numpy()
+        NT, KC = -(-N // 128), -(-K // 512)
+        unit = 36864
+        want = np.zeros(NT * KC * unit, np.uint8)
         for t in range(NT):
-            for kt in range(KT):
-                for j in range(4):
-                    for c in range(4):
-                        rows = t * 128 + np.arange(32) + 32 * c
-                        for kb in range(4):
-                            col = kt * 16 + 4 * j + kb
-                            ok = (rows < N) & (col < K // 16)
-                            want[t, kt, j, :, c, kb] = np.where(ok, sc[np.minimum(rows, N - 1), min(col, K // 16 - 1)], 0)
-        assert np.array_equal(prep, want.ravel())
+            for c in range(KC):
+                base = (t * KC + c) * unit
+                for a in range(2):
+                    for r in range(128):
+                        row = t * 128 + r
+                        for b in range(128):
+                            col = c * 256 + a * 128 + b
+                            if row < N and col < K // 2:
+                                want[base + a * 16384 + r * 128 + ((((b >> 4) ^ (r & 7)) << 4) | (b & 15))] = codes[row, col]
+                for j in range(8):
+                    for l in range(32):
+                        for cc in range(4):
+                            for kb in range(4):
+                                row, blk = t * 128 + l + 32 * cc, c * 32 + 4 * j + kb
+                                if row < N and blk < K // 16:
+                                    want[base + 32768 + j * 512 + l * 16 + 4 * cc + kb] = sc[row, blk]
+        assert np.array_equal(prep, want)
