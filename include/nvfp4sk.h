@@ -142,6 +142,31 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *
                                         nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_linear_noalloc -- nvfp4_linear for callers that cannot allocate.
+ * (The pages have no counterpart: this is a deployment variant.)
+ *
+ * Some callers cannot call cudaMalloc or take memory from a caching
+ * allocator: a plugin inside a host runtime that owns all device memory, a
+ * serving loop that must never enter an allocator on its latency path, or
+ * code with no allocator at hand.  This variant takes no workspace: its
+ * split-K scratch is a fixed array inside the library (every GPU that loads
+ * the library holds nvfp4_linear_noalloc_scratch_bytes() of it until the
+ * process exits).  Same arguments and results as nvfp4_linear otherwise.
+ * Limits: N <= 524288 (larger N is rejected with
+ * NVFP4SK_ERR_UNSUPPORTED_SHAPE); the grid is capped at 160 CTAs.
+ * The first call on a device looks up the array's device address (and sets
+ * kernel attributes); make that first call before any stream capture.
+ * All calls on a device share the one array, and each call clears its
+ * arrival counters first: calls whose GPU work can overlap (unordered
+ * streams) race on it and must not be issued.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t nvfp4_linear_noalloc_scratch_bytes(void);
+NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const float *g_a, int64_t M,
+                                                const uint8_t *w_prepared, const float *g_w, int64_t N, int64_t K,
+                                                const void *residual, void *y, int64_t ldy,
+                                                nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * tree_attn_fp8kv -- attention of the T tree nodes over the FP8 paged KV
  * cache with the ancestor mask (section "Tree multi-token prediction": the
  * target model verifies all candidates of the tree in one forward pass;

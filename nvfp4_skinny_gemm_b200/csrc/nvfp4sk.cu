@@ -592,3 +592,93 @@ nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, ui
 }
 
 }  // extern "C"
+
+// ============================================================================
+// nvfp4_linear_noalloc: the NVFP4 linear for callers that cannot allocate.
+//
+// The scratch nvfp4_linear keeps in a caller-owned workspace (split-K arrival
+// counters, partial tiles) lives here in one file-scope device array instead,
+// sized for LIN_NOALLOC_MAX_CTAS CTAs and LIN_MAX_NT weight tiles.  The
+// array's name is only a host-side stand-in: the device address is obtained
+// with cudaGetSymbolAddress, once per device, on the first call made on that
+// device.  Every call on a device shares the one array, so calls whose GPU
+// work overlaps (different streams, no ordering) race on it.
+// ============================================================================
+namespace {
+constexpr int LIN_NOALLOC_MAX_CTAS = 160;
+constexpr size_t LIN_NOALLOC_SCRATCH_BYTES = LIN_COUNTER_BYTES + (size_t)LIN_NOALLOC_MAX_CTAS * 2 * 128 * 16 * 4;
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_linear_noalloc_scratch[LIN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+uint8_t *g_noalloc_ptr[MAX_DEV];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(uint8_t **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= MAX_DEV) return fail(NVFP4SK_ERR_DEVICE, "device id %d out of range", dev);
+    if (!g_noalloc_ptr[dev]) {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_linear_noalloc_scratch);
+            if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(linear scratch)");
+            g_noalloc_ptr[dev] = (uint8_t *)p;
+        }
+    }
+    *out = g_noalloc_ptr[dev];
+    return NVFP4SK_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_linear_noalloc_scratch_bytes(void) { return LIN_NOALLOC_SCRATCH_BYTES; }
+
+nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const float *g_a, int64_t M,
+                                    const uint8_t *w_prepared, const float *g_w, int64_t N, int64_t K,
+                                    const void *residual, void *y, int64_t ldy, nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!a_prepared || !g_a || !w_prepared || !g_w || !y) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (M < 1 || M > 16 || N < 1 || K < 64 || K % 64 != 0 || ldy < N)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, N >= 1, K %% 64 == 0, ldy >= N");
+    if (N > LIN_MAX_NT * 128)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "N = %lld exceeds the built-in scratch of nvfp4_linear_noalloc (at most %lld output features)",
+                    (long long)N, (long long)(LIN_MAX_NT * 128));
+    if (!al16(a_prepared) || !al16(w_prepared))
+        return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands must be 16-byte aligned");
+    uint8_t *scratch = nullptr;
+    if (int rc = noalloc_scratch(&scratch)) return rc;
+    const int64_t NT = cdiv(N, 128), KC = cdiv(K, LIN_KC), U = NT * KC;
+    const int G = (int)std::min<int64_t>(std::min<int64_t>(linear_grid(*d, U), LIN_NOALLOC_MAX_CTAS), U);
+    cudaStream_t st = (cudaStream_t)stream;
+    // the arrival counters must read zero when the kernel starts
+    cudaError_t e = cudaMemsetAsync(scratch, 0, (size_t)NT * 4 * sizeof(int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(linear scratch counters)");
+    LinearParams p;
+    p.w = w_prepared;
+    p.a = a_prepared;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.residual = (const __nv_bfloat16 *)residual;
+    p.y = (__nv_bfloat16 *)y;
+    p.counters = (int *)scratch;
+    p.partial = (float *)(scratch + LIN_COUNTER_BYTES);
+    p.ldy = ldy;
+    p.U = U;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.NT = (int)NT;
+    p.KC = (int)KC;
+    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, st, 1, p),
+                    "nvfp4_linear_kernel (no-alloc)");
+}
+
+}  // extern "C"

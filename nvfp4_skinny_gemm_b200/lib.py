@@ -42,6 +42,8 @@ _SIGS = {
     "nvfp4_prepare_weight": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "nvfp4_linear_noalloc_scratch_bytes": (_sz, []),
+    "nvfp4_linear_noalloc": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
     "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
     "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
                                _vp, _f32, _vp, _vp, _sz, _vp]),
