@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--ctx", type=int, default=23552)
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--kernel-case", default=None,
                     choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "attn", "restore", "quantize"],
                     help="run one kernel on a small case (for ncu captures) instead of the step")
@@ -264,6 +266,11 @@ def run_ours(args, world, rank, local):
         for _ in range(max(3, args.warmup)):
             graph.replay()
         torch.cuda.synchronize()
+        if args.profile_range:
+            torch.cuda.profiler.start()
+            graph.replay()
+            torch.cuda.synchronize()
+            torch.cuda.profiler.stop()
 
         # ---- device-timed step
         barrier(world)

@@ -174,8 +174,10 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const
  *
  * q: bf16, node i head hq at q[i*ld_q + hq*D + d] (ld_q >= Hq*D, even).
  * Cache (one layer): k_pool u8 [n_pool_pages][Hkv][page_size][D]
- *   (token-major pages); v_pool u8 [n_pool_pages][Hkv][D][page_size]
- *   (dimension-major pages).  Position p lives in page page_table[p /
+ *   (token-major pages); v_pool u8 [n_pool_pages][Hkv][D*page_size], each
+ *   (page, head) plane cut into tiles of 8 dimensions x 16 slots (128
+ *   bytes): dimension d, slot t at byte ((d/8)*(page_size/16) + t/16)*128 +
+ *   (d%8)*16 + t%16 of the plane.  Position p lives in page page_table[p /
  *   page_size], slot p % page_size.  Context positions are 0..ctx_len-1; the
  *   tree nodes' own K/V are at ctx_len + i (node i).
  * page_table: i32 [ceil((ctx_len+T)/page_size)] physical page ids.
@@ -184,7 +186,12 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const
  * Node i, head hq (KV head h = hq / (Hq/Hkv)) attends to every context
  *   position and to the tree positions of {i} and its ancestors:
  *   out = softmax_p(sm_scale * q . K_p) . V_p, bf16 [T][Hq][D] (dense).
- * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 7.
+ * Slots of the last page past position ctx_len+T-1 may hold any bytes
+ *   (NaN codes included); they do not reach the output.  A page id outside
+ *   [0, n_pool_pages) skips that page (its positions get no weight) and is
+ *   flagged NVFP4SK_ERR_OUT_OF_RANGE in the device status, as is a parent id
+ *   outside [-1, T).
+ * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 8.
  * ws: tree_attn_workspace_bytes(...) bytes.
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
@@ -231,7 +238,8 @@ NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, i
 /* Append T new tokens' K and V (bf16, token i head h at k_new[i*ld_new +
  * h*D + d]) to the cache at positions ctx_len .. ctx_len+T-1 as
  * E4M3(fp32(x / scale[h])) (round-to-nearest-even, saturating); the FP8 KV
- * cache write of section "NVFP4 and FP8".  Layouts as tree_attn_fp8kv. */
+ * cache write of section "NVFP4 and FP8".  Layouts as tree_attn_fp8kv;
+ * D % 8 == 0 and page_size % 16 == 0. */
 NVFP4SK_API nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_new, int T, int Hkv, int D,
                              uint8_t *k_pool, uint8_t *v_pool, int64_t n_pool_pages, int page_size,
                              const int32_t *page_table, int64_t ctx_len, const float *k_scale,
@@ -265,6 +273,12 @@ NVFP4SK_API int64_t nvfp4sk_get_option(int option);
  * = E4M3 code (RNE, satfinite).  Either output may be NULL. */
 NVFP4SK_API nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, uint8_t *e4m3,
                                     nvfp4sk_stream_t stream);
+
+/* Diagnostic (failure detection; the pages have no counterpart): one launch
+ * whose single device wait can never be satisfied.  The wait gives up after
+ * the NVFP4SK_OPT_TIMEOUT_NS limit; the next nvfp4sk_get_device_status
+ * returns NVFP4SK_ERR_TIMEOUT with site 900, and the context stays usable. */
+NVFP4SK_API nvfp4sk_status nvfp4sk_debug_wait_timeout(nvfp4sk_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -1,21 +1,31 @@
 // attn.cuh -- tree-masked attention of the draft-tree nodes over the FP8
-// paged KV cache (flash-decoding: split over the context, then combine).
+// paged KV cache on sm_100a tensor cores (flash-decoding: split over the
+// context, then combine).
 //
 // Grid (splits, Hkv); one CTA = one KV head x one contiguous range of pages.
-// Warps 0..group-1 each own one query head of the group and all 16 nodes
-// (16 MMA rows); the last warp is the producer: per page it loads the K page
-// (8 KB, 2-D TMA with 128-byte swizzle) and the V page (8 KB, 1-D bulk copy,
-// stored dimension-major) into a ring of shared-memory stages.
-//
-// Both contractions run on FP8 tensor-core MMAs (mma.sync m16n8k32 e4m3,
-// fp32 accumulate), reading the cached E4M3 codes straight from shared
-// memory; the per-head K/V scales are applied to scores / outputs instead.
-// The bf16 query (scaled per row by a power of two) and the probabilities
-// (scaled by 256) are each written as a sum of two E4M3 terms hi + lo, so
-// each contraction is two MMAs and the operands keep ~8 significant bits.
-// Token and dimension orders inside a page are permuted (consistently for
-// Q, K, P and V) so that every fragment is one conflict-free 16-byte load.
-// Softmax is online in the log2 domain; rows are reduced with quad shuffles.
+// The 128 MMA rows are (query head w of the group, node i) -> row 16*w + i
+// (rows past group*16 are zero padding).  Per page of 64 tokens:
+//   S = Q K^T   tcgen05.mma kind::f8f6f4, M=128, N=64, K=32 per instruction;
+//               Q enters as two E4M3 terms (hi + lo) of the row-scaled bf16
+//               query, K as the cached E4M3 codes (128-byte-swizzled TMA
+//               tile); fp32 S in tensor memory.
+//   softmax     one thread per row: S row -> registers (tcgen05.ld), ancestor
+//               mask on the page that holds the tree, running max in the
+//               log2 domain, P' = 2^(s - m + 6) as two E4M3 terms (hi + lo)
+//               stored to shared memory in the MMA's core-matrix layout.
+//               O is rescaled in tensor memory only when a row max grows by
+//               more than 2^2.
+//   O += P V    M=128, N=144, K=32: the V pages are kept in HBM in the
+//               core-matrix layout, so one bulk copy lands the operand; 16
+//               extra operand rows (one of them all ones) make column 128 of
+//               O the row sum of P', accumulated in fp32 by the tensor core.
+// Two softmax warpgroups take alternate pages, each with its own S and O
+// accumulators in tensor memory and its own running max, so that two pages
+// are in the exponent / packing stage at once; their results are merged in
+// the epilogue.
+// Warp roles: 0 producer (TMA K page + bulk V page into an 8-stage ring),
+// 1 TMEM allocation + single-thread MMA issue, 2-5 and 6-9 softmax.
+// The split results (O / l, m, l per row) are merged by the combine kernel.
 #pragma once
 #include "common.cuh"
 
@@ -24,12 +34,155 @@ namespace nvfp4sk {
 constexpr int ATT_D = 128;
 constexpr int ATT_P = 64;
 constexpr int ATT_T = 16;
-constexpr int ATT_STAGES = 4;
-constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;     // 8 KB, token-major
-constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;     // 8 KB, dimension-major
-constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES;
-constexpr uint32_t ATT_SMEM_BYTES = ATT_STAGES * ATT_STAGE_BYTES + 1024 + 256;
+constexpr int ATT_ROWS = 128;
+constexpr int ATT_STAGES = 8;
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_MAX_SPLITS = 1024;
+constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;                 // 8 KB token-major page
+constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB core-matrix page
+constexpr uint32_t ATT_ONES_BYTES = 16 * ATT_P;                 // 16 operand rows: ones, then zeros
+constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES + ATT_ONES_BYTES;   // 17 KB
+constexpr uint32_t ATT_Q_BYTES = ATT_ROWS * ATT_D;              // one E4M3 term of Q
+constexpr uint32_t ATT_PB_BYTES = ATT_ROWS * ATT_P;             // one E4M3 term of P
+constexpr uint32_t ATT_OFF_Q = ATT_STAGES * ATT_STAGE_BYTES;    // Q hi | Q lo
+constexpr uint32_t ATT_OFF_P = ATT_OFF_Q + 2 * ATT_Q_BYTES;     // P[2 groups] x (hi | lo)
+constexpr uint32_t ATT_OFF_X = ATT_OFF_P + 4 * ATT_PB_BYTES;    // float exchange [2][2][128]
+constexpr uint32_t ATT_OFF_BAR = ATT_OFF_X + 2048;
+constexpr uint32_t ATT_SMEM_BYTES = ATT_OFF_BAR + 256 + 1024;
+constexpr uint32_t ATT_TMEM_COLS = 512;
+constexpr uint32_t ATT_NO = ATT_D + 16;                         // O columns: 128 dims + row sum block
+constexpr uint32_t ATT_TM_S0 = 0, ATT_TM_S1 = 64;
+constexpr uint32_t ATT_TM_O0 = 128, ATT_TM_O1 = 288;
+constexpr float ATT_TAU = 2.0f;       // log2 growth of a row max that triggers an O rescale
+constexpr float ATT_PSHIFT = 6.0f;    // P' = 2^(s - m + 6) <= 2^(6 + TAU) = 256 < 448
 constexpr float LOG2E = 1.4426950408889634f;
+static_assert(ATT_STAGE_BYTES % 1024 == 0, "K tiles need 1024-byte alignment (128-byte swizzle atoms)");
+static_assert(ATT_TM_O1 + ATT_NO <= ATT_TMEM_COLS && ATT_TM_O0 + ATT_NO <= ATT_TM_O1, "tensor memory budget");
+
+// Byte of (dim d, slot t) inside a V page plane: 8-dim x 16-slot core matrices
+// of 128 bytes, ordered [d/8][t/16][d%8][t%16].
+__host__ __device__ __forceinline__ uint32_t v_offset(uint32_t d, uint32_t t)
+{
+    return ((d >> 3) * (ATT_P / 16) + (t >> 4)) * 128u + (d & 7u) * 16u + (t & 15u);
+}
+
+// Instruction descriptor, kind::f8f6f4: fp32 accumulate (bits 4-5 = 1), A and
+// B E4M3 (format 0), K-major, N>>3 in bits 17-22, M>>4 in bits 24-28.
+constexpr uint32_t att_idesc(uint32_t M, uint32_t N) { return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24); }
+
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t tmem_ld_x1(uint32_t taddr)
+{
+    uint32_t v;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// packed halves: lower half <- lo, upper half <- hi
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi)
+{
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t h)
+{
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h));
+    return d;
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c)
+{
+    uint32_t d;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)c));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Four non-negative values -> E4M3 codes hi (bytes 0..3) and lo with x ~= hi + lo:
+// x is rounded to f16 (11 bits), hi = E4M3(x), lo = E4M3(x - hi) (exact f16 difference).
+__device__ __forceinline__ void split4_f16(float x0, float x1, float x2, float x3, uint32_t &hi, uint32_t &lo)
+{
+    const uint32_t a = f32x2_to_f16x2(x0, x1), b = f32x2_to_f16x2(x2, x3);
+    const uint32_t ha = f16x2_to_e4m3x2(a), hb = f16x2_to_e4m3x2(b);
+    const uint32_t la = f16x2_to_e4m3x2(hsub2_u32(a, e4m3x2_to_f16x2(ha)));
+    const uint32_t lb = f16x2_to_e4m3x2(hsub2_u32(b, e4m3x2_to_f16x2(hb)));
+    hi = ha | (hb << 16);
+    lo = la | (lb << 16);
+}
+
+// x0, x1 -> (hi, lo) E4M3 pairs (byte 0 = x0, byte 1 = x1) with x ~= hi + lo, in fp32.
+__device__ __forceinline__ void split2_f32(float x0, float x1, uint32_t &hi2, uint32_t &lo2)
+{
+    hi2 = cvt_e4m3x2(x0, x1) & 0xFFFFu;
+    const uint32_t hh = e4m3x2_to_f16x2(hi2);
+    const float h0 = __half2float(__ushort_as_half((unsigned short)(hh & 0xFFFFu)));
+    const float h1 = __half2float(__ushort_as_half((unsigned short)(hh >> 16)));
+    lo2 = cvt_e4m3x2(x0 - h0, x1 - h1) & 0xFFFFu;
+}
 
 struct AttnParams {
     const __nv_bfloat16 *q;
@@ -48,57 +201,24 @@ struct AttnParams {
     int T, Hq, Hkv, group, S, n_log_pages;
 };
 
-__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm(
-        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ float fast_exp2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// x -> (hi, lo) E4M3 codes with x ~= value(hi) + value(lo)
-__device__ __forceinline__ void split_e4m3(float x, uint32_t &hi, uint32_t &lo)
-{
-    hi = cvt_e4m3x2(x, 0.f) & 0xFFu;
-    const float r = x - e4m3_to_float(hi);
-    lo = cvt_e4m3x2(r, 0.f) & 0xFFu;
-}
-
-// two floats -> two (hi, lo) pairs packed into bytes [0..1] of hi2 / lo2
-__device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint32_t &hi2, uint32_t &lo2, float &sum)
-{
-    const uint32_t h = cvt_e4m3x2(x0, x1);          // byte0 = x0, byte1 = x1
-    uint32_t hh;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"((uint16_t)h));
-    const float h0 = __half2float(__ushort_as_half((unsigned short)(hh & 0xFFFFu)));
-    const float h1 = __half2float(__ushort_as_half((unsigned short)(hh >> 16)));
-    const float r0 = x0 - h0, r1 = x1 - h1;
-    const uint32_t l = cvt_e4m3x2(r0, r1);
-    uint32_t ll;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(ll) : "h"((uint16_t)l));
-    sum += (h0 + h1) + (__half2float(__ushort_as_half((unsigned short)(ll & 0xFFFFu))) +
-                        __half2float(__ushort_as_half((unsigned short)(ll >> 16))));
-    hi2 = h & 0xFFFFu;
-    lo2 = l & 0xFFFFu;
-}
-
-__global__ void __launch_bounds__(8 * 32, 1)
+__global__ void __launch_bounds__(ATT_THREADS, 1)
     tree_attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const AttnParams p)
 {
     extern __shared__ uint8_t att_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(att_smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ATT_STAGES * ATT_STAGE_BYTES);
-    uint64_t *empty = full + ATT_STAGES;
-    volatile int *s_valid = reinterpret_cast<volatile int *>(empty + ATT_STAGES);
-    volatile int *s_abort = s_valid + ATT_STAGES;
+    uint64_t *kv_full = reinterpret_cast<uint64_t *>(smem + ATT_OFF_BAR);
+    uint64_t *kv_empty = kv_full + ATT_STAGES;
+    uint64_t *s_full = kv_empty + ATT_STAGES;   // [2]
+    uint64_t *s_free = s_full + 2;              // [2]
+    uint64_t *p_full = s_free + 2;              // [2]
+    uint64_t *p_free = p_full + 2;              // [2]
+    uint64_t *q_ready = p_free + 2;
+    uint64_t *o_done = q_ready + 1;
+    uint64_t *drain = o_done + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    volatile uint8_t *s_page_ok = reinterpret_cast<volatile uint8_t *>(tmem_holder + 2);   // [ATT_STAGES]
+    float *xch = reinterpret_cast<float *>(smem + ATT_OFF_X);                             // [2][2][128]
 
     const int h = blockIdx.y, split = blockIdx.x;
     const int group = p.group;
@@ -109,284 +229,399 @@ __global__ void __launch_bounds__(8 * 32, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < ATT_STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], group);
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_free[b], 4);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&p_free[b], 1);
+        }
+        mbar_init(q_ready, 8);
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
         *s_abort = 0;
         fence_barrier_init();
     }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, ATT_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
     pdl_wait();
     pdl_launch_dependents();
 
-    if ((int)warp == group) {
+    if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            int issued = 0;
             for (int i = 0; i < n_pages; ++i) {
                 const int st = i % ATT_STAGES;
                 if (i >= ATT_STAGES &&
-                    !mbar_wait(&empty[st], (uint32_t)(((i / ATT_STAGES) & 1) ^ 1), 301, s_abort))
+                    !mbar_wait(&kv_empty[st], (uint32_t)(((i / ATT_STAGES) - 1) & 1), 301, s_abort))
                     break;
                 const int32_t pg = p.page_table[pg0 + i];
-                const bool valid = pg >= 0 && pg < p.n_pool_pages;
-                s_valid[st] = valid ? 1 : 0;
                 uint8_t *dst = smem + st * ATT_STAGE_BYTES;
-                if (valid) {
-                    mbar_arrive_expect_tx(&full[st], ATT_STAGE_BYTES);
-                    tma_load_2d(dst, &tm_k, &full[st], 0, (int32_t)(((int64_t)pg * p.Hkv + h) * ATT_P));
+                const bool ok = pg >= 0 && pg < p.n_pool_pages;
+                s_page_ok[st] = ok ? 1 : 0;
+                if (ok) {
+                    mbar_arrive_expect_tx(&kv_full[st], ATT_K_BYTES + ATT_V_BYTES);
+                    tma_load_2d(dst, &tm_k, &kv_full[st], 0, (int32_t)(((int64_t)pg * p.Hkv + h) * ATT_P));
                     bulk_load(dst + ATT_K_BYTES, p.v_pool + ((int64_t)pg * p.Hkv + h) * ATT_V_BYTES, ATT_V_BYTES,
-                              &full[st]);
+                              &kv_full[st]);
                 } else {
                     report_error(ERRBIT_RANGE, 302);
-                    mbar_arrive(&full[st]);
+                    mbar_arrive(&kv_full[st]);        // page skipped: its scores are masked out
                 }
+                issued = i + 1;
             }
             if (*s_abort) {
-                for (int i = n_pages > ATT_STAGES ? n_pages - ATT_STAGES : 0; i < n_pages; ++i)
-                    mbar_wait(&full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 303);
+                for (int i = issued > ATT_STAGES ? issued - ATT_STAGES : 0; i < issued; ++i)
+                    mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 303);
             }
         }
-        return;
-    }
-    if ((int)warp > group) return;
-
-    // ---------------------------------------------------------------- compute
-    const int hq = h * group + (int)warp;
-    const int g = (int)(lane >> 2), c = (int)(lane & 3);
-    const int T = p.T;
-    const int64_t L = p.ctx_len;
-
-    // query fragments: rows g (node g) and g+8 (node g+8), dims 32c..32c+31
-    float qv[2][32];
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = att_idesc(128, ATT_P);
+            constexpr uint32_t idesc_o = att_idesc(128, ATT_NO);
+            const uint32_t q_hi = smem_u32(smem + ATT_OFF_Q), q_lo = q_hi + ATT_Q_BYTES;
+            bool o_init[2] = {false, false};
+            bool ok = mbar_wait(q_ready, 0, 310, s_abort);
+            tc_fence_after();
+            auto issue_pv = [&](int j) -> bool {
+                const int g = j & 1;
+                if (!mbar_wait(&p_full[g], (uint32_t)((j >> 1) & 1), 311, s_abort)) return false;
+                tc_fence_after();
+                if (s_page_ok[j % ATT_STAGES]) {
+                    const uint32_t v_s = smem_u32(smem + (j % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES);
+                    const uint32_t p_hi = smem_u32(smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES), p_lo = p_hi + ATT_PB_BYTES;
+                    const uint32_t o_t = tmem_base + (g ? ATT_TM_O1 : ATT_TM_O0);
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const int node = g + 8 * rr;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (node < T) w = *reinterpret_cast<const uint4 *>(p.q + node * p.ld_q + (int64_t)hq * ATT_D + 32 * c + 8 * i);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                qv[rr][8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
-                qv[rr][8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
-            }
-        }
-    }
-    float c_row[2];
-    uint32_t anc[2];
-    uint32_t qa_hi[4][4], qa_lo[4][4];   // [k-step][reg]
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        float amax = 0.f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(qv[rr][k]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-        // power-of-two row scale 2^(7 - floor(log2 amax)) puts the row max in [128, 256)
-        int e = 0;
-        if (amax > 0.f) e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-        e = max(-100, min(100, e));
-        const float qs = amax > 0.f ? __uint_as_float((uint32_t)(127 + 7 - e) << 23) : 1.f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) qv[rr][k] *= qs;
-        c_row[rr] = __fdiv_rn(p.k_scale[h] * p.sm_scale * LOG2E, qs);
-        // ancestor mask of node g + 8 rr
-        uint32_t m = 0;
-        const int node = g + 8 * rr;
-        if (node < T) {
-            int a = node;
-            for (int it = 0; it < ATT_T && a >= 0; ++it) {
-                if (a >= T) {                      // malformed tree: parent id out of range
-                    report_error(ERRBIT_RANGE, 305);
-                    break;
-                }
-                m |= 1u << a;
-                a = p.parent[a];
-            }
-        }
-        anc[rr] = m;
-    }
-    // dims of k-step t = 2u + v: a0/b0 <-> 32c + 16u + 8v + 0..3, a2/b1 <-> +4..7
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int base = 16 * (t >> 1) + 8 * (t & 1);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                uint32_t hw = 0, lw = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t hb, lb;
-                    split_e4m3(qv[rr][base + 4 * half + j], hb, lb);
-                    hw |= hb << (8 * j);
-                    lw |= lb << (8 * j);
-                }
-                qa_hi[t][2 * half + rr] = hw;   // reg order: a0 (g,lo-k) a1 (g+8,lo-k) a2 (g,hi-k) a3 (g+8,hi-k)
-                qa_lo[t][2 * half + rr] = lw;
-            }
-        }
-    }
-
-    float O[16][4];
-#pragma unroll
-    for (int nd = 0; nd < 16; ++nd)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) O[nd][e] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-
-    for (int i = 0; i < n_pages; ++i) {
-        const int st = i % ATT_STAGES;
-        if (!mbar_wait(&full[st], (uint32_t)((i / ATT_STAGES) & 1), 304, s_abort)) break;
-        if (s_valid[st]) {
-            const uint8_t *kt = smem + st * ATT_STAGE_BYTES;
-            const uint8_t *vt = kt + ATT_K_BYTES;
-            const int64_t pos0 = (int64_t)(pg0 + i) * ATT_P;
-            float sacc[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-            // k-steps outermost so that consecutive MMAs update different n-tiles
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                uint4 kw[8];
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                    const int tok = 16 * (g >> 1) + 8 * (nt >> 2) + 4 * ((nt & 3) >> 1) + 2 * (nt & 1) + (g & 1);
-                    kw[nt] = *reinterpret_cast<const uint4 *>(kt + tok * 128 + (((2 * c + u) ^ (tok & 7)) << 4));
-                }
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_hi[2 * u], kw[nt].x, kw[nt].y);
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_hi[2 * u + 1], kw[nt].z, kw[nt].w);
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_lo[2 * u], kw[nt].x, kw[nt].y);
-#pragma unroll
-                for (int nt = 0; nt < 8; ++nt) mma_e4m3_16832(sacc[nt], qa_lo[2 * u + 1], kw[nt].z, kw[nt].w);
-            }
-            // scale, mask, row max
-            const bool tail = pos0 + ATT_P > L;
-            float tmax[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int rr = e >> 1;
-                    float s2 = sacc[nt][e] * c_row[rr];
-                    if (tail) {
-                        const int tok = 16 * c + 8 * (nt >> 2) + 4 * ((nt & 3) >> 1) + 2 * (nt & 1) + (e & 1);
-                        const int64_t pos = pos0 + tok;
-                        bool vis = pos < L;
-                        if (!vis) {
-                            const int64_t j = pos - L;
-                            vis = j < T && ((anc[rr] >> j) & 1u);
-                        }
-                        if (!vis) s2 = -INFINITY;
+                    for (int t = 0; t < ATT_P / 32; ++t) {
+                        const uint64_t vd = smem_desc(v_s + 256 * t, 128, 512, SWZ_NONE);
+                        mma_f8f6f4(o_t, smem_desc(p_hi + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o,
+                                   (o_init[g] || t > 0) ? 1u : 0u);
+                        mma_f8f6f4(o_t, smem_desc(p_lo + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o, 1u);
                     }
-                    sacc[nt][e] = s2;
-                    tmax[rr] = fmaxf(tmax[rr], s2);
+                    o_init[g] = true;
                 }
-            }
-            float alpha[2], muse[2];
+                tc_commit(&p_free[g]);
+                tc_commit(&kv_empty[j % ATT_STAGES]);
+                return true;
+            };
+            for (int i = 0; i < n_pages && ok; ++i) {
+                const int st = i % ATT_STAGES, g = i & 1;
+                if (!mbar_wait(&kv_full[st], (uint32_t)((i / ATT_STAGES) & 1), 312, s_abort)) { ok = false; break; }
+                if (i >= 2 && !mbar_wait(&s_free[g], (uint32_t)(((i - 2) >> 1) & 1), 313, s_abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t k_s = smem_u32(smem + st * ATT_STAGE_BYTES);
+                const uint32_t s_t = tmem_base + (g ? ATT_TM_S1 : ATT_TM_S0);
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                tmax[rr] = fmaxf(tmax[rr], __shfl_xor_sync(0xFFFFFFFFu, tmax[rr], 1));
-                tmax[rr] = fmaxf(tmax[rr], __shfl_xor_sync(0xFFFFFFFFu, tmax[rr], 2));
-                const float mn = fmaxf(m_run[rr], tmax[rr]);
-                muse[rr] = mn == -INFINITY ? 0.f : mn;
-                alpha[rr] = fast_exp2(m_run[rr] - muse[rr]);
-                m_run[rr] = mn;
-            }
-            // probabilities x 256 as (hi, lo) E4M3 pairs, packed into PV A fragments
-            uint32_t pa_hi[2][4], pa_lo[2][4];
-            float psum[2] = {0.f, 0.f};
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {          // a0/a1 (n-tiles 4w,4w+1) a2/a3 (4w+2,4w+3)
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int nA = 4 * w + 2 * half, nB = nA + 1;
-                        const float x0 = fast_exp2(sacc[nA][2 * rr] - muse[rr]) * 256.f;
-                        const float x1 = fast_exp2(sacc[nA][2 * rr + 1] - muse[rr]) * 256.f;
-                        const float x2 = fast_exp2(sacc[nB][2 * rr] - muse[rr]) * 256.f;
-                        const float x3 = fast_exp2(sacc[nB][2 * rr + 1] - muse[rr]) * 256.f;
-                        uint32_t h01, l01, h23, l23;
-                        split_e4m3x2(x0, x1, h01, l01, psum[rr]);
-                        split_e4m3x2(x2, x3, h23, l23, psum[rr]);
-                        pa_hi[w][2 * half + rr] = h01 | (h23 << 16);
-                        pa_lo[w][2 * half + rr] = l01 | (l23 << 16);
-                    }
+                for (int t = 0; t < ATT_D / 32; ++t) {
+                    const uint64_t kd = smem_desc(k_s + 32 * t, 16, 1024, SWZ_128B);
+                    mma_f8f6f4(s_t, smem_desc(q_hi + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, t > 0 ? 1u : 0u);
+                    mma_f8f6f4(s_t, smem_desc(q_lo + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, 1u);
                 }
+                tc_commit(&s_full[g]);
+                if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
             }
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) l_run[rr] = l_run[rr] * alpha[rr] + psum[rr];
-            // four dimension tiles at a time: their MMAs are independent
-#pragma unroll
-            for (int nd0 = 0; nd0 < 16; nd0 += 4) {
-                uint4 x[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int nd = nd0 + k;
-                    O[nd][0] *= alpha[0]; O[nd][1] *= alpha[0];
-                    O[nd][2] *= alpha[1]; O[nd][3] *= alpha[1];
-                    x[k] = *reinterpret_cast<const uint4 *>(vt + (8 * nd + g) * ATT_P + 16 * c);
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_hi[0], x[k].x, x[k].y);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_hi[1], x[k].z, x[k].w);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_lo[0], x[k].x, x[k].y);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_e4m3_16832(O[nd0 + k], pa_lo[1], x[k].z, x[k].w);
+            if (ok && n_pages > 0) ok = issue_pv(n_pages - 1);
+            if (ok) {
+                tc_commit(o_done);
+            } else {
+                tc_commit(drain);
+                mbar_wait(drain, 0, 314);
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+    } else {
+        // ------------------------------------------------------------ softmax groups
+        const int g = (int)(warp - 2) >> 2;                   // 0: even pages, 1: odd pages
+        const uint32_t qd = warp & 3;                         // TMEM sub-partition
+        const int r = (int)(32 * qd + lane);                  // MMA row
+        const int w = r >> 4, node = r & 15;
+        const bool row_ok = w < group;
+        const int hq = h * group + w;
+        const int T = p.T;
+        const int64_t L = p.ctx_len;
+        const uint32_t row_t = tmem_base + ((32u * qd) << 16);
+        const uint32_t s_t = row_t + (g ? ATT_TM_S1 : ATT_TM_S0);
+        const uint32_t o_t = row_t + (g ? ATT_TM_O1 : ATT_TM_O0);
+
+        // ---- Q -> two E4M3 terms, row scaled by a power of two into [128, 256);
+        //      group g converts dims 64g .. 64g+63 of row r
+        float c_row;
+        uint32_t anc = 0;
+        {
+            const bool has_q = row_ok && node < T;
+            uint4 qraw[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                qraw[k] = has_q ? *reinterpret_cast<const uint4 *>(p.q + node * p.ld_q + (int64_t)hq * ATT_D + 64 * g + 8 * k)
+                                : make_uint4(0, 0, 0, 0);
+            float amax = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t wd[4] = {qraw[k].x, qraw[k].y, qraw[k].z, qraw[k].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(wd[j] << 16)),
+                                             fabsf(__uint_as_float(wd[j] & 0xFFFF0000u))));
+            }
+            xch[g * 128 + r] = amax;
+            // the ones block of every stage: operand row 128 (16 bytes per 16-token chunk) = 1.0, rest 0
+            {
+                const int st_i = (int)(threadIdx.x - 64);     // 0..255
+                uint8_t *ones = smem + (st_i >> 5) * ATT_STAGE_BYTES + ATT_K_BYTES + ATT_V_BYTES;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t off = (uint32_t)(st_i & 31) * 32u + 16u * j;
+                    const uint32_t v = (off < 512u && (off & 127u) == 0u) ? 0x38383838u : 0u;
+                    *reinterpret_cast<uint4 *>(ones + off) = make_uint4(v, v, v, v);
+                }
+            }
+            named_bar_sync(1, 256);
+            amax = fmaxf(xch[r], xch[128 + r]);
+            int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 0;
+            e = max(-120, min(127, e));
+            const float qs = amax > 0.f ? __uint_as_float((uint32_t)(127 + 7 - e) << 23) : 1.f;
+            c_row = __fdiv_rn(p.k_scale[h] * p.sm_scale * LOG2E, qs);
+            uint8_t *qh = smem + ATT_OFF_Q, *ql = qh + ATT_Q_BYTES;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {                   // 16-byte chunk c = dims 16c .. 16c+15
+                const uint32_t c = 4u * (uint32_t)g + (uint32_t)cc;
+                const uint32_t wv[8] = {qraw[2 * cc].x,     qraw[2 * cc].y,     qraw[2 * cc].z,     qraw[2 * cc].w,
+                                        qraw[2 * cc + 1].x, qraw[2 * cc + 1].y, qraw[2 * cc + 1].z, qraw[2 * cc + 1].w};
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t h01, l01, h23, l23;
+                    split2_f32(__uint_as_float(wv[2 * j] << 16) * qs, __uint_as_float(wv[2 * j] & 0xFFFF0000u) * qs,
+                               h01, l01);
+                    split2_f32(__uint_as_float(wv[2 * j + 1] << 16) * qs,
+                               __uint_as_float(wv[2 * j + 1] & 0xFFFF0000u) * qs, h23, l23);
+                    hw[j] = h01 | (h23 << 16);
+                    lw[j] = l01 | (l23 << 16);
+                }
+                const uint32_t off = (uint32_t)r * 128u + ((c ^ ((uint32_t)r & 7u)) << 4);
+                *reinterpret_cast<uint4 *>(qh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(ql + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            if (has_q) {
+                int a = node;
+                for (int it = 0; it < ATT_T && a >= 0; ++it) {
+                    if (a >= T) {                              // malformed tree: parent id out of range
+                        report_error(ERRBIT_RANGE, 305);
+                        break;
+                    }
+                    anc |= 1u << a;
+                    a = p.parent[a];
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
+
+        float m_ref = -INFINITY;
+        bool ok = true;
+        int32_t pid = g < n_pages ? p.page_table[pg0 + g] : -1;
+        for (int i = g; i < n_pages; i += 2) {
+            const bool vpage = pid >= 0 && pid < p.n_pool_pages;
+            if (i + 2 < n_pages) pid = p.page_table[pg0 + i + 2];
+            bool w_ok = true;
+            if (lane == 0) w_ok = mbar_wait(&s_full[g], (uint32_t)((i >> 1) & 1), 320, s_abort);
+            if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t s[64];
+            {
+                uint32_t (&s0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&s[0]);
+                uint32_t (&s1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&s[32]);
+                tmem_ld_x32(s_t, s0);
+                tmem_ld_x32(s_t + 32u, s1);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[g]);
+            if (!vpage) {                                      // no product for this page
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[g]);
+                continue;
+            }
+            const int64_t pos0 = (int64_t)(pg0 + i) * ATT_P;
+            if (pos0 + ATT_P > L) {
+                const int t0 = (int)(pos0 - L);                // tree slot of column 0 (> -64)
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const int tj = t0 + j;                     // negative: context position
+                    const bool vis = tj < 0 || (tj < T && ((anc >> (tj & 31)) & 1u));
+                    if (!vis) s[j] = 0xFF800000u;             // -inf
+                }
+            }
+            float mr = __uint_as_float(s[0]);
+#pragma unroll
+            for (int j = 1; j < 64; ++j) mr = fmaxf(mr, __uint_as_float(s[j]));
+            const float mx = mr * c_row;
+            const bool need = mx > m_ref + ATT_TAU;
+            const bool resc = need && m_ref > -INFINITY;
+            bool waited = false;
+            if (__any_sync(0xFFFFFFFFu, resc)) {
+                // every product of this group so far must be in O before it is rescaled
+                bool r_ok = true;
+                if (lane == 0) r_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 321, s_abort);
+                if (!__shfl_sync(0xFFFFFFFFu, r_ok ? 1 : 0, 0)) { ok = false; break; }
+                waited = true;
+                tc_fence_after();
+                const float alpha = resc ? fast_exp2(m_ref - mx) : 1.f;
+#pragma unroll 1
+                for (uint32_t col = 0; col < ATT_NO; col += 16) {
+                    uint32_t o[16];
+                    tmem_ld_32x32b_x16(o_t + col, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                    tmem_st_x16(o_t + col, o);
+                }
+                tmem_wait_st();
+            }
+            if (need) m_ref = mx;
+            const float nb = m_ref > -INFINITY ? ATT_PSHIFT - m_ref : 0.f;
+            uint32_t ph[16], pl[16];
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                split4_f16(fast_exp2(fmaf(__uint_as_float(s[j]), c_row, nb)),
+                           fast_exp2(fmaf(__uint_as_float(s[j + 1]), c_row, nb)),
+                           fast_exp2(fmaf(__uint_as_float(s[j + 2]), c_row, nb)),
+                           fast_exp2(fmaf(__uint_as_float(s[j + 3]), c_row, nb)), ph[j >> 2], pl[j >> 2]);
+            if (pos0 + ATT_P > L + T) {
+                // slots past the last written token may hold any byte (NaN codes
+                // included); zero their V so that 0 * V stays 0 in the product
+                const bool k_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
+                if (!__all_sync(0xFFFFFFFFu, k_ok)) { ok = false; break; }
+                uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
+                for (int t = (int)(L + T - pos0); t < ATT_P; ++t) vs[v_offset((uint32_t)r, (uint32_t)t)] = 0;
+            }
+            // the P buffer of this group's previous page must have been consumed
+            if (!waited && i >= 2) {
+                bool f_ok = true;
+                if (lane == 0) f_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 322, s_abort);
+                if (!__shfl_sync(0xFFFFFFFFu, f_ok ? 1 : 0, 0)) { ok = false; break; }
+            }
+            uint8_t *pb = smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {                      // tokens 16c .. 16c+15
+                const uint32_t off = (((uint32_t)r >> 3) * 4u + (uint32_t)c) * 128u + ((uint32_t)r & 7u) * 16u;
+                *reinterpret_cast<uint4 *>(pb + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+                *reinterpret_cast<uint4 *>(pb + ATT_PB_BYTES + off) =
+                    make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[g]);
+        }
+
+        // ---- merge the two groups' (m, O) and write the split result:
+        //      o = O / l (V code units), m, l; group g writes dims 64g .. 64g+63
+        bool d_ok = ok && n_pages > 0;
+        if (d_ok && lane == 0) d_ok = mbar_wait(o_done, 0, 323, s_abort);
+        d_ok = __shfl_sync(0xFFFFFFFFu, d_ok ? 1 : 0, 0) != 0;
+        xch[256 + g * 128 + r] = m_ref;
+        named_bar_sync(1, 256);
+        const float mA = xch[256 + r], mB = xch[384 + r];
+        const int64_t prow = (((int64_t)h * p.S + split) * group) * 16 + r;
+        if (d_ok) {
+            tc_fence_after();
+            const float M = fmaxf(mA, mB);
+            const float wA = mA > -INFINITY ? fast_exp2(mA - M) : 0.f;
+            const float wB = mB > -INFINITY ? fast_exp2(mB - M) : 0.f;
+            const float lA = __uint_as_float(tmem_ld_x1(row_t + ATT_TM_O0 + 128u));
+            const float lB = __uint_as_float(tmem_ld_x1(row_t + ATT_TM_O1 + 128u));
+            tmem_wait_ld();
+            const float l = (wA > 0.f ? wA * lA : 0.f) + (wB > 0.f ? wB * lB : 0.f);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float ca = wA > 0.f ? wA * inv : 0.f, cb = wB > 0.f ? wB * inv : 0.f;
+            float *dst = p.part_o + prow * ATT_D;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t col = 64u * (uint32_t)g + 32u * cc;
+                uint32_t oa[32], ob[32];
+                tmem_ld_x32(row_t + ATT_TM_O0 + col, oa);
+                tmem_ld_x32(row_t + ATT_TM_O1 + col, ob);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        float v[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float a = ca > 0.f ? ca * __uint_as_float(oa[j + k]) : 0.f;
+                            const float b = cb > 0.f ? cb * __uint_as_float(ob[j + k]) : 0.f;
+                            v[k] = a + b;
+                        }
+                        __stcg(reinterpret_cast<float4 *>(dst + col + j), make_float4(v[0], v[1], v[2], v[3]));
+                    }
+                }
+            }
+            if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M - ATT_PSHIFT, l));
+        } else if (n_pages == 0 && row_ok && g == 0) {
+            __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(0.f, 0.f));
+        }
     }
 
-    // partial result of this split: o = O / l (V code units), m, l
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        l_run[rr] += __shfl_xor_sync(0xFFFFFFFFu, l_run[rr], 1);
-        l_run[rr] += __shfl_xor_sync(0xFFFFFFFFu, l_run[rr], 2);
-    }
-    const int64_t rowbase = (((int64_t)h * p.S + split) * group + warp) * 16;
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const int node = g + 8 * rr;
-        const float inv = l_run[rr] > 0.f ? 1.f / l_run[rr] : 0.f;
-        float *dst = p.part_o + (rowbase + node) * ATT_D;
-#pragma unroll
-        for (int nd = 0; nd < 16; ++nd)
-            __stcg(reinterpret_cast<float2 *>(dst + 8 * nd + 2 * c),
-                   make_float2(O[nd][2 * rr] * inv, O[nd][2 * rr + 1] * inv));
-        if (c == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + (rowbase + node) * 2), make_float2(m_run[rr], l_run[rr]));
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, ATT_TMEM_COLS);
     }
 }
 
 // out[i][hq][:] = sum_s w_s o_s / sum_s w_s * v_scale[h],  w_s = l_s 2^(m_s - M)
 __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnParams p)
 {
+    __shared__ float w_s[ATT_MAX_SPLITS];
+    __shared__ float red[ATT_D / 32];
     pdl_wait();
     pdl_launch_dependents();
     const int i = blockIdx.x, hq = blockIdx.y, d = threadIdx.x;
     const int h = hq / p.group, w = hq % p.group;
-    float M = -INFINITY;
-    for (int s = 0; s < p.S; ++s) {
-        const int64_t r = (((int64_t)h * p.S + s) * p.group + w) * 16 + i;
-        M = fmaxf(M, __ldcg(p.part_ml + 2 * r));
+    const int S = p.S;
+    auto row = [&](int s) { return (((int64_t)h * S + s) * p.group + w) * 16 + i; };
+    float mloc = -INFINITY;
+    for (int s = d; s < S; s += ATT_D) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * row(s)));
+        w_s[s] = ml.y > 0.f ? ml.x : -INFINITY;
+        if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
     }
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < p.S; ++s) {
-        const int64_t r = (((int64_t)h * p.S + s) * p.group + w) * 16 + i;
-        const float m = __ldcg(p.part_ml + 2 * r), l = __ldcg(p.part_ml + 2 * r + 1);
-        if (l > 0.f) {
-            const float ws = l * fast_exp2(m - M);
-            num += ws * __ldcg(p.part_o + r * ATT_D + d);
-            den += ws;
-        }
+    mloc = warp_max(mloc);
+    if ((d & 31) == 0) red[d >> 5] = mloc;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float dloc = 0.f;
+    for (int s = d; s < S; s += ATT_D) {
+        const float m = w_s[s];
+        float ws = 0.f;
+        if (m > -INFINITY) ws = __ldcg(p.part_ml + 2 * row(s) + 1) * fast_exp2(m - M);
+        w_s[s] = ws;
+        dloc += ws;
+    }
+    dloc = warp_sum(dloc);
+    if ((d & 31) == 0) red[d >> 5] = dloc;
+    __syncthreads();
+    const float den = (red[0] + red[1]) + (red[2] + red[3]);
+    float num = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < S; ++s) {
+        const float ws = w_s[s];
+        if (ws > 0.f) num += ws * __ldcg(p.part_o + row(s) * ATT_D + d);
     }
     const float o = den > 0.f ? num / den * p.v_scale[h] : 0.f;
     p.out[((int64_t)i * p.Hq + hq) * ATT_D + d] = __float2bfloat16_rn(o);

@@ -7,8 +7,10 @@
 namespace nvfp4sk {
 
 // One CTA per (node i, KV head h); thread d writes K[d] and V[d] of that
-// token as E4M3(fp32(x / scale[h])) into the paged pools (K token-major, V
-// dimension-major pages).
+// token as E4M3(fp32(x / scale[h])) into the paged pools.  K pages are
+// token-major; a V (page, head) plane is cut into 8-dimension x 16-slot tiles
+// of 128 bytes, tile (d/8, slot/16) at index (d/8)*(P/16) + slot/16, rows d%8
+// of 16 slot bytes inside (the operand image the attention PV product reads).
 __global__ void __launch_bounds__(128) kv_append_kernel(const __nv_bfloat16 *__restrict__ k_new,
                                                         const __nv_bfloat16 *__restrict__ v_new, int64_t ld_new,
                                                         int Hkv, int D, uint8_t *__restrict__ k_pool,
@@ -32,8 +34,8 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __nv_bfloat16 *__r
         const float kx = __bfloat162float(k_new[(int64_t)i * ld_new + (int64_t)h * D + d]);
         const float vx = __bfloat162float(v_new[(int64_t)i * ld_new + (int64_t)h * D + d]);
         k_pool[(((int64_t)pg * Hkv + h) * P + slot) * D + d] = (uint8_t)(cvt_e4m3x2(__fdiv_rn(kx, ks), 0.f) & 0xFFu);
-        v_pool[((int64_t)pg * Hkv + h) * (int64_t)D * P + (int64_t)d * P + slot] =
-            (uint8_t)(cvt_e4m3x2(__fdiv_rn(vx, vs), 0.f) & 0xFFu);
+        const int64_t v_byte = ((int64_t)(d >> 3) * (P >> 4) + (slot >> 4)) * 128 + (d & 7) * 16 + (slot & 15);
+        v_pool[((int64_t)pg * Hkv + h) * (int64_t)D * P + v_byte] = (uint8_t)(cvt_e4m3x2(__fdiv_rn(vx, vs), 0.f) & 0xFFu);
     }
 }
 

@@ -192,7 +192,7 @@ size_t linear_ws(int64_t G, int64_t NT) { (void)NT; return LIN_COUNTER_BYTES + u
 int attn_splits(const DevInfo &d, int Hkv, int64_t n_log)
 {
     int64_t S = g_opt_attn_splits > 0 ? g_opt_attn_splits : std::max<int64_t>(1, d.sms / std::max(1, Hkv));
-    return (int)std::max<int64_t>(1, std::min<int64_t>(S, n_log));
+    return (int)std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(S, ATT_MAX_SPLITS), n_log));
 }
 size_t attn_ws(int Hkv, int S, int group)
 {
@@ -416,10 +416,10 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     if (int rc = device_info(&d)) return rc;
     if (!q || !k_pool || !v_pool || !page_table || !parent || !k_scale || !v_scale || !out)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 7 ||
+    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 8 ||
         ctx_len < 0 || n_pool_pages < 1 || ld_q < (int64_t)Hq * D || n_pool_pages * Hkv * ATT_P > INT32_MAX)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
-                    "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 7, ld_q >= Hq*D");
+                    "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 8, ld_q >= Hq*D");
     if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool))
         return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes) and the pools must be 16-byte aligned");
     const int64_t n_log = cdiv(ctx_len + T, ATT_P);
@@ -453,7 +453,7 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     p.S = S;
     p.n_log_pages = (int)n_log;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, Hkv), dim3((group + 1) * 32), ATT_SMEM_BYTES, st, 1, tk, p);
+    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, Hkv), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, 1, tk, p);
     if (e != cudaSuccess) return cuda_fail(e, "tree_attn_split_kernel");
     return launched(launch(tree_attn_combine_kernel, dim3(T, Hq), dim3(ATT_D), 0, st, 1, p),
                     "tree_attn_combine_kernel");
@@ -541,8 +541,9 @@ nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_ne
     if (int rc = device_info(&d)) return rc;
     if (!k_new || !v_new || !k_pool || !v_pool || !page_table || !k_scale || !v_scale)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (T < 1 || Hkv < 1 || D < 1 || page_size < 1 || ctx_len < 0 || ld_new < (int64_t)Hkv * D || n_pool_pages < 1)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "bad shape");
+    if (T < 1 || Hkv < 1 || D < 8 || D % 8 || page_size < 16 || page_size % 16 || ctx_len < 0 ||
+        ld_new < (int64_t)Hkv * D || n_pool_pages < 1)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need T, Hkv >= 1, D % 8 == 0, page_size % 16 == 0, ld_new >= Hkv*D");
     return launched(launch(kv_append_kernel, dim3(T, Hkv), dim3(128), 0, (cudaStream_t)stream, 1,
                            (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new, ld_new, Hkv, D, k_pool,
                            v_pool, n_pool_pages, page_size, page_table, ctx_len, k_scale, v_scale),
@@ -589,6 +590,14 @@ nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, ui
     const int grid = (int)std::min<int64_t>(cdiv(n, 256), 16 * d->sms);
     return launched(launch(debug_encode_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, x, n, e2m1, e4m3),
                     "debug_encode_kernel");
+}
+
+nvfp4sk_status nvfp4sk_debug_wait_timeout(nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    return launched(launch(debug_wait_timeout_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream, 1),
+                    "debug_wait_timeout_kernel");
 }
 
 }  // extern "C"

@@ -374,4 +374,21 @@ __global__ void debug_encode_kernel(const float *__restrict__ x, int64_t n, uint
     }
 }
 
+// ---- diagnostics: a bounded wait that runs out -----------------------------
+// Waits on an mbarrier that nothing arrives at.  The wait gives up after the
+// per-wait limit (NVFP4SK_OPT_TIMEOUT_NS), records a timeout at site 900 in the
+// device error word and the kernel returns normally: the host sees the failure
+// through nvfp4sk_get_device_status and the context stays usable.
+__global__ void debug_wait_timeout_kernel()
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, 900);
+    __syncthreads();
+}
+
 }  // namespace nvfp4sk

@@ -106,12 +106,24 @@ def fp8_codes(x: np.ndarray, scale: float) -> np.ndarray:
     return torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
+def v_plane_offsets(D: int = HEAD_DIM, P: int = PAGE) -> np.ndarray:
+    """[D, P] byte offsets of (dimension d, slot t) inside one (page, head)
+    plane of the V pool: the plane is cut into tiles of 8 dimensions x 16 slots
+    (128 bytes), tile (d // 8, t // 16) stored at tile index
+    (d // 8) * (P // 16) + t // 16, row d % 8 of 16 slot bytes inside."""
+    assert D % 8 == 0 and P % 16 == 0
+    d = np.arange(D)[:, None]
+    t = np.arange(P)[None, :]
+    return ((d // 8) * (P // 16) + t // 16) * 128 + (d % 8) * 16 + t % 16
+
+
 class KVCache:
     """A synthetic FP8 paged cache for one layer.
 
     k_pool u8 [n_pages, Hkv, P, D] (token-major pages), v_pool u8
-    [n_pages, Hkv, D, P] (dimension-major pages), page_table i32 over the
-    logical pages covering ctx_len + T positions, k_scale/v_scale f32 [Hkv].
+    [n_pages, Hkv, D * P] (tiled planes, see v_plane_offsets), page_table i32
+    over the logical pages covering ctx_len + T positions, k_scale/v_scale
+    f32 [Hkv].
     """
 
     def __init__(self, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, T):
@@ -121,11 +133,13 @@ class KVCache:
 
 def kv_cache(workload: int, ctx_len: int, T: int = TREE_NODES, Hkv: int = N_KV_HEADS,
              D: int = HEAD_DIM, P: int = PAGE, extra_pages: int = 0, fill_tree: bool = True,
-             sub: int = 0) -> KVCache:
+             sub: int = 0, unused_nan: bool = False) -> KVCache:
     """K/V ~ N(0,1) for positions 0..ctx_len+T-1, per-(head, K|V) scale =
     amax over the context / 448, stored as FP8 in a randomly permuted pool.
     If fill_tree, the tree slots ctx_len..ctx_len+T-1 are filled too (with the
-    same scales, saturating); otherwise they are left as zero bytes."""
+    same scales, saturating); otherwise they are left as zero bytes.  Pool
+    bytes that hold no position are random finite codes, or the E4M3 NaN code
+    0x7F if unused_nan (a pool that was never cleared)."""
     g = rng(workload, 800, sub)
     total = ctx_len + T
     n_log = (total + P - 1) // P
@@ -138,7 +152,11 @@ def kv_cache(workload: int, ctx_len: int, T: int = TREE_NODES, Hkv: int = N_KV_H
     page_table = g.permutation(n_pages)[:n_log].astype(np.int32)
     # unused pool bytes get random codes (never NaN) so that stray reads show
     k_pool = g.integers(0, 0x7E, (n_pages, Hkv, P, D), dtype=np.uint8)
-    v_pool = g.integers(0, 0x7E, (n_pages, Hkv, D, P), dtype=np.uint8)
+    v_pool = g.integers(0, 0x7E, (n_pages, Hkv, D * P), dtype=np.uint8)
+    if unused_nan:
+        k_pool[:] = 0x7F
+        v_pool[:] = 0x7F
+    off = v_plane_offsets(D, P)
     upto = total if fill_tree else ctx_len
     for h in range(Hkv):
         kc = fp8_codes(k[:upto, h], k_scale[h])          # [pos, D]
@@ -147,12 +165,12 @@ def kv_cache(workload: int, ctx_len: int, T: int = TREE_NODES, Hkv: int = N_KV_H
             n = min(P, upto - p)
             pg = page_table[p // P]
             k_pool[pg, h, :n, :] = kc[p:p + n]
-            v_pool[pg, h, :, :n] = vc[p:p + n].T
+            v_pool[pg, h, off[:, :n].ravel()] = vc[p:p + n].T.ravel()
     if not fill_tree:
         for i in range(T):
             p = ctx_len + i
             k_pool[page_table[p // P], :, p % P, :] = 0
-            v_pool[page_table[p // P], :, :, p % P] = 0
+            v_pool[page_table[p // P], :, off[:, p % P]] = 0
     return KVCache(k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, T)
 
 

@@ -59,6 +59,7 @@ _SIGS = {
     "nvfp4sk_set_option": (_int, [_int, _i64]),
     "nvfp4sk_get_option": (_i64, [_int]),
     "nvfp4sk_debug_encode": (_int, [_vp, _i64, _vp, _vp, _vp]),
+    "nvfp4sk_debug_wait_timeout": (_int, [_vp]),
 }
 
 
@@ -202,7 +203,7 @@ def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, str
 def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None, out=None,
               ld_q=None, T=None, Hq=None, ws=None, stream=None):
     """q bf16 [T, Hq, D] (or a strided [T, >= Hq*D] view with ld_q); pools u8
-    [pages, Hkv, P, D] / [pages, Hkv, D, P]; returns bf16 [T, Hq, D]."""
+    [pages, Hkv, P, D] / [pages, Hkv, D*P] (tiled V planes); returns bf16 [T, Hq, D]."""
     n_pages, Hkv, P, D = k_pool.shape
     if T is None:
         T, Hq = q.shape[0], q.shape[1]

@@ -147,7 +147,7 @@ class VerifyModel:
         return self.kv[l, 0].view(self.n_pool, I.N_KV_HEADS, I.PAGE, I.HEAD_DIM)
 
     def v_pool(self, l):
-        return self.kv[l, 1].view(self.n_pool, I.N_KV_HEADS, I.HEAD_DIM, I.PAGE)
+        return self.kv[l, 1].view(self.n_pool, I.N_KV_HEADS, I.HEAD_DIM * I.PAGE)
 
     # ------------------------------------------------------------------ ops
     def restore(self):

@@ -166,13 +166,15 @@ def linear_sampled(a_codes, a_scales, g_a, w_codes, w_scales, g_w, idx_m, idx_n)
 
 # ---------------------------------------------------------------- attention
 def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None):
-    """q [T, Hq, D]; k_pool u8 [pages, Hkv, P, D]; v_pool u8 [pages, Hkv, D, P]."""
+    """q [T, Hq, D]; k_pool u8 [pages, Hkv, P, D]; v_pool u8 [pages, Hkv, D*P]
+    (8-dimension x 16-slot tiles of 128 bytes, tile (d//8, slot//16) at index
+    (d//8)*(P//16) + slot//16)."""
     q = _f32(q)
     T, Hq, D = q.shape
     k_pool = np.ascontiguousarray(k_pool, np.uint8)
     v_pool = np.ascontiguousarray(v_pool, np.uint8)
     n_pages, Hkv, P, D2 = k_pool.shape
-    assert D2 == D and v_pool.shape == (n_pages, Hkv, D, P)
+    assert D2 == D and v_pool.shape == (n_pages, Hkv, D * P) and D % 8 == 0 and P % 16 == 0
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(D)
     out = np.zeros((T, Hq, D), np.float64)

@@ -234,7 +234,10 @@ EXPORT void oracle_nvfp4_linear_sampled(const uint8_t *a_codes, const uint8_t *a
 /* target forward; "NVFP4 and FP8": FP8 KV cache; "KV-cache reuse": pages).  */
 /*                                                                           */
 /* Cache layout (per layer): K pool uint8 [n_pages][Hkv][P][D] (token-major  */
-/* page), V pool uint8 [n_pages][Hkv][D][P] (dimension-major page).  Logical */
+/* page), V pool uint8 [n_pages][Hkv][D*P]: a (page, head) plane of V is cut */
+/* into 8-dimension x 16-slot tiles of 128 bytes, tile (d/8, slot/16) at     */
+/* tile index (d/8)*(P/16) + slot/16, rows d%8 of 16 slots inside (v_byte    */
+/* below; needs D % 8 == 0 and P % 16 == 0).  Logical                        */
 /* position p lives in physical page page_table[p / P], slot p % P.  The     */
 /* tree nodes' own K/V sit at positions L .. L+T-1 (node i at L+i).          */
 /* Node i sees every context position p < L and the tree positions of its    */
@@ -243,6 +246,13 @@ EXPORT void oracle_nvfp4_linear_sampled(const uint8_t *a_codes, const uint8_t *a
 /*   s_p = sm_scale * sum_d q[d] * k_scale[h] * value(K code)                */
 /*   o   = sum_p softmax(s)_p * v_scale[h] * value(V code)   (fp64)          */
 /* ------------------------------------------------------------------------ */
+
+/* byte offset of (dimension d, slot) inside one V plane */
+static int64_t v_byte(int d, int slot, int P)
+{
+    int64_t tile = (int64_t)(d / 8) * (P / 16) + slot / 16;
+    return tile * 128 + (d % 8) * 16 + slot % 16;
+}
 
 static int is_ancestor(const int32_t *parent, int j, int i)
 {
@@ -257,7 +267,7 @@ EXPORT int oracle_tree_attn(const float *q, int T, int Hq, int Hkv, int D,
                             const float *k_scale, const float *v_scale, double sm_scale,
                             double *out)
 {
-    if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+    if (Hkv <= 0 || Hq % Hkv != 0 || D % 8 != 0 || P % 16 != 0) return -1;
     int group = Hq / Hkv;
     int64_t total = L + T;
     int bad = 0;
@@ -291,7 +301,7 @@ EXPORT int oracle_tree_attn(const float *q, int T, int Hq, int Hkv, int D,
                 int64_t pg = page_table[p / P];
                 const uint8_t *vb = v_pool + (pg * Hkv + h) * (int64_t)D * P;
                 for (int d = 0; d < D; ++d)
-                    o[d] += w * ((double)v_scale[h] * oracle_e4m3_value(vb[(int64_t)d * P + p % P]));
+                    o[d] += w * ((double)v_scale[h] * oracle_e4m3_value(vb[v_byte(d, (int)(p % P), P)]));
             }
             for (int d = 0; d < D; ++d) o[d] /= den;
             free(s);
@@ -309,6 +319,7 @@ EXPORT int oracle_kv_append(const float *k_new, const float *v_new, int T, int H
                             const int32_t *page_table, int64_t L,
                             const float *k_scale, const float *v_scale)
 {
+    if (D % 8 != 0 || P % 16 != 0) return -1;
     for (int i = 0; i < T; ++i) {
         int64_t p = L + i, pg = page_table[p / P], slot = p % P;
         if (pg < 0 || pg >= n_pages) return -7;
@@ -317,7 +328,7 @@ EXPORT int oracle_kv_append(const float *k_new, const float *v_new, int T, int H
                 double kx = f32((double)k_new[((int64_t)i * Hkv + h) * D + d] / (double)k_scale[h]);
                 double vx = f32((double)v_new[((int64_t)i * Hkv + h) * D + d] / (double)v_scale[h]);
                 k_pool[((pg * Hkv + h) * P + slot) * D + d] = (uint8_t)oracle_e4m3_encode(kx);
-                v_pool[(pg * Hkv + h) * (int64_t)D * P + (int64_t)d * P + slot] = (uint8_t)oracle_e4m3_encode(vx);
+                v_pool[(pg * Hkv + h) * (int64_t)D * P + v_byte(d, (int)slot, P)] = (uint8_t)oracle_e4m3_encode(vx);
             }
     }
     return 0;

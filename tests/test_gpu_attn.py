@@ -42,6 +42,7 @@ def _tree(kind, T, seed):
 @pytest.mark.parametrize("T,Hq,Hkv,L,kind", [
     (16, 24, 4, 0, "tree"), (16, 24, 4, 37, "tree"), (16, 24, 4, 1000, "tree"), (1, 24, 4, 100, "chain"),
     (5, 8, 2, 200, "chain"), (16, 6, 1, 64, "star"), (16, 24, 4, 4096, "tree"), (9, 14, 2, 127, "tree"),
+    (16, 32, 4, 300, "tree"), (3, 8, 1, 63, "chain"), (16, 24, 4, 48, "tree"),
 ])
 def test_attention_small(oracle, T, Hq, Hkv, L, kind):
     cuda()
@@ -72,6 +73,22 @@ def test_attention_full_context(oracle):
     print(f"config3: max abs err {err.max():.3e}, rel-Frobenius {rel:.3e}, max |o| {np.abs(want).max():.3e}")
     assert err.max() <= ATTN_ABS_TOL
     assert rel <= 2e-2
+
+
+@pytest.mark.parametrize("L", [1000, 1008, 4080])
+def test_unused_pool_bytes_may_be_nan(oracle, L):
+    """A pool that was never cleared: every byte that holds no position is the
+    E4M3 NaN code, including the slots of the last page past the tree."""
+    cuda()
+    cache = inputs.kv_cache(74, L, extra_pages=4, unused_nan=True)
+    parent = inputs.tree_parent(74)
+    q = inputs.query_bf16(74)
+    got = _run_gpu(q, cache, parent)
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, L, parent,
+                            cache.k_scale, cache.v_scale)
+    assert np.isfinite(got).all()
+    err = np.abs(got - want)
+    assert np.all(err <= ATTN_ABS_TOL + 2.0 ** -8 * np.abs(want)), err.max()
 
 
 def test_page_permutation_bit_identical():

@@ -5,9 +5,10 @@
 (2) a tree equals running each root-to-node path as its own chain;
 (3) one node with no context returns its own V;
 (4) identical keys give the mean of the visible V;
-(5) pure-Python brute force at L=3, D=4, T=4;
+(5) pure-Python brute force at L=3, D=8, T=4;
 (6) a random permutation of the physical pool (with the page table) changes
-    nothing; bytes outside the visible positions change nothing.
+    nothing; bytes outside the visible positions change nothing;
+(7) the tiled V plane layout: hand-computed byte offsets, a bijection.
 """
 import math
 
@@ -22,12 +23,13 @@ def _dense(cache, Hkv, D, P):
     total = cache.ctx_len + cache.T
     kp = torch.from_numpy(cache.k_pool.copy()).view(torch.float8_e4m3fn).double().numpy()
     vp = torch.from_numpy(cache.v_pool.copy()).view(torch.float8_e4m3fn).double().numpy()
+    off = inputs.v_plane_offsets(D, P)
     K = np.zeros((total, Hkv, D))
     V = np.zeros((total, Hkv, D))
     for p in range(total):
         pg = cache.page_table[p // P]
         K[p] = kp[pg, :, p % P, :] * cache.k_scale[:, None]
-        V[p] = vp[pg, :, :, p % P] * cache.v_scale[:, None]
+        V[p] = vp[pg][:, off[:, p % P]] * cache.v_scale[:, None]
     return K, V
 
 
@@ -37,7 +39,7 @@ def _run(oracle, q, cache, parent):
 
 
 def test_chain_equals_causal_sdpa(oracle):
-    T, Hq, Hkv, D, P, L = 5, 6, 2, 16, 8, 21
+    T, Hq, Hkv, D, P, L = 5, 6, 2, 16, 16, 21
     cache = inputs.kv_cache(100, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=3)
     q = inputs.query_bf16(100, T, Hq, D).float().numpy()
     out = _run(oracle, q, cache, inputs.chain_parent(T))
@@ -64,12 +66,13 @@ def test_tree_equals_per_path_chains(oracle):
         # a fresh cache: same context pages, the path's tree slots in order
         n_log = (L + d + P - 1) // P
         kp = np.zeros((n_log, Hkv, P, D), np.uint8)
-        vp = np.zeros((n_log, Hkv, D, P), np.uint8)
+        vp = np.zeros((n_log, Hkv, D * P), np.uint8)
+        off = inputs.v_plane_offsets(D, P)
         for p in range(L + d):
             src = p if p < L else L + path[p - L]
             spg, sslot = cache.page_table[src // P], src % P
             kp[p // P, :, p % P, :] = cache.k_pool[spg, :, sslot, :]
-            vp[p // P, :, :, p % P] = cache.v_pool[spg, :, :, sslot]
+            vp[p // P][:, off[:, p % P]] = cache.v_pool[spg][:, off[:, sslot]]
         sub = oracle.tree_attn(q[path], kp, vp, np.arange(n_log, dtype=np.int32), L,
                                inputs.chain_parent(d), cache.k_scale, cache.v_scale)
         assert np.allclose(sub[-1], out[i], rtol=1e-12, atol=1e-14), i
@@ -77,7 +80,7 @@ def test_tree_equals_per_path_chains(oracle):
 
 
 def test_single_node_no_context_returns_v0(oracle):
-    Hq, Hkv, D, P = 2, 1, 8, 4
+    Hq, Hkv, D, P = 2, 1, 8, 16
     cache = inputs.kv_cache(102, 0, T=1, Hkv=Hkv, D=D, P=P)
     cache.k_scale[:] = 0.5
     cache.v_scale[:] = 0.25
@@ -89,7 +92,7 @@ def test_single_node_no_context_returns_v0(oracle):
 
 
 def test_identical_keys_give_mean_of_visible_v(oracle):
-    T, Hq, Hkv, D, P, L = 6, 2, 1, 8, 8, 13
+    T, Hq, Hkv, D, P, L = 6, 2, 1, 8, 16, 13
     cache = inputs.kv_cache(103, L, T=T, Hkv=Hkv, D=D, P=P)
     for p in range(L + T):
         cache.k_pool[cache.page_table[p // P], 0, p % P, :] = 0x30   # same key everywhere
@@ -105,7 +108,7 @@ def test_identical_keys_give_mean_of_visible_v(oracle):
 
 
 def test_bruteforce_tiny(oracle):
-    T, Hq, Hkv, D, P, L = 4, 2, 1, 4, 2, 3
+    T, Hq, Hkv, D, P, L = 4, 2, 1, 8, 16, 3
     cache = inputs.kv_cache(104, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=2)
     parent = np.array([-1, 0, 0, 2], np.int32)
     q = inputs.query_bf16(104, T, Hq, D).float().numpy()
@@ -123,7 +126,7 @@ def test_bruteforce_tiny(oracle):
 
 
 def test_page_permutation_and_unseen_bytes_do_not_matter(oracle):
-    T, Hq, Hkv, D, P, L = 16, 6, 2, 16, 8, 45
+    T, Hq, Hkv, D, P, L = 16, 6, 2, 16, 16, 45
     cache = inputs.kv_cache(105, L, T=T, Hkv=Hkv, D=D, P=P, extra_pages=5)
     parent = inputs.tree_parent(105, T)
     q = inputs.query_bf16(105, T, Hq, D).float().numpy()
@@ -138,10 +141,21 @@ def test_page_permutation_and_unseen_bytes_do_not_matter(oracle):
     # scribble over every byte that no node may see
     used = {(cache.page_table[p // P], p % P) for p in range(L + T)}
     kp3, vp3 = cache.k_pool.copy(), cache.v_pool.copy()
+    off = inputs.v_plane_offsets(D, P)
     for pg in range(kp3.shape[0]):
         for slot in range(P):
             if (pg, slot) not in used:
                 kp3[pg, :, slot, :] = 0x7E
-                vp3[pg, :, :, slot] = 0x7E
+                vp3[pg][:, off[:, slot]] = 0x7E
     out3 = oracle.tree_attn(q, kp3, vp3, cache.page_table, L, parent, cache.k_scale, cache.v_scale)
     assert np.array_equal(out, out3)
+
+
+def test_v_plane_layout():
+    off = inputs.v_plane_offsets(16, 32)
+    # tile (d//8, t//16) at index (d//8)*2 + t//16, 128 bytes; row d%8 of 16 bytes
+    assert off[0, 0] == 0 and off[0, 15] == 15 and off[1, 0] == 16 and off[7, 15] == 127
+    assert off[0, 16] == 128 and off[8, 0] == 256 and off[9, 17] == 401 and off[15, 31] == 511
+    for D, P in [(8, 16), (16, 32), (128, 64)]:
+        o = inputs.v_plane_offsets(D, P)
+        assert sorted(o.ravel().tolist()) == list(range(D * P))

@@ -46,7 +46,7 @@ def test_kv_append_matches_torch_cast(oracle):
             wk = torch.from_numpy(qk).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
             wv = torch.from_numpy(qv).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
             assert np.array_equal(kp[pg, h, slot], wk)
-            assert np.array_equal(vp[pg, h, :, slot], wv)
+            assert np.array_equal(vp[pg, h, inputs.v_plane_offsets(D, P)[:, slot]], wv)
     # context untouched
     for p in range(L):
         pg, slot = cache.page_table[p // P], p % P
