@@ -23,8 +23,10 @@
 // accumulators in tensor memory and its own running max, so that two pages
 // are in the exponent / packing stage at once; their results are merged in
 // the epilogue.
-// Warp roles: 0 producer (TMA K page + bulk V page into an 8-stage ring),
-// 1 TMEM allocation + single-thread MMA issue, 2-5 and 6-9 softmax.
+// Warp roles: 0 producer (lane s feeds stage s of an 8-stage ring: TMA K page
+// + bulk V page), 1 TMEM allocation + QK issue (one thread), 10 PV issue (one
+// thread), 2-5 and 6-9 softmax.  The two issuers run independently, so a
+// group's next scores never wait behind the other group's product.
 // The split results (O / l, m, l per row) are merged by the combine kernel.
 #pragma once
 #include "common.cuh"
@@ -36,7 +38,7 @@ constexpr int ATT_P = 64;
 constexpr int ATT_T = 16;
 constexpr int ATT_ROWS = 128;
 constexpr int ATT_STAGES = 8;
-constexpr int ATT_THREADS = 320;
+constexpr int ATT_THREADS = 352;
 constexpr int ATT_MAX_SPLITS = 1024;
 constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;                 // 8 KB token-major page
 constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB core-matrix page
@@ -214,8 +216,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     uint64_t *p_free = p_full + 2;              // [2]
     uint64_t *q_ready = p_free + 2;
     uint64_t *o_done = q_ready + 1;
-    uint64_t *drain = o_done + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *drain = o_done + 1;                // [2]: QK issuer, PV issuer
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 2);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     volatile uint8_t *s_page_ok = reinterpret_cast<volatile uint8_t *>(tmem_holder + 2);   // [ATT_STAGES]
     float *xch = reinterpret_cast<float *>(smem + ATT_OFF_X);                             // [2][2][128]
@@ -240,7 +242,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         mbar_init(q_ready, 8);
         mbar_init(o_done, 1);
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -257,10 +260,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < n_pages; ++i) {
-                const int st = i % ATT_STAGES;
+        // lane st feeds stage st (pages st, st + 8, ...): the copies of
+        // different stages are issued by different threads, which keeps
+        // several page loads in flight per SM.
+        if (lane < ATT_STAGES) {
+            const int st = (int)lane;
+            int last = -1;
+            for (int i = st; i < n_pages; i += ATT_STAGES) {
                 if (i >= ATT_STAGES &&
                     !mbar_wait(&kv_empty[st], (uint32_t)(((i / ATT_STAGES) - 1) & 1), 301, s_abort))
                     break;
@@ -277,25 +283,49 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     report_error(ERRBIT_RANGE, 302);
                     mbar_arrive(&kv_full[st]);        // page skipped: its scores are masked out
                 }
-                issued = i + 1;
+                last = i;
             }
-            if (*s_abort) {
-                for (int i = issued > ATT_STAGES ? issued - ATT_STAGES : 0; i < issued; ++i)
-                    mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 303);
-            }
+            // on abort, let this stage's last copy land before the CTA exits
+            if (*s_abort && last >= 0) mbar_wait(&kv_full[st], (uint32_t)((last / ATT_STAGES) & 1), 303);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ QK issuer
+        // S = Q K^T of page i into the S buffer of group i & 1, as soon as the
+        // page has landed and the group has read that buffer's previous page
         if (lane == 0) {
             constexpr uint32_t idesc_s = att_idesc(128, ATT_P);
-            constexpr uint32_t idesc_o = att_idesc(128, ATT_NO);
             const uint32_t q_hi = smem_u32(smem + ATT_OFF_Q), q_lo = q_hi + ATT_Q_BYTES;
-            bool o_init[2] = {false, false};
             bool ok = mbar_wait(q_ready, 0, 310, s_abort);
-            tc_fence_after();
-            auto issue_pv = [&](int j) -> bool {
+            for (int i = 0; i < n_pages && ok; ++i) {
+                const int st = i % ATT_STAGES, g = i & 1;
+                if (!mbar_wait(&kv_full[st], (uint32_t)((i / ATT_STAGES) & 1), 312, s_abort)) { ok = false; break; }
+                if (i >= 2 && !mbar_wait(&s_free[g], (uint32_t)(((i - 2) >> 1) & 1), 313, s_abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t k_s = smem_u32(smem + st * ATT_STAGE_BYTES);
+                const uint32_t s_t = tmem_base + (g ? ATT_TM_S1 : ATT_TM_S0);
+#pragma unroll
+                for (int t = 0; t < ATT_D / 32; ++t) {
+                    const uint64_t kd = smem_desc(k_s + 32 * t, 16, 1024, SWZ_128B);
+                    mma_f8f6f4(s_t, smem_desc(q_hi + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, t > 0 ? 1u : 0u);
+                    mma_f8f6f4(s_t, smem_desc(q_lo + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, 1u);
+                }
+                tc_commit(&s_full[g]);
+            }
+            // every QK product is complete before tensor memory is released
+            tc_commit(&drain[0]);
+            mbar_wait(&drain[0], 0, 314);
+        }
+        __syncwarp();
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ PV issuer
+        // O_g += P V of page j once group g has written P (hi, lo) for it
+        if (lane == 0) {
+            constexpr uint32_t idesc_o = att_idesc(128, ATT_NO);
+            bool o_init[2] = {false, false};
+            bool ok = true;
+            for (int j = 0; j < n_pages && ok; ++j) {
                 const int g = j & 1;
-                if (!mbar_wait(&p_full[g], (uint32_t)((j >> 1) & 1), 311, s_abort)) return false;
+                if (!mbar_wait(&p_full[g], (uint32_t)((j >> 1) & 1), 311, s_abort)) { ok = false; break; }
                 tc_fence_after();
                 if (s_page_ok[j % ATT_STAGES]) {
                     const uint32_t v_s = smem_u32(smem + (j % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES);
@@ -312,30 +342,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 }
                 tc_commit(&p_free[g]);
                 tc_commit(&kv_empty[j % ATT_STAGES]);
-                return true;
-            };
-            for (int i = 0; i < n_pages && ok; ++i) {
-                const int st = i % ATT_STAGES, g = i & 1;
-                if (!mbar_wait(&kv_full[st], (uint32_t)((i / ATT_STAGES) & 1), 312, s_abort)) { ok = false; break; }
-                if (i >= 2 && !mbar_wait(&s_free[g], (uint32_t)(((i - 2) >> 1) & 1), 313, s_abort)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t k_s = smem_u32(smem + st * ATT_STAGE_BYTES);
-                const uint32_t s_t = tmem_base + (g ? ATT_TM_S1 : ATT_TM_S0);
-#pragma unroll
-                for (int t = 0; t < ATT_D / 32; ++t) {
-                    const uint64_t kd = smem_desc(k_s + 32 * t, 16, 1024, SWZ_128B);
-                    mma_f8f6f4(s_t, smem_desc(q_hi + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, t > 0 ? 1u : 0u);
-                    mma_f8f6f4(s_t, smem_desc(q_lo + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, 1u);
-                }
-                tc_commit(&s_full[g]);
-                if (i >= 1 && !issue_pv(i - 1)) { ok = false; break; }
             }
-            if (ok && n_pages > 0) ok = issue_pv(n_pages - 1);
             if (ok) {
                 tc_commit(o_done);
             } else {
-                tc_commit(drain);
-                mbar_wait(drain, 0, 314);
+                tc_commit(&drain[1]);
+                mbar_wait(&drain[1], 0, 315);
             }
         }
         __syncwarp();
@@ -583,48 +595,77 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
 }
 
-// out[i][hq][:] = sum_s w_s o_s / sum_s w_s * v_scale[h],  w_s = l_s 2^(m_s - M)
+// out[i][hq][:] = sum_s w_s o_s / sum_s w_s * v_scale[h],  w_s = l_s 2^(m_s - M).
+// One CTA per (node, query head), 4 warps: warp j sums splits j, j+4, ... for
+// all 128 dims (4 per lane); the partial rows of its first 16 splits are
+// requested before the weights are known, so the kernel waits on about one
+// round of L2 loads.  Warp sums are added in warp order (deterministic).
+constexpr int CMB_PF = 16;
 __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnParams p)
 {
     __shared__ float w_s[ATT_MAX_SPLITS];
+    __shared__ float l_s[ATT_MAX_SPLITS];
     __shared__ float red[ATT_D / 32];
+    __shared__ float4 xs[4][ATT_D / 4];
     pdl_wait();
     pdl_launch_dependents();
-    const int i = blockIdx.x, hq = blockIdx.y, d = threadIdx.x;
+    const int i = blockIdx.x, hq = blockIdx.y, tid = threadIdx.x;
+    const int wp = tid >> 5, lane = tid & 31;
     const int h = hq / p.group, w = hq % p.group;
     const int S = p.S;
     auto row = [&](int s) { return (((int64_t)h * S + s) * p.group + w) * 16 + i; };
+    float4 pv[CMB_PF];
+#pragma unroll
+    for (int k = 0; k < CMB_PF; ++k) {
+        const int s = wp + 4 * k;
+        pv[k] = s < S ? __ldcg(reinterpret_cast<const float4 *>(p.part_o + row(s) * ATT_D) + lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float mloc = -INFINITY;
-    for (int s = d; s < S; s += ATT_D) {
+    for (int s = tid; s < S; s += ATT_D) {
         const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * row(s)));
         w_s[s] = ml.y > 0.f ? ml.x : -INFINITY;
+        l_s[s] = ml.y;
         if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
     }
     mloc = warp_max(mloc);
-    if ((d & 31) == 0) red[d >> 5] = mloc;
+    if (lane == 0) red[wp] = mloc;
     __syncthreads();
     const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     __syncthreads();
     float dloc = 0.f;
-    for (int s = d; s < S; s += ATT_D) {
+    for (int s = tid; s < S; s += ATT_D) {
         const float m = w_s[s];
-        float ws = 0.f;
-        if (m > -INFINITY) ws = __ldcg(p.part_ml + 2 * row(s) + 1) * fast_exp2(m - M);
+        const float ws = m > -INFINITY ? l_s[s] * fast_exp2(m - M) : 0.f;
         w_s[s] = ws;
         dloc += ws;
     }
     dloc = warp_sum(dloc);
-    if ((d & 31) == 0) red[d >> 5] = dloc;
+    if (lane == 0) red[wp] = dloc;
     __syncthreads();
     const float den = (red[0] + red[1]) + (red[2] + red[3]);
-    float num = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < S; ++s) {
-        const float ws = w_s[s];
-        if (ws > 0.f) num += ws * __ldcg(p.part_o + row(s) * ATT_D + d);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < CMB_PF; ++k) {
+        const int s = wp + 4 * k;
+        const float ws = s < S ? w_s[s] : 0.f;
+        if (ws > 0.f) {
+            acc.x += ws * pv[k].x; acc.y += ws * pv[k].y; acc.z += ws * pv[k].z; acc.w += ws * pv[k].w;
+        }
     }
+    for (int s = wp + 4 * CMB_PF; s < S; s += 4) {
+        const float ws = w_s[s];
+        if (ws > 0.f) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.part_o + row(s) * ATT_D) + lane);
+            acc.x += ws * v.x; acc.y += ws * v.y; acc.z += ws * v.z; acc.w += ws * v.w;
+        }
+    }
+    xs[wp][lane] = acc;
+    __syncthreads();
+    const float *xf = reinterpret_cast<const float *>(xs);
+    const float num = (xf[tid] + xf[ATT_D + tid]) + (xf[2 * ATT_D + tid] + xf[3 * ATT_D + tid]);
     const float o = den > 0.f ? num / den * p.v_scale[h] : 0.f;
-    p.out[((int64_t)i * p.Hq + hq) * ATT_D + d] = __float2bfloat16_rn(o);
+    p.out[((int64_t)i * p.Hq + hq) * ATT_D + tid] = __float2bfloat16_rn(o);
 }
 
 }  // namespace nvfp4sk

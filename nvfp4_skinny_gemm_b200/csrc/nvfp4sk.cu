@@ -543,7 +543,7 @@ nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_ne
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (T < 1 || Hkv < 1 || D < 8 || D % 8 || page_size < 16 || page_size % 16 || ctx_len < 0 ||
         ld_new < (int64_t)Hkv * D || n_pool_pages < 1)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need T, Hkv >= 1, D % 8 == 0, page_size % 16 == 0, ld_new >= Hkv*D");
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need T, Hkv >= 1, D %% 8 == 0, page_size %% 16 == 0, ld_new >= Hkv*D");
     return launched(launch(kv_append_kernel, dim3(T, Hkv), dim3(128), 0, (cudaStream_t)stream, 1,
                            (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new, ld_new, Hkv, D, k_pool,
                            v_pool, n_pool_pages, page_size, page_table, ctx_len, k_scale, v_scale),
