@@ -37,29 +37,29 @@ constexpr int ATT_D = 128;
 constexpr int ATT_P = 64;
 constexpr int ATT_T = 16;
 constexpr int ATT_ROWS = 128;
-constexpr int ATT_STAGES = 8;
+constexpr int ATT_STAGES = 10;
 constexpr int ATT_THREADS = 352;
 constexpr int ATT_MAX_SPLITS = 1024;
 constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;                 // 8 KB token-major page
 constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB core-matrix page
 constexpr uint32_t ATT_ONES_BYTES = 16 * ATT_P;                 // 16 operand rows: ones, then zeros
 constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES + ATT_ONES_BYTES;   // 17 KB
-constexpr uint32_t ATT_Q_BYTES = ATT_ROWS * ATT_D;              // one E4M3 term of Q
 constexpr uint32_t ATT_PB_BYTES = ATT_ROWS * ATT_P;             // one E4M3 term of P
-constexpr uint32_t ATT_OFF_Q = ATT_STAGES * ATT_STAGE_BYTES;    // Q hi | Q lo
-constexpr uint32_t ATT_OFF_P = ATT_OFF_Q + 2 * ATT_Q_BYTES;     // P[2 groups] x (hi | lo)
+constexpr uint32_t ATT_OFF_P = ATT_STAGES * ATT_STAGE_BYTES;    // P[2 groups] x (hi | lo)
 constexpr uint32_t ATT_OFF_X = ATT_OFF_P + 4 * ATT_PB_BYTES;    // float exchange [2][2][128]
 constexpr uint32_t ATT_OFF_BAR = ATT_OFF_X + 2048;
-constexpr uint32_t ATT_SMEM_BYTES = ATT_OFF_BAR + 256 + 1024;
+constexpr uint32_t ATT_SMEM_BYTES = ATT_OFF_BAR + 512 + 1024;
 constexpr uint32_t ATT_TMEM_COLS = 512;
 constexpr uint32_t ATT_NO = ATT_D + 16;                         // O columns: 128 dims + row sum block
 constexpr uint32_t ATT_TM_S0 = 0, ATT_TM_S1 = 64;
 constexpr uint32_t ATT_TM_O0 = 128, ATT_TM_O1 = 288;
+constexpr uint32_t ATT_TM_Q = 448;                              // Q hi 448..479, Q lo 480..511 (A operand)
 constexpr float ATT_TAU = 2.0f;       // log2 growth of a row max that triggers an O rescale
 constexpr float ATT_PSHIFT = 6.0f;    // P' = 2^(s - m + 6) <= 2^(6 + TAU) = 256 < 448
 constexpr float LOG2E = 1.4426950408889634f;
 static_assert(ATT_STAGE_BYTES % 1024 == 0, "K tiles need 1024-byte alignment (128-byte swizzle atoms)");
-static_assert(ATT_TM_O1 + ATT_NO <= ATT_TMEM_COLS && ATT_TM_O0 + ATT_NO <= ATT_TM_O1, "tensor memory budget");
+static_assert(ATT_TM_O1 + ATT_NO <= ATT_TM_Q && ATT_TM_O0 + ATT_NO <= ATT_TM_O1 && ATT_TM_Q + 64 <= ATT_TMEM_COLS,
+              "tensor memory budget");
 
 // Byte of (dim d, slot t) inside a V page plane: 8-dim x 16-slot core matrices
 // of 128 bytes, ordered [d/8][t/16][d%8][t%16].
@@ -80,6 +80,18 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// same, with the A operand read from tensor memory (lane = row, 4 E4M3 per column)
+__device__ __forceinline__ void mma_f8f6f4_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -251,6 +263,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         tmem_alloc(tmem_holder, ATT_TMEM_COLS);
         tmem_relinquish();
     }
+    if (threadIdx.x == 32) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_k) : "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -294,7 +307,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // page has landed and the group has read that buffer's previous page
         if (lane == 0) {
             constexpr uint32_t idesc_s = att_idesc(128, ATT_P);
-            const uint32_t q_hi = smem_u32(smem + ATT_OFF_Q), q_lo = q_hi + ATT_Q_BYTES;
+            const uint32_t q_hi = tmem_base + ATT_TM_Q, q_lo = q_hi + 32u;
             bool ok = mbar_wait(q_ready, 0, 310, s_abort);
             for (int i = 0; i < n_pages && ok; ++i) {
                 const int st = i % ATT_STAGES, g = i & 1;
@@ -306,8 +319,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
                 for (int t = 0; t < ATT_D / 32; ++t) {
                     const uint64_t kd = smem_desc(k_s + 32 * t, 16, 1024, SWZ_128B);
-                    mma_f8f6f4(s_t, smem_desc(q_hi + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, t > 0 ? 1u : 0u);
-                    mma_f8f6f4(s_t, smem_desc(q_lo + 32 * t, 16, 1024, SWZ_128B), kd, idesc_s, 1u);
+                    mma_f8f6f4_ta(s_t, q_hi + 8u * t, kd, idesc_s, t > 0 ? 1u : 0u);
+                    mma_f8f6f4_ta(s_t, q_lo + 8u * t, kd, idesc_s, 1u);
                 }
                 tc_commit(&s_full[g]);
             }
@@ -371,6 +384,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         uint32_t anc = 0;
         {
             const bool has_q = row_ok && node < T;
+            const int par_l = (int)lane < T ? p.parent[lane] : -1;
             uint4 qraw[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -387,15 +401,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             xch[g * 128 + r] = amax;
             // the ones block of every stage: operand row 128 (16 bytes per 16-token chunk) = 1.0, rest 0
-            {
-                const int st_i = (int)(threadIdx.x - 64);     // 0..255
-                uint8_t *ones = smem + (st_i >> 5) * ATT_STAGE_BYTES + ATT_K_BYTES + ATT_V_BYTES;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t off = (uint32_t)(st_i & 31) * 32u + 16u * j;
-                    const uint32_t v = (off < 512u && (off & 127u) == 0u) ? 0x38383838u : 0u;
-                    *reinterpret_cast<uint4 *>(ones + off) = make_uint4(v, v, v, v);
-                }
+            for (int idx = (int)threadIdx.x - 64; idx < ATT_STAGES * (int)(ATT_ONES_BYTES / 16); idx += 256) {
+                const uint32_t off = (uint32_t)(idx % (ATT_ONES_BYTES / 16)) * 16u;
+                const uint32_t v = (off < 512u && (off & 127u) == 0u) ? 0x38383838u : 0u;
+                *reinterpret_cast<uint4 *>(smem + (idx / (ATT_ONES_BYTES / 16)) * ATT_STAGE_BYTES + ATT_K_BYTES +
+                                           ATT_V_BYTES + off) = make_uint4(v, v, v, v);
             }
             named_bar_sync(1, 256);
             amax = fmaxf(xch[r], xch[128 + r]);
@@ -403,39 +413,43 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             e = max(-120, min(127, e));
             const float qs = amax > 0.f ? __uint_as_float((uint32_t)(127 + 7 - e) << 23) : 1.f;
             c_row = __fdiv_rn(p.k_scale[h] * p.sm_scale * LOG2E, qs);
-            uint8_t *qh = smem + ATT_OFF_Q, *ql = qh + ATT_Q_BYTES;
+            // A operand of S = Q K^T in tensor memory: row r in lane r, dims 4c .. 4c+3
+            // in column c; this group writes columns 16g .. 16g+15 of each term
+            uint32_t hw[16], lw[16];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {                   // 16-byte chunk c = dims 16c .. 16c+15
-                const uint32_t c = 4u * (uint32_t)g + (uint32_t)cc;
-                const uint32_t wv[8] = {qraw[2 * cc].x,     qraw[2 * cc].y,     qraw[2 * cc].z,     qraw[2 * cc].w,
-                                        qraw[2 * cc + 1].x, qraw[2 * cc + 1].y, qraw[2 * cc + 1].z, qraw[2 * cc + 1].w};
-                uint32_t hw[4], lw[4];
+            for (int k = 0; k < 8; ++k) {                      // dims 64g + 8k .. 64g + 8k + 7
+                const uint32_t wv[4] = {qraw[k].x, qraw[k].y, qraw[k].z, qraw[k].w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 2; ++j) {
                     uint32_t h01, l01, h23, l23;
                     split2_f32(__uint_as_float(wv[2 * j] << 16) * qs, __uint_as_float(wv[2 * j] & 0xFFFF0000u) * qs,
                                h01, l01);
                     split2_f32(__uint_as_float(wv[2 * j + 1] << 16) * qs,
                                __uint_as_float(wv[2 * j + 1] & 0xFFFF0000u) * qs, h23, l23);
-                    hw[j] = h01 | (h23 << 16);
-                    lw[j] = l01 | (l23 << 16);
+                    hw[2 * k + j] = h01 | (h23 << 16);
+                    lw[2 * k + j] = l01 | (l23 << 16);
                 }
-                const uint32_t off = (uint32_t)r * 128u + ((c ^ ((uint32_t)r & 7u)) << 4);
-                *reinterpret_cast<uint4 *>(qh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(ql + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
-            if (has_q) {
-                int a = node;
-                for (int it = 0; it < ATT_T && a >= 0; ++it) {
-                    if (a >= T) {                              // malformed tree: parent id out of range
-                        report_error(ERRBIT_RANGE, 305);
-                        break;
-                    }
-                    anc |= 1u << a;
-                    a = p.parent[a];
+            tmem_st_x16(row_t + ATT_TM_Q + 16u * (uint32_t)g, hw);
+            tmem_st_x16(row_t + ATT_TM_Q + 32u + 16u * (uint32_t)g, lw);
+            tmem_wait_st();
+            // ancestors of this node: walk the parent array held one entry per lane
+            {
+                int a = has_q ? node : -1;
+                bool bad = false;
+#pragma unroll 1
+                for (int it = 0; it < ATT_T; ++it) {
+                    const bool act = a >= 0 && !bad;
+                    if (act && a >= T) bad = true;             // malformed tree: parent id out of range
+                    const bool take = act && !bad;
+                    if (take) anc |= 1u << a;
+                    const int nxt = __shfl_sync(0xFFFFFFFFu, par_l, take ? a : 0);
+                    a = take ? nxt : -1;
                 }
+                if (bad) report_error(ERRBIT_RANGE, 305);
             }
             fence_proxy_async_smem();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(q_ready);
         }
