@@ -192,6 +192,10 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const
  *   flagged NVFP4SK_ERR_OUT_OF_RANGE in the device status, as is a parent id
  *   outside [-1, T).
  * Supported: D == 128, page_size == 64, 1 <= T <= 16, Hq/Hkv <= 8.
+ * act_prepared (nullable): the bf16 output rows are also NVFP4-quantised with
+ *   the static tensor scale *g_act into the prepared activation image that
+ *   nvfp4_linear reads (K = Hq*D, row i = node i), exactly as
+ *   nvfp4_quantize_act(out, g_in = g_act) would; g_act must then be non-NULL.
  * ws: tree_attn_workspace_bytes(...) bytes.
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
@@ -199,8 +203,8 @@ NVFP4SK_API nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, i
                                const uint8_t *k_pool, const uint8_t *v_pool, int64_t n_pool_pages,
                                int page_size, const int32_t *page_table, int64_t ctx_len,
                                const int32_t *parent, const float *k_scale, const float *v_scale,
-                               float sm_scale, void *out, void *ws, size_t ws_bytes,
-                               nvfp4sk_stream_t stream);
+                               float sm_scale, void *out, const float *g_act, uint8_t *act_prepared,
+                               void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * kv_page_restore -- restore cached KV pages of a reused prompt prefix into
@@ -223,18 +227,20 @@ NVFP4SK_API nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_
  * kernel that produces them).
  * ---------------------------------------------------------------------- */
 /* y = x / sqrt(mean(x^2) + eps) * w rounded to bf16, then NVFP4-quantised
- * exactly as nvfp4_quantize_act (dynamic g), with the same outputs.  x bf16
+ * exactly as nvfp4_quantize_act, with the same outputs: g_in NULL = dynamic
+ * tensor scale (amax over the whole y), else the static scale *g_in (a
+ * calibrated checkpoint's; one launch with no grid-wide reduction).  x bf16
  * [rows][n] (row stride n), w bf16 [n].  rows <= 16, n % 64 == 0, n <= 8192. */
 NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows,
-                                                  int64_t n, uint8_t *codes, uint8_t *scales, float *g_out,
-                                                  uint8_t *act_prepared, void *ws, size_t ws_bytes,
+                                                  int64_t n, const float *g_in, uint8_t *codes, uint8_t *scales,
+                                                  float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
                                                   nvfp4sk_stream_t stream);
 /* h = silu(gu[:, :F]) * gu[:, F:] rounded to bf16, then NVFP4-quantised
- * (dynamic g), same outputs.  gu bf16 [rows][2F].  rows <= 16, F % 64 == 0,
- * rows * F <= 524288. */
-NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes,
-                                                 uint8_t *scales, float *g_out, uint8_t *act_prepared, void *ws,
-                                                 size_t ws_bytes, nvfp4sk_stream_t stream);
+ * (g_in NULL = dynamic g, else static *g_in), same outputs.  gu bf16
+ * [rows][2F].  rows <= 16, F % 64 == 0, rows * F <= 524288. */
+NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, const float *g_in,
+                                                 uint8_t *codes, uint8_t *scales, float *g_out, uint8_t *act_prepared,
+                                                 void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
 /* Append T new tokens' K and V (bf16, token i head h at k_new[i*ld_new +
  * h*D + d]) to the cache at positions ctx_len .. ctx_len+T-1 as
  * E4M3(fp32(x / scale[h])) (round-to-nearest-even, saturating); the FP8 KV

@@ -30,6 +30,7 @@
 // The split results (O / l, m, l per row) are merged by the combine kernel.
 #pragma once
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace nvfp4sk {
 
@@ -209,6 +210,8 @@ struct AttnParams {
     float *part_o;        // [Hkv][S][group*16][128]
     float *part_ml;       // [Hkv][S][group*16][2]
     __nv_bfloat16 *out;   // [T][Hq][D]
+    const float *g_act;   // static tensor scale of the fused NVFP4 output (with act)
+    uint8_t *act;         // nullable: prepared NVFP4 activation of out, K = Hq*D
     int64_t ctx_len;
     int64_t n_pool_pages;
     float sm_scale;
@@ -679,7 +682,23 @@ __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnPara
     const float *xf = reinterpret_cast<const float *>(xs);
     const float num = (xf[tid] + xf[ATT_D + tid]) + (xf[2 * ATT_D + tid] + xf[3 * ATT_D + tid]);
     const float o = den > 0.f ? num / den * p.v_scale[h] : 0.f;
-    p.out[((int64_t)i * p.Hq + hq) * ATT_D + tid] = __float2bfloat16_rn(o);
+    const __nv_bfloat16 ob = __float2bfloat16_rn(o);
+    p.out[((int64_t)i * p.Hq + hq) * ATT_D + tid] = ob;
+    if (p.act) {
+        // NVFP4 of the bf16 output row with the static tensor scale: the 8 blocks of
+        // 16 dims of this head are blocks hq*8 .. hq*8+7 of row i (K = Hq*D)
+        __shared__ float orow[ATT_D];
+        orow[tid] = __bfloat162float(ob);
+        __syncthreads();
+        if (tid < ATT_D / 16) {
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = orow[16 * tid + k];
+            uint2 pk;
+            const uint32_t sc = quant_block16(v, *p.g_act, pk);
+            store_prepared(p.act, i, (int64_t)hq * (ATT_D / 16) + tid, pk, sc);
+        }
+    }
 }
 
 }  // namespace nvfp4sk

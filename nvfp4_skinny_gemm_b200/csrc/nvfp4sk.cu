@@ -282,7 +282,7 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
                     "x, its row stride and act_prepared must be 16-byte aligned, codes 8-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t nblk = rows * (K / 16);
-    if (nblk <= QSMALL_MAX_BLOCKS) {
+    if (nblk <= QSMALL_MAX_BLOCKS && !g_in) {
         const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
         cudaError_t e = x_dtype == NVFP4SK_BF16
                             ? launch(quant_fused_kernel<__nv_bfloat16, 0>, dim3(cs), dim3(QTHREADS), 0, st, cs,
@@ -409,8 +409,9 @@ size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, i
 nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D, const uint8_t *k_pool,
                                const uint8_t *v_pool, int64_t n_pool_pages, int page_size,
                                const int32_t *page_table, int64_t ctx_len, const int32_t *parent,
-                               const float *k_scale, const float *v_scale, float sm_scale, void *out, void *ws,
-                               size_t ws_bytes, nvfp4sk_stream_t stream)
+                               const float *k_scale, const float *v_scale, float sm_scale, void *out,
+                               const float *g_act, uint8_t *act_prepared, void *ws, size_t ws_bytes,
+                               nvfp4sk_stream_t stream)
 {
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
@@ -420,8 +421,9 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
         ctx_len < 0 || n_pool_pages < 1 || ld_q < (int64_t)Hq * D || n_pool_pages * Hkv * ATT_P > INT32_MAX)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
                     "need D == 128, page_size == 64, 1 <= T <= 16, Hq %% Hkv == 0, Hq/Hkv <= 8, ld_q >= Hq*D");
-    if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool))
-        return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes) and the pools must be 16-byte aligned");
+    if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool) || !al16(act_prepared))
+        return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes), the pools and act_prepared must be 16-byte aligned");
+    if (act_prepared && !g_act) return fail(NVFP4SK_ERR_INVALID_ARG, "act_prepared needs the static scale g_act");
     const int64_t n_log = cdiv(ctx_len + T, ATT_P);
     const int group = Hq / Hkv;
     const int S = attn_splits(*d, Hkv, n_log);
@@ -443,6 +445,8 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     p.part_o = (float *)ws;
     p.part_ml = (float *)((uint8_t *)ws + up256((size_t)Hkv * S * group * 16 * ATT_D * 4));
     p.out = (__nv_bfloat16 *)out;
+    p.g_act = g_act;
+    p.act = act_prepared;
     p.ctx_len = ctx_len;
     p.n_pool_pages = n_pool_pages;
     p.sm_scale = sm_scale;
@@ -491,8 +495,8 @@ nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_t *src_ids, 
 
 // ---------------------------------------------------------------- glue
 nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows, int64_t n,
-                                      uint8_t *codes, uint8_t *scales, float *g_out, uint8_t *act_prepared, void *ws,
-                                      size_t ws_bytes, nvfp4sk_stream_t stream)
+                                      const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
+                                      uint8_t *act_prepared, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
     DevInfo *d;
@@ -504,6 +508,11 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
     if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
         (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "x, w, act_prepared must be 16-byte aligned, codes 8-byte aligned");
+    if (g_in)
+        return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows), dim3(RTHREADS), 0,
+                               (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, n,
+                               g_in, codes, scales, g_out, act_prepared),
+                        "rmsnorm_quant_static_kernel");
     const int cs = rows <= 8 ? 8 : 16;
     return launched(launch(rmsnorm_quant_kernel, dim3(cs), dim3(RTHREADS), 0, (cudaStream_t)stream, cs,
                            (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, rows, n, codes, scales, g_out,
@@ -511,8 +520,8 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
                     "rmsnorm_quant_kernel");
 }
 
-nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, uint8_t *codes, uint8_t *scales,
-                                     float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
+nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, const float *g_in, uint8_t *codes,
+                                     uint8_t *scales, float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
                                      nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
@@ -525,6 +534,12 @@ nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, ui
     if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "gu, act_prepared must be 16-byte aligned, codes 8-byte aligned");
     const int64_t nblk = rows * (F / 16);
+    if (g_in)
+        return launched(launch(swiglu_quant_static_kernel,
+                               dim3((unsigned)std::min<int64_t>(4 * d->sms, cdiv(nblk, QBIG_THREADS_STATIC))),
+                               dim3(QBIG_THREADS_STATIC), 0, (cudaStream_t)stream, 1, (const __nv_bfloat16 *)gu, rows,
+                               F, g_in, codes, scales, g_out, act_prepared),
+                        "swiglu_quant_static_kernel");
     const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
     return launched(launch(quant_fused_kernel<__nv_bfloat16, 1>, dim3(cs), dim3(QTHREADS), 0, (cudaStream_t)stream,
                            cs, (const __nv_bfloat16 *)gu, rows, F, 2 * F, (const float *)nullptr, codes, scales,

@@ -16,6 +16,7 @@ constexpr int QNB = 4;                 // max 16-blocks per thread of the fused 
 constexpr int64_t QSMALL_MAX_BLOCKS = (int64_t)QCL_MAX * QTHREADS * QNB;
 constexpr int RTHREADS = 256;          // threads per CTA of the fused RMSNorm path
 constexpr int RNB = 2;                 // 16-blocks per thread of a row (n <= 8192)
+constexpr int QBIG_THREADS_STATIC = 256;
 
 __device__ __forceinline__ float tensor_scale_from_amax(float amax)
 {
@@ -288,6 +289,70 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         }
     }
     cluster_sync_all();
+}
+
+// ---- static tensor scale: no grid-wide reduction, one launch --------------
+// RMSNorm + quantise with a given g: one CTA per row, each thread up to RNB
+// 16-blocks; only the row's sum of squares is reduced (within the CTA).
+__global__ void __launch_bounds__(RTHREADS)
+    rmsnorm_quant_static_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
+                                int64_t n, const float *__restrict__ g_in, uint8_t *__restrict__ codes,
+                                uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
+{
+    __shared__ float s_red[33];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t r = blockIdx.x;
+    const int64_t kb = n / 16;
+    float v[RNB][16];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < RNB; ++j) {
+        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
+        if (c < kb) {
+            load16<__nv_bfloat16>(x + r * n + c * 16, v[j]);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) ss += v[j][k] * v[j][k];
+        }
+    }
+    const float g = *g_in;
+    const float tot = block_sum(ss, s_red);
+    const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
+    if (r == 0 && threadIdx.x == 0) *g_out = g;
+#pragma unroll
+    for (int j = 0; j < RNB; ++j) {
+        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
+        if (c < kb) {
+            float wv[16];
+            load16<__nv_bfloat16>(w + c * 16, wv);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[j][k] = round_bf16(__fmul_rn(__fmul_rn(v[j][k], inv), wv[k]));
+            uint2 pk;
+            const uint32_t sc = quant_block16(v[j], g, pk);
+            store_block(codes, scales, act, r, c, n, pk, sc);
+        }
+    }
+}
+
+// SwiGLU + quantise with a given g: one thread per 16-block, grid-stride.
+__global__ void __launch_bounds__(QBIG_THREADS_STATIC)
+    swiglu_quant_static_kernel(const __nv_bfloat16 *__restrict__ gu, int64_t rows, int64_t F,
+                               const float *__restrict__ g_in, uint8_t *__restrict__ codes,
+                               uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const float g = *g_in;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const int64_t kb = F / 16, nblk = rows * kb;
+    for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblk; b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = b / kb, c = b % kb;
+        float v[16];
+        load16_swiglu(gu + r * 2 * F + c * 16, gu + r * 2 * F + F + c * 16, v);
+        uint2 pk;
+        const uint32_t sc = quant_block16(v, g, pk);
+        store_block(codes, scales, act, r, c, F, pk, sc);
+    }
 }
 
 // ---- large tensors: amax partials, then encode ----------------------------

@@ -46,10 +46,10 @@ _SIGS = {
     "nvfp4_linear_noalloc": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
     "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
     "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
-                               _vp, _f32, _vp, _vp, _sz, _vp]),
+                               _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kv_page_restore": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
-    "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kv_append_fp8": (_int, [_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp, _vp]),
     "argmax_workspace_bytes": (_sz, [_i64, _i64]),
     "argmax_rows_bf16": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
@@ -201,9 +201,11 @@ def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, str
 
 
 def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None, out=None,
-              ld_q=None, T=None, Hq=None, ws=None, stream=None):
+              ld_q=None, T=None, Hq=None, ws=None, stream=None, g_act=None, act=None):
     """q bf16 [T, Hq, D] (or a strided [T, >= Hq*D] view with ld_q); pools u8
-    [pages, Hkv, P, D] / [pages, Hkv, D*P] (tiled V planes); returns bf16 [T, Hq, D]."""
+    [pages, Hkv, P, D] / [pages, Hkv, D*P] (tiled V planes); returns bf16 [T, Hq, D].
+    With act (prepared activation buffer) and g_act (static tensor scale), the
+    output is also quantised to NVFP4 in the same launch."""
     n_pages, Hkv, P, D = k_pool.shape
     if T is None:
         T, Hq = q.shape[0], q.shape[1]
@@ -216,7 +218,7 @@ def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, 
     wp, wn = _ws(ws, load().tree_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)), "attn")
     _call("tree_attn_fp8kv", q.data_ptr(), ld_q, T, Hq, Hkv, D, k_pool.data_ptr(), v_pool.data_ptr(), n_pages, P,
           page_table.data_ptr(), int(ctx_len), parent.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
-          float(sm_scale), out.data_ptr(), wp, wn, _stream(stream))
+          float(sm_scale), out.data_ptr(), _p(g_act), _p(act), wp, wn, _stream(stream))
     return out
 
 
@@ -226,20 +228,21 @@ def kv_page_restore(src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, st
           page_bytes, src_pool.numel() // page_bytes, dst_pool.numel() // page_bytes, _stream(stream))
 
 
-def rmsnorm_quantize(x, w, eps, out, act=None, stream=None):
-    """out = (codes or None, scales or None, g); act: prepared buffer or None."""
+def rmsnorm_quantize(x, w, eps, out, act=None, stream=None, g_in=None):
+    """out = (codes or None, scales or None, g); act: prepared buffer or None;
+    g_in: static tensor scale (device [1]) or None for the dynamic one."""
     rows, n = x.shape
     codes, scales, g = out
-    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, _p(codes), _p(scales),
-          g.data_ptr(), _p(act), None, 0, _stream(stream))
+    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, _p(g_in), _p(codes),
+          _p(scales), g.data_ptr(), _p(act), None, 0, _stream(stream))
     return out
 
 
-def swiglu_quantize(gu, out, act=None, stream=None):
+def swiglu_quantize(gu, out, act=None, stream=None, g_in=None):
     rows, F2 = gu.shape
     codes, scales, g = out
-    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, _p(codes), _p(scales), g.data_ptr(), _p(act),
-          None, 0, _stream(stream))
+    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, _p(g_in), _p(codes), _p(scales), g.data_ptr(),
+          _p(act), None, 0, _stream(stream))
     return out
 
 

@@ -71,9 +71,15 @@ class VerifyModel:
     tensor t -> inputs.weight_fp32(4, t, N, K, sub=l)), which the oracle
     reproduces."""
 
+    SITES = 4      # quantisation sites per layer: norm1, attention out, norm2, SwiGLU
+
     def __init__(self, n_layers=I.N_LAYERS, ctx_len=I.CTX_MAX, T=I.TREE_NODES, weights="device",
                  prefix_frac=0.96, device="cuda", lm_head=True, seed=42):
         self.dev = torch.device(device)
+        # activation tensor scales: dynamic (amax/2688 per call) until calibrate()
+        # turns them into static per-site scales, as a calibrated checkpoint has
+        self.static = False
+        self._record = False
         self.n_layers, self.L, self.T = n_layers, ctx_len, T
         self.eps = 1e-6
         H, F, Hq, Hkv, D, P = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM, I.PAGE
@@ -133,6 +139,7 @@ class VerifyModel:
         self.q_f = Act(F, self.dev)
         self.logits = torch.empty(T, I.VOCAB, dtype=torch.bfloat16, device=self.dev)
         self.ids = torch.empty(T, dtype=torch.int32, device=self.dev)
+        self.G = torch.ones(n_layers * self.SITES + 1, dtype=torch.float32, device=self.dev)
 
     def _random_fp8(self, shape, *seed):
         """Random finite E4M3 bytes (never the NaN codes 0x7F / 0xFF)."""
@@ -153,31 +160,65 @@ class VerifyModel:
     def restore(self):
         nv.kv_page_restore(self.src.view(-1), self.src_ids, self.kv.view(-1), self.dst_ids, PAGE_BYTES)
 
+    # ------------------------------------------------------------------ scales
+    def _site(self, i):
+        """Static scale of quantisation site i (device [1]), or None when dynamic."""
+        return self.G[i:i + 1] if self.static else None
+
+    def _note(self, i, act):
+        if self._record:
+            self.G[i:i + 1].copy_(act.g)
+
+    def calibrate(self, restore=True):
+        """Run one step with dynamic tensor scales and keep each site's scale as
+        its static g_in from then on (one activation scale per quantised tensor
+        of the checkpoint)."""
+        self.static, self._record = False, True
+        self.step(restore=restore)
+        self._record, self.static = False, True
+
     def layer(self, l):
         lay, T = self.layers[l], self.T
-        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l], self.eps, self.q_h.out, act=self.q_h.buf)
-        self._linear(self.q_h, lay["qkv"], self.qkv)
+        s0 = l * self.SITES
+        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l], self.eps, self.q_h.out, act=self.q_h.buf,
+                            g_in=self._site(s0))
+        self._note(s0, self.q_h)
+        self._linear(self.q_h.buf, self.q_h.g, lay["qkv"], self.qkv)
         qd = I.N_Q_HEADS * I.HEAD_DIM
         kd = I.N_KV_HEADS * I.HEAD_DIM
         nv.kv_append(self.qkv[:, qd:], self.qkv[:, qd + kd:], self.qkv.stride(0), T, self.k_pool(l),
                      self.v_pool(l), self.page_table, self.L, self.k_scale[l], self.v_scale[l])
-        nv.tree_attn(self.qkv, self.k_pool(l), self.v_pool(l), self.page_table, self.L, self.parent,
-                     self.k_scale[l], self.v_scale[l], out=self.attn, ld_q=self.qkv.stride(0), T=T,
-                     Hq=I.N_Q_HEADS)
-        nv.quantize(self.attn, out=self.q_a.out, act=self.q_a.buf, canonical=False)
-        self._linear(self.q_a, lay["o"], self.h, residual=self.h)
-        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l + 1], self.eps, self.q_h.out, act=self.q_h.buf)
-        self._linear(self.q_h, lay["gate_up"], self.gu)
-        nv.swiglu_quantize(self.gu, self.q_f.out, act=self.q_f.buf)
-        self._linear(self.q_f, lay["down"], self.h, residual=self.h)
+        if self.static:
+            # attention output quantised in the combine launch with the static scale
+            g_a = self._site(s0 + 1)
+            nv.tree_attn(self.qkv, self.k_pool(l), self.v_pool(l), self.page_table, self.L, self.parent,
+                         self.k_scale[l], self.v_scale[l], out=self.attn, ld_q=self.qkv.stride(0), T=T,
+                         Hq=I.N_Q_HEADS, g_act=g_a, act=self.q_a.buf)
+        else:
+            nv.tree_attn(self.qkv, self.k_pool(l), self.v_pool(l), self.page_table, self.L, self.parent,
+                         self.k_scale[l], self.v_scale[l], out=self.attn, ld_q=self.qkv.stride(0), T=T,
+                         Hq=I.N_Q_HEADS)
+            nv.quantize(self.attn, out=self.q_a.out, act=self.q_a.buf, canonical=False)
+            self._note(s0 + 1, self.q_a)
+            g_a = self.q_a.g
+        self._linear(self.q_a.buf, g_a, lay["o"], self.h, residual=self.h)
+        nv.rmsnorm_quantize(self.h, self.norm_w[2 * l + 1], self.eps, self.q_h.out, act=self.q_h.buf,
+                            g_in=self._site(s0 + 2))
+        self._note(s0 + 2, self.q_h)
+        self._linear(self.q_h.buf, self.q_h.g, lay["gate_up"], self.gu)
+        nv.swiglu_quantize(self.gu, self.q_f.out, act=self.q_f.buf, g_in=self._site(s0 + 3))
+        self._note(s0 + 3, self.q_f)
+        self._linear(self.q_f.buf, self.q_f.g, lay["down"], self.h, residual=self.h)
 
     def head(self):
-        nv.rmsnorm_quantize(self.h, self.norm_w[-1], self.eps, self.q_h.out, act=self.q_h.buf)
-        self._linear(self.q_h, self.lm_head, self.logits)
+        i = self.n_layers * self.SITES
+        nv.rmsnorm_quantize(self.h, self.norm_w[-1], self.eps, self.q_h.out, act=self.q_h.buf, g_in=self._site(i))
+        self._note(i, self.q_h)
+        self._linear(self.q_h.buf, self.q_h.g, self.lm_head, self.logits)
         nv.argmax(self.logits, self.ids)
 
-    def _linear(self, q, lin, y, residual=None):
-        nv.linear(q.buf, q.g, self.T, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
+    def _linear(self, act, g, lin, y, residual=None):
+        nv.linear(act, g, self.T, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
 
     def step(self, restore=True):
         """One verify step on the current self.h / self.parent; result in self.ids."""
@@ -188,11 +229,17 @@ class VerifyModel:
         if self.lm_head is not None:
             self.head()
 
-    LAUNCHES_PER_LAYER = 11          # norm-q, qkv, kv-append, attn split+combine, q, o, norm-q, gate_up, swiglu-q, down
     LAUNCHES_HEAD = 3                # norm-q, lm head, argmax
 
+    @property
+    def launches_per_layer(self):
+        """norm-q, qkv, kv-append, attention split + combine, [quantise], o,
+        norm-q, gate_up, swiglu-q, down (the attention output is quantised in
+        the combine launch when the scales are static)."""
+        return 10 if self.static else 11
+
     def launches_per_step(self, restore=True):
-        return (1 if restore else 0) + self.n_layers * self.LAUNCHES_PER_LAYER + \
+        return (1 if restore else 0) + self.n_layers * self.launches_per_layer + \
             (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     # ------------------------------------------------------------------ bytes

@@ -161,3 +161,22 @@ def test_bad_page_id_and_parent_are_flagged():
     rc, site = nv.device_status()
     assert rc == -7 and site == 305, (rc, site)
     assert nv.device_status()[0] == 0
+
+
+def test_fused_nvfp4_output_matches_separate_quantisation():
+    """With a static tensor scale the combine launch also writes the NVFP4
+    prepared activation of its bf16 output: byte-identical to quantising the
+    bf16 output in a separate call (same recipe, same values)."""
+    cuda()
+    L, T, Hq = 700, 16, 24
+    cache = inputs.kv_cache(80, L)
+    parent = inputs.tree_parent(80)
+    q = to_dev(inputs.query_bf16(80))
+    kp, vp, pt, ks, vs = _dev_cache(cache)
+    g = to_dev(np.array([0.0006], np.float32))
+    act = nv.act_buffer(Hq * 128)
+    out = nv.tree_attn(q, kp, vp, pt, L, to_dev(parent), ks, vs, g_act=g, act=act)
+    ref_act = nv.act_buffer(Hq * 128)
+    nv.quantize(out.view(T, Hq * 128), g_in=g, act=ref_act, canonical=False)
+    assert torch.equal(act, ref_act)
+    assert nv.device_status()[0] == 0

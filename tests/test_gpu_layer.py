@@ -1,0 +1,99 @@
+"""Per-layer parity of the verify step (teacher-forced): one decoder layer of
+the 64-layer stack run through the library (VerifyModel.layer) against the
+same layer composed from the oracle's pieces on the same bf16 input, the same
+NVFP4 weights (quantised from the same fp32 values) and the same FP8 cache.
+
+The oracle side follows the layer definition step by step:
+  y1 = bf16(RMSNorm(h)), qkv = bf16(NVFP4(y1) x W_qkv^T), FP8 append of the
+  tree's K/V, a = bf16(tree attention), h1 = bf16(h + NVFP4(a) x W_o^T),
+  y2 = bf16(RMSNorm(h1)), gu = bf16(NVFP4(y2) x W_gu^T),
+  s = bf16(SwiGLU(gu)), h2 = bf16(h1 + NVFP4(s) x W_down^T),
+with every NVFP4 activation quantised with the tensor scale the GPU used
+(static scales) or its own amax/2688 (dynamic scales).
+
+Tolerance: each piece is gated elsewhere (linear rel-Frobenius <= 1e-3 after
+bf16 rounding, attention <= 2e-3 absolute, quantisation bit-exact).  Composed,
+a bf16 rounding difference upstream can flip an E2M1 code downstream (one
+grid step of one element), so the layer output is gated at 1e-2
+rel-Frobenius, and the attention output and QKV activations at their own
+bars (attention: 2e-3 + 2^-8 |o|) against the oracle fed with the GPU's own
+inputs to those ops.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import cuda, rel_fro
+from nvfp4_skinny_gemm_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+@pytest.mark.parametrize("static", [False, True])
+def test_one_layer_teacher_forced(oracle, static):
+    cuda()
+    from nvfp4_skinny_gemm_b200.step import VerifyModel
+    L, T = 1024, I.TREE_NODES
+    m = VerifyModel(n_layers=1, ctx_len=L, weights="host", lm_head=False)
+    h0 = I.bf16_normal(4, 300, (T, I.HIDDEN)) * 0.5
+    parent = I.tree_parent(4)
+    m.parent.copy_(torch.from_numpy(parent))
+    m.restore()
+    if static:
+        m.h.copy_(h0)
+        m.calibrate(restore=False)
+    m.h.copy_(h0)
+    kp = m.k_pool(0).cpu().numpy().copy()
+    vp = m.v_pool(0).cpu().numpy().copy()
+    m.layer(0)
+    torch.cuda.synchronize()
+    h2_gpu = m.h.float().cpu().numpy()
+    qkv_gpu = m.qkv.float().cpu().numpy()
+    attn_gpu = m.attn.float().cpu().numpy()
+    G = m.G.cpu().numpy()
+
+    # ---- oracle composition
+    wq = {}
+    for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items()):
+        wq[name] = oracle.quantize(I.weight_fp32(4, t, N, K, sub=0))
+
+    def lin(x_bf16, name, site):
+        ac, asc, ga = oracle.quantize(x_bf16, g_in=float(G[site]) if static else None)
+        wc, wsc, gw = wq[name]
+        return oracle.linear(ac, asc, ga, wc, wsc, gw)
+
+    h = h0.float().numpy()
+    ones = np.ones(I.HIDDEN, np.float32)
+    y1 = _bf16(oracle.rmsnorm(h, ones, eps=m.eps))
+    qkv = _bf16(lin(y1, "qkv", 0))
+    assert rel_fro(qkv_gpu, qkv) <= 1e-2, rel_fro(qkv_gpu, qkv)
+    # attention from the GPU's own QKV output (teacher-forced), gated at 2e-3
+    qd, kd = I.N_Q_HEADS * I.HEAD_DIM, I.N_KV_HEADS * I.HEAD_DIM
+    k_new = qkv_gpu[:, qd:qd + kd].reshape(T, I.N_KV_HEADS, I.HEAD_DIM)
+    v_new = qkv_gpu[:, qd + kd:].reshape(T, I.N_KV_HEADS, I.HEAD_DIM)
+    ks, vs = m.k_scale[0].cpu().numpy(), m.v_scale[0].cpu().numpy()
+    pt = m.page_table_h
+    oracle.kv_append(k_new, v_new, kp, vp, pt, L, ks, vs)
+    assert np.array_equal(m.k_pool(0).cpu().numpy(), kp)
+    assert np.array_equal(m.v_pool(0).cpu().numpy(), vp)
+    a = oracle.tree_attn(qkv_gpu[:, :qd].reshape(T, I.N_Q_HEADS, I.HEAD_DIM), kp, vp, pt, L, parent, ks, vs)
+    # the cache holds uniformly random E4M3 codes, so outputs reach |o| ~ 9: the
+    # bar adds the bf16 output rounding (2^-9 |o|) and the two-term operand
+    # error, as for the other small attention cases
+    err_a = np.abs(attn_gpu.reshape(a.shape) - a)
+    assert np.all(err_a <= 2e-3 + 2.0 ** -8 * np.abs(a)), err_a.max()
+    # rest of the layer from the GPU's attention output
+    a = attn_gpu.reshape(T, qd)
+    h1 = _bf16(h + lin(a, "o", 1))
+    y2 = _bf16(oracle.rmsnorm(h1, ones, eps=m.eps))
+    gu = _bf16(lin(y2, "gate_up", 2))
+    s = _bf16(oracle.swiglu(gu))
+    h2 = _bf16(h1 + lin(s, "down", 3))
+    err = rel_fro(h2_gpu, h2)
+    print(f"layer parity ({'static' if static else 'dynamic'} scales): rel-Frobenius {err:.2e}")
+    assert err <= 1e-2
+    assert np.isfinite(h2_gpu).all()

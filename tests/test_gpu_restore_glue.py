@@ -67,7 +67,9 @@ def _dequant_err(oracle, codes, scales, g, want):
     return np.linalg.norm(deq - want) / np.linalg.norm(want)
 
 
-def test_rmsnorm_quantize(oracle):
+@pytest.mark.parametrize("g_static", [None, 0.0019])
+def test_rmsnorm_quantize(oracle, g_static):
+    """g_static None: dynamic tensor scale; else the one-launch static-scale path."""
     cuda()
     rows, n = 16, inputs.HIDDEN
     x = inputs.bf16_normal(92, 0, (rows, n)) * 3
@@ -75,30 +77,33 @@ def test_rmsnorm_quantize(oracle):
     out = (torch.empty(rows, n // 2, dtype=torch.uint8, device="cuda"),
            torch.empty(rows, n // 16, dtype=torch.uint8, device="cuda"),
            torch.empty(1, dtype=torch.float32, device="cuda"))
-    nv.rmsnorm_quantize(to_dev(x), to_dev(w), 1e-6, out)
+    g_in = None if g_static is None else to_dev(np.array([g_static], np.float32))
+    nv.rmsnorm_quantize(to_dev(x), to_dev(w), 1e-6, out, g_in=g_in)
     y = oracle.rmsnorm(x.float().numpy(), w.float().numpy(), eps=1e-6)
     # codes = NVFP4 of the bf16-rounded RMSNorm output: compare with the oracle's
     # quantisation of the oracle's bf16-rounded output (differences only where
     # the fp32 RMSNorm lands on the other side of a bf16 rounding boundary)
     yb = torch.from_numpy(y).float().to(torch.bfloat16).float().numpy()
-    oc, osc, og = oracle.quantize(yb)
+    oc, osc, og = oracle.quantize(yb, g_in=g_static)
     assert abs(float(out[2].cpu()[0]) - og) <= 1e-6 * og
     assert np.mean(out[0].cpu().numpy() != oc) < 2e-3
     assert np.mean(out[1].cpu().numpy() != osc) < 2e-3
     assert _dequant_err(oracle, *out, y) < 0.12           # NVFP4 quantisation noise of N(0,1) data
 
 
-def test_swiglu_quantize(oracle):
+@pytest.mark.parametrize("g_static", [None, 0.015])
+def test_swiglu_quantize(oracle, g_static):
     cuda()
     rows, F = 16, inputs.FFN
     gu = inputs.bf16_normal(93, 0, (rows, 2 * F)) * 2
     out = (torch.empty(rows, F // 2, dtype=torch.uint8, device="cuda"),
            torch.empty(rows, F // 16, dtype=torch.uint8, device="cuda"),
            torch.empty(1, dtype=torch.float32, device="cuda"))
-    nv.swiglu_quantize(to_dev(gu), out)
+    g_in = None if g_static is None else to_dev(np.array([g_static], np.float32))
+    nv.swiglu_quantize(to_dev(gu), out, g_in=g_in)
     h = oracle.swiglu(gu.float().numpy())
     hb = torch.from_numpy(h).float().to(torch.bfloat16).float().numpy()
-    oc, osc, og = oracle.quantize(hb)
+    oc, osc, og = oracle.quantize(hb, g_in=g_static)
     assert abs(float(out[2].cpu()[0]) - og) <= 1e-6 * og
     assert np.mean(out[0].cpu().numpy() != oc) < 2e-3
     assert np.mean(out[1].cpu().numpy() != osc) < 2e-3
