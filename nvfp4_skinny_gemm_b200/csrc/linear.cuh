@@ -22,9 +22,12 @@
 // Work unit = one weight unit.  The NT x KC units are cut into
 // G = min(#SMs, units) contiguous ranges (stream-K split-K), so every CTA
 // streams the same number of weight bytes.  A tile whose K range is split
-// over several CTAs is reduced by the CTA that finishes it last (per-tile,
-// per-sub-partition arrival counter); partial sums are added in contributor
-// order, so results do not depend on timing.
+// over several CTAs is reduced by its owner, the CTA holding its first K
+// chunk (which reaches that tile last): the other contributors publish fp32
+// partial sums and bump a per-tile, per-sub-partition arrival counter; the
+// owner polls the counter and loads their partials while its own products
+// are still in flight, then adds them in contributor order, so results do
+// not depend on timing.
 //
 // Warp roles (192 threads, one CTA per SM):
 //   warp 0   producer: weight units of the first stages are requested before
@@ -41,6 +44,7 @@ namespace nvfp4sk {
 
 constexpr int LIN_STAGES = 4;
 constexpr int LIN_THREADS = 192;
+constexpr int LIN_PF = 7;                         // split-K partials prefetched by a tile's owner
 constexpr int LIN_KC = 512;                       // K elements per unit / chunk
 constexpr int LIN_KSTEPS = LIN_KC / 64;           // MMA steps per unit
 constexpr uint32_t LIN_W_ATOM = 128 * 128;        // 128 rows x 256 E2M1, swizzled
@@ -79,6 +83,34 @@ struct LinearParams {
     int64_t U;                     // NT * KC
     int M, N, NT, KC;
 };
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait (bounded) until *p == want; returns false and records a timeout otherwise.
+__device__ __forceinline__ bool poll_counter(const int *p, int want, uint32_t site, volatile int *abort)
+{
+    if (ld_acquire_gpu(p) == want) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 8; ++i)
+            if (ld_acquire_gpu(p) == want) return true;
+        if (abort && *abort) return false;
+        if (globaltimer() - t0 > g_timeout_ns) {
+            report_error(ERRBIT_TIMEOUT, site);
+            if (abort) *abort = 1;
+            return false;
+        }
+    }
+}
 
 __device__ __forceinline__ int64_t lin_start(int64_t c, int64_t U, int64_t G) { return c * U / G; }
 __device__ __forceinline__ int64_t lin_cta_of(int64_t u, int64_t U, int64_t G) { return ((u + 1) * G + U - 1) / U - 1; }
@@ -223,7 +255,36 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             const int64_t t = u / KC, ka = u % KC;
             const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
             const uint32_t b = (uint32_t)(seg & 1);
+            const bool whole = ka == 0 && kend == KC;
+            const int64_t first = whole ? c : lin_cta_of(t * KC, U, G);
+            const int64_t last = whole ? c : lin_cta_of(t * KC + KC - 1, U, G);
+            // Split tile: the CTA holding its first K chunk owns it.  That chunk
+            // range ends the owner's own range, so the owner reaches this tile
+            // last; it polls the other contributors' arrivals and loads their
+            // partial sums while its own products are still in flight, then adds
+            // them to its accumulator in contributor order.
+            const bool owner = !whole && c == first;
+            float part[LIN_PF][16];
             bool ok = true;
+            if (owner) {
+                if (lane == 0) ok = poll_counter(p.counters + t * 4 + q, (int)(last - first), 107, s_abort);
+                ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                __threadfence();
+#pragma unroll
+                for (int k = 0; k < LIN_PF; ++k) {
+                    const int64_t cc = first + 1 + k;
+                    if (cc <= last) {
+                        const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
+                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const float4 f = __ldcg(Q + v);
+                            part[k][4 * v] = f.x; part[k][4 * v + 1] = f.y; part[k][4 * v + 2] = f.z; part[k][4 * v + 3] = f.w;
+                        }
+                    }
+                }
+            }
             if (lane == 0) ok = mbar_wait(&accf[b], (uint32_t)((seg >> 1) & 1), 106, s_abort);
             ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
@@ -235,22 +296,45 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[b]);
             const int64_t n = t * 128 + row;
-            if (ka == 0 && kend == KC) {
+            if (whole || owner) {
+                float acc[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc[m] = __uint_as_float(r[m]);
+                if (owner) {
+#pragma unroll
+                    for (int k = 0; k < LIN_PF; ++k)
+                        if (first + 1 + k <= last) {
+#pragma unroll
+                            for (int m = 0; m < 16; ++m) acc[m] = __fadd_rn(acc[m], part[k][m]);
+                        }
+                    // tiles split over more than LIN_PF + 1 CTAs: the rest, in order
+                    for (int64_t cc = first + 1 + LIN_PF; cc <= last; ++cc) {
+                        const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
+                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const float4 f = __ldcg(Q + v);
+                            acc[4 * v] = __fadd_rn(acc[4 * v], f.x);
+                            acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], f.y);
+                            acc[4 * v + 2] = __fadd_rn(acc[4 * v + 2], f.z);
+                            acc[4 * v + 3] = __fadd_rn(acc[4 * v + 3], f.w);
+                        }
+                    }
+                    if (lane == 0) p.counters[t * 4 + q] = 0;
+                }
                 if (n < p.N) {
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
                         if (m < M) {
-                            float o = __fmul_rn(__uint_as_float(r[m]), gs);
+                            float o = __fmul_rn(acc[m], gs);
                             if (p.residual) o = __fadd_rn(o, __bfloat162float(p.residual[m * p.ldy + n]));
                             p.y[m * p.ldy + n] = __float2bfloat16_rn(o);
                         }
                     }
                 }
             } else {
-                // split-K fix-up, per warp: each warp owns rows 32q..32q+31 of the
-                // tile and its own arrival counter, so no cross-warp barrier is needed.
-                // Partial slots are [128 rows][16 tokens] fp32: a lane's 16 values
-                // are 64 contiguous bytes (four 16-byte stores / loads).
+                // contributor: publish the partial sum, then one release add on the
+                // tile's arrival counter (per warp: each warp owns rows 32q..32q+31)
                 const int slot = (t == first_tile_of_me) ? 0 : 1;
                 float4 *P = reinterpret_cast<float4 *>(p.partial + ((c * 2 + slot) * 128 + row) * 16);
 #pragma unroll
@@ -259,53 +343,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                 __threadfence();
                 __syncwarp();
-                const int64_t first = lin_cta_of(t * KC, U, G), last = lin_cta_of(t * KC + KC - 1, U, G);
-                int is_last = 0;
-                if (lane == 0) is_last = (atomicAdd(p.counters + t * 4 + q, 1) == (int)(last - first)) ? 1 : 0;
-                is_last = __shfl_sync(0xFFFFFFFFu, is_last, 0);
-                if (is_last) {
-                    __threadfence();
-                    float acc[16];
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-                    // contributors in order; up to 8 of them loaded before summing
-                    for (int64_t c0 = first; c0 <= last; c0 += 8) {
-                        float4 part[8][4];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int64_t cc = c0 + k;
-                            if (cc <= last) {
-                                const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
-                                const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
-#pragma unroll
-                                for (int v = 0; v < 4; ++v) part[k][v] = __ldcg(Q + v);
-                            }
-                        }
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            if (c0 + k <= last) {
-#pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    acc[4 * v] = __fadd_rn(acc[4 * v], part[k][v].x);
-                                    acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], part[k][v].y);
-                                    acc[4 * v + 2] = __fadd_rn(acc[4 * v + 2], part[k][v].z);
-                                    acc[4 * v + 3] = __fadd_rn(acc[4 * v + 3], part[k][v].w);
-                                }
-                            }
-                        }
-                    }
-                    if (n < p.N) {
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            if (m < M) {
-                                float o = __fmul_rn(acc[m], gs);
-                                if (p.residual) o = __fadd_rn(o, __bfloat162float(p.residual[m * p.ldy + n]));
-                                p.y[m * p.ldy + n] = __float2bfloat16_rn(o);
-                            }
-                        }
-                    }
-                    if (lane == 0) p.counters[t * 4 + q] = 0;
-                }
+                if (lane == 0) red_release_gpu_add(p.counters + t * 4 + q, 1);
             }
             u += kend - ka;
         }
