@@ -55,12 +55,18 @@ constexpr uint32_t LIN_A_UNIT = 2 * LIN_A_ATOM + LIN_KSTEPS * LIN_SF_IMG;    // 
 constexpr uint32_t LIN_STAGE_BYTES = LIN_W_UNIT + LIN_A_UNIT;                // 45056 = 44 * 1024
 constexpr uint32_t LIN_OFF_BAR = LIN_STAGES * LIN_STAGE_BYTES;
 constexpr uint32_t LIN_SMEM_BYTES = LIN_OFF_BAR + 256 + 1024;
-constexpr uint32_t LIN_TMEM_COLS = 256;
-// TMEM columns: acc[b] at 16*b (16 fp32 columns = 16 tokens); weight scales
-// SFA[r] at 32 + 32*r and activation scales SFB[r] at 96 + 32*r, 4 columns
-// per MMA step.  Scale-factor column addresses handed to the MMA stay
-// multiples of 4.
-constexpr uint32_t TM_ACC = 0, TM_SFA = 32, TM_SFB = 96;
+constexpr uint32_t LIN_TMEM_COLS = 512;
+constexpr int LIN_NACC = 1;                       // independent accumulators per tile (MMA j -> j % LIN_NACC)
+constexpr int LIN_SFB_SLOTS = 11;                 // activation-scale chunks kept resident in TMEM
+// TMEM columns: accumulator a of buffer b at 16*(LIN_NACC*b + a) (16 fp32
+// columns = 16 tokens; the MMAs of a tile rotate over the LIN_NACC
+// accumulators so that consecutive products do not wait on each other, and
+// the epilogue adds them in a fixed order); weight scales SFA[r] and
+// activation scales SFB[r] 32 columns each (4 per MMA step), resident
+// activation scales of up to LIN_SFB_SLOTS K chunks after them.  Scale-factor
+// column addresses handed to the MMA stay multiples of 4.
+constexpr uint32_t TM_ACC = 0, TM_SFA = 32 * LIN_NACC, TM_SFB = TM_SFA + 64, TM_SFB_RES = TM_SFB + 64;
+static_assert(TM_SFB_RES + 32 * LIN_SFB_SLOTS <= LIN_TMEM_COLS, "tensor memory budget");
 
 // Instruction descriptor (kind::mxf4nvf4): A/B format E2M1 (1) in bits 7-9 and
 // 10-12, K-major A and B, N>>3 in bits 17-22, scale format UE4M3 (0) in
@@ -200,13 +206,21 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             constexpr uint32_t idesc = lin_idesc(128, 16);
             int64_t i = 0, seg = 0;
             bool ok = true;
+            // The activation scales of K chunk kc are the same for every weight tile:
+            // when this CTA sweeps all K chunks at least four times (an LM-head-like
+            // shape: many tiles, short K), each chunk's scales are copied into tensor
+            // memory once (slot kc - kc0 mod KC) and reused by every later tile.
+            // (Measured: with less reuse the per-unit copies are as fast.)
+            const bool sfb_resident = n_units >= 4 * (int64_t)KC && KC <= LIN_SFB_SLOTS;
+            const int64_t kc0 = u0 % KC;
+            uint32_t sfb_loaded = 0;
             for (int64_t u = u0; u < u1 && ok; ++seg) {
                 const int64_t ka = u % KC;
                 const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
                 const uint32_t b = (uint32_t)(seg & 1);
                 if (!mbar_wait(&acce[b], (uint32_t)(((seg >> 1) & 1) ^ 1), 103, s_abort)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + TM_ACC + 16 * b;
+                const uint32_t d_tmem = tmem_base + TM_ACC + 16 * LIN_NACC * b;
                 for (int64_t kc = ka; kc < kend; ++kc, ++i) {
                     const int s = (int)(i % LIN_STAGES);
                     if (!mbar_wait(&full[s], (uint32_t)((i / LIN_STAGES) & 1), 104, s_abort)) { ok = false; break; }
@@ -215,19 +229,30 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     const uint32_t w_s = smem_u32(smem + s * LIN_STAGE_BYTES);
                     const uint32_t a_s = w_s + LIN_W_UNIT;
                     const uint32_t sfa_s = w_s + 2 * LIN_W_ATOM, sfb_s = a_s + 2 * LIN_A_ATOM;
-                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * r, sfb_t = tmem_base + TM_SFB + 32 * r;
+                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * r;
+                    uint32_t sfb_t = tmem_base + TM_SFB + 32 * r;
+                    bool copy_sfb = true;
+                    if (sfb_resident) {
+                        const uint32_t slot = (uint32_t)((kc - kc0 + KC) % KC);
+                        sfb_t = tmem_base + TM_SFB_RES + 32 * slot;
+                        copy_sfb = !((sfb_loaded >> slot) & 1u);
+                        sfb_loaded |= 1u << slot;
+                    }
 #pragma unroll
-                    for (int j = 0; j < LIN_KSTEPS; ++j) {
+                    for (int j = 0; j < LIN_KSTEPS; ++j)
                         tmem_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
-                        tmem_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
+                    if (copy_sfb) {
+#pragma unroll
+                        for (int j = 0; j < LIN_KSTEPS; ++j)
+                            tmem_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
                     }
 #pragma unroll
                     for (int j = 0; j < LIN_KSTEPS; ++j) {
                         const uint32_t atom = (uint32_t)(j >> 2), ko = 32u * (uint32_t)(j & 3);
                         const uint64_t adesc = smem_desc(w_s + atom * LIN_W_ATOM + ko, 16, 1024, SWZ_128B);
                         const uint64_t bdesc = smem_desc(a_s + atom * LIN_A_ATOM + ko, 16, 1024, SWZ_128B);
-                        mma_mxf4nvf4(d_tmem, adesc, bdesc, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
-                                     (kc > ka || j > 0) ? 1u : 0u);
+                        mma_mxf4nvf4(d_tmem + 16 * (j % LIN_NACC), adesc, bdesc, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+                                     (kc > ka || j >= LIN_NACC) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -290,7 +315,23 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             uint32_t r[16];
-            tmem_ld_32x32b_x16(tmem_base + ((32u * q) << 16) + TM_ACC + 16 * b, r);
+            {
+                const uint32_t acc_t = tmem_base + ((32u * q) << 16) + TM_ACC + 16 * LIN_NACC * b;
+                tmem_ld_32x32b_x16(acc_t, r);
+                if (LIN_NACC > 1) {
+                    uint32_t r2[LIN_NACC > 1 ? LIN_NACC - 1 : 1][16];
+#pragma unroll
+                    for (int a = 1; a < LIN_NACC; ++a) tmem_ld_32x32b_x16(acc_t + 16 * a, r2[a - 1]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        float v = __uint_as_float(r[m]);
+#pragma unroll
+                        for (int a = 1; a < LIN_NACC; ++a) v = __fadd_rn(v, __uint_as_float(r2[a - 1][m]));
+                        r[m] = __float_as_uint(v);
+                    }
+                }
+            }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
