@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ctx", type=int, default=23552)
     ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--chain", type=int, default=0,
+                    help="verify a linear-MTP chain of this many tokens instead of the 16-node tree")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
@@ -220,7 +222,8 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": len(vals), "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"64-layer 27B-class verify step, 16-node tree, ctx {args.ctx} FP8 paged KV, "
+            "config": {"workload": f"{args.layers}-layer 27B-class verify step, "
+                               f"{f'linear-MTP chain of {T}' if args.chain else '16-node tree'}, ctx {args.ctx} FP8 paged KV, "
                                    f"NVFP4 W4A4 linears + LM head, kv_page_restore of 96% prefix",
                        "layers": args.layers, "ctx": args.ctx, "tree_nodes": 16, "parallelism": "replicas"},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
@@ -235,10 +238,11 @@ def run_ours(args, world, rank, local):
     from nvfp4_skinny_gemm_b200.step import VerifyModel
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    model = VerifyModel(n_layers=args.layers, ctx_len=args.ctx, weights="device", device=dev)
-    h0 = I.bf16_normal(4, 300, (I.TREE_NODES, I.HIDDEN)).pin_memory()
-    par0 = torch.from_numpy(I.tree_parent(4)).pin_memory()
-    ids_host = torch.empty(I.TREE_NODES, dtype=torch.int32).pin_memory()
+    T = args.chain or I.TREE_NODES
+    model = VerifyModel(n_layers=args.layers, ctx_len=args.ctx, T=T, weights="device", device=dev)
+    h0 = I.bf16_normal(4, 300, (T, I.HIDDEN)).pin_memory()
+    par0 = torch.from_numpy(I.chain_parent(T) if args.chain else I.tree_parent(4)).pin_memory()
+    ids_host = torch.empty(T, dtype=torch.int32).pin_memory()
     stream = torch.cuda.Stream(device=dev)
 
     def load_inputs():
@@ -330,9 +334,10 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": t_dev / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate); fp8 e4m3 KV",
         "data": "synthetic",
-        "config": {"workload": f"64-layer 27B-class verify step, 16-node tree, ctx {args.ctx} FP8 paged KV, "
+        "config": {"workload": f"{args.layers}-layer 27B-class verify step, "
+                               f"{f'linear-MTP chain of {T}' if args.chain else '16-node tree'}, ctx {args.ctx} FP8 paged KV, "
                                f"NVFP4 W4A4 linears + LM head, kv_page_restore of 96% prefix",
-                   "layers": args.layers, "ctx": args.ctx, "tree_nodes": 16, "hidden": I.HIDDEN,
+                   "layers": args.layers, "ctx": args.ctx, "tree_nodes": T, "hidden": I.HIDDEN,
                    "weights_gb": round(sum(l.nbytes for lay in model.layers for l in lay.values()) / 1e9
                                        + model.lm_head.nbytes / 1e9, 3),
                    "l2": "inputs larger than L2 (11.4 GB of weights streamed per step)",

@@ -234,3 +234,64 @@ def ancestors(parent, i):
         out.append(i)
         i = int(parent[i])
     return out
+
+
+# ---------------------------------------------------------------- greedy tree acceptance
+# The step after the verify forward ("Tree multi-token prediction": the target
+# model verifies the tree's candidates in one pass and the runtime accepts the
+# matching path; temperature 0, so acceptance is exact): node 0 (the root, the
+# last accepted token) is accepted; node i >= 1 is accepted when its parent is
+# accepted and its draft token equals the target's greedy choice after the
+# parent.  The accepted path ends at the deepest accepted node (lowest index
+# among equally deep ones); the next token is the target's choice after it.
+def tree_accept_greedy(draft_tokens, target_argmax, parent):
+    """Returns (path [root .. end] as a list of node indices, next token)."""
+    T = len(parent)
+    accepted = [False] * T
+    depth = [0] * T
+    for i in range(T):                       # parents precede children
+        p = int(parent[i])
+        if p < 0:
+            accepted[i] = i == 0
+            depth[i] = 0
+        else:
+            depth[i] = depth[p] + 1
+            accepted[i] = accepted[p] and int(draft_tokens[i]) == int(target_argmax[p])
+    end = 0
+    for i in range(T):
+        if accepted[i] and depth[i] > depth[end]:
+            end = i
+    path = []
+    i = end
+    while i >= 0:
+        path.append(i)
+        i = int(parent[i])
+    path.reverse()
+    return path, int(target_argmax[end])
+
+
+def kv_compact_accepted(k_pool, v_pool, page_table, ctx_len, path):
+    """In place on one layer's pools (k [pages, Hkv, P, D], v [pages, Hkv, D*P]
+    in the tiled plane layout): the K/V of path node path[k], stored at logical
+    position ctx_len + path[k], is moved to position ctx_len + k, so that the
+    accepted tokens follow the context contiguously.  Each moved token is read
+    before anything is written."""
+    n_pages, Hkv, P, D = k_pool.shape
+
+    def v_off(d, t):                         # tile (d//8, t//16) of 8 x 16 bytes
+        return ((d // 8) * (P // 16) + t // 16) * 128 + (d % 8) * 16 + t % 16
+
+    def where(pos):
+        return int(page_table[pos // P]), pos % P
+
+    ks, vs = [], []
+    for node in path:
+        pg, sl = where(ctx_len + node)
+        ks.append(k_pool[pg, :, sl, :].copy())
+        vs.append(np.array([[v_pool[pg, h, v_off(d, sl)] for d in range(D)] for h in range(Hkv)], np.uint8))
+    for k in range(len(path)):
+        pg, sl = where(ctx_len + k)
+        k_pool[pg, :, sl, :] = ks[k]
+        for h in range(Hkv):
+            for d in range(D):
+                v_pool[pg, h, v_off(d, sl)] = vs[k][h, d]

@@ -33,14 +33,16 @@ def _bf16(x):
     return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
 
 
-@pytest.mark.parametrize("static", [False, True])
-def test_one_layer_teacher_forced(oracle, static):
+@pytest.mark.parametrize("static,T,chain", [(False, 16, False), (True, 16, False), (True, 4, True)])
+def test_one_layer_teacher_forced(oracle, static, T, chain):
+    """16-node tree (the verify step) and a linear-MTP chain of 4 tokens (the
+    pages' baseline variant) through the same kernels."""
     cuda()
     from nvfp4_skinny_gemm_b200.step import VerifyModel
-    L, T = 1024, I.TREE_NODES
-    m = VerifyModel(n_layers=1, ctx_len=L, weights="host", lm_head=False)
+    L = 1024
+    m = VerifyModel(n_layers=1, ctx_len=L, T=T, weights="host", lm_head=False)
     h0 = I.bf16_normal(4, 300, (T, I.HIDDEN)) * 0.5
-    parent = I.tree_parent(4)
+    parent = I.chain_parent(T) if chain else I.tree_parent(4)
     m.parent.copy_(torch.from_numpy(parent))
     m.restore()
     if static:
