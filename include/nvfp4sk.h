@@ -250,6 +250,36 @@ NVFP4SK_API nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, i
                              uint8_t *k_pool, uint8_t *v_pool, int64_t n_pool_pages, int page_size,
                              const int32_t *page_table, int64_t ctx_len, const float *k_scale,
                              const float *v_scale, nvfp4sk_stream_t stream);
+/* ------------------------------------------------------------------------
+ * Greedy acceptance of the verified tree (section "Tree multi-token
+ * prediction": the target model verifies the candidates in one pass and the
+ * runtime accepts the matching path; greedy decoding makes it exact).
+ * Node 0 (the root, the last accepted token) is accepted; node i >= 1 is
+ * accepted when its parent is accepted and draft_tokens[i] ==
+ * target_argmax[parent[i]] (target_argmax[j]: the target's greedy token after
+ * node j, e.g. from argmax_rows_bf16 of the LM head).  path (device i32 [T])
+ * receives the node indices from the root to the deepest accepted node (lowest
+ * index among equally deep ones), n_accepted (device i32 [1]) its length,
+ * next_token (device i32 [1]) the target's token after that node.  parent
+ * must be topologically ordered (parent[0] == -1, 0 <= parent[i] < i); else
+ * only the root is accepted and NVFP4SK_ERR_OUT_OF_RANGE is flagged in the
+ * device status.  1 <= T <= 32.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API nvfp4sk_status tree_accept_greedy(const int32_t *draft_tokens, const int32_t *target_argmax,
+                                              const int32_t *parent, int T, int32_t *path, int32_t *n_accepted,
+                                              int32_t *next_token, nvfp4sk_stream_t stream);
+/* Move the accepted tokens' K/V next to the context in every layer: for k <
+ * *n_accepted, the K and V bytes of logical position ctx_len + path[k] go to
+ * position ctx_len + k (all are read before any is written).  Pools as
+ * tree_attn_fp8kv; layer l's pools start at k_pool + l*layer_stride and
+ * v_pool + l*layer_stride (bytes).  path / n_accepted as written by
+ * tree_accept_greedy (device memory, so the two calls need no host sync).
+ * Ids outside the pool or the tree are skipped and flagged
+ * NVFP4SK_ERR_OUT_OF_RANGE.  D <= 128, D % 8 == 0, page_size % 16 == 0. */
+NVFP4SK_API nvfp4sk_status kv_compact_accepted(uint8_t *k_pool, uint8_t *v_pool, int64_t layer_stride, int n_layers,
+                                               int Hkv, int D, int64_t n_pool_pages, int page_size,
+                                               const int32_t *page_table, int64_t ctx_len, const int32_t *path,
+                                               const int32_t *n_accepted, int T, nvfp4sk_stream_t stream);
 /* idx[r] = argmax_j x[r*ld + j] over bf16 values, lowest index on ties. */
 NVFP4SK_API size_t argmax_workspace_bytes(int64_t rows, int64_t n);
 NVFP4SK_API nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t ld, int32_t *idx, void *ws,

@@ -102,3 +102,113 @@ __global__ void __launch_bounds__(AMX_THREADS) argmax_rows_kernel(const __nv_bfl
 }
 
 }  // namespace nvfp4sk
+
+namespace nvfp4sk {
+
+// ---- greedy acceptance of the verified tree -------------------------------
+// One warp.  Node 0 (the root: the last accepted token) is accepted; node
+// i >= 1 is accepted when its parent is accepted and its draft token equals
+// the target's greedy choice after the parent.  The accepted path runs from
+// the root to the deepest accepted node (lowest index among equally deep
+// ones); the next token is the target's choice after that node.  A parent
+// array that is not topologically ordered (parent[0] != -1, or parent[i]
+// outside [0, i)) is flagged (site 501) and only the root is accepted.
+constexpr int ACC_MAX_T = 32;
+
+__global__ void __launch_bounds__(32) tree_accept_kernel(const int32_t *__restrict__ tok,
+                                                         const int32_t *__restrict__ amax,
+                                                         const int32_t *__restrict__ parent, int T,
+                                                         int32_t *__restrict__ path, int32_t *__restrict__ n_acc,
+                                                         int32_t *__restrict__ next_tok)
+{
+    __shared__ int s_par[ACC_MAX_T], s_tok[ACC_MAX_T], s_amax[ACC_MAX_T];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int i = threadIdx.x;
+    if (i < T) {
+        s_par[i] = parent[i];
+        s_tok[i] = tok[i];
+        s_amax[i] = amax[i];
+    }
+    __syncwarp();
+    if (i != 0) return;
+    bool bad = s_par[0] != -1;
+    for (int j = 1; j < T; ++j) bad |= s_par[j] < 0 || s_par[j] >= j;
+    uint32_t acc_mask = 1u;
+    int depth[ACC_MAX_T];
+    depth[0] = 0;
+    int end = 0;
+    if (!bad) {
+        for (int j = 1; j < T; ++j) {
+            const int p = s_par[j];
+            depth[j] = depth[p] + 1;
+            if (((acc_mask >> p) & 1u) && s_tok[j] == s_amax[p]) {
+                acc_mask |= 1u << j;
+                if (depth[j] > depth[end]) end = j;
+            }
+        }
+    } else {
+        report_error(ERRBIT_RANGE, 501);
+    }
+    const int n = depth[end] + 1;
+    for (int k = n - 1, a = end; k >= 0; --k, a = k >= 0 ? s_par[a] : a) path[k] = a;
+    *n_acc = n;
+    *next_tok = s_amax[end];
+}
+
+// ---- move the accepted tokens' K/V next to the context --------------------
+// Grid (layers, KV heads), one thread per dimension: the K and V bytes of the
+// accepted path's tokens (tree slots ctx_len + path[k]) are read first, then
+// written to positions ctx_len + k, in every layer.
+__global__ void __launch_bounds__(128) kv_compact_kernel(uint8_t *__restrict__ k_base, uint8_t *__restrict__ v_base,
+                                                         int64_t layer_stride, int Hkv, int D,
+                                                         int64_t n_pool_pages, int P,
+                                                         const int32_t *__restrict__ page_table, int64_t ctx_len,
+                                                         const int32_t *__restrict__ path,
+                                                         const int32_t *__restrict__ n_acc, int T)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int l = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+    const int n = min(max(*n_acc, 0), T);
+    uint8_t *kp = k_base + (int64_t)l * layer_stride, *vp = v_base + (int64_t)l * layer_stride;
+    uint8_t kr[ACC_MAX_T], vr[ACC_MAX_T];
+    bool ok = true;
+    auto locate = [&](int64_t pos, int64_t &pg, int &slot) {
+        pg = page_table[pos / P];
+        slot = (int)(pos % P);
+        return pg >= 0 && pg < n_pool_pages;
+    };
+#pragma unroll 1
+    for (int k = 0; k < n; ++k) {
+        const int node = path[k];
+        int64_t pg;
+        int slot;
+        if (node < 0 || node >= T || !locate(ctx_len + node, pg, slot)) {
+            if (d == 0) report_error(ERRBIT_RANGE, 502);
+            ok = false;
+            break;
+        }
+        if (d < D) {
+            kr[k] = kp[((pg * Hkv + h) * P + slot) * D + d];
+            vr[k] = vp[(pg * Hkv + h) * (int64_t)D * P + ((d >> 3) * (P >> 4) + (slot >> 4)) * 128 + (d & 7) * 16 + (slot & 15)];
+        }
+    }
+    __syncthreads();
+    if (!__syncthreads_and(ok ? 1 : 0)) return;
+#pragma unroll 1
+    for (int k = 0; k < n; ++k) {
+        int64_t pg;
+        int slot;
+        if (!locate(ctx_len + k, pg, slot)) {
+            if (d == 0) report_error(ERRBIT_RANGE, 502);
+            return;
+        }
+        if (d < D) {
+            kp[((pg * Hkv + h) * P + slot) * D + d] = kr[k];
+            vp[(pg * Hkv + h) * (int64_t)D * P + ((d >> 3) * (P >> 4) + (slot >> 4)) * 128 + (d & 7) * 16 + (slot & 15)] = vr[k];
+        }
+    }
+}
+
+}  // namespace nvfp4sk

@@ -607,6 +607,38 @@ nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, ui
                     "debug_encode_kernel");
 }
 
+nvfp4sk_status tree_accept_greedy(const int32_t *draft_tokens, const int32_t *target_argmax, const int32_t *parent,
+                                  int T, int32_t *path, int32_t *n_accepted, int32_t *next_token,
+                                  nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!draft_tokens || !target_argmax || !parent || !path || !n_accepted || !next_token)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (T < 1 || T > ACC_MAX_T) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= T <= 32");
+    return launched(launch(tree_accept_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream, 1, draft_tokens,
+                           target_argmax, parent, T, path, n_accepted, next_token),
+                    "tree_accept_kernel");
+}
+
+nvfp4sk_status kv_compact_accepted(uint8_t *k_pool, uint8_t *v_pool, int64_t layer_stride, int n_layers, int Hkv,
+                                   int D, int64_t n_pool_pages, int page_size, const int32_t *page_table,
+                                   int64_t ctx_len, const int32_t *path, const int32_t *n_accepted, int T,
+                                   nvfp4sk_stream_t stream)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    if (!k_pool || !v_pool || !page_table || !path || !n_accepted) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (n_layers < 1 || Hkv < 1 || D < 8 || D > 128 || D % 8 || page_size < 16 || page_size % 16 || T < 1 ||
+        T > ACC_MAX_T || ctx_len < 0 || n_pool_pages < 1 || layer_stride < 0)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "need n_layers, Hkv >= 1, 8 <= D <= 128, D %% 8 == 0, page_size %% 16 == 0, 1 <= T <= 32");
+    return launched(launch(kv_compact_kernel, dim3(n_layers, Hkv), dim3(128), 0, (cudaStream_t)stream, 1, k_pool,
+                           v_pool, layer_stride, Hkv, D, n_pool_pages, page_size, page_table, ctx_len, path,
+                           n_accepted, T),
+                    "kv_compact_kernel");
+}
+
 nvfp4sk_status nvfp4sk_debug_wait_timeout(nvfp4sk_stream_t stream)
 {
     DevInfo *d;

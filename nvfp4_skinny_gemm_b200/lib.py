@@ -60,6 +60,8 @@ _SIGS = {
     "nvfp4sk_get_option": (_i64, [_int]),
     "nvfp4sk_debug_encode": (_int, [_vp, _i64, _vp, _vp, _vp]),
     "nvfp4sk_debug_wait_timeout": (_int, [_vp]),
+    "tree_accept_greedy": (_int, [_vp, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
+    "kv_compact_accepted": (_int, [_vp, _vp, _i64, _int, _int, _int, _i64, _int, _vp, _i64, _vp, _vp, _int, _vp]),
 }
 
 
@@ -252,6 +254,26 @@ def kv_append(k_new, v_new, ld_new, T, k_pool, v_pool, page_table, ctx_len, k_sc
           v_new.data_ptr() if hasattr(v_new, "data_ptr") else v_new, ld_new, T, Hkv, D, k_pool.data_ptr(),
           v_pool.data_ptr(), n_pages, P, page_table.data_ptr(), int(ctx_len), k_scale.data_ptr(),
           v_scale.data_ptr(), _stream(stream))
+
+
+def tree_accept(draft_tokens, target_argmax, parent, out=None, stream=None):
+    """Greedy acceptance: returns device tensors (path i32 [T], n i32 [1], next i32 [1])."""
+    T = parent.numel()
+    if out is None:
+        dev = parent.device
+        out = (torch.empty(T, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
+               torch.empty(1, dtype=torch.int32, device=dev))
+    path, n, nxt = out
+    _call("tree_accept_greedy", draft_tokens.data_ptr(), target_argmax.data_ptr(), parent.data_ptr(), T,
+          path.data_ptr(), n.data_ptr(), nxt.data_ptr(), _stream(stream))
+    return out
+
+
+def kv_compact(k_base, v_base, layer_stride, n_layers, Hkv, D, n_pool_pages, P, page_table, ctx_len, path, n, T,
+               stream=None):
+    """Move the accepted tokens' K/V to ctx_len .. in every layer (see kv_compact_accepted)."""
+    _call("kv_compact_accepted", k_base, v_base, int(layer_stride), n_layers, Hkv, D, int(n_pool_pages), P,
+          page_table.data_ptr(), int(ctx_len), path.data_ptr(), n.data_ptr(), T, _stream(stream))
 
 
 def argmax(x, idx=None, ws=None, stream=None):

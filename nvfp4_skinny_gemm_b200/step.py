@@ -217,6 +217,16 @@ class VerifyModel:
         self._linear(self.q_h.buf, self.q_h.g, self.lm_head, self.logits)
         nv.argmax(self.logits, self.ids)
 
+    def accept(self, draft_tokens):
+        """Greedy acceptance after a step (self.ids = the target's token after each
+        node) and compaction of the accepted tokens' K/V next to the context in
+        every layer.  Returns device tensors (path, n_accepted, next_token)."""
+        out = nv.tree_accept(draft_tokens, self.ids, self.parent)
+        k0, v0 = self.kv[0, 0], self.kv[0, 1]
+        nv.kv_compact(k0.data_ptr(), v0.data_ptr(), self.kv[0].nbytes, self.n_layers, I.N_KV_HEADS, I.HEAD_DIM,
+                      self.n_pool, I.PAGE, self.page_table, self.L, out[0], out[1], self.T)
+        return out
+
     def _linear(self, act, g, lin, y, residual=None):
         nv.linear(act, g, self.T, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
 
