@@ -509,7 +509,7 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
         (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "x, w, act_prepared must be 16-byte aligned, codes 8-byte aligned");
     if (g_in)
-        return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows), dim3(RTHREADS), 0,
+        return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, RS_SPLIT), dim3(RS_THREADS), 0,
                                (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, n,
                                g_in, codes, scales, g_out, act_prepared),
                         "rmsnorm_quant_static_kernel");

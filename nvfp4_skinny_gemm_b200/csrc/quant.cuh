@@ -292,45 +292,47 @@ __global__ void __launch_bounds__(RTHREADS, 1)
 }
 
 // ---- static tensor scale: no grid-wide reduction, one launch --------------
-// RMSNorm + quantise with a given g: one CTA per row, each thread up to RNB
-// 16-blocks; only the row's sum of squares is reduced (within the CTA).
-__global__ void __launch_bounds__(RTHREADS)
+// RMSNorm + quantise with a given g: RSPLIT CTAs per row; each CTA reduces
+// the whole row's sum of squares (the row is 10 KB, read from L2 by every
+// CTA of the row) and encodes its share of the row's 16-blocks, one block per
+// thread.
+constexpr int RS_SPLIT = 4;
+constexpr int RS_THREADS = 128;
+__global__ void __launch_bounds__(RS_THREADS)
     rmsnorm_quant_static_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
                                 int64_t n, const float *__restrict__ g_in, uint8_t *__restrict__ codes,
                                 uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
 {
-    __shared__ float s_red[33];
+    __shared__ float s_red[RS_THREADS / 32];
     pdl_wait();
     pdl_launch_dependents();
     const int64_t r = blockIdx.x;
     const int64_t kb = n / 16;
-    float v[RNB][16];
+    const __nv_bfloat16 *xr = x + r * n;
     float ss = 0.f;
+    for (int64_t c = threadIdx.x; c < kb; c += RS_THREADS) {
+        float v[16];
+        load16<__nv_bfloat16>(xr + c * 16, v);
 #pragma unroll
-    for (int j = 0; j < RNB; ++j) {
-        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
-        if (c < kb) {
-            load16<__nv_bfloat16>(x + r * n + c * 16, v[j]);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) ss += v[j][k] * v[j][k];
-        }
+        for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
     }
-    const float g = *g_in;
-    const float tot = block_sum(ss, s_red);
+    ss = warp_sum(ss);
+    if (lane_id() == 0) s_red[warp_id()] = ss;
+    __syncthreads();
+    const float tot = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
     const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
-    if (r == 0 && threadIdx.x == 0) *g_out = g;
+    const float g = *g_in;
+    if (r == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+    const int64_t b0 = blockIdx.y * kb / RS_SPLIT, b1 = (blockIdx.y + 1) * kb / RS_SPLIT;
+    for (int64_t c = b0 + threadIdx.x; c < b1; c += RS_THREADS) {
+        float v[16], wv[16];
+        load16<__nv_bfloat16>(xr + c * 16, v);
+        load16<__nv_bfloat16>(w + c * 16, wv);
 #pragma unroll
-    for (int j = 0; j < RNB; ++j) {
-        const int64_t c = threadIdx.x + (int64_t)j * blockDim.x;
-        if (c < kb) {
-            float wv[16];
-            load16<__nv_bfloat16>(w + c * 16, wv);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) v[j][k] = round_bf16(__fmul_rn(__fmul_rn(v[j][k], inv), wv[k]));
-            uint2 pk;
-            const uint32_t sc = quant_block16(v[j], g, pk);
-            store_block(codes, scales, act, r, c, n, pk, sc);
-        }
+        for (int k = 0; k < 16; ++k) v[k] = round_bf16(__fmul_rn(__fmul_rn(v[k], inv), wv[k]));
+        uint2 pk;
+        const uint32_t sc = quant_block16(v, g, pk);
+        store_block(codes, scales, act, r, c, n, pk, sc);
     }
 }
 
