@@ -48,3 +48,18 @@ def test_header_is_plain_c():
     hdr = lib.HEADER
     r = subprocess.run(["gcc", "-std=c99", "-fsyntax-only", "-x", "c", hdr], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_binding_arity_matches_header():
+    """Every ctypes signature of the binding has as many arguments as the C
+    declaration in include/nvfp4sk.h (a missing one shifts the stream handle)."""
+    import re
+    from nvfp4_skinny_gemm_b200 import lib
+    txt = open(lib.HEADER).read()
+    seen = 0
+    for m in re.finditer(r"NVFP4SK_API [^(]*?\b([a-z_0-9]+)\(([^)]*)\);", txt, re.S):
+        name, args = m.group(1), m.group(2).strip()
+        n = 0 if args in ("", "void") else len(args.split(","))
+        assert len(lib._SIGS[name][1]) == n, (name, n, len(lib._SIGS[name][1]))
+        seen += 1
+    assert seen == len(lib._SIGS)
