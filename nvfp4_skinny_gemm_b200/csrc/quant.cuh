@@ -304,8 +304,8 @@ __global__ void __launch_bounds__(RS_THREADS)
                                 uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
 {
     __shared__ float s_red[RS_THREADS / 32];
-    pdl_wait();
     pdl_launch_dependents();
+    pdl_wait();
     const int64_t r = blockIdx.x;
     const int64_t kb = n / 16;
     const __nv_bfloat16 *xr = x + r * n;
@@ -342,8 +342,8 @@ __global__ void __launch_bounds__(QBIG_THREADS_STATIC)
                                const float *__restrict__ g_in, uint8_t *__restrict__ codes,
                                uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
 {
-    pdl_wait();
     pdl_launch_dependents();
+    pdl_wait();
     const float g = *g_in;
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
     const int64_t kb = F / 16, nblk = rows * kb;
