@@ -19,8 +19,7 @@
  *   [OFP8] OCP 8-bit Floating Point Specification (OFP8), E4M3 ("fn": no
  *          infinities, S.1111.111 is NaN, max finite 448).
  * The pages name the formats but do not spell out the bit-level recipe; the
- * readings taken where they are silent are listed in the design doc and repeated
- * in the comments below.
+ * readings taken where they are silent are stated in the comments below.
  *
  * Arithmetic: fp64 throughout.  Where the quantisation recipe is defined as a
  * sequence of IEEE fp32 operations, each single fp32 operation is emulated by
@@ -354,7 +353,7 @@ EXPORT int oracle_kv_page_restore(const uint8_t *src_pool, const int32_t *src_id
 
 /* ------------------------------------------------------------------------ */
 /* Layer glue of the dense 27B-class verify step (not on the pages; the      */
-/* readings are listed in the design doc): RMSNorm, SwiGLU.                       */
+/* readings are stated with each function): RMSNorm, SwiGLU.                 */
 /* ------------------------------------------------------------------------ */
 
 /* y = x / sqrt(mean(x^2) + eps) * w, per row of length n. */
