@@ -11,8 +11,8 @@
  *   - section "NVFP4 and FP8: smaller weights, faster decoding": low-batch
  *     decode is DRAM-bandwidth bound; weights AND activations are NVFP4,
  *     the LM head included; the KV cache is FP8;
- *   - section "KV-cache reuse between agent steps": the runtime finds reused
- *     prompt prefixes and restores their cached attention KV pages;
+ *   - section "KV-cache reuse between agent steps": a prompt prefix seen before
+ *     is detected and its KV pages are copied back from the cache;
  *   - section "Tree multi-token prediction": candidates are organised into a
  *     16-node tree (8 draft steps, top-2 per depth) and verified in ONE
  *     forward pass of the target model.
@@ -252,8 +252,8 @@ NVFP4SK_API nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, i
                              const float *v_scale, nvfp4sk_stream_t stream);
 /* ------------------------------------------------------------------------
  * Greedy acceptance of the verified tree (section "Tree multi-token
- * prediction": the target model verifies the candidates in one pass and the
- * runtime accepts the matching path; greedy decoding makes it exact).
+ * prediction": all candidates are checked by one target pass and the path
+ * that agrees with the target is kept; with greedy decoding that is exact).
  * Node 0 (the root, the last accepted token) is accepted; node i >= 1 is
  * accepted when its parent is accepted and draft_tokens[i] ==
  * target_argmax[parent[i]] (target_argmax[j]: the target's greedy token after

@@ -237,9 +237,9 @@ def ancestors(parent, i):
 
 
 # ---------------------------------------------------------------- greedy tree acceptance
-# The step after the verify forward ("Tree multi-token prediction": the target
-# model verifies the tree's candidates in one pass and the runtime accepts the
-# matching path; temperature 0, so acceptance is exact): node 0 (the root, the
+# The step after the verify forward ("Tree multi-token prediction": one target
+# pass checks every candidate of the tree and the path that agrees with the
+# target is kept; at temperature 0 that is exact): node 0 (the root, the
 # last accepted token) is accepted; node i >= 1 is accepted when its parent is
 # accepted and its draft token equals the target's greedy choice after the
 # parent.  The accepted path ends at the deepest accepted node (lowest index
