@@ -13,6 +13,12 @@ between agent steps"); the 16-node tree is verified in one forward pass
 ("Tree multi-token prediction"); weights, activations and the LM head are
 NVFP4 and the cache is FP8 ("NVFP4 and FP8").
 
+Suffix prefill (VerifyModel.prefill) writes the K/V of the prompt tokens that
+the prefix cache does not hold ("KV-cache reuse between agent steps": only the
+new suffix is prefilled) through the same kernels, 16 tokens at a time: each
+group of 16 is a chain (causal) tree over everything before it, which is
+causal attention over the whole suffix split at group boundaries.
+
 All buffers are allocated once, so a step can be captured in a CUDA graph.
 """
 from __future__ import annotations
@@ -26,6 +32,17 @@ from . import inputs as I
 from . import lib as nv
 
 PAGE_BYTES = I.N_KV_HEADS * I.PAGE * I.HEAD_DIM      # one (layer, K|V, page) plane: 32 KB
+PREFILL_CHUNK = 16                                   # rows per skinny launch (linear M, attention T)
+
+
+def prefill_chunks(start: int, S: int, C: int = PREFILL_CHUNK):
+    """Row groups of a suffix prefill: (row0, rows, ctx_len) for rows
+    row0 .. row0+rows-1 of the S suffix tokens, which sit at positions
+    start+row0 ..; ctx_len = start+row0 is the context each group attends to
+    in full before its own causal chain."""
+    if start < 0 or S < 0 or C < 1:
+        raise ValueError("need start >= 0, S >= 0, C >= 1")
+    return [(r, min(C, S - r), start + r) for r in range(0, S, C)]
 
 
 class Linear:
@@ -227,8 +244,117 @@ class VerifyModel:
                       self.n_pool, I.PAGE, self.page_table, self.L, out[0], out[1], self.T)
         return out
 
-    def _linear(self, act, g, lin, y, residual=None):
-        nv.linear(act, g, self.T, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
+    def _linear(self, act, g, lin, y, residual=None, M=None):
+        nv.linear(act, g, self.T if M is None else M, lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
+
+    # ------------------------------------------------------------------ prefill
+    def _prefill_buffers(self, S):
+        """Per-suffix buffers, kept for later calls of up to the same length."""
+        pf = getattr(self, "_pf", None)
+        if pf is not None and pf["cap"] >= S:
+            return pf
+        H, F, Hq, Hkv, D, C = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM, PREFILL_CHUNK
+        cap = -(-S // C) * C
+        n = cap // C
+        dev = self.dev
+        pf = {
+            "cap": cap,
+            "qkv": torch.empty(cap, (Hq + 2 * Hkv) * D, dtype=torch.bfloat16, device=dev),
+            "attn": torch.empty(cap, Hq * D, dtype=torch.bfloat16, device=dev),
+            "gu": torch.empty(C, 2 * F, dtype=torch.bfloat16, device=dev),
+            "q_h": [Act(H, dev) for _ in range(n)],
+            "q_a": [Act(Hq * D, dev) for _ in range(n)],
+            "q_f": [Act(F, dev) for _ in range(n)],
+            "parent": torch.from_numpy(I.chain_parent(C)).to(dev),
+            "logits": torch.empty(1, I.VOCAB, dtype=torch.bfloat16, device=dev),
+            "ids": torch.empty(1, dtype=torch.int32, device=dev),
+        }
+        self._pf = pf
+        return pf
+
+    def prefill(self, h: torch.Tensor, start: int, layers=None):
+        """Prefill the S = h.shape[0] suffix tokens at positions start .. start+S-1.
+
+        h: bf16 [S, HIDDEN] (contiguous, on the model's device) holds the
+        tokens' input hidden states and is overwritten with the last layer's
+        output.  Every layer's K/V of the suffix lands in the paged FP8 cache
+        (positions start .. in the page table), so that a verify step at
+        ctx_len = start + S sees it.  Returns the device int32 [1] argmax of
+        the last token's logits (the token that follows the suffix), or None
+        without an LM head or for S == 0.
+
+        layers: the layers to run, in order (default all); the head runs only
+        when they end with the last layer.  Running range(0, k) and then
+        range(k, n_layers) gives the same result as one call.
+
+        Needs static activation scales (calibrate()): with them, quantising a
+        row does not depend on the other rows, so 16-row groups give the
+        result of one pass over all S rows.
+
+        Order inside a layer: each op runs over all row groups before the
+        next op starts, so a linear's weights are read from HBM once and
+        from L2 for the later groups; all groups' K/V are appended before any
+        group attends, and group c attends to the context (start + 16c
+        tokens, the earlier groups included) plus its own chain."""
+        if not self.static:
+            raise RuntimeError("prefill needs static activation scales: call calibrate() first")
+        S = h.shape[0]
+        if h.dtype != torch.bfloat16 or h.dim() != 2 or h.shape[1] != I.HIDDEN or not h.is_contiguous():
+            raise ValueError("h must be a contiguous bf16 [S, HIDDEN] tensor")
+        if start < 0 or start + S > self.n_log * I.PAGE:
+            raise ValueError(f"positions {start} .. {start + S - 1} exceed the page table "
+                             f"({self.n_log} pages of {I.PAGE})")
+        layers = range(self.n_layers) if layers is None else list(layers)
+        if any(not 0 <= l < self.n_layers for l in layers):
+            raise ValueError("layer index out of range")
+        if S == 0:
+            return None
+        pf = self._prefill_buffers(S)
+        groups = prefill_chunks(start, S)
+        qd = I.N_Q_HEADS * I.HEAD_DIM
+        kd = I.N_KV_HEADS * I.HEAD_DIM
+        qkv, attn, gu = pf["qkv"], pf["attn"], pf["gu"]
+        for l in layers:
+            lay, s0 = self.layers[l], l * self.SITES
+            kp, vp = self.k_pool(l), self.v_pool(l)
+            for c, (r, t, _) in enumerate(groups):
+                a = pf["q_h"][c]
+                nv.rmsnorm_quantize(h[r:r + t], self.norm_w[2 * l], self.eps, a.out, act=a.buf,
+                                    g_in=self._site(s0))
+                self._linear(a.buf, a.g, lay["qkv"], qkv[r:r + t], M=t)
+            nv.kv_append(qkv[:S, qd:], qkv[:S, qd + kd:], qkv.stride(0), S, kp, vp, self.page_table, start,
+                         self.k_scale[l], self.v_scale[l])
+            for c, (r, t, ctx) in enumerate(groups):
+                a = pf["q_a"][c]
+                nv.tree_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, pf["parent"], self.k_scale[l],
+                             self.v_scale[l], out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS,
+                             g_act=self._site(s0 + 1), act=a.buf)
+                self._linear(a.buf, self._site(s0 + 1), lay["o"], h[r:r + t], residual=h[r:r + t], M=t)
+                a = pf["q_h"][c]
+                nv.rmsnorm_quantize(h[r:r + t], self.norm_w[2 * l + 1], self.eps, a.out, act=a.buf,
+                                    g_in=self._site(s0 + 2))
+            for c, (r, t, _) in enumerate(groups):
+                a, f = pf["q_h"][c], pf["q_f"][c]
+                self._linear(a.buf, a.g, lay["gate_up"], gu[:t], M=t)
+                nv.swiglu_quantize(gu[:t], f.out, act=f.buf, g_in=self._site(s0 + 3))
+            for c, (r, t, _) in enumerate(groups):
+                f = pf["q_f"][c]
+                self._linear(f.buf, f.g, lay["down"], h[r:r + t], residual=h[r:r + t], M=t)
+        if self.lm_head is None or len(layers) == 0 or layers[-1] != self.n_layers - 1:
+            return None
+        i = self.n_layers * self.SITES
+        a = pf["q_h"][0]
+        nv.rmsnorm_quantize(h[S - 1:S], self.norm_w[-1], self.eps, a.out, act=a.buf, g_in=self._site(i))
+        self._linear(a.buf, a.g, self.lm_head, pf["logits"], M=1)
+        nv.argmax(pf["logits"], pf["ids"])
+        return pf["ids"]
+
+    def prefill_launches(self, S):
+        """Kernel launches of prefill(S rows): per layer and row group norm-q,
+        qkv, attention split + combine, o, norm-q, gate_up, swiglu-q, down,
+        plus one K/V append per layer; then the head on the last row."""
+        n = len(prefill_chunks(0, S))
+        return 0 if S == 0 else self.n_layers * (9 * n + 1) + (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     def step(self, restore=True):
         """One verify step on the current self.h / self.parent; result in self.ids."""

@@ -1,0 +1,123 @@
+"""Suffix prefill on the GPU (VerifyModel.prefill): S prompt tokens that the
+prefix cache does not hold go through every layer 16 rows at a time, each
+group attending to the context before it (earlier groups included) plus its
+own causal chain.
+
+(1) Per layer, teacher-forced against the oracle run over all S rows at once
+    (no groups): RMSNorm + NVFP4 with the static site scales, the NVFP4
+    linears with M = S, the FP8 append of the S tokens' K/V (bit-exact pool),
+    causal attention as ONE chain of S tokens after the context, SwiGLU.  The
+    bars are those of the one-layer verify test (rel-Frobenius 1e-2 on the
+    composed outputs; attention 2e-3 + 2^-8 |o| against the oracle fed the
+    GPU's own Q and cache).  S = 20 spans a full group and a ragged one.
+(2) The whole call with the LM head: the returned token is the first argmax
+    of the last row's logits; two calls over layer ranges [0, 1) and [1, 2)
+    give the bits of one call; a second run gives the same bits.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import cuda, rel_fro
+from nvfp4_skinny_gemm_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+def _bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def _calibrated(L, weights, lm_head):
+    from nvfp4_skinny_gemm_b200.step import VerifyModel
+    m = VerifyModel(n_layers=2, ctx_len=L, T=I.TREE_NODES, weights=weights, lm_head=lm_head)
+    m.parent.copy_(torch.from_numpy(I.tree_parent(4)))
+    m.restore()
+    m.h.copy_(I.bf16_normal(4, 300, (I.TREE_NODES, I.HIDDEN)) * 0.5)
+    m.calibrate(restore=False)
+    m.restore()
+    return m
+
+
+def test_prefill_layers_teacher_forced(oracle):
+    cuda()
+    L, S = 1024, 20
+    start = L - S
+    m = _calibrated(L, "host", lm_head=False)
+    G = m.G.cpu().numpy()
+    hs = (I.bf16_normal(4, 301, (S, I.HIDDEN)) * 0.5).cuda()
+    ones = np.ones(I.HIDDEN, np.float32)
+    qd, kd = I.N_Q_HEADS * I.HEAD_DIM, I.N_KV_HEADS * I.HEAD_DIM
+    pt = m.page_table_h
+    for l in range(m.n_layers):
+        s0 = l * m.SITES
+        kp = m.k_pool(l).cpu().numpy().copy()
+        vp = m.v_pool(l).cpu().numpy().copy()
+        h = hs.float().cpu().numpy()
+        assert m.prefill(hs, start, layers=[l]) is None
+        torch.cuda.synchronize()
+        qkv_gpu = m._pf["qkv"][:S].float().cpu().numpy()
+        attn_gpu = m._pf["attn"][:S].float().cpu().numpy()
+        h2_gpu = hs.float().cpu().numpy()
+
+        wq = {name: oracle.quantize(I.weight_fp32(4, t, N, K, sub=l))
+              for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items())}
+
+        def lin(x_bf16, name, site):
+            ac, asc, ga = oracle.quantize(x_bf16, g_in=float(G[site]))
+            return oracle.linear(ac, asc, ga, *wq[name])
+
+        y1 = _bf16(oracle.rmsnorm(h, ones, eps=m.eps))
+        qkv = _bf16(lin(y1, "qkv", s0))
+        assert rel_fro(qkv_gpu, qkv) <= 1e-2, (l, rel_fro(qkv_gpu, qkv))
+        ks, vs = m.k_scale[l].cpu().numpy(), m.v_scale[l].cpu().numpy()
+        oracle.kv_append(qkv_gpu[:, qd:qd + kd].reshape(S, I.N_KV_HEADS, I.HEAD_DIM),
+                         qkv_gpu[:, qd + kd:].reshape(S, I.N_KV_HEADS, I.HEAD_DIM), kp, vp, pt, start, ks, vs)
+        assert np.array_equal(m.k_pool(l).cpu().numpy(), kp)
+        assert np.array_equal(m.v_pool(l).cpu().numpy(), vp)
+        # one causal chain of all S tokens after the context, no groups
+        a = oracle.tree_attn(qkv_gpu[:, :qd].reshape(S, I.N_Q_HEADS, I.HEAD_DIM), kp, vp, pt, start,
+                             I.chain_parent(S), ks, vs)
+        err_a = np.abs(attn_gpu.reshape(a.shape) - a)
+        assert np.all(err_a <= 2e-3 + 2.0 ** -8 * np.abs(a)), (l, err_a.max())
+        h1 = _bf16(h + lin(attn_gpu, "o", s0 + 1))
+        y2 = _bf16(oracle.rmsnorm(h1, ones, eps=m.eps))
+        gu = _bf16(lin(y2, "gate_up", s0 + 2))
+        s = _bf16(oracle.swiglu(gu))
+        h2 = _bf16(h1 + lin(s, "down", s0 + 3))
+        err = rel_fro(h2_gpu, h2)
+        print(f"prefill layer {l}: rel-Frobenius {err:.2e}")
+        assert err <= 1e-2 and np.isfinite(h2_gpu).all()
+
+
+def test_prefill_head_ranges_determinism():
+    cuda()
+    L, S = 1024, 37
+    start = L - S
+    m = _calibrated(L, "device", lm_head=True)
+    h0 = (I.bf16_normal(4, 302, (S, I.HIDDEN)) * 0.5).cuda()
+    kv0 = m.kv.clone()
+
+    def run(ranges):
+        m.kv.copy_(kv0)
+        h = h0.clone()
+        for r in ranges:
+            ids = m.prefill(h, start, layers=r)
+        torch.cuda.synchronize()
+        return h, ids.clone(), m.kv.clone(), m._pf["logits"].clone()
+
+    h_a, ids_a, kv_a, lg_a = run([None])
+    h_b, ids_b, kv_b, lg_b = run([None])
+    h_c, ids_c, kv_c, lg_c = run([range(0, 1), range(1, 2)])
+    assert torch.equal(h_a, h_b) and torch.equal(kv_a, kv_b) and torch.equal(ids_a, ids_b)
+    assert torch.equal(h_a, h_c) and torch.equal(kv_a, kv_c) and torch.equal(ids_a, ids_c)
+    assert torch.isfinite(lg_a.float()).all()
+    lg = lg_a.float().cpu().numpy()[0]
+    assert int(ids_a.cpu()[0]) == int(np.flatnonzero(lg == lg.max())[0])
+    # only the suffix's cache positions changed, in both layers
+    changed = (kv_a != kv0).cpu().numpy()             # [layers, 2, pool pages, 32 KB]
+    P = I.PAGE
+    pages = {int(m.page_table_h[p // P]) for p in range(start, L)}
+    assert changed[:, :, sorted(pages)].any(axis=(2, 3)).all()
+    others = [pg for pg in range(m.n_pool) if pg not in pages]
+    assert not changed[:, :, others].any()

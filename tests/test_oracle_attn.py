@@ -8,7 +8,11 @@
 (5) pure-Python brute force at L=3, D=8, T=4;
 (6) a random permutation of the physical pool (with the page table) changes
     nothing; bytes outside the visible positions change nothing;
-(7) the tiled V plane layout: hand-computed byte offsets, a bijection.
+(7) the tiled V plane layout: hand-computed byte offsets, a bijection;
+(8) causal attention over a suffix of S tokens, split into row groups of at
+    most 16 that each attend to the context before them plus their own chain
+    (the suffix prefill's decomposition), gives the same rows as the chain of
+    all S tokens at once, bit for bit.
 """
 import math
 
@@ -159,3 +163,25 @@ def test_v_plane_layout():
     for D, P in [(8, 16), (16, 32), (128, 64)]:
         o = inputs.v_plane_offsets(D, P)
         assert sorted(o.ravel().tolist()) == list(range(D * P))
+
+
+def test_suffix_groups_equal_whole_causal(oracle):
+    """Row group (r, t) of a causal suffix sees positions < start + r + i for
+    its row i, which is a chain of t tokens after a context of start + r: the
+    oracle visits the same positions in the same order, so the results match
+    exactly.  S = 37 gives two full groups and a ragged one."""
+    from nvfp4_skinny_gemm_b200.step import prefill_chunks
+    S, Hq, Hkv, D, P, start = 37, 4, 2, 16, 16, 29
+    cache = inputs.kv_cache(104, start, T=S, Hkv=Hkv, D=D, P=P, extra_pages=2)
+    q = inputs.query_bf16(104, S, Hq, D).float().numpy()
+    whole = _run(oracle, q, cache, inputs.chain_parent(S))
+    groups = prefill_chunks(start, S)
+    assert [t for _, t, _ in groups] == [16, 16, 5]
+    for r, t, ctx in groups:
+        part = oracle.tree_attn(q[r:r + t], cache.k_pool, cache.v_pool, cache.page_table, ctx,
+                                inputs.chain_parent(t), cache.k_scale, cache.v_scale)
+        assert np.array_equal(part, whole[r:r + t]), (r, t)
+    # the check has teeth: rows that skip the earlier rows of their own group differ
+    wrong = oracle.tree_attn(q[16:32], cache.k_pool, cache.v_pool, cache.page_table, start + 16,
+                             np.full(16, -1, np.int32), cache.k_scale, cache.v_scale)
+    assert not np.allclose(wrong, whole[16:32])
