@@ -10,6 +10,10 @@ the step's inputs (16 hidden rows + parent array, pinned) and the
 device->host read of the 16 argmax ids.  Weights (11.4 GB) far exceed L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+`--prefill S` times instead the suffix prefill of the last S prompt tokens
+(positions ctx - S .. ctx - 1, after the restored prefix) through all layers
+plus the last token's LM head, one CUDA graph per prefill, on one GPU.
 """
 from __future__ import annotations
 
@@ -43,6 +47,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--chain", type=int, default=0,
                     help="verify a linear-MTP chain of this many tokens instead of the 16-node tree")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time the suffix prefill of this many tokens instead of the verify step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
@@ -365,6 +371,90 @@ def run_ours(args, world, rank, local):
     del graph, lin_graph
 
 
+# ------------------------------------------------------------------ suffix prefill
+def run_prefill(args):
+    """Suffix prefill of S = args.prefill tokens after ctx - S cached tokens,
+    timed with CUDA events around graph replays (weights far exceed L2).
+
+    Roofline: the FLOPs the prefill must do (the NVFP4 linears over S rows, the
+    LM head over the last row, QK^T and PV of the causal attention) at the
+    tensor peaks of their types (FP4 linears, FP8 attention: the measured
+    sustained bf16 GEMM peak times the nominal ratios 4 and 2)."""
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    from nvfp4_skinny_gemm_b200.step import VerifyModel
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    S, L = args.prefill, args.ctx
+    start = L - S
+    model = VerifyModel(n_layers=args.layers, ctx_len=L, weights="device", device=dev)
+    h_in = (I.bf16_normal(4, 303, (S, I.HIDDEN)) * 0.5).to(dev)
+    h = torch.empty_like(h_in)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        model.h.copy_(I.bf16_normal(4, 300, (I.TREE_NODES, I.HIDDEN)).to(dev))
+        model.parent.copy_(torch.from_numpy(I.tree_parent(4)).to(dev))
+        model.step()                                       # eager: allocates workspaces
+        model.calibrate()                                  # restore + one dynamic-scale step
+        h.copy_(h_in)
+        model.prefill(h, start)                            # eager: allocates the prefill buffers
+        torch.cuda.synchronize()
+        rc, site = nv.device_status(stream)
+        assert rc == 0, f"device status {rc} at site {site}"
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            h.copy_(h_in)
+            ids = model.prefill(h, start)
+        for _ in range(max(3, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        clocks = Clocks(dev)
+        time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        t = e0.elapsed_time(e1) * 1e-3 / args.steps
+        rc, site = nv.device_status(stream)
+        assert rc == 0, f"device status {rc} at site {site}"
+        assert ids is not None and 0 <= int(ids.cpu()[0]) < I.VOCAB
+
+    lin_flops = 2.0 * S * sum(N * K for (K, N) in I.LAYER_LINEARS.values()) * args.layers \
+        + 2.0 * I.VOCAB * I.HIDDEN
+    visible = S * (start + 1) + S * (S - 1) / 2                    # sum over rows of the positions seen
+    attn_flops = 4.0 * I.HEAD_DIM * I.N_Q_HEADS * visible * args.layers
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    bf16 = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    kind = "measured" if "bf16_tflops_sustained" in peaks else "fallback"
+    ideal = lin_flops / (4 * bf16 * 1e12) + attn_flops / (2 * bf16 * 1e12)
+    flops = lin_flops + attn_flops
+    line = {
+        "metric": "suffix prefill tokens/s", "value": S / t, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate); fp8 e4m3 KV", "data": "synthetic",
+        "config": {"workload": f"{args.layers}-layer suffix prefill of {S} tokens after {start} cached tokens, "
+                               f"16-row groups through the skinny kernels, LM head on the last token",
+                   "layers": args.layers, "ctx": L, "suffix": S, "parallelism": "single GPU",
+                   "l2": "inputs larger than L2 (11.4 GB of weights)"},
+        "roofline": {"bound": "tensor", "achieved": round(flops / t / 1e12, 1),
+                     "peak": round(flops / ideal / 1e12, 1), "unit": "TFLOP/s", "frac": round(ideal / t, 4),
+                     "peak_source": f"{kind} sustained bf16 GEMM x 4 (FP4 linears) and x 2 (FP8 attention), "
+                                    f"weighted by their FLOPs",
+                     "linear_tflop": round(lin_flops / 1e12, 2), "attention_tflop": round(attn_flops / 1e12, 2),
+                     "traffic": None},
+        "clocks": clk,
+        "gpu_launches": model.prefill_launches(S) * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+
+
 # ------------------------------------------------------------------ single-kernel cases
 def run_kernel_case(args):
     """A few launches of one kernel on a small case (a few GB at most): the
@@ -430,6 +520,9 @@ def main():
     if args.kernel_case:
         torch.cuda.set_device(0)
         run_kernel_case(args)
+        return
+    if args.prefill > 0 and args.impl == "ours":
+        run_prefill(args)
         return
     world, rank, local = dist_setup(args)
     try:
