@@ -86,12 +86,16 @@ class VerifyModel:
     seeded per layer) -- same distribution as the host generator, used for
     timing; weights="host": the seeded numpy generator of `inputs` (layer l,
     tensor t -> inputs.weight_fp32(4, t, N, K, sub=l)), which the oracle
-    reproduces."""
+    reproduces.
+
+    first_layer: the model holds layers first_layer .. first_layer+n_layers-1
+    of the stack (their weights; the cache and the scales are the slice's
+    own), e.g. one layer deep in the 64-layer stack for a per-layer check."""
 
     SITES = 4      # quantisation sites per layer: norm1, attention out, norm2, SwiGLU
 
     def __init__(self, n_layers=I.N_LAYERS, ctx_len=I.CTX_MAX, T=I.TREE_NODES, weights="device",
-                 prefix_frac=0.96, device="cuda", lm_head=True, seed=42):
+                 prefix_frac=0.96, device="cuda", lm_head=True, seed=42, first_layer=0):
         self.dev = torch.device(device)
         # activation tensor scales: dynamic (amax/2688 per call) until calibrate()
         # turns them into static per-site scales, as a calibrated checkpoint has
@@ -102,7 +106,7 @@ class VerifyModel:
         H, F, Hq, Hkv, D, P = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM, I.PAGE
         self.layers = []
         gen = torch.Generator(device=self.dev)
-        for l in range(n_layers):
+        for l in range(first_layer, first_layer + n_layers):
             lay = {}
             for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items()):
                 if weights == "host":

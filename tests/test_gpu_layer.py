@@ -2,6 +2,8 @@
 the 64-layer stack run through the library (VerifyModel.layer) against the
 same layer composed from the oracle's pieces on the same bf16 input, the same
 NVFP4 weights (quantised from the same fp32 values) and the same FP8 cache.
+Layers 0 (1,024 cached tokens, both scale modes, tree and chain), 31 (8,192)
+and 63 (23,552): a one-layer model holding that layer's weights.
 
 The oracle side follows the layer definition step by step:
   y1 = bf16(RMSNorm(h)), qkv = bf16(NVFP4(y1) x W_qkv^T), FP8 append of the
@@ -33,14 +35,15 @@ def _bf16(x):
     return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
 
 
-@pytest.mark.parametrize("static,T,chain", [(False, 16, False), (True, 16, False), (True, 4, True)])
-def test_one_layer_teacher_forced(oracle, static, T, chain):
+@pytest.mark.parametrize("static,T,chain,L,layer", [(False, 16, False, 1024, 0), (True, 16, False, 1024, 0),
+                                                   (True, 4, True, 1024, 0), (True, 16, False, 8192, 31),
+                                                   (True, 16, False, 23552, 63)])
+def test_one_layer_teacher_forced(oracle, static, T, chain, L, layer):
     """16-node tree (the verify step) and a linear-MTP chain of 4 tokens (the
     pages' baseline variant) through the same kernels."""
     cuda()
     from nvfp4_skinny_gemm_b200.step import VerifyModel
-    L = 1024
-    m = VerifyModel(n_layers=1, ctx_len=L, T=T, weights="host", lm_head=False)
+    m = VerifyModel(n_layers=1, ctx_len=L, T=T, weights="host", lm_head=False, first_layer=layer)
     h0 = I.bf16_normal(4, 300, (T, I.HIDDEN)) * 0.5
     parent = I.chain_parent(T) if chain else I.tree_parent(4)
     m.parent.copy_(torch.from_numpy(parent))
@@ -61,7 +64,7 @@ def test_one_layer_teacher_forced(oracle, static, T, chain):
     # ---- oracle composition
     wq = {}
     for t, (name, (K, N)) in enumerate(I.LAYER_LINEARS.items()):
-        wq[name] = oracle.quantize(I.weight_fp32(4, t, N, K, sub=0))
+        wq[name] = oracle.quantize(I.weight_fp32(4, t, N, K, sub=layer))
 
     def lin(x_bf16, name, site):
         ac, asc, ga = oracle.quantize(x_bf16, g_in=float(G[site]) if static else None)
@@ -96,6 +99,6 @@ def test_one_layer_teacher_forced(oracle, static, T, chain):
     s = _bf16(oracle.swiglu(gu))
     h2 = _bf16(h1 + lin(s, "down", 3))
     err = rel_fro(h2_gpu, h2)
-    print(f"layer parity ({'static' if static else 'dynamic'} scales): rel-Frobenius {err:.2e}")
+    print(f"layer {layer} at {L} tokens ({'static' if static else 'dynamic'} scales): rel-Frobenius {err:.2e}")
     assert err <= 1e-2
     assert np.isfinite(h2_gpu).all()
