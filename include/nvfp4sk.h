@@ -24,7 +24,10 @@
  *     stated otherwise; the library allocates nothing per call.
  *   - Calls are asynchronous on `stream` (a cudaStream_t) and return before
  *     the GPU work ends.  Host-side argument checks return an error code and
- *     launch nothing.  Device-side problems (a page id out of range, a wait
+ *     launch nothing; they run before the current device is looked up, so a
+ *     bad argument reports the same code with or without a usable GPU, and a
+ *     well-formed call without an sm_100 device returns NVFP4SK_ERR_DEVICE
+ *     (or NVFP4SK_ERR_CUDA when no device is visible).  Device-side problems (a page id out of range, a wait
  *     that ran out) never trap: the kernel skips the access, records the
  *     problem in a device error word and returns; nvfp4sk_get_device_status()
  *     reports and clears it.

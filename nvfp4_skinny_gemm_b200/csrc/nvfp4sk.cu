@@ -266,8 +266,6 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
                                   const float *g_in, uint8_t *codes, uint8_t *scales, float *g_out,
                                   uint8_t *act_prepared, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!x || !g_out || (!act_prepared && (!codes || !scales)))
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer (need codes+scales and/or act_prepared)");
     if (x_dtype != NVFP4SK_BF16 && x_dtype != NVFP4SK_FP32) return fail(NVFP4SK_ERR_INVALID_ARG, "bad dtype");
@@ -280,6 +278,8 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
         (reinterpret_cast<uintptr_t>(act_prepared) & 15u) != 0)
         return fail(NVFP4SK_ERR_MISALIGNED,
                     "x, its row stride and act_prepared must be 16-byte aligned, codes 8-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t nblk = rows * (K / 16);
     if (nblk <= QSMALL_MAX_BLOCKS && !g_in) {
@@ -318,13 +318,13 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
 nvfp4sk_status nvfp4_prepare_act(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,
                                  uint8_t *act_prepared, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!codes || !scales || !act_prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (rows < 1 || rows > 16 || K < 64 || K % 64 != 0)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, K %% 64 == 0");
     if ((reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "codes 8-byte aligned, act_prepared 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int64_t nblk = rows * (K / 16);
     const int grid = (int)std::min<int64_t>(cdiv(nblk, 256), 4 * d->sms);
     return launched(launch(prepare_act_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, codes, scales, rows,
@@ -337,11 +337,11 @@ size_t nvfp4_prepared_weight_bytes(int64_t N, int64_t K) { return (size_t)cdiv(N
 nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K,
                                     uint8_t *prepared, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!codes || !scales || !prepared) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (N < 1 || K < 64 || K % 64 != 0) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need N >= 1, K %% 64 == 0");
     if (!al16(prepared)) return fail(NVFP4SK_ERR_MISALIGNED, "prepared buffer must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int64_t total = (int64_t)nvfp4_prepared_weight_bytes(N, K);
     const int grid = (int)std::min<int64_t>(cdiv(total, 256), 16 * d->sms);
     return launched(launch(prepare_weight_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, codes, scales, N,
@@ -364,13 +364,13 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t
                             const float *g_w, int64_t N, int64_t K, const void *residual, void *y, int64_t ldy,
                             void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!a_prepared || !g_a || !w_prepared || !g_w || !y) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (M < 1 || M > 16 || N < 1 || N > LIN_MAX_NT * 128 || K < 64 || K % 64 != 0 || ldy < N)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, 1 <= N <= 524288, K %% 64 == 0, ldy >= N");
     if (!al16(a_prepared) || !al16(w_prepared))
         return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int64_t NT = cdiv(N, 128), KC = cdiv(K, LIN_KC), U = NT * KC;
     const int G = linear_grid(*d, U);
     const size_t need = linear_ws(G, NT);
@@ -413,8 +413,6 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
                                const float *g_act, uint8_t *act_prepared, void *ws, size_t ws_bytes,
                                nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!q || !k_pool || !v_pool || !page_table || !parent || !k_scale || !v_scale || !out)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_T || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > 8 ||
@@ -424,6 +422,8 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool) || !al16(act_prepared))
         return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes), the pools and act_prepared must be 16-byte aligned");
     if (act_prepared && !g_act) return fail(NVFP4SK_ERR_INVALID_ARG, "act_prepared needs the static scale g_act");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int64_t n_log = cdiv(ctx_len + T, ATT_P);
     const int group = Hq / Hkv;
     const int S = attn_splits(*d, Hkv, n_log);
@@ -468,13 +468,13 @@ nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_t *src_ids, 
                                const int32_t *dst_ids, int64_t n, int64_t page_bytes, int64_t n_src_pages,
                                int64_t n_dst_pages, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (n == 0) return NVFP4SK_OK;
     if (!src_pool || !src_ids || !dst_pool || !dst_ids) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (n < 0 || page_bytes < 16 || page_bytes % 16 != 0 || n_src_pages < 1 || n_dst_pages < 1)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need n >= 0, page_bytes %% 16 == 0");
     if (!al16(src_pool) || !al16(dst_pool)) return fail(NVFP4SK_ERR_MISALIGNED, "pools must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     RestoreParams p;
     p.src = src_pool;
     p.src_ids = src_ids;
@@ -499,8 +499,6 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
                                       uint8_t *act_prepared, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!x || !w || !g_out || (!act_prepared && (!codes || !scales)))
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (rows < 1 || rows > 16 || n < 64 || n % 64 != 0 || n > (int64_t)RTHREADS * RNB * 16)
@@ -508,6 +506,8 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
     if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
         (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "x, w, act_prepared must be 16-byte aligned, codes 8-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     if (g_in)
         return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, RS_SPLIT), dim3(RS_THREADS), 0,
                                (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, n,
@@ -525,14 +525,14 @@ nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, co
                                      nvfp4sk_stream_t stream)
 {
     (void)ws; (void)ws_bytes;
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!gu || !g_out || (!act_prepared && (!codes || !scales)))
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (rows < 1 || rows > 16 || F < 64 || F % 64 != 0 || rows * (F / 16) > QSMALL_MAX_BLOCKS)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, F %% 64 == 0, rows*F <= 524288");
     if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "gu, act_prepared must be 16-byte aligned, codes 8-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int64_t nblk = rows * (F / 16);
     if (g_in)
         return launched(launch(swiglu_quant_static_kernel,
@@ -552,13 +552,13 @@ nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_ne
                              const int32_t *page_table, int64_t ctx_len, const float *k_scale, const float *v_scale,
                              nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!k_new || !v_new || !k_pool || !v_pool || !page_table || !k_scale || !v_scale)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (T < 1 || Hkv < 1 || D < 8 || D % 8 || page_size < 16 || page_size % 16 || ctx_len < 0 ||
         ld_new < (int64_t)Hkv * D || n_pool_pages < 1)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need T, Hkv >= 1, D %% 8 == 0, page_size %% 16 == 0, ld_new >= Hkv*D");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     return launched(launch(kv_append_kernel, dim3(T, Hkv), dim3(128), 0, (cudaStream_t)stream, 1,
                            (const __nv_bfloat16 *)k_new, (const __nv_bfloat16 *)v_new, ld_new, Hkv, D, k_pool,
                            v_pool, n_pool_pages, page_size, page_table, ctx_len, k_scale, v_scale),
@@ -578,11 +578,11 @@ size_t argmax_workspace_bytes(int64_t rows, int64_t n)
 nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t ld, int32_t *idx, void *ws,
                                 size_t ws_bytes, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!x || !idx) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (rows < 1 || rows > AMX_MAX_ROWS || n < 1 || n > INT32_MAX || ld < n)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 4096, ld >= n");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const size_t need = argmax_workspace_bytes(rows, n);
     if (!ws || ws_bytes < need) return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes", need);
     const int nch = argmax_chunks(n);
@@ -598,10 +598,10 @@ nvfp4sk_status argmax_rows_bf16(const void *x, int64_t rows, int64_t n, int64_t 
 nvfp4sk_status nvfp4sk_debug_encode(const float *x, int64_t n, uint8_t *e2m1, uint8_t *e4m3,
                                     nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!x || n < 0) return fail(NVFP4SK_ERR_INVALID_ARG, "bad arguments");
     if (n == 0) return NVFP4SK_OK;
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     const int grid = (int)std::min<int64_t>(cdiv(n, 256), 16 * d->sms);
     return launched(launch(debug_encode_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream, 1, x, n, e2m1, e4m3),
                     "debug_encode_kernel");
@@ -611,11 +611,11 @@ nvfp4sk_status tree_accept_greedy(const int32_t *draft_tokens, const int32_t *ta
                                   int T, int32_t *path, int32_t *n_accepted, int32_t *next_token,
                                   nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!draft_tokens || !target_argmax || !parent || !path || !n_accepted || !next_token)
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (T < 1 || T > ACC_MAX_T) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= T <= 32");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     return launched(launch(tree_accept_kernel, dim3(1), dim3(32), 0, (cudaStream_t)stream, 1, draft_tokens,
                            target_argmax, parent, T, path, n_accepted, next_token),
                     "tree_accept_kernel");
@@ -626,13 +626,13 @@ nvfp4sk_status kv_compact_accepted(uint8_t *k_pool, uint8_t *v_pool, int64_t lay
                                    int64_t ctx_len, const int32_t *path, const int32_t *n_accepted, int T,
                                    nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!k_pool || !v_pool || !page_table || !path || !n_accepted) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (n_layers < 1 || Hkv < 1 || D < 8 || D > 128 || D % 8 || page_size < 16 || page_size % 16 || T < 1 ||
         T > ACC_MAX_T || ctx_len < 0 || n_pool_pages < 1 || layer_stride < 0)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
                     "need n_layers, Hkv >= 1, 8 <= D <= 128, D %% 8 == 0, page_size %% 16 == 0, 1 <= T <= 32");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     return launched(launch(kv_compact_kernel, dim3(n_layers, Hkv), dim3(128), 0, (cudaStream_t)stream, 1, k_pool,
                            v_pool, layer_stride, Hkv, D, n_pool_pages, page_size, page_table, ctx_len, path,
                            n_accepted, T),
@@ -699,8 +699,6 @@ nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const float *g_a,
                                     const uint8_t *w_prepared, const float *g_w, int64_t N, int64_t K,
                                     const void *residual, void *y, int64_t ldy, nvfp4sk_stream_t stream)
 {
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
     if (!a_prepared || !g_a || !w_prepared || !g_w || !y) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
     if (M < 1 || M > 16 || N < 1 || K < 64 || K % 64 != 0 || ldy < N)
         return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, N >= 1, K %% 64 == 0, ldy >= N");
@@ -710,6 +708,8 @@ nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const float *g_a,
                     (long long)N, (long long)(LIN_MAX_NT * 128));
     if (!al16(a_prepared) || !al16(w_prepared))
         return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
     uint8_t *scratch = nullptr;
     if (int rc = noalloc_scratch(&scratch)) return rc;
     const int64_t NT = cdiv(N, 128), KC = cdiv(K, LIN_KC), U = NT * KC;

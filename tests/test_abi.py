@@ -63,3 +63,89 @@ def test_binding_arity_matches_header():
         assert len(lib._SIGS[name][1]) == n, (name, n, len(lib._SIGS[name][1]))
         seen += 1
     assert seen == len(lib._SIGS)
+
+
+# Fake device addresses: every call below is rejected by a host-side check
+# before the library looks at the device, so nothing is dereferenced or
+# launched (on a machine with or without a GPU).
+A = 1 << 20                 # 16-byte aligned, non-null
+MIS = A + 8                 # 8 bytes off a 16-byte boundary
+
+
+def _rc(name, *args):
+    return getattr(lib.load(), name)(*args)
+
+
+def test_host_checks_reject_bad_arguments_before_the_device():
+    E_ARG, E_SHAPE, E_ALIGN = -1, -2, -3
+    cases = [
+        # nvfp4_quantize_act(x, dtype, rows, K, ld_x, g_in, codes, scales, g_out, act, ws, ws_bytes, stream)
+        (E_ARG, "nvfp4_quantize_act", None, 0, 16, 64, 64, None, A, A, None, None, A, 1 << 20, None),
+        (E_ARG, "nvfp4_quantize_act", A, 7, 16, 64, 64, None, A, A, A, None, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_quantize_act", A, 0, 16, 24, 24, None, A, A, A, None, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_quantize_act", A, 0, 17, 64, 64, None, None, None, A, A, A, 1 << 20, None),
+        (E_ALIGN, "nvfp4_quantize_act", MIS, 0, 16, 64, 64, None, A, A, A, None, A, 1 << 20, None),
+        # nvfp4_prepare_act(codes, scales, rows, K, act, stream)
+        (E_SHAPE, "nvfp4_prepare_act", A, A, 17, 64, A, None),
+        (E_ALIGN, "nvfp4_prepare_act", A, A, 16, 64, MIS, None),
+        # nvfp4_prepare_weight(codes, scales, N, K, prepared, stream)
+        (E_SHAPE, "nvfp4_prepare_weight", A, A, 128, 100, A, None),
+        (E_ALIGN, "nvfp4_prepare_weight", A, A, 128, 128, MIS, None),
+        # nvfp4_linear(a, g_a, M, w, g_w, N, K, residual, y, ldy, ws, ws_bytes, stream)
+        (E_ARG, "nvfp4_linear", None, A, 16, A, A, 128, 128, None, A, 128, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear", A, A, 17, A, A, 128, 128, None, A, 128, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear", A, A, 16, A, A, 524289, 128, None, A, 524289, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear", A, A, 16, A, A, 128, 96, None, A, 128, A, 1 << 20, None),
+        (E_ALIGN, "nvfp4_linear", MIS, A, 16, A, A, 128, 128, None, A, 128, A, 1 << 20, None),
+        # nvfp4_linear_noalloc(a, g_a, M, w, g_w, N, K, residual, y, ldy, stream)
+        (E_SHAPE, "nvfp4_linear_noalloc", A, A, 16, A, A, 524289, 128, None, A, 524289, None),
+        # tree_attn_fp8kv(q, ld_q, T, Hq, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, parent,
+        #                 k_scale, v_scale, sm_scale, out, g_act, act, ws, ws_bytes, stream)
+        (E_SHAPE, "tree_attn_fp8kv", A, 3072, 17, 24, 4, 128, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
+         None, A, 1 << 20, None),
+        (E_SHAPE, "tree_attn_fp8kv", A, 3072, 16, 24, 4, 64, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
+         None, A, 1 << 20, None),
+        (E_SHAPE, "tree_attn_fp8kv", A, 3072, 16, 36, 4, 128, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
+         None, A, 1 << 20, None),
+        (E_ALIGN, "tree_attn_fp8kv", MIS, 3072, 16, 24, 4, 128, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
+         None, A, 1 << 20, None),
+        (E_ARG, "tree_attn_fp8kv", A, 3072, 16, 24, 4, 128, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
+         A, A, 1 << 20, None),
+        # kv_page_restore(src, src_ids, dst, dst_ids, n, page_bytes, n_src, n_dst, stream)
+        (E_SHAPE, "kv_page_restore", A, A, A, A, 4, 15, 8, 8, None),
+        (E_ALIGN, "kv_page_restore", MIS, A, A, A, 4, 32768, 8, 8, None),
+        # nvfp4_rmsnorm_quantize(x, w, eps, rows, n, g_in, codes, scales, g_out, act, ws, ws_bytes, stream)
+        (E_SHAPE, "nvfp4_rmsnorm_quantize", A, A, 1e-6, 16, 8256, None, A, A, A, None, None, 0, None),
+        # nvfp4_swiglu_quantize(gu, rows, F, g_in, codes, scales, g_out, act, ws, ws_bytes, stream)
+        (E_SHAPE, "nvfp4_swiglu_quantize", A, 0, 17408, None, A, A, A, None, None, 0, None),
+        # kv_append_fp8(k, v, ld, T, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, k_s, v_s, stream)
+        (E_SHAPE, "kv_append_fp8", A, A, 4096, 16, 4, 12, A, A, 8, 64, A, 100, A, A, None),
+        # argmax_rows_bf16(x, rows, n, ld, idx, ws, ws_bytes, stream)
+        (E_SHAPE, "argmax_rows_bf16", A, 5000, 151936, 151936, A, A, 1 << 24, None),
+        # tree_accept_greedy(draft, target, parent, T, path, n, next, stream)
+        (E_SHAPE, "tree_accept_greedy", A, A, A, 33, A, A, A, None),
+        # kv_compact_accepted(k, v, layer_stride, n_layers, Hkv, D, n_pool, P, page_table, ctx_len, path, n, T, stream)
+        (E_SHAPE, "kv_compact_accepted", A, A, 1 << 20, 64, 4, 136, 8, 64, A, 100, A, A, 16, None),
+        # nvfp4sk_debug_encode(x, n, e2m1, e4m3, stream)
+        (E_ARG, "nvfp4sk_debug_encode", A, -1, A, A, None),
+    ]
+    for want, name, *args in cases:
+        got = _rc(name, *args)
+        assert got == want, (name, args, got, lib.load().nvfp4sk_last_error())
+        assert lib.load().nvfp4sk_last_error(), name
+    # an empty restore is a no-op that needs no device
+    assert _rc("kv_page_restore", A, A, A, A, 0, 32768, 8, 8, None) == 0
+
+
+def test_calls_fail_loudly_without_a_gpu():
+    """Without a device the library reports an error (no CPU fallback), and
+    the binding raises it."""
+    import pytest
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc = _rc("nvfp4sk_debug_wait_timeout", None)
+    assert rc in (-5, -8), rc
+    assert lib.load().nvfp4sk_last_error()
+    with pytest.raises(lib.NvFp4Error):
+        lib._call("nvfp4sk_debug_wait_timeout", None)
