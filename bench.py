@@ -363,6 +363,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": model.launches_per_step() * args.steps,
     }
     line["step_hbm_gbs"] = round(step_bytes / (t_dev / args.steps) / 1e9, 1)
+    line["node_tokens_per_s"] = round(T * value, 1)      # candidate tokens verified per second
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, desc = oracle_sample(args.ctx, args.layers)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
