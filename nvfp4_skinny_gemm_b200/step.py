@@ -296,8 +296,8 @@ class VerifyModel:
         result of one pass over all S rows.
 
         Order inside a layer: each op runs over all row groups before the
-        next op starts, so a linear's weights are read from HBM once and
-        from L2 for the later groups; all groups' K/V are appended before any
+        next op starts, so a linear's weights can stay in L2 for the later
+        groups; all groups' K/V are appended before any
         group attends, and group c attends to the context (start + 16c
         tokens, the earlier groups included) plus its own chain."""
         if not self.static:
@@ -305,6 +305,8 @@ class VerifyModel:
         S = h.shape[0]
         if h.dtype != torch.bfloat16 or h.dim() != 2 or h.shape[1] != I.HIDDEN or not h.is_contiguous():
             raise ValueError("h must be a contiguous bf16 [S, HIDDEN] tensor")
+        if h.device != self.dev:
+            raise ValueError(f"h is on {h.device}, the model on {self.dev}")
         if start < 0 or start + S > self.n_log * I.PAGE:
             raise ValueError(f"positions {start} .. {start + S - 1} exceed the page table "
                              f"({self.n_log} pages of {I.PAGE})")

@@ -71,6 +71,8 @@ def test_prefill_arguments(monkeypatch):
     with pytest.raises(ValueError):
         m.prefill(h.float(), 100)
     with pytest.raises(ValueError):
+        m.prefill(h.to("meta"), 100)                 # another device than the model's
+    with pytest.raises(ValueError):
         m.prefill(torch.zeros(8, 2 * I.HIDDEN, dtype=torch.bfloat16)[:, ::2], 100)
     m.static = False
     with pytest.raises(RuntimeError):
