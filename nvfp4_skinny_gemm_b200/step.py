@@ -305,7 +305,7 @@ class VerifyModel:
         S = h.shape[0]
         if h.dtype != torch.bfloat16 or h.dim() != 2 or h.shape[1] != I.HIDDEN or not h.is_contiguous():
             raise ValueError("h must be a contiguous bf16 [S, HIDDEN] tensor")
-        if h.device != self.dev:
+        if h.device.type != self.dev.type or (self.dev.index is not None and h.device.index != self.dev.index):
             raise ValueError(f"h is on {h.device}, the model on {self.dev}")
         if start < 0 or start + S > self.n_log * I.PAGE:
             raise ValueError(f"positions {start} .. {start + S - 1} exceed the page table "
