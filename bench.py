@@ -373,6 +373,17 @@ def run_ours(args, world, rank, local):
 
 
 # ------------------------------------------------------------------ suffix prefill
+def prefill_flops(S, start, layers):
+    """FLOPs a suffix prefill of S tokens after `start` cached tokens must do:
+    (NVFP4 linears over S rows + the LM head over the last row, QK^T and PV
+    of causal attention: row i sees start + i + 1 positions)."""
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    lin = 2.0 * S * sum(N * K for (K, N) in I.LAYER_LINEARS.values()) * layers + 2.0 * I.VOCAB * I.HIDDEN
+    visible = S * (start + 1) + S * (S - 1) / 2
+    attn = 4.0 * I.HEAD_DIM * I.N_Q_HEADS * visible * layers
+    return lin, attn
+
+
 def run_prefill(args):
     """Suffix prefill of S = args.prefill tokens after ctx - S cached tokens,
     timed with CUDA events around graph replays (weights far exceed L2).
@@ -424,10 +435,7 @@ def run_prefill(args):
         assert rc == 0, f"device status {rc} at site {site}"
         assert ids is not None and 0 <= int(ids.cpu()[0]) < I.VOCAB
 
-    lin_flops = 2.0 * S * sum(N * K for (K, N) in I.LAYER_LINEARS.values()) * args.layers \
-        + 2.0 * I.VOCAB * I.HIDDEN
-    visible = S * (start + 1) + S * (S - 1) / 2                    # sum over rows of the positions seen
-    attn_flops = 4.0 * I.HEAD_DIM * I.N_Q_HEADS * visible * args.layers
+    lin_flops, attn_flops = prefill_flops(S, start, args.layers)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     bf16 = float(peaks.get("bf16_tflops_sustained", 1400.0))

@@ -32,3 +32,37 @@ def test_clock_sampler_parses_and_flags_throttling():
     assert d["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     c.proc = None
     assert c.stop()["sm_mhz"] is None
+
+
+def test_prefill_flops_brute_force():
+    """bench.prefill_flops against a count over rows, positions and weights."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    S, start, layers = 7, 11, 3
+    lin, attn = bench.prefill_flops(S, start, layers)
+    macs = 0
+    for _ in range(layers):
+        for K, N in I.LAYER_LINEARS.values():
+            macs += S * N * K
+    macs += I.VOCAB * I.HIDDEN                       # LM head, last row only
+    assert lin == 2 * macs
+    seen = sum(len(range(0, start + i + 1)) for i in range(S))
+    # QK^T and PV: 2 x D multiply-adds per (row, head, visible position)
+    assert attn == layers * I.N_Q_HEADS * seen * 2 * 2 * I.HEAD_DIM
+
+
+def test_verify_step_algorithmic_linear_bytes(monkeypatch):
+    """The bytes the bench divides by for the linears' roofline: per launch the
+    weight codes + E4M3 scales, the activation codes + scales, the bf16 output
+    (and the residual read of O and down), 64 layers + LM head at 16 rows."""
+    from fake_lib import fake_model
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    m, _ = fake_model(monkeypatch, 64, 1024)
+    T, tot = 16, 0
+    for name, (K, N) in list(I.LAYER_LINEARS.items()) * 64:
+        res = 2 if name in ("o", "down") else 1
+        tot += N * K // 2 + N * K // 16 + T * K // 2 + T * K // 16 + res * T * N * 2
+    K, N = I.HIDDEN, I.VOCAB
+    tot += N * K // 2 + N * K // 16 + T * K // 2 + T * K // 16 + T * N * 2
+    assert m.linear_bytes() == tot == 11_528_946_688
