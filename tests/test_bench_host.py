@@ -69,14 +69,15 @@ def test_verify_step_algorithmic_linear_bytes(monkeypatch):
 
 
 def test_verify_step_attention_and_restore_bytes(monkeypatch):
-    """K+V bytes read per step (64 layers x 4 heads x 128 dims x 2 for K and
-    V over the context and the 16 tree slots) and the restore's read + write
-    of the reused prefix pages (32 KB planes, K and V, every layer)."""
+    """K+V bytes read per step (layers x 4 heads x 128 dims x 2 for K and V
+    over the context and the 16 tree slots) and the restore's read + write of
+    the reused prefix pages (32 KB planes, K and V, every layer)."""
     import math
     from fake_lib import fake_model
+    n = 2                                            # both counts are linear in the layers
     for L in (1024, 8192, 23552):
-        m, _ = fake_model(monkeypatch, 64, L)
-        assert m.attn_bytes() == 64 * 2 * (L + 16) * 4 * 128
+        m, _ = fake_model(monkeypatch, n, L)
+        assert m.attn_bytes() == n * 2 * (L + 16) * 4 * 128
         pages = math.ceil(round(0.96 * L) / 64)
-        assert m.restore_bytes() == 2 * 64 * 2 * pages * 32768
+        assert m.restore_bytes() == 2 * n * 2 * pages * 32768
     assert pages == 354                              # 22,610 prefix tokens at 23,552
