@@ -63,9 +63,10 @@ def test_single_rank_helpers_need_no_process_group():
 
 
 def test_reference_arm_under_two_gloo_ranks():
-    """`bench.py --impl reference` launched like the driver launches N > 1
-    (torch.distributed.run, 127.0.0.1): rank 0 alone times the oracle and
-    prints one JSON line; the other rank exits 0 without work."""
+    """`bench.py --impl reference` launched for N > 1 ranks the way a
+    multi-GPU run is launched (torch.distributed.run, one node, 127.0.0.1):
+    rank 0 alone times the oracle and prints one JSON line; the other rank
+    exits 0 without work."""
     import json
     import subprocess
     port = _free_port()
