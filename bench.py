@@ -211,6 +211,21 @@ def oracle_sample(ctx, layers, seconds_hint=15.0):
     return 1.0 / step, threads, desc
 
 
+def oracle_sample_one_thread(ctx, layers, timeout=600):
+    """The same bounded oracle sample on one OpenMP thread, in a fresh Python
+    process (fork + exec, no CUDA state).  Returns its steps/s, or None if it
+    could not run: the multi-threaded figure stays the reported baseline."""
+    code = (f"import json, sys; sys.path.insert(0, {ROOT!r}); import bench; "
+            f"v, t, _ = bench.oracle_sample({int(ctx)}, {int(layers)}); print(json.dumps([v, t]))")
+    env = dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES="")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=timeout)
+        v, threads = json.loads(r.stdout.strip().splitlines()[-1])
+        return float(v) if threads == 1 else None
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
     if rank != 0:
@@ -366,7 +381,8 @@ def run_ours(args, world, rank, local):
     line["node_tokens_per_s"] = round(T * value, 1)      # candidate tokens verified per second
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, desc = oracle_sample(args.ctx, args.layers)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                                "value_one_thread": oracle_sample_one_thread(args.ctx, args.layers)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, lin_graph

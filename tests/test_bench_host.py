@@ -81,3 +81,13 @@ def test_verify_step_attention_and_restore_bytes(monkeypatch):
         pages = math.ceil(round(0.96 * L) / 64)
         assert m.restore_bytes() == 2 * n * 2 * pages * 32768
     assert pages == 354                              # 22,610 prefix tokens at 23,552
+
+
+def test_oracle_sample_on_one_thread():
+    """The single-thread CPU baseline runs the same sample in a child process
+    limited to one OpenMP thread (smaller than the multi-threaded figure)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    v1 = bench.oracle_sample_one_thread(1024, 2)
+    assert v1 is not None and v1 > 0
+    assert bench.oracle_sample_one_thread(1024, 2, timeout=0.01) is None
