@@ -47,7 +47,7 @@ def _worker(rank, world, port, out):
 def test_barrier_and_max_over_ranks_two_gloo_ranks():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()          # no fork of this multi-threaded process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == pytest.approx(2.25) and out[1][0] == pytest.approx(2.25)
