@@ -86,13 +86,18 @@ def load(path: str = LIB_PATH):
     return _lib
 
 
-def _p(t):
-    if t is None:
-        return None
+def _d(t):
+    """Device address of a CUDA tensor; an int passes through as a raw device
+    address.  A host tensor raises here rather than reaching a kernel."""
     if isinstance(t, int):
         return t
-    assert t.is_cuda, "device tensor expected"
+    if not t.is_cuda:
+        raise ValueError(f"a device tensor is expected, got one on {t.device}")
     return t.data_ptr()
+
+
+def _p(t):
+    return None if t is None else _d(t)
 
 
 def _stream(stream=None):
@@ -173,8 +178,8 @@ def quantize(x: torch.Tensor, g_in: torch.Tensor | None = None, out=None, act: t
                torch.empty(1, dtype=torch.float32, device=x.device))
     codes, scales, g = out
     wp, wn = _ws(ws, load().nvfp4_quantize_workspace_bytes(rows, K), "quantize")
-    _call("nvfp4_quantize_act", x.data_ptr(), dt, rows, K, x.stride(0), _p(g_in), _p(codes), _p(scales),
-          g.data_ptr(), _p(act), wp, wn, _stream(stream))
+    _call("nvfp4_quantize_act", _d(x), dt, rows, K, x.stride(0), _p(g_in), _p(codes), _p(scales),
+          _d(g), _p(act), wp, wn, _stream(stream))
     return codes, scales, g
 
 
@@ -182,13 +187,13 @@ def prepare_act(codes: torch.Tensor, scales: torch.Tensor, K: int, act=None, str
     rows = codes.shape[0]
     if act is None:
         act = act_buffer(K, codes.device)
-    _call("nvfp4_prepare_act", codes.data_ptr(), scales.data_ptr(), rows, K, act.data_ptr(), _stream(stream))
+    _call("nvfp4_prepare_act", _d(codes), _d(scales), rows, K, _d(act), _stream(stream))
     return act
 
 
 def prepare_weight(codes: torch.Tensor, scales: torch.Tensor, N: int, K: int, stream=None):
     out = torch.empty(load().nvfp4_prepared_weight_bytes(N, K), dtype=torch.uint8, device=codes.device)
-    _call("nvfp4_prepare_weight", codes.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(stream))
+    _call("nvfp4_prepare_weight", _d(codes), _d(scales), N, K, _d(out), _stream(stream))
     return out
 
 
@@ -197,8 +202,8 @@ def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, str
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=a_act.device)
     wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K), "linear")
-    _call("nvfp4_linear", a_act.data_ptr(), g_a.data_ptr(), M, w_prep.data_ptr(), g_w.data_ptr(), N, K,
-          _p(residual), y.data_ptr(), y.stride(0), wp, wn, _stream(stream))
+    _call("nvfp4_linear", _d(a_act), _d(g_a), M, _d(w_prep), _d(g_w), N, K,
+          _p(residual), _d(y), y.stride(0), wp, wn, _stream(stream))
     return y
 
 
@@ -218,15 +223,15 @@ def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, 
     if out is None:
         out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=q.device)
     wp, wn = _ws(ws, load().tree_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)), "attn")
-    _call("tree_attn_fp8kv", q.data_ptr(), ld_q, T, Hq, Hkv, D, k_pool.data_ptr(), v_pool.data_ptr(), n_pages, P,
-          page_table.data_ptr(), int(ctx_len), parent.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
-          float(sm_scale), out.data_ptr(), _p(g_act), _p(act), wp, wn, _stream(stream))
+    _call("tree_attn_fp8kv", _d(q), ld_q, T, Hq, Hkv, D, _d(k_pool), _d(v_pool), n_pages, P,
+          _d(page_table), int(ctx_len), _d(parent), _d(k_scale), _d(v_scale),
+          float(sm_scale), _d(out), _p(g_act), _p(act), wp, wn, _stream(stream))
     return out
 
 
 def kv_page_restore(src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, stream=None):
     n = src_ids.numel() if n is None else n
-    _call("kv_page_restore", src_pool.data_ptr(), src_ids.data_ptr(), dst_pool.data_ptr(), dst_ids.data_ptr(), n,
+    _call("kv_page_restore", _d(src_pool), _d(src_ids), _d(dst_pool), _d(dst_ids), n,
           page_bytes, src_pool.numel() // page_bytes, dst_pool.numel() // page_bytes, _stream(stream))
 
 
@@ -235,25 +240,25 @@ def rmsnorm_quantize(x, w, eps, out, act=None, stream=None, g_in=None):
     g_in: static tensor scale (device [1]) or None for the dynamic one."""
     rows, n = x.shape
     codes, scales, g = out
-    _call("nvfp4_rmsnorm_quantize", x.data_ptr(), w.data_ptr(), float(eps), rows, n, _p(g_in), _p(codes),
-          _p(scales), g.data_ptr(), _p(act), None, 0, _stream(stream))
+    _call("nvfp4_rmsnorm_quantize", _d(x), _d(w), float(eps), rows, n, _p(g_in), _p(codes),
+          _p(scales), _d(g), _p(act), None, 0, _stream(stream))
     return out
 
 
 def swiglu_quantize(gu, out, act=None, stream=None, g_in=None):
     rows, F2 = gu.shape
     codes, scales, g = out
-    _call("nvfp4_swiglu_quantize", gu.data_ptr(), rows, F2 // 2, _p(g_in), _p(codes), _p(scales), g.data_ptr(),
+    _call("nvfp4_swiglu_quantize", _d(gu), rows, F2 // 2, _p(g_in), _p(codes), _p(scales), _d(g),
           _p(act), None, 0, _stream(stream))
     return out
 
 
 def kv_append(k_new, v_new, ld_new, T, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, stream=None):
     n_pages, Hkv, P, D = k_pool.shape
-    _call("kv_append_fp8", k_new.data_ptr() if hasattr(k_new, "data_ptr") else k_new,
-          v_new.data_ptr() if hasattr(v_new, "data_ptr") else v_new, ld_new, T, Hkv, D, k_pool.data_ptr(),
-          v_pool.data_ptr(), n_pages, P, page_table.data_ptr(), int(ctx_len), k_scale.data_ptr(),
-          v_scale.data_ptr(), _stream(stream))
+    _call("kv_append_fp8", _d(k_new),
+          _d(v_new), ld_new, T, Hkv, D, _d(k_pool),
+          _d(v_pool), n_pages, P, _d(page_table), int(ctx_len), _d(k_scale),
+          _d(v_scale), _stream(stream))
 
 
 def tree_accept(draft_tokens, target_argmax, parent, out=None, stream=None):
@@ -264,8 +269,8 @@ def tree_accept(draft_tokens, target_argmax, parent, out=None, stream=None):
         out = (torch.empty(T, dtype=torch.int32, device=dev), torch.empty(1, dtype=torch.int32, device=dev),
                torch.empty(1, dtype=torch.int32, device=dev))
     path, n, nxt = out
-    _call("tree_accept_greedy", draft_tokens.data_ptr(), target_argmax.data_ptr(), parent.data_ptr(), T,
-          path.data_ptr(), n.data_ptr(), nxt.data_ptr(), _stream(stream))
+    _call("tree_accept_greedy", _d(draft_tokens), _d(target_argmax), _d(parent), T,
+          _d(path), _d(n), _d(nxt), _stream(stream))
     return out
 
 
@@ -273,7 +278,7 @@ def kv_compact(k_base, v_base, layer_stride, n_layers, Hkv, D, n_pool_pages, P, 
                stream=None):
     """Move the accepted tokens' K/V to ctx_len .. in every layer (see kv_compact_accepted)."""
     _call("kv_compact_accepted", k_base, v_base, int(layer_stride), n_layers, Hkv, D, int(n_pool_pages), P,
-          page_table.data_ptr(), int(ctx_len), path.data_ptr(), n.data_ptr(), T, _stream(stream))
+          _d(page_table), int(ctx_len), _d(path), _d(n), T, _stream(stream))
 
 
 def argmax(x, idx=None, ws=None, stream=None):
@@ -281,7 +286,7 @@ def argmax(x, idx=None, ws=None, stream=None):
     if idx is None:
         idx = torch.empty(rows, dtype=torch.int32, device=x.device)
     wp, wn = _ws(ws, load().argmax_workspace_bytes(rows, n), "argmax")
-    _call("argmax_rows_bf16", x.data_ptr(), rows, n, x.stride(0), idx.data_ptr(), wp, wn, _stream(stream))
+    _call("argmax_rows_bf16", _d(x), rows, n, x.stride(0), _d(idx), wp, wn, _stream(stream))
     return idx
 
 
@@ -289,5 +294,5 @@ def debug_encode(x: torch.Tensor, stream=None):
     n = x.numel()
     e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
     e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
-    _call("nvfp4sk_debug_encode", x.data_ptr(), n, e2.data_ptr(), e4.data_ptr(), _stream(stream))
+    _call("nvfp4sk_debug_encode", _d(x), n, _d(e2), _d(e4), _stream(stream))
     return e2, e4

@@ -149,3 +149,36 @@ def test_calls_fail_loudly_without_a_gpu():
     assert lib.load().nvfp4sk_last_error()
     with pytest.raises(lib.NvFp4Error):
         lib._call("nvfp4sk_debug_wait_timeout", None)
+
+
+def test_binding_rejects_host_tensors():
+    """Every tensor argument of the C ABI is a device pointer: the binding
+    raises on a host tensor instead of passing its address to a kernel."""
+    import pytest
+    import torch
+
+    class HostWs:                                   # stands in for a device workspace
+        def get(self, n):
+            return torch.zeros(max(int(n), 256), dtype=torch.uint8)
+
+    h = lambda *s, dt=torch.uint8: torch.zeros(*s, dtype=dt)
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    g = torch.ones(1)
+    calls = [
+        lambda: lib.rmsnorm_quantize(bf(16, 64), bf(64), 1e-6, (None, None, g), act=h(8192)),
+        lambda: lib.swiglu_quantize(bf(16, 128), (None, None, g), act=h(8192)),
+        lambda: lib.prepare_weight(h(128, 32), h(128, 4), 128, 64),
+        lambda: lib.prepare_act(h(16, 32), h(16, 4), 64, act=h(8192)),
+        lambda: lib.kv_page_restore(h(64), h(1, dt=torch.int32), h(64), h(1, dt=torch.int32), 32),
+        lambda: lib.kv_append(bf(16, 384), bf(16, 384), 384, 16, h(2, 1, 64, 128), h(2, 1, 8192),
+                              h(2, dt=torch.int32), 0, g, g),
+        lambda: lib.tree_accept(h(16, dt=torch.int32), h(16, dt=torch.int32), h(16, dt=torch.int32),
+                                out=(h(16, dt=torch.int32), h(1, dt=torch.int32), h(1, dt=torch.int32))),
+        lambda: lib.linear(h(8192), g, 16, h(36864), g, 128, 512, y=bf(16, 128), ws=HostWs()),
+        lambda: lib.tree_attn(bf(16, 24, 128), h(2, 4, 64, 128), h(2, 4, 8192), h(2, dt=torch.int32), 10,
+                              h(16, dt=torch.int32), g, g, out=bf(16, 24, 128), ws=HostWs()),
+        lambda: lib.argmax(bf(16, 4096), idx=h(16, dt=torch.int32), ws=HostWs()),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(ValueError, match="device tensor"):
+            call()
