@@ -355,6 +355,24 @@ class VerifyModel:
         nv.argmax(pf["logits"], pf["ids"])
         return pf["ids"]
 
+    def turn(self, h_suffix: torch.Tensor, draft_tokens: torch.Tensor | None = None):
+        """One agent turn's forward work: restore the reused prefix pages,
+        prefill the suffix (the S = ctx_len - prefix_tokens positions the
+        restore does not hold; h_suffix is overwritten), then verify the tree
+        in self.h / self.parent at ctx_len, and with draft tokens accept the
+        longest matching path.  Needs static activation scales (calibrate()),
+        as prefill() does.  Returns (token after the suffix, ids of the verify
+        step, and the acceptance tuple of accept() or None)."""
+        S = h_suffix.shape[0]
+        if S != self.L - self.prefix_tokens:
+            raise ValueError(f"the suffix has {self.L - self.prefix_tokens} tokens after the "
+                             f"{self.prefix_tokens}-token prefix, got {S}")
+        self.restore()
+        nxt = self.prefill(h_suffix, self.prefix_tokens)
+        self.step(restore=False)
+        acc = self.accept(draft_tokens) if draft_tokens is not None else None
+        return nxt, self.ids, acc
+
     def prefill_launches(self, S):
         """Kernel launches of prefill(S rows): per layer and row group norm-q,
         qkv, attention split + combine, o, norm-q, gate_up, swiglu-q, down,

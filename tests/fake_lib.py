@@ -54,6 +54,8 @@ class FakeLib:
         self.m = None
         self.wmap = {}
         self.start = 0            # first labelled cache position (earlier ones are context)
+        self.restores = 0
+        self.accepted = None
 
     # ---- helpers
     def rows(self, x, n=None):
@@ -92,6 +94,17 @@ class FakeLib:
 
     def kv_page_restore(self, src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, stream=None):
         self.launches += 1
+        self.restores += 1
+
+    def tree_accept(self, draft_tokens, target_argmax, parent, out=None, stream=None):
+        self.launches += 1
+        self.accepted = (self.get(draft_tokens.view(-1, 1)), self.get(target_argmax.view(-1, 1)))
+        return ("path", "n", "next")
+
+    def kv_compact(self, k_base, v_base, layer_stride, n_layers, Hkv, D, n_pool_pages, P, page_table, ctx_len,
+                   path, n, T, stream=None):
+        self.launches += 1
+        assert (path, n) == ("path", "n") and ctx_len == self.m.L and n_layers == self.m.n_layers
 
     def quantize(self, x, g_in=None, out=None, act=None, canonical=True, ws=None, stream=None):
         self.launches += 1
@@ -201,20 +214,22 @@ def scale_label(L, static, site, rows):
     return L("site", site) if static else L("dynamic", *rows)
 
 
-def expected_layers(L, n_layers, start, S, parent, h, static=True):
+def expected_layers(L, n_layers, start, S, parent, h, static=True, ctx_kv=None):
     """Labels the layer definition gives for S rows at cache positions
-    start .. start+S-1, row i attending to the rows parent makes visible,
+    start .. start+S-1, row i attending to the labelled context ctx_kv[l]
+    (a list per layer, default none) and to the rows parent makes visible,
     with no grouping of rows anywhere.  Returns (h labels, {(layer, pos): kv})."""
     sites = step.VerifyModel.SITES
     kv = {}
     for l in range(n_layers):
+        ctx = list(ctx_kv[l]) if ctx_kv is not None else []
         s0 = l * sites
         n_sc = scale_label(L, static, s0, h)
         y1 = [L("norm", 2 * l, n_sc, v) for v in h]
         qkv = [L("linear", l, "qkv", n_sc, v, None) for v in y1]
         for r in range(S):
             kv[(l, start + r)] = L("kv", qkv[r])
-        att = [L("attn", qkv[r], *[kv[(l, start + j)] for j in ancestors(parent, r)]) for r in range(S)]
+        att = [L("attn", qkv[r], *ctx, *[kv[(l, start + j)] for j in ancestors(parent, r)]) for r in range(S)]
         a_sc = scale_label(L, static, s0 + 1, att)
         aq = [L("quant", a_sc, v) for v in att]
         h1 = [L("linear", l, "o", a_sc, aq[r], h[r]) for r in range(S)]

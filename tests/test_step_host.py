@@ -44,3 +44,34 @@ def test_launch_count_of_the_benchmarked_step(monkeypatch):
     m.parent.copy_(torch.from_numpy(I.tree_parent(4)))
     m.step()
     assert fake.launches == m.launches_per_step() == 644
+
+
+def test_agent_turn_restore_prefill_verify_accept(monkeypatch):
+    """turn(): one restore, the suffix prefilled at positions prefix .. ctx-1,
+    then the verify step whose every node attends to the whole prefilled
+    suffix (and its ancestors), then acceptance on the step's argmax."""
+    L, n_layers = 1000, 2
+    m, fake = fake_model(monkeypatch, n_layers, L)
+    S = L - m.prefix_tokens
+    fake.start = m.prefix_tokens
+    h_suf = torch.zeros(S, I.HIDDEN, dtype=torch.bfloat16)
+    suf_in = [fake.L("suffix", r) for r in range(S)]
+    fake.put(h_suf, suf_in)
+    parent = I.tree_parent(4)
+    m.parent.copy_(torch.from_numpy(parent))
+    tree_in = [fake.L("node", r) for r in range(16)]
+    fake.put(m.h, tree_in)
+    draft = torch.zeros(16, dtype=torch.int32)
+    fake.put(draft.view(-1, 1), [fake.L("draft", r) for r in range(16)])
+    nxt, ids, acc = m.turn(h_suf, draft)
+    assert fake.restores == 1 and acc == ("path", "n", "next")
+    _, suf_kv = expected_layers(fake.L, n_layers, m.prefix_tokens, S, I.chain_parent(S), suf_in)
+    ctx = [[suf_kv[(l, m.prefix_tokens + r)] for r in range(S)] for l in range(n_layers)]
+    h_exp, tree_kv = expected_layers(fake.L, n_layers, L, 16, parent, tree_in, ctx_kv=ctx)
+    assert fake.get(m.h) == h_exp
+    assert all(fake.kv[k] == v for k, v in {**suf_kv, **tree_kv}.items())
+    assert fake.accepted[0] == [fake.L("draft", r) for r in range(16)]
+    assert fake.accepted[1] == fake.get(m.ids.view(-1, 1))
+    assert fake.launches == 1 + m.prefill_launches(S) + m.launches_per_step(restore=False) + 2
+    with pytest.raises(ValueError):
+        m.turn(h_suf[:-1])
