@@ -295,3 +295,56 @@ def kv_compact_accepted(k_pool, v_pool, page_table, ctx_len, path):
         for h in range(Hkv):
             for d in range(D):
                 v_pool[pg, h, v_off(d, sl)] = vs[k][h, d]
+
+
+# ---------------------------------------------------------------- one decoder layer
+def bf16(x):
+    """Nearest bf16 of each value, as an fp64 array: round to fp32 first (as
+    the kernels hold their results), then to the upper 16 bits of the fp32
+    pattern, ties to even.  Finite, in-range inputs only."""
+    f = np.asarray(x, np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def decoder_layer(h, norm_w1, norm_w2, weights, G, k_pool, v_pool, page_table, ctx_len, parent, k_scale,
+                  v_scale, Hq, eps=1e-6):
+    """One pre-norm decoder layer of the verify step on the T rows of h, as
+    the step composes it ("NVFP4 and FP8": NVFP4 weights and activations, FP8
+    KV cache; "Tree multi-token prediction": the T rows are the tree's nodes):
+
+        y1 = bf16(RMSNorm(h)),            qkv = bf16(NVFP4(y1) x W_qkv^T),
+        FP8 append of the rows' K/V at ctx_len .., a = bf16(tree attention),
+        h1 = bf16(h + NVFP4(a) x W_o^T),  y2 = bf16(RMSNorm(h1)),
+        gu = bf16(NVFP4(y2) x W_gu^T),    s = bf16(SwiGLU(gu)),
+        h2 = bf16(h1 + NVFP4(s) x W_down^T).
+
+    weights: name -> (codes, scales, g) of 'qkv', 'o', 'gate_up', 'down';
+    G: the four activation scales (norm1, attention out, norm2, SwiGLU) of a
+    calibrated checkpoint, or None for the dynamic amax/2688 of each tensor.
+    The pools (k [pages, Hkv, P, D], v [pages, Hkv, D*P]) are updated in place.
+    Returns a dict of every intermediate (fp64 arrays of bf16 values)."""
+    h = np.asarray(h, np.float64)
+    T = h.shape[0]
+    _, Hkv, _, D = k_pool.shape
+    qd, kd = Hq * D, Hkv * D
+
+    def lin(x, name, site):
+        ac, asc, ga = quantize(x, g_in=None if G is None else float(G[site]))
+        return linear(ac, asc, ga, *weights[name])
+
+    r = {"h": h}
+    r["y1"] = bf16(rmsnorm(h, norm_w1, eps))
+    r["qkv"] = bf16(lin(r["y1"], "qkv", 0))
+    kv_append(r["qkv"][:, qd:qd + kd].reshape(T, Hkv, D), r["qkv"][:, qd + kd:].reshape(T, Hkv, D),
+              k_pool, v_pool, page_table, ctx_len, k_scale, v_scale)
+    a = tree_attn(r["qkv"][:, :qd].reshape(T, Hq, D), k_pool, v_pool, page_table, ctx_len, parent,
+                  k_scale, v_scale)
+    r["attn"] = bf16(a.reshape(T, qd))
+    r["h1"] = bf16(h + lin(r["attn"], "o", 1))
+    r["y2"] = bf16(rmsnorm(r["h1"], norm_w2, eps))
+    r["gu"] = bf16(lin(r["y2"], "gate_up", 2))
+    r["s"] = bf16(swiglu(r["gu"]))
+    r["h2"] = bf16(r["h1"] + lin(r["s"], "down", 3))
+    return r
