@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ctx", type=int, default=23552)
+    ap.add_argument("--sweep", default="1024,8192,23552",
+                    help="context lengths of the verify-step sweep (same weights), '' for none")
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--chain", type=int, default=0,
                     help="verify a linear-MTP chain of this many tokens instead of the 16-node tree")
@@ -53,7 +55,8 @@ def parse():
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--kernel-case", default=None,
-                    choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "attn", "restore", "quantize"],
+                    choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "linear_o", "linear_down",
+                             "linear_m1_2048", "attn", "restore", "quantize"],
                     help="run one kernel on a small case (for ncu captures) instead of the step")
     return ap.parse_args()
 
@@ -230,8 +233,6 @@ def oracle_sample_one_thread(ctx, layers, timeout=600):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    for _ in range(args.warmup):
-        pass
     vals, desc, threads = [], "", 1
     t0 = time.perf_counter()
     for _ in range(max(1, args.steps)):
@@ -241,7 +242,10 @@ def run_reference(args, world, rank):
             break
     v = float(np.median(vals))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": len(vals), "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+            "steps": len(vals), "warmup": args.warmup, "ms_per_step": 1e3 / v,
+            "ms_per_step_kind": "estimate: each step times a bounded oracle sample and extrapolates it "
+                                "to a whole verify step (no step runs in full)",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{args.layers}-layer 27B-class verify step, "
                                f"{f'linear-MTP chain of {T}' if args.chain else '16-node tree'}, ctx {args.ctx} FP8 paged KV, "
@@ -253,6 +257,50 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------------ our arm
+def capture(stream, fn):
+    """One CUDA graph of fn()'s launches on `stream`."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def time_graph(graph, stream, reps, warm=3):
+    """Seconds per replay: CUDA events on the launching stream around `reps`
+    back-to-back replays, after `warm` untimed ones."""
+    for _ in range(warm):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e-3 / reps
+
+
+def linear_launches(model):
+    """The step's 257 linear launches (same operands, shapes and order)."""
+    for lay in model.layers:
+        model._linear(model.q_h.buf, model.q_h.g, lay["qkv"], model.qkv)
+        model._linear(model.q_a.buf, model.q_a.g, lay["o"], model.h, residual=model.h)
+        model._linear(model.q_h.buf, model.q_h.g, lay["gate_up"], model.gu)
+        model._linear(model.q_f.buf, model.q_f.g, lay["down"], model.h, residual=model.h)
+    model._linear(model.q_h.buf, model.q_h.g, model.lm_head, model.logits)
+
+
+def attention_launches(model):
+    """The step's attention calls (split + combine, with the fused static NVFP4
+    output), one per layer over that layer's pools, back to back."""
+    from nvfp4_skinny_gemm_b200 import inputs as I
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    for l in range(model.n_layers):
+        nv.tree_attn(model.qkv, model.k_pool(l), model.v_pool(l), model.page_table, model.L, model.parent,
+                     model.k_scale[l], model.v_scale[l], out=model.attn, ld_q=model.qkv.stride(0), T=model.T,
+                     Hq=I.N_Q_HEADS, g_act=model._site(l * model.SITES + 1), act=model.q_a.buf)
+
+
 def run_ours(args, world, rank, local):
     from nvfp4_skinny_gemm_b200 import inputs as I
     from nvfp4_skinny_gemm_b200 import lib as nv
@@ -280,17 +328,9 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         rc, site = nv.device_status(stream)
         assert rc == 0, f"device status {rc} at site {site}"
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            model.step()
-        lin_graph = torch.cuda.CUDAGraph()                 # the dominant kernel alone, same launches
-        with torch.cuda.graph(lin_graph, stream=stream):
-            for lay in model.layers:
-                model._linear(model.q_h.buf, model.q_h.g, lay["qkv"], model.qkv)
-                model._linear(model.q_a.buf, model.q_a.g, lay["o"], model.h, residual=model.h)
-                model._linear(model.q_h.buf, model.q_h.g, lay["gate_up"], model.gu)
-                model._linear(model.q_f.buf, model.q_f.g, lay["down"], model.h, residual=model.h)
-            model._linear(model.q_h.buf, model.q_h.g, model.lm_head, model.logits)
+        graph = capture(stream, model.step)
+        lin_graph = capture(stream, lambda: linear_launches(model))     # the dominant kernel alone, same launches
+        attn_graph = capture(stream, lambda: attention_launches(model))  # the attention pairs alone
         load_inputs()
         for _ in range(max(3, args.warmup)):
             graph.replay()
@@ -318,20 +358,24 @@ def run_ours(args, world, rank, local):
         rc, site = nv.device_status(stream)
         assert rc == 0, f"device status {rc} at site {site}"
 
-        # ---- dominant kernel: all linear launches of one step, back to back
+        # ---- dominant kernel: all linear launches of one step, back to back;
+        #      then the 64 attention launch pairs of one step, back to back
         reps = max(3, min(20, args.steps))
-        for _ in range(2):
-            lin_graph.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            lin_graph.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        t_lin = e0.elapsed_time(e1) * 1e-3 / reps
+        t_lin = time_graph(lin_graph, stream, reps)
+        t_attn = time_graph(attn_graph, stream, reps)
         n_lin = 4 * model.n_layers + 1
 
-        # ---- end to end: pinned host inputs in, argmax ids out, every step
+        # ---- the step without the per-step prefix restore (the pages restore
+        #      once per agent turn; the benchmarked step includes it)
+        nr_graph = capture(stream, lambda: model.step(restore=False))
+        t_nr = max_over_ranks(time_graph(nr_graph, stream, args.steps), world)
+        del nr_graph
+
+        # ---- end to end: pinned host inputs in, argmax ids out, every step.
+        #      (1) queued back to back (stream throughput); (2) the host waits
+        #      for each step's ids before issuing the next, as a decode loop
+        #      that drafts the next tree from them must
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
         e0.record(stream)
@@ -343,12 +387,26 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         t_e2e = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            load_inputs()
+            graph.replay()
+            ids_host.copy_(model.ids, non_blocking=True)
+            stream.synchronize()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t_e2e_sync = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world)
 
     peak, peak_kind = measured_peak()
     lin_bytes = model.linear_bytes()
     achieved = lin_bytes / t_lin / 1e9
     traffic = recorded_traffic()
     step_bytes = model.step_bytes()
+    attn_bytes = model.attn_bytes()
+    attn_gbs = attn_bytes / t_attn / 1e9
     value = world * args.steps / t_dev
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -371,21 +429,62 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_step": lin_bytes, "launches": n_lin,
                      "us_per_step_of_linears": round(t_lin * 1e6, 1),
                      "traffic": traffic},
+        "roofline_attn": {"kernel": f"tree_attn_split_kernel + tree_attn_combine_kernel ({model.n_layers} launch "
+                                    f"pairs of one step, back to back)",
+                          "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
+                          "frac": round(attn_gbs / peak, 4),
+                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                          "algorithmic_bytes_per_step": attn_bytes,
+                          "algorithmic_bytes_per_launch_pair": attn_bytes // model.n_layers,
+                          "us_per_launch_pair": round(t_attn / model.n_layers * 1e6, 2), "traffic": None},
+        "no_restore": {"value": world / t_nr, "unit": UNIT, "ms_per_step": round(t_nr * 1e3, 3),
+                       "note": "the same step without the per-step kv_page_restore of the prefix "
+                               "(the pages restore once per agent turn)"},
         "clocks": clk,
         "e2e": {"value": world * args.steps / t_e2e, "unit": UNIT,
                 "h2d_bytes_per_step": h0.numel() * 2 + par0.numel() * 4,
-                "d2h_bytes_per_step": ids_host.numel() * 4},
+                "d2h_bytes_per_step": ids_host.numel() * 4,
+                "mode": "steps queued back to back (stream throughput)"},
+        "e2e_sync": {"value": world * args.steps / t_e2e_sync, "unit": UNIT,
+                     "ms_per_step": round(t_e2e_sync / args.steps * 1e3, 3),
+                     "mode": "the host waits for each step's argmax ids before issuing the next step"},
         "gpu_launches": model.launches_per_step() * args.steps,
     }
     line["step_hbm_gbs"] = round(step_bytes / (t_dev / args.steps) / 1e9, 1)
     line["node_tokens_per_s"] = round(T * value, 1)      # candidate tokens verified per second
+
+    # ---- context sweep of the verify step (same weights; cache and page table rebuilt)
+    del graph, lin_graph, attn_graph
+    sweep = [{"ctx": args.ctx, "value": value, "ms_per_step": line["ms_per_step"],
+              "step_hbm_gbs": line["step_hbm_gbs"], "pct_of_peak": line["step_pct_of_peak"]}]
+    if args.sweep:
+        for c in [int(x) for x in args.sweep.split(",") if int(x) != args.ctx]:
+            with torch.cuda.stream(stream):
+                model.set_context(c)
+                load_inputs()
+                model.step()
+                torch.cuda.synchronize()
+                g2 = capture(stream, model.step)
+                t_c = max_over_ranks(time_graph(g2, stream, args.steps), world)
+                rc, site = nv.device_status(stream)
+                assert rc == 0, f"device status {rc} at site {site}"
+                del g2
+            sb = model.step_bytes()
+            sweep.append({"ctx": c, "value": world / t_c, "ms_per_step": round(t_c * 1e3, 3),
+                          "step_hbm_gbs": round(sb / t_c / 1e9, 1), "pct_of_peak": round(100 * sb / t_c / 1e9 / peak, 1)})
+        sweep.sort(key=lambda d: d["ctx"])
+    line["sweep"] = sweep
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, desc = oracle_sample(args.ctx, args.layers)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+        runs = [oracle_sample(args.ctx, args.layers) for _ in range(3)]
+        v = float(np.median([r[0] for r in runs]))
+        threads, desc = runs[0][1], runs[0][2]
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc + "; median of 3 runs",
+                                "runs": [r[0] for r in runs],
                                 "value_one_thread": oracle_sample_one_thread(args.ctx, args.layers)}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, lin_graph
 
 
 # ------------------------------------------------------------------ suffix prefill
@@ -492,7 +591,9 @@ def run_kernel_case(args):
     case = args.kernel_case
     if case.startswith("linear"):
         K, N = {"linear_lmhead": (I.HIDDEN, I.VOCAB), "linear_gate_up": I.LAYER_LINEARS["gate_up"],
-                "linear_qkv": I.LAYER_LINEARS["qkv"]}[case]
+                "linear_qkv": I.LAYER_LINEARS["qkv"], "linear_o": I.LAYER_LINEARS["o"],
+                "linear_down": I.LAYER_LINEARS["down"], "linear_m1_2048": (2048, 2048)}[case]
+        M = 1 if case == "linear_m1_2048" else 16
         ncopy = max(1, math.ceil(400e6 / (N * K * 9 // 16)))     # rotate copies: > L2 per sweep
         ws = []
         for _ in range(ncopy):
@@ -500,11 +601,11 @@ def run_kernel_case(args):
             sc = torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g)
             ws.append((nv.prepare_weight(c, sc, N, K), torch.full((1,), 0.01, device=dev)))
             del c, sc
-        a = torch.randn(16, K, device=dev, generator=g).to(torch.bfloat16)
+        a = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
         act = nv.act_buffer(K)
         _, _, ga = nv.quantize(a, act=act)
-        y = torch.empty(16, N, dtype=torch.bfloat16, device=dev)
-        fn = lambda i: nv.linear(act, ga, 16, ws[i % ncopy][0], ws[i % ncopy][1], N, K, y=y)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: nv.linear(act, ga, M, ws[i % ncopy][0], ws[i % ncopy][1], N, K, y=y)
         nbytes = N * K * 9 // 16
     elif case == "attn":
         cache = I.kv_cache(3, I.CTX_MAX)

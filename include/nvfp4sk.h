@@ -37,8 +37,12 @@
  *     zero when a call starts: zero-fill such a workspace once when it is
  *     allocated and do not lend it to another kind of call (tree_attn_fp8kv
  *     and nvfp4_quantize_act leave partial results in theirs); every
- *     successful call leaves its counters zero again.  Calls that share one
- *     workspace must be stream-ordered.
+ *     successful call leaves its counters zero again.  A call whose device
+ *     status later reads non-zero (a wait that ran out, above all) may leave
+ *     counters non-zero: after nvfp4sk_get_device_status returns an error,
+ *     zero every nvfp4_linear and argmax_rows_bf16 workspace again before its
+ *     next use (the ctypes binding does this for its default workspaces).
+ *     Calls that share one workspace must be stream-ordered.
  *   - Scalars such as tensor scales are device pointers, so no call syncs.
  *   - Error codes are negative; nvfp4sk_last_error() gives a message for the
  *     last failing call of the calling thread.
@@ -136,7 +140,8 @@ NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint
  * K % 64 == 0, 1 <= N <= 524288; prepared operands 16-byte aligned.
  * residual: NULL or bf16 [M][ldy] added before rounding (may alias y).
  * y: bf16 [M][ldy], ldy >= N.
- * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes (see workspace rule).
+ * ws: nvfp4_linear_workspace_bytes(M, N, K) bytes, zero-filled at allocation
+ *   and again after a failing device status (the workspace rule above).
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t M,
@@ -208,6 +213,16 @@ NVFP4SK_API nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, i
                                const int32_t *parent, const float *k_scale, const float *v_scale,
                                float sm_scale, void *out, const float *g_act, uint8_t *act_prepared,
                                void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
+
+/* Conversion of V pages written token-major (plane = [page_size slots][D]
+ * bytes, the same layout as the K pool) into the tiled plane layout that
+ * tree_attn_fp8kv reads (see above), for caches filled elsewhere.  n_planes
+ * (page, head) planes of D*page_size bytes each, contiguous in both buffers;
+ * plane i of v_tiled receives plane i of v_token_major.  The bytes are only
+ * moved (no arithmetic).  D % 8 == 0, page_size % 16 == 0, D*page_size <=
+ * 16384, buffers 16-byte aligned and not overlapping. */
+NVFP4SK_API nvfp4sk_status kv_v_pages_to_tiled(const uint8_t *v_token_major, uint8_t *v_tiled, int64_t n_planes,
+                                               int D, int page_size, nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * kv_page_restore -- restore cached KV pages of a reused prompt prefix into

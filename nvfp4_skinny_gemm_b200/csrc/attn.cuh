@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 last = i;
             }
             // on abort, let this stage's last copy land before the CTA exits
-            if (*s_abort && last >= 0) mbar_wait(&kv_full[st], (uint32_t)((last / ATT_STAGES) & 1), 303);
+            if (*s_abort && last >= 0) mbar_wait_drain(&kv_full[st], (uint32_t)((last / ATT_STAGES) & 1), 303);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ QK issuer
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
             // every QK product is complete before tensor memory is released
             tc_commit(&drain[0]);
-            mbar_wait(&drain[0], 0, 314);
+            mbar_wait_drain(&drain[0], 0, 314);
         }
         __syncwarp();
     } else if (warp == 10) {
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_commit(o_done);
             } else {
                 tc_commit(&drain[1]);
-                mbar_wait(&drain[1], 0, 315);
+                mbar_wait_drain(&drain[1], 0, 315);
             }
         }
         __syncwarp();

@@ -101,6 +101,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     }
 }
 
+// Drain wait: the wait a kernel makes, after an abort, for its own copies or
+// tensor-core products still in flight before it releases shared or tensor
+// memory.  Its limit never drops below DRAIN_FLOOR_NS, whatever the per-wait
+// limit the caller set, so that a tiny limit cannot free memory that an
+// in-flight operation still writes.
+constexpr uint64_t DRAIN_FLOOR_NS = 100000000ull;   // 100 ms
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint32_t site)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    const uint64_t lim = g_timeout_ns > DRAIN_FLOOR_NS ? g_timeout_ns : DRAIN_FLOOR_NS;
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer() - t0 > lim) {
+            report_error(ERRBIT_TIMEOUT, site);
+            return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------------------
 // Async proxy: TMA tiled loads, 1-D bulk copies, proxy fences
 // ----------------------------------------------------------------------------

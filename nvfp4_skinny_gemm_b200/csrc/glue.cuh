@@ -39,6 +39,40 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __nv_bfloat16 *__r
     }
 }
 
+// Token-major V planes -> the tiled plane layout the attention reads.  One CTA
+// per (page, head) plane of P slots x D dimensions: the plane is staged in
+// shared memory with 16-byte loads, then each 16-byte output row (dimension
+// d, slots 16j .. 16j+15) is gathered from it and stored with one 16-byte
+// write.  D % 8 == 0, P % 16 == 0, D * P <= KVT_MAX_PLANE.
+constexpr int KVT_MAX_PLANE = 16384;
+__global__ void __launch_bounds__(256) kv_v_to_tiled_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                                            int D, int P)
+{
+    __shared__ __align__(16) uint8_t plane[KVT_MAX_PLANE];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t bytes = (int64_t)D * P;
+    const uint8_t *s = src + blockIdx.x * bytes;
+    uint8_t *o = dst + blockIdx.x * bytes;
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += blockDim.x)
+        *reinterpret_cast<uint4 *>(plane + 16 * i) = *reinterpret_cast<const uint4 *>(s + 16 * i);
+    __syncthreads();
+    const int tiles_t = P / 16;
+    for (int64_t row = threadIdx.x; row < bytes / 16; row += blockDim.x) {
+        // output row `row`: tile (d / 8, j) = row / 8 with j fastest, line d % 8 = row % 8
+        const int tile = (int)(row >> 3), d = (tile / tiles_t) * 8 + (int)(row & 7), j = tile % tiles_t;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) v |= (uint32_t)plane[(16 * j + 4 * q + b) * D + d] << (8 * b);
+            w[q] = v;
+        }
+        *reinterpret_cast<uint4 *>(o + 16 * row) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // argmax over bf16 rows: grid (chunks, rows); each CTA reduces its chunk to
 // (value, index), the last CTA of a row (arrival counter) reduces the chunk
 // results in chunk order.  Ties resolve to the lowest index.

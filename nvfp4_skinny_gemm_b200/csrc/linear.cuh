@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             if (*s_abort) {
                 // let every copy still in flight land before the CTA exits
                 for (int64_t i = issued > LIN_STAGES ? issued - LIN_STAGES : 0; i < issued; ++i)
-                    mbar_wait(&full[i % LIN_STAGES], (uint32_t)((i / LIN_STAGES) & 1), 102);
+                    mbar_wait_drain(&full[i % LIN_STAGES], (uint32_t)((i / LIN_STAGES) & 1), 102);
             }
         } else {
             pdl_wait();
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             if (!ok) {
                 // drain: wait for every MMA issued so far before TMEM is freed
                 tc_commit(drain);
-                mbar_wait(drain, 0, 105);
+                mbar_wait_drain(drain, 0, 105);
             }
         }
         __syncwarp();

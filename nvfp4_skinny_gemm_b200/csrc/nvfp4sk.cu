@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -48,7 +49,7 @@ int cuda_fail(cudaError_t e, const char *what)
 struct DevInfo {
     int sms = 0;
     int major = 0, minor = 0;
-    bool ready = false;
+    std::atomic<bool> ready{false};   // set (release) after the fields above are filled
 };
 constexpr int MAX_DEV = 64;
 DevInfo g_dev[MAX_DEV];
@@ -71,9 +72,9 @@ int device_info(DevInfo **out)
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= MAX_DEV) return fail(NVFP4SK_ERR_DEVICE, "device id %d out of range", dev);
     DevInfo &d = g_dev[dev];
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!d.ready) {
+        if (!d.ready.load(std::memory_order_relaxed)) {
             if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
                 return cuda_fail(e, "cudaDeviceGetAttribute");
             cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -95,7 +96,7 @@ int device_info(DevInfo **out)
             unsigned long long t = (unsigned long long)g_opt_timeout_ns;
             if ((e = cudaMemcpyToSymbol(g_timeout_ns, &t, sizeof t)) != cudaSuccess)
                 return cuda_fail(e, "cudaMemcpyToSymbol(timeout)");
-            d.ready = true;
+            d.ready.store(true, std::memory_order_release);
         }
     }
     *out = &d;
@@ -565,6 +566,26 @@ nvfp4sk_status kv_append_fp8(const void *k_new, const void *v_new, int64_t ld_ne
                     "kv_append_kernel");
 }
 
+nvfp4sk_status kv_v_pages_to_tiled(const uint8_t *v_token_major, uint8_t *v_tiled, int64_t n_planes, int D,
+                                   int page_size, nvfp4sk_stream_t stream)
+{
+    if (n_planes == 0) return NVFP4SK_OK;
+    if (!v_token_major || !v_tiled) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (n_planes < 0 || n_planes > INT32_MAX || D < 8 || D % 8 || page_size < 16 || page_size % 16 ||
+        (int64_t)D * page_size > KVT_MAX_PLANE)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need D %% 8 == 0, page_size %% 16 == 0, D*page_size <= %d",
+                    KVT_MAX_PLANE);
+    if (!al16(v_token_major) || !al16(v_tiled)) return fail(NVFP4SK_ERR_MISALIGNED, "planes must be 16-byte aligned");
+    const uint8_t *a = v_token_major, *b = v_tiled;
+    const int64_t total = n_planes * D * page_size;
+    if (a < b + total && b < a + total) return fail(NVFP4SK_ERR_INVALID_ARG, "source and destination overlap");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    return launched(launch(kv_v_to_tiled_kernel, dim3((unsigned)n_planes), dim3(256), 0, (cudaStream_t)stream, 1,
+                           v_token_major, v_tiled, D, page_size),
+                    "kv_v_to_tiled_kernel");
+}
+
 // Argmax workspace: arrival counters int32 [rows] at offset 0 (fixed
 // capacity), then per-chunk values fp32 [rows][nch] and indices i32 [rows][nch].
 constexpr int64_t AMX_MAX_ROWS = 4096;
@@ -668,7 +689,9 @@ constexpr size_t LIN_NOALLOC_SCRATCH_BYTES = LIN_COUNTER_BYTES + (size_t)LIN_NOA
 static __device__ __align__(256) uint8_t g_linear_noalloc_scratch[LIN_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-uint8_t *g_noalloc_ptr[MAX_DEV];
+// Device address of the scratch array per device id; published with a release
+// store once looked up, read with acquire loads (no lock on the fast path).
+std::atomic<uint8_t *> g_noalloc_ptr[MAX_DEV];
 std::mutex g_noalloc_mu;
 
 int noalloc_scratch(uint8_t **out)
@@ -677,16 +700,19 @@ int noalloc_scratch(uint8_t **out)
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= MAX_DEV) return fail(NVFP4SK_ERR_DEVICE, "device id %d out of range", dev);
-    if (!g_noalloc_ptr[dev]) {
+    uint8_t *p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
-            void *p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_linear_noalloc_scratch);
-            if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(linear scratch)");
-            g_noalloc_ptr[dev] = (uint8_t *)p;
+        p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            void *a = nullptr;
+            e = cudaGetSymbolAddress(&a, g_linear_noalloc_scratch);
+            if (e != cudaSuccess || !a) return cuda_fail(e, "cudaGetSymbolAddress(linear scratch)");
+            p = (uint8_t *)a;
+            g_noalloc_ptr[dev].store(p, std::memory_order_release);
         }
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return NVFP4SK_OK;
 }
 }  // namespace

@@ -48,6 +48,7 @@ _SIGS = {
     "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
                                _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kv_page_restore": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
+    "kv_v_pages_to_tiled": (_int, [_vp, _vp, _i64, _int, _int, _vp]),
     "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kv_append_fp8": (_int, [_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp, _vp]),
@@ -150,10 +151,28 @@ def get_option(opt):
     return load().nvfp4sk_get_option(opt)
 
 
+# default workspaces whose arrival counters must read zero when a call starts
+_COUNTER_KINDS = ("linear", "argmax")
+
+
+def _rezero_counter_workspaces():
+    """Zero the default linear / argmax workspaces of every device: a call whose
+    device wait ran out can leave their arrival counters non-zero, and the next
+    call on the same workspace would count stale arrivals."""
+    for (dev, kind), ws in _default_ws.items():
+        if kind in _COUNTER_KINDS and ws.buf is not None:
+            ws.buf.zero_()
+
+
 def device_status(stream=None):
-    """(status code, site): synchronises the stream, reads and clears the error word."""
+    """(status code, site): synchronises the stream, reads and clears the error
+    word.  On a non-zero status the default linear and argmax workspaces are
+    zeroed again (stream-ordered on the current stream), as the C ABI's
+    workspace rule asks of every caller-owned workspace after a failure."""
     site = _int(0)
     rc = load().nvfp4sk_get_device_status(_stream(stream), ctypes.byref(site))
+    if rc != 0:
+        _rezero_counter_workspaces()
     return rc, site.value
 
 
@@ -233,6 +252,16 @@ def kv_page_restore(src_pool, src_ids, dst_pool, dst_ids, page_bytes, n=None, st
     n = src_ids.numel() if n is None else n
     _call("kv_page_restore", _d(src_pool), _d(src_ids), _d(dst_pool), _d(dst_ids), n,
           page_bytes, src_pool.numel() // page_bytes, dst_pool.numel() // page_bytes, _stream(stream))
+
+
+def v_pages_to_tiled(v_token_major, v_tiled=None, stream=None):
+    """Token-major V planes u8 [n, page_size, D] -> the tiled plane layout the
+    attention reads, u8 [n, D*page_size] (a byte permutation)."""
+    n, P, D = v_token_major.shape
+    if v_tiled is None:
+        v_tiled = torch.empty(n, D * P, dtype=torch.uint8, device=v_token_major.device)
+    _call("kv_v_pages_to_tiled", _d(v_token_major), _d(v_tiled), n, D, P, _stream(stream))
+    return v_tiled
 
 
 def rmsnorm_quantize(x, w, eps, out, act=None, stream=None, g_in=None):

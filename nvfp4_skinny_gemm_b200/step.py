@@ -129,25 +129,8 @@ class VerifyModel:
             del w
         torch.cuda.empty_cache()
 
-        # paged FP8 cache: planes (layer, K|V) x pool pages x 32 KB
-        self.n_log = math.ceil((ctx_len + T) / P)
-        self.n_pool = self.n_log + 8
-        g = I.rng(4, 500)
-        self.page_table_h = g.permutation(self.n_pool)[:self.n_log].astype(np.int32)
-        self.page_table = torch.from_numpy(self.page_table_h).to(self.dev)
-        self.kv = self._random_fp8((n_layers, 2, self.n_pool, PAGE_BYTES), 4, 501)
-        self.k_scale = torch.full((n_layers, Hkv), 0.02, dtype=torch.float32, device=self.dev)
-        self.v_scale = torch.full((n_layers, Hkv), 0.02, dtype=torch.float32, device=self.dev)
-        # prefix cache (hot cache of the previous agent turn) and restore ids
-        self.prefix_tokens = int(round(prefix_frac * ctx_len))
-        self.n_prefix_pages = math.ceil(self.prefix_tokens / P)
-        self.n_src = self.n_prefix_pages + 16
-        self.src = self._random_fp8((n_layers, 2, self.n_src, PAGE_BYTES), 4, 502)
-        src_pages = g.permutation(self.n_src)[:self.n_prefix_pages]
-        planes = np.arange(n_layers * 2)[:, None]
-        self.src_ids = torch.from_numpy((planes * self.n_src + src_pages[None, :]).ravel().astype(np.int32)).to(self.dev)
-        self.dst_ids = torch.from_numpy(
-            (planes * self.n_pool + self.page_table_h[None, :self.n_prefix_pages]).ravel().astype(np.int32)).to(self.dev)
+        self.prefix_frac, self._cache_seed = prefix_frac, seed + first_layer
+        self.set_context(ctx_len)
 
         # activations (static buffers)
         self.h = torch.empty(T, H, dtype=torch.bfloat16, device=self.dev)
@@ -162,13 +145,57 @@ class VerifyModel:
         self.ids = torch.empty(T, dtype=torch.int32, device=self.dev)
         self.G = torch.ones(n_layers * self.SITES + 1, dtype=torch.float32, device=self.dev)
 
-    def _random_fp8(self, shape, *seed):
-        """Random finite E4M3 bytes (never the NaN codes 0x7F / 0xFF)."""
+    def set_context(self, ctx_len):
+        """(Re)build the paged FP8 cache for ctx_len cached tokens, keeping the
+        weights: planes (layer, K|V) x pool pages x 32 KB in a randomly
+        permuted pool, the prefix cache holding round(prefix_frac * ctx_len)
+        tokens, and the restore ids.  CUDA graphs captured before hold the old
+        buffers and must be captured again."""
+        P, T, n_layers = I.PAGE, self.T, self.n_layers
+        self.kv = self.src = None
+        if self.dev.type == "cuda":
+            torch.cuda.empty_cache()
+        self.L = ctx_len
+        self.n_log = math.ceil((ctx_len + T) / P)
+        self.n_pool = self.n_log + 8
+        g = I.rng(4, 500)
+        self.page_table_h = g.permutation(self.n_pool)[:self.n_log].astype(np.int32)
+        self.page_table = torch.from_numpy(self.page_table_h).to(self.dev)
+        # prefix cache (hot cache of the previous agent turn) and restore ids
+        self.prefix_tokens = int(round(self.prefix_frac * ctx_len))
+        self.n_prefix_pages = math.ceil(self.prefix_tokens / P)
+        self.n_src = self.n_prefix_pages + 16
+        self.kv = torch.empty(n_layers, 2, self.n_pool, PAGE_BYTES, dtype=torch.uint8, device=self.dev)
+        self.src = torch.empty(n_layers, 2, self.n_src, PAGE_BYTES, dtype=torch.uint8, device=self.dev)
+        self.k_scale = torch.empty(n_layers, I.N_KV_HEADS, dtype=torch.float32, device=self.dev)
+        self.v_scale = torch.empty(n_layers, I.N_KV_HEADS, dtype=torch.float32, device=self.dev)
+        self._fill_cache(self._cache_seed)
+        src_pages = g.permutation(self.n_src)[:self.n_prefix_pages]
+        planes = np.arange(n_layers * 2)[:, None]
+        self.src_ids = torch.from_numpy((planes * self.n_src + src_pages[None, :]).ravel().astype(np.int32)).to(self.dev)
+        self.dst_ids = torch.from_numpy(
+            (planes * self.n_pool + self.page_table_h[None, :self.n_prefix_pages]).ravel().astype(np.int32)).to(self.dev)
+
+    def _fill_cache(self, seed):
+        """Cache contents as in the single-layer attention workload: K and V
+        ~ N(0,1), stored as FP8 E4M3 with one scale per (layer, KV head, K|V)
+        = amax/448 over that head's live and prefix-cache planes (so the
+        restored pages and the live ones share a scale), cast with torch's
+        float8_e4m3fn conversion.  Drawn on the GPU (torch generator)."""
+        Hkv = I.N_KV_HEADS
         gen = torch.Generator(device=self.dev)
-        gen.manual_seed(int(np.random.default_rng([42, *seed]).integers(1 << 62)))
-        x = torch.randint(0, 0x7E, shape, dtype=torch.uint8, device=self.dev, generator=gen)
-        sign = torch.randint(0, 2, shape, dtype=torch.uint8, device=self.dev, generator=gen)
-        return x | (sign << 7)
+        gen.manual_seed(int(np.random.default_rng([42, 4, 501, seed]).integers(1 << 62)))
+        for l in range(self.n_layers):
+            for kv, scale in ((0, self.k_scale), (1, self.v_scale)):
+                live = torch.randn(self.n_pool, Hkv, PAGE_BYTES // Hkv, generator=gen, device=self.dev)
+                pre = torch.randn(self.n_src, Hkv, PAGE_BYTES // Hkv, generator=gen, device=self.dev)
+                amax = torch.maximum(live.abs().amax(dim=(0, 2)), pre.abs().amax(dim=(0, 2)))
+                sc = amax / 448.0
+                scale[l].copy_(sc)
+                for buf, x in ((self.kv, live), (self.src, pre)):
+                    buf[l, kv].view(-1, Hkv, PAGE_BYTES // Hkv).copy_(
+                        (x / sc[None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8))
+                del live, pre
 
     # ------------------------------------------------------------------ pools
     def k_pool(self, l):

@@ -194,6 +194,7 @@ def fake_model(monkeypatch, n_layers, ctx_len, T=16, lm_head=True, static=True):
     fake = FakeLib()
     monkeypatch.setattr(step, "nv", fake)
     monkeypatch.setattr(step.torch, "randn", lambda *a, **k: FakeWeight(*a))
+    monkeypatch.setattr(step.VerifyModel, "_fill_cache", lambda self, seed: None)
     monkeypatch.setattr(step.Linear, "from_fp32",
                         staticmethod(lambda w: step.Linear(object(), torch.ones(1), *w.shape)))
     m = step.VerifyModel(n_layers=n_layers, ctx_len=ctx_len, T=T, weights="device", device="cpu",

@@ -126,6 +126,11 @@ def test_host_checks_reject_bad_arguments_before_the_device():
         (E_SHAPE, "tree_accept_greedy", A, A, A, 33, A, A, A, None),
         # kv_compact_accepted(k, v, layer_stride, n_layers, Hkv, D, n_pool, P, page_table, ctx_len, path, n, T, stream)
         (E_SHAPE, "kv_compact_accepted", A, A, 1 << 20, 64, 4, 136, 8, 64, A, 100, A, A, 16, None),
+        # kv_v_pages_to_tiled(src, dst, n_planes, D, page_size, stream)
+        (E_SHAPE, "kv_v_pages_to_tiled", A, A + (1 << 20), 4, 12, 64, None),
+        (E_SHAPE, "kv_v_pages_to_tiled", A, A + (1 << 20), 4, 256, 128, None),
+        (E_ALIGN, "kv_v_pages_to_tiled", MIS, A + (1 << 20), 4, 128, 64, None),
+        (E_ARG, "kv_v_pages_to_tiled", A, A + 8192, 4, 128, 64, None),
         # nvfp4sk_debug_encode(x, n, e2m1, e4m3, stream)
         (E_ARG, "nvfp4sk_debug_encode", A, -1, A, A, None),
     ]
@@ -178,7 +183,37 @@ def test_binding_rejects_host_tensors():
         lambda: lib.tree_attn(bf(16, 24, 128), h(2, 4, 64, 128), h(2, 4, 8192), h(2, dt=torch.int32), 10,
                               h(16, dt=torch.int32), g, g, out=bf(16, 24, 128), ws=HostWs()),
         lambda: lib.argmax(bf(16, 4096), idx=h(16, dt=torch.int32), ws=HostWs()),
+        lambda: lib.v_pages_to_tiled(h(2, 64, 128), h(2, 8192)),
     ]
     for i, call in enumerate(calls):
         with pytest.raises(ValueError, match="device tensor"):
             call()
+
+
+def test_failing_status_rezeroes_counter_workspaces(monkeypatch):
+    """After a failing device status the binding zeroes its default linear and
+    argmax workspaces (their arrival counters may be stale after a wait ran
+    out) and leaves the others alone; a clean status touches nothing."""
+    import torch
+
+    class FakeWs:
+        def __init__(self):
+            self.buf = torch.full((64,), 7, dtype=torch.uint8)
+
+    spaces = {(0, k): FakeWs() for k in ("linear", "argmax", "attn", "quantize")}
+    monkeypatch.setattr(lib, "_default_ws", spaces)
+    state = {"rc": 0}
+
+    class FakeLib:
+        def nvfp4sk_get_device_status(self, stream, site):
+            return state["rc"]
+
+    monkeypatch.setattr(lib, "load", lambda path=None: FakeLib())
+    monkeypatch.setattr(lib, "_stream", lambda s=None: None)
+    assert lib.device_status()[0] == 0
+    assert all(int(w.buf.min()) == 7 for w in spaces.values())
+    state["rc"] = -6
+    assert lib.device_status()[0] == -6
+    for (_, kind), w in spaces.items():
+        want = 0 if kind in ("linear", "argmax") else 7
+        assert int(w.buf.min()) == want and int(w.buf.max()) == want, kind

@@ -86,11 +86,15 @@ def test_one_layer_teacher_forced(oracle, static, T, chain, L, layer):
     assert np.array_equal(m.k_pool(0).cpu().numpy(), kp)
     assert np.array_equal(m.v_pool(0).cpu().numpy(), vp)
     a = oracle.tree_attn(qkv_gpu[:, :qd].reshape(T, I.N_Q_HEADS, I.HEAD_DIM), kp, vp, pt, L, parent, ks, vs)
-    # the cache holds uniformly random E4M3 codes, so outputs reach |o| ~ 9: the
-    # bar adds the bf16 output rounding (2^-9 |o|) and the two-term operand
-    # error, as for the other small attention cases
+    # the cache holds N(0,1) K/V in FP8 with amax/448 scales, as the
+    # single-layer attention workload does: at 23,552 cached tokens the stated
+    # bar (2e-3 absolute) applies as it is; shorter contexts give larger
+    # outputs and also allow the bf16 output rounding and the two-term operand
+    # error, as the other small attention cases do
     err_a = np.abs(attn_gpu.reshape(a.shape) - a)
-    assert np.all(err_a <= 2e-3 + 2.0 ** -8 * np.abs(a)), err_a.max()
+    bar = 2e-3 if L >= I.CTX_MAX else 2e-3 + 2.0 ** -8 * np.abs(a)
+    print(f"layer {layer} at {L} tokens: attention max abs err {err_a.max():.2e}, max |o| {np.abs(a).max():.2e}")
+    assert np.all(err_a <= bar), err_a.max()
     # rest of the layer from the GPU's attention output
     a = attn_gpu.reshape(T, qd)
     h1 = _bf16(h + lin(a, "o", 1))
