@@ -137,6 +137,11 @@ NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint
  * a_prepared, g_a: activation from nvfp4_quantize_act (act_prepared) or the
  *   fused quantisers; 1 <= M <= 16 rows.
  * w_prepared, g_w: weight from nvfp4_prepare_weight (+ its tensor scale).
+ *   With programmatic dependent launch on (the default) the first weight
+ *   units are requested before the preceding kernel on the stream has
+ *   finished, and the kernel lets its own dependents start at once: the
+ *   weights must not be written by a kernel that may still run (see
+ *   tree_attn_fp8kv for the rule).
  * K % 64 == 0, 1 <= N <= 524288; prepared operands 16-byte aligned.
  * residual: NULL or bf16 [M][ldy] added before rounding (may alias y).
  * y: bf16 [M][ldy], ldy >= N.
@@ -205,6 +210,16 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const
  *   nvfp4_linear reads (K = Hq*D, row i = node i), exactly as
  *   nvfp4_quantize_act(out, g_in = g_act) would; g_act must then be non-NULL.
  * ws: tree_attn_workspace_bytes(...) bytes.
+ * Ordering: with programmatic dependent launch on (NVFP4SK_OPT_PDL, the
+ *   default), the kernel reads page_table and starts loading context pages
+ *   (positions < ctx_len) before the preceding kernel on the stream has
+ *   finished, as nvfp4_linear does with its weights.  No kernel that may
+ *   still run when this one starts may write them: the immediately preceding
+ *   kernel, and, when that kernel lets its dependents start before it waits
+ *   on its own predecessor (nvfp4_linear and the static-scale quantisers do),
+ *   that predecessor in turn.  kv_append_fp8 waits first, so "append, then
+ *   attention" is safe.  Everything else (q, parent, the scales, the tree
+ *   slots) is read after the preceding kernel has finished.
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
 NVFP4SK_API nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D,

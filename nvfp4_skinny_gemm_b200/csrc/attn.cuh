@@ -271,18 +271,29 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    pdl_wait();
+    // Every role but the producer waits for the preceding kernel here (the
+    // queries, the tree and the scales may be its output); the producer waits
+    // only before its first tree page, see below.
+    if (warp != 0) pdl_wait();
     pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         // lane st feeds stage st (pages st, st + 8, ...): the copies of
         // different stages are issued by different threads, which keeps
-        // several page loads in flight per SM.
+        // several page loads in flight per SM.  Context pages of the first
+        // round are requested before the wait on the preceding kernel (the
+        // context and the page table are not written by it; the tree slots,
+        // which the K/V append of the same step writes, are loaded after it).
         if (lane < ATT_STAGES) {
             const int st = (int)lane;
             int last = -1;
+            bool waited = false;
             for (int i = st; i < n_pages; i += ATT_STAGES) {
+                if (!waited && (i >= ATT_STAGES || (int64_t)(pg0 + i + 1) * ATT_P > p.ctx_len)) {
+                    pdl_wait();
+                    waited = true;
+                }
                 if (i >= ATT_STAGES &&
                     !mbar_wait(&kv_empty[st], (uint32_t)(((i / ATT_STAGES) - 1) & 1), 301, s_abort))
                     break;
@@ -301,8 +312,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 }
                 last = i;
             }
+            if (!waited) pdl_wait();
             // on abort, let this stage's last copy land before the CTA exits
             if (*s_abort && last >= 0) mbar_wait_drain(&kv_full[st], (uint32_t)((last / ATT_STAGES) & 1), 303);
+        } else {
+            pdl_wait();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ QK issuer
