@@ -291,7 +291,7 @@ def linear_launches(model):
 
 
 def attention_launches(model):
-    """The step's attention calls (split + combine, with the fused static NVFP4
+    """The step's attention calls (split with the fused combine, and the static NVFP4
     output), one per layer over that layer's pools, back to back."""
     from nvfp4_skinny_gemm_b200 import inputs as I
     from nvfp4_skinny_gemm_b200 import lib as nv
@@ -330,7 +330,7 @@ def run_ours(args, world, rank, local):
         assert rc == 0, f"device status {rc} at site {site}"
         graph = capture(stream, model.step)
         lin_graph = capture(stream, lambda: linear_launches(model))     # the dominant kernel alone, same launches
-        attn_graph = capture(stream, lambda: attention_launches(model))  # the attention pairs alone
+        attn_graph = capture(stream, lambda: attention_launches(model))  # the attention calls alone
         load_inputs()
         for _ in range(max(3, args.warmup)):
             graph.replay()
@@ -359,7 +359,7 @@ def run_ours(args, world, rank, local):
         assert rc == 0, f"device status {rc} at site {site}"
 
         # ---- dominant kernel: all linear launches of one step, back to back;
-        #      then the 64 attention launch pairs of one step, back to back
+        #      then the 64 attention calls of one step, back to back
         reps = max(3, min(20, args.steps))
         t_lin = time_graph(lin_graph, stream, reps)
         t_attn = time_graph(attn_graph, stream, reps)
@@ -429,14 +429,14 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_step": lin_bytes, "launches": n_lin,
                      "us_per_step_of_linears": round(t_lin * 1e6, 1),
                      "traffic": traffic},
-        "roofline_attn": {"kernel": f"tree_attn_split_kernel + tree_attn_combine_kernel ({model.n_layers} launch "
-                                    f"pairs of one step, back to back)",
+        "roofline_attn": {"kernel": f"tree_attn_split_kernel with the fused combine ({model.n_layers} calls of "
+                                    f"one step, back to back)",
                           "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
                           "frac": round(attn_gbs / peak, 4),
                           "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                           "algorithmic_bytes_per_step": attn_bytes,
-                          "algorithmic_bytes_per_launch_pair": attn_bytes // model.n_layers,
-                          "us_per_launch_pair": round(t_attn / model.n_layers * 1e6, 2), "traffic": None},
+                          "algorithmic_bytes_per_call": attn_bytes // model.n_layers,
+                          "us_per_call": round(t_attn / model.n_layers * 1e6, 2), "traffic": None},
         "no_restore": {"value": world / t_nr, "unit": UNIT, "ms_per_step": round(t_nr * 1e3, 3),
                        "note": "the same step without the per-step kv_page_restore of the prefix "
                                "(the pages restore once per agent turn)"},

@@ -32,16 +32,17 @@
  *     problem in a device error word and returns; nvfp4sk_get_device_status()
  *     reports and clears it.
  *   - A "workspace" is caller-owned device scratch of at least the size the
- *     matching *_workspace_bytes() query returns.  The nvfp4_linear and
- *     argmax_rows_bf16 workspaces start with arrival counters that must read
- *     zero when a call starts: zero-fill such a workspace once when it is
- *     allocated and do not lend it to another kind of call (tree_attn_fp8kv
- *     and nvfp4_quantize_act leave partial results in theirs); every
+ *     matching *_workspace_bytes() query returns.  The nvfp4_linear,
+ *     argmax_rows_bf16 and tree_attn_fp8kv workspaces start with arrival
+ *     counters that must read zero when a call starts: zero-fill such a
+ *     workspace once when it is allocated and do not lend it to another kind
+ *     of call (nvfp4_quantize_act leaves partial results in its own); every
  *     successful call leaves its counters zero again.  A call whose device
  *     status later reads non-zero (a wait that ran out, above all) may leave
  *     counters non-zero: after nvfp4sk_get_device_status returns an error,
- *     zero every nvfp4_linear and argmax_rows_bf16 workspace again before its
- *     next use (the ctypes binding does this for its default workspaces).
+ *     zero every nvfp4_linear, argmax_rows_bf16 and tree_attn_fp8kv workspace
+ *     again before its next use (the ctypes binding does this for its
+ *     default workspaces).
  *     Calls that share one workspace must be stream-ordered.
  *   - Scalars such as tensor scales are device pointers, so no call syncs.
  *   - Error codes are negative; nvfp4sk_last_error() gives a message for the
@@ -155,6 +156,27 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *
                                         nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_linear_wide -- the same NVFP4 linear for many tokens at once: the
+ * linears of the suffix prefill (section "KV-cache reuse between agent
+ * steps": after the reused prefix is restored only the new suffix of the
+ * prompt is prefilled, hundreds of tokens in one forward pass).
+ * Y[s][n] = bf16( g_a*g_w * sum_b s_a[s,b] s_w[n,b] sum_{k in b} a[s,k] w[n,k]
+ * (+ residual[s][n]) ), fp32 accumulation, for s < S.
+ *
+ * a_prepared: the S x K activation in the weight tile image, i.e. what
+ *   nvfp4_prepare_weight(codes, scales, S, K, ...) writes for its canonical
+ *   NVFP4 codes and scales (tokens take the place of weight rows);
+ *   nvfp4_prepared_weight_bytes(S, K) bytes.  g_a: its tensor scale.
+ * w_prepared, g_w: as nvfp4_linear.  S >= 1, N >= 1, K % 64 == 0.
+ * residual: NULL or bf16 [S][ldy] added before rounding (may alias y).
+ * y: bf16 [S][ldy], ldy >= N.  No workspace: every output tile is computed
+ * whole by one CTA (tiles of 128 weight rows x 256 tokens).
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API nvfp4sk_status nvfp4_linear_wide(const uint8_t *a_prepared, const float *g_a, int64_t S,
+                                             const uint8_t *w_prepared, const float *g_w, int64_t N, int64_t K,
+                                             const void *residual, void *y, int64_t ldy, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_linear_noalloc -- nvfp4_linear for callers that cannot allocate.
  * (The pages have no counterpart: this is a deployment variant.)
  *
@@ -209,7 +231,9 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const
  *   the static tensor scale *g_act into the prepared activation image that
  *   nvfp4_linear reads (K = Hq*D, row i = node i), exactly as
  *   nvfp4_quantize_act(out, g_in = g_act) would; g_act must then be non-NULL.
- * ws: tree_attn_workspace_bytes(...) bytes.
+ * ws: tree_attn_workspace_bytes(...) bytes, zero-filled at allocation (it
+ *   starts with the per-head arrival counters of the fused combine; see the
+ *   workspace rule above).
  * Ordering: with programmatic dependent launch on (NVFP4SK_OPT_PDL, the
  *   default), the kernel reads page_table and starts loading context pages
  *   (positions < ctx_len) before the preceding kernel on the stream has
@@ -228,6 +252,30 @@ NVFP4SK_API nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, i
                                const int32_t *parent, const float *k_scale, const float *v_scale,
                                float sm_scale, void *out, const float *g_act, uint8_t *act_prepared,
                                void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * causal_attn_fp8kv -- the attention of the suffix prefill (section "KV-cache
+ * reuse between agent steps": the new suffix of the prompt is prefilled
+ * after the reused prefix pages are restored): T <= 128 new tokens at
+ * positions ctx_len .. ctx_len+T-1, whose K/V are already in the cache
+ * (kv_append_fp8), attend causally: token i, head hq sees every position up
+ * to ctx_len + i.  Same layouts, scales and output as tree_attn_fp8kv with a
+ * chain (parent[i] = i-1), computed 128 queries of one query head per CTA
+ * (grid: splits x Hq), so each K/V page is read once per 128 queries.
+ * Longer suffixes are cut into blocks of up to 128 tokens, block b at
+ * ctx_len = start + 128 b.  Hq % Hkv == 0, Hq <= 64; D == 128,
+ * page_size == 64.  No NVFP4 output.
+ * ws: causal_attn_workspace_bytes(...) bytes, zero-filled at allocation
+ *   (arrival counters at its start, as for tree_attn_fp8kv).
+ * Ordering with programmatic dependent launch: as tree_attn_fp8kv (context
+ *   pages before the preceding kernel finishes, the T new positions after).
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t causal_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len);
+NVFP4SK_API nvfp4sk_status causal_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D,
+                                             const uint8_t *k_pool, const uint8_t *v_pool, int64_t n_pool_pages,
+                                             int page_size, const int32_t *page_table, int64_t ctx_len,
+                                             const float *k_scale, const float *v_scale, float sm_scale, void *out,
+                                             void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
 
 /* Conversion of V pages written token-major (plane = [page_size slots][D]
  * bytes, the same layout as the K pool) into the tiled plane layout that
@@ -263,14 +311,17 @@ NVFP4SK_API nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_
  * exactly as nvfp4_quantize_act, with the same outputs: g_in NULL = dynamic
  * tensor scale (amax over the whole y), else the static scale *g_in (a
  * calibrated checkpoint's; one launch with no grid-wide reduction).  x bf16
- * [rows][n] (row stride n), w bf16 [n].  rows <= 16, n % 64 == 0, n <= 8192. */
+ * [rows][n] (row stride n), w bf16 [n].  rows <= 16, n % 64 == 0, n <= 8192;
+ * with a static g_in and only the canonical outputs (act_prepared NULL) any
+ * number of rows (the suffix prefill). */
 NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows,
                                                   int64_t n, const float *g_in, uint8_t *codes, uint8_t *scales,
                                                   float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
                                                   nvfp4sk_stream_t stream);
 /* h = silu(gu[:, :F]) * gu[:, F:] rounded to bf16, then NVFP4-quantised
  * (g_in NULL = dynamic g, else static *g_in), same outputs.  gu bf16
- * [rows][2F].  rows <= 16, F % 64 == 0, rows * F <= 524288. */
+ * [rows][2F].  rows <= 16, F % 64 == 0, rows * F <= 524288; with a static
+ * g_in and only the canonical outputs any number of rows. */
 NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, const float *g_in,
                                                  uint8_t *codes, uint8_t *scales, float *g_out, uint8_t *act_prepared,
                                                  void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);

@@ -2,32 +2,43 @@
 // paged KV cache on sm_100a tensor cores (flash-decoding: split over the
 // context, then combine).
 //
-// Grid (splits, Hkv); one CTA = one KV head x one contiguous range of pages.
-// The 128 MMA rows are (query head w of the group, node i) -> row 16*w + i
-// (rows past group*16 are zero padding).  Per page of 64 tokens:
+// Tree mode (the verify step): grid (splits, Hkv); one CTA = one KV head x
+// one contiguous range of pages.  The 128 MMA rows are (query head w of the
+// group, node i) -> row 16*w + i (rows past group*16 are zero padding), and a
+// node sees the tree slots of its ancestors and itself.  Causal mode (the
+// suffix prefill): grid (splits, Hq); the 128 MMA rows are up to 128 queries
+// of one query head, query i at position ctx_len + i sees every position up
+// to its own.  Per page of 64 tokens:
 //   S = Q K^T   tcgen05.mma kind::f8f6f4, M=128, N=64, K=32 per instruction;
 //               Q enters as two E4M3 terms (hi + lo) of the row-scaled bf16
 //               query, K as the cached E4M3 codes (128-byte-swizzled TMA
 //               tile); fp32 S in tensor memory.
 //   softmax     one thread per row: S row -> registers (tcgen05.ld), ancestor
 //               mask on the page that holds the tree, running max in the
-//               log2 domain, P' = 2^(s - m + 6) as two E4M3 terms (hi + lo)
-//               stored to shared memory in the MMA's core-matrix layout.
-//               O is rescaled in tensor memory only when a row max grows by
-//               more than 2^2.
-//   O += P V    M=128, N=144, K=32: the V pages are kept in HBM in the
-//               core-matrix layout, so one bulk copy lands the operand; 16
-//               extra operand rows (one of them all ones) make column 128 of
-//               O the row sum of P', accumulated in fp32 by the tensor core.
+//               log2 domain, P' = 2^(s - m) in f16 (ex2.approx.f16x2 on the
+//               f16-rounded exponent), stored to shared memory in the MMA's
+//               core-matrix layout.  O is rescaled in tensor memory only when
+//               a row max grows by more than 2^2.
+//   O += P V    tcgen05.mma kind::f16, M=128, N=144, K=16: the page's V codes
+//               (kept in HBM in a tiled core-matrix layout, one bulk copy per
+//               page) are widened E4M3 -> f16 (exact) into the operand image
+//               by the softmax threads; 16 extra operand rows (one of them all
+//               ones) make column 128 of O the row sum of P', accumulated in
+//               fp32 by the tensor core.
 // Two softmax warpgroups take alternate pages, each with its own S and O
 // accumulators in tensor memory and its own running max, so that two pages
-// are in the exponent / packing stage at once; their results are merged in
-// the epilogue.
+// are in the exponent stage at once; their results are merged in the
+// epilogue.
 // Warp roles: 0 producer (lane s feeds stage s of an 8-stage ring: TMA K page
-// + bulk V page), 1 TMEM allocation + QK issue (one thread), 10 PV issue (one
-// thread), 2-5 and 6-9 softmax.  The two issuers run independently, so a
-// group's next scores never wait behind the other group's product.
-// The split results (O / l, m, l per row) are merged by the combine kernel.
+// + bulk V page; context pages are requested before the wait on the
+// preceding kernel), 1 TMEM allocation + QK issue (one thread), 10 PV issue
+// (one thread), 2-5 and 6-9 softmax.  The two issuers run independently, so
+// a group's next scores never wait behind the other group's product.
+// Combine: when the grid fits on the GPU at once (splits x Hkv <= #SMs, one
+// CTA per SM), the CTAs of a KV head publish their split results (O / l, m,
+// l per row), meet on a per-head arrival counter and each CTA then finishes
+// a slice of the head's rows (fused combine, no second launch); otherwise
+// tree_attn_combine_kernel merges the split results.
 #pragma once
 #include "common.cuh"
 #include "quant.cuh"
@@ -38,29 +49,32 @@ constexpr int ATT_D = 128;
 constexpr int ATT_P = 64;
 constexpr int ATT_T = 16;
 constexpr int ATT_ROWS = 128;
-constexpr int ATT_STAGES = 10;
+constexpr int ATT_STAGES = 8;
 constexpr int ATT_THREADS = 352;
 constexpr int ATT_MAX_SPLITS = 1024;
 constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;                 // 8 KB token-major page
-constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB core-matrix page
-constexpr uint32_t ATT_ONES_BYTES = 16 * ATT_P;                 // 16 operand rows: ones, then zeros
-constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES + ATT_ONES_BYTES;   // 17 KB
-constexpr uint32_t ATT_PB_BYTES = ATT_ROWS * ATT_P;             // one E4M3 term of P
-constexpr uint32_t ATT_OFF_P = ATT_STAGES * ATT_STAGE_BYTES;    // P[2 groups] x (hi | lo)
-constexpr uint32_t ATT_OFF_X = ATT_OFF_P + 4 * ATT_PB_BYTES;    // float exchange [2][2][128]
-constexpr uint32_t ATT_OFF_BAR = ATT_OFF_X + 2048;
+constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB tiled page
+constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES; // 16 KB
+constexpr uint32_t ATT_NO = ATT_D + 16;                         // O columns: 128 dims + row sum block
+constexpr uint32_t ATT_P16_BYTES = ATT_ROWS * ATT_P * 2;        // P of one page in f16: 16 KB
+constexpr uint32_t ATT_V16_BYTES = ATT_NO * ATT_P * 2;          // V of one page in f16 + ones block: 18 KB
+constexpr uint32_t ATT_OFF_P = ATT_STAGES * ATT_STAGE_BYTES;    // P[2 groups]
+constexpr uint32_t ATT_OFF_V16 = ATT_OFF_P + 2 * ATT_P16_BYTES; // V16[2 groups]
+constexpr uint32_t ATT_OFF_X = ATT_OFF_V16 + 2 * ATT_V16_BYTES; // float exchange [2][2][128]
+constexpr uint32_t ATT_OFF_C = ATT_OFF_X + 2048;                // combine: bf16 rows as float [2][128]
+constexpr uint32_t ATT_OFF_BAR = ATT_OFF_C + 1024;
 constexpr uint32_t ATT_SMEM_BYTES = ATT_OFF_BAR + 512 + 1024;
 constexpr uint32_t ATT_TMEM_COLS = 512;
-constexpr uint32_t ATT_NO = ATT_D + 16;                         // O columns: 128 dims + row sum block
 constexpr uint32_t ATT_TM_S0 = 0, ATT_TM_S1 = 64;
 constexpr uint32_t ATT_TM_O0 = 128, ATT_TM_O1 = 288;
 constexpr uint32_t ATT_TM_Q = 448;                              // Q hi 448..479, Q lo 480..511 (A operand)
 constexpr float ATT_TAU = 2.0f;       // log2 growth of a row max that triggers an O rescale
-constexpr float ATT_PSHIFT = 6.0f;    // P' = 2^(s - m + 6) <= 2^(6 + TAU) = 256 < 448
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr uint32_t ATT_CNT_BYTES = 256;                         // per-head arrival counters (fused combine)
 static_assert(ATT_STAGE_BYTES % 1024 == 0, "K tiles need 1024-byte alignment (128-byte swizzle atoms)");
 static_assert(ATT_TM_O1 + ATT_NO <= ATT_TM_Q && ATT_TM_O0 + ATT_NO <= ATT_TM_O1 && ATT_TM_Q + 64 <= ATT_TMEM_COLS,
               "tensor memory budget");
+static_assert(ATT_SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 // Byte of (dim d, slot t) inside a V page plane: 8-dim x 16-slot core matrices
 // of 128 bytes, ordered [d/8][t/16][d%8][t%16].
@@ -69,8 +83,9 @@ __host__ __device__ __forceinline__ uint32_t v_offset(uint32_t d, uint32_t t)
     return ((d >> 3) * (ATT_P / 16) + (t >> 4)) * 128u + (d & 7u) * 16u + (t & 15u);
 }
 
-// Instruction descriptor, kind::f8f6f4: fp32 accumulate (bits 4-5 = 1), A and
-// B E4M3 (format 0), K-major, N>>3 in bits 17-22, M>>4 in bits 24-28.
+// Instruction descriptor: fp32 accumulate (bits 4-5 = 1), A and B format 0
+// (E4M3 under kind::f8f6f4, f16 under kind::f16), K-major, N>>3 in bits
+// 17-22, M>>4 in bits 24-28.
 constexpr uint32_t att_idesc(uint32_t M, uint32_t N) { return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24); }
 
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -95,49 +110,6 @@ __device__ __forceinline__ void mma_f8f6f4_ta(uint32_t d_tmem, uint32_t a_tmem, 
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-
-__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ uint32_t tmem_ld_x1(uint32_t taddr)
-{
-    uint32_t v;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float fast_exp2(float x)
 {
@@ -170,23 +142,32 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c)
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)c));
     return d;
 }
-__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b)
+__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t h)
 {
     uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(d) : "r"(h));
     return d;
 }
 
-// Four non-negative values -> E4M3 codes hi (bytes 0..3) and lo with x ~= hi + lo:
-// x is rounded to f16 (11 bits), hi = E4M3(x), lo = E4M3(x - hi) (exact f16 difference).
-__device__ __forceinline__ void split4_f16(float x0, float x1, float x2, float x3, uint32_t &hi, uint32_t &lo)
+// D[tmem] (+)= A x B^T, A and B f16 in shared memory (K-major), fp32 accumulate.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate)
 {
-    const uint32_t a = f32x2_to_f16x2(x0, x1), b = f32x2_to_f16x2(x2, x3);
-    const uint32_t ha = f16x2_to_e4m3x2(a), hb = f16x2_to_e4m3x2(b);
-    const uint32_t la = f16x2_to_e4m3x2(hsub2_u32(a, e4m3x2_to_f16x2(ha)));
-    const uint32_t lb = f16x2_to_e4m3x2(hsub2_u32(b, e4m3x2_to_f16x2(hb)));
-    hi = ha | (hb << 16);
-    lo = la | (lb << 16);
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Byte offset of (row r, column k) in a K-major f16 operand image without
+// swizzle: core matrices of 8 rows x 8 columns (16-byte rows), 8 core
+// matrices along K per 64 columns (leading byte offset 128), row groups 1 KB
+// apart (stride byte offset 1024).
+__device__ __forceinline__ uint32_t f16_core_offset(uint32_t r, uint32_t k)
+{
+    return ((r >> 3) * 8u + (k >> 3)) * 128u + (r & 7u) * 16u + (k & 7u) * 2u;
 }
 
 // x0, x1 -> (hi, lo) E4M3 pairs (byte 0 = x0, byte 1 = x1) with x ~= hi + lo, in fp32.
@@ -215,7 +196,13 @@ struct AttnParams {
     int64_t ctx_len;
     int64_t n_pool_pages;
     float sm_scale;
+    int *cnt;             // [grid.y] arrival counters of the fused combine (zero at call start)
     int T, Hq, Hkv, group, S, n_log_pages;
+    int fuse;             // 1: fused combine in the split kernel
+    int causal;           // 0: tree (grid.y = KV heads, rows 16 w + node of the group's query heads);
+                          // 1: causal chain (grid.y = query heads, row = query, T <= 128)
+    int rows_w;           // rows per query head in a CTA: 16 (tree) or 128 (causal)
+    int nheads;           // query heads per CTA: group (tree) or 1 (causal)
 };
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
@@ -237,8 +224,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     volatile uint8_t *s_page_ok = reinterpret_cast<volatile uint8_t *>(tmem_holder + 2);   // [ATT_STAGES]
     float *xch = reinterpret_cast<float *>(smem + ATT_OFF_X);                             // [2][2][128]
 
-    const int h = blockIdx.y, split = blockIdx.x;
+    const int ch = blockIdx.y, split = blockIdx.x;      // CTA head: a KV head (tree) or a query head (causal)
     const int group = p.group;
+    const int h = p.causal ? ch / group : ch;             // KV head
+    const int hq0 = p.causal ? ch : ch * group;           // first query head of the CTA's rows
+    const int rows_cta = p.nheads * p.rows_w;
     const uint32_t warp = warp_id(), lane = lane_id();
     const int pg0 = (int)((int64_t)split * p.n_log_pages / p.S);
     const int pg1 = (int)((int64_t)(split + 1) * p.n_log_pages / p.S);
@@ -318,6 +308,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else {
             pdl_wait();
         }
+        __syncwarp();          // reconverge before the CTA-wide barrier below
     } else if (warp == 1) {
         // ------------------------------------------------------------ QK issuer
         // S = Q K^T of page i into the S buffer of group i & 1, as soon as the
@@ -348,7 +339,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         __syncwarp();
     } else if (warp == 10) {
         // ------------------------------------------------------------ PV issuer
-        // O_g += P V of page j once group g has written P (hi, lo) for it
+        // O_g += P V of page j once group g has written P and the widened V
         if (lane == 0) {
             constexpr uint32_t idesc_o = att_idesc(128, ATT_NO);
             bool o_init[2] = {false, false};
@@ -358,16 +349,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if (!mbar_wait(&p_full[g], (uint32_t)((j >> 1) & 1), 311, s_abort)) { ok = false; break; }
                 tc_fence_after();
                 if (s_page_ok[j % ATT_STAGES]) {
-                    const uint32_t v_s = smem_u32(smem + (j % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES);
-                    const uint32_t p_hi = smem_u32(smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES), p_lo = p_hi + ATT_PB_BYTES;
+                    const uint32_t p_s = smem_u32(smem + ATT_OFF_P + g * ATT_P16_BYTES);
+                    const uint32_t v_s = smem_u32(smem + ATT_OFF_V16 + g * ATT_V16_BYTES);
                     const uint32_t o_t = tmem_base + (g ? ATT_TM_O1 : ATT_TM_O0);
 #pragma unroll
-                    for (int t = 0; t < ATT_P / 32; ++t) {
-                        const uint64_t vd = smem_desc(v_s + 256 * t, 128, 512, SWZ_NONE);
-                        mma_f8f6f4(o_t, smem_desc(p_hi + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o,
-                                   (o_init[g] || t > 0) ? 1u : 0u);
-                        mma_f8f6f4(o_t, smem_desc(p_lo + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o, 1u);
-                    }
+                    for (int t = 0; t < ATT_P / 16; ++t)
+                        mma_f16(o_t, smem_desc(p_s + 256 * t, 128, 1024, SWZ_NONE),
+                                smem_desc(v_s + 256 * t, 128, 1024, SWZ_NONE), idesc_o, (o_init[g] || t > 0) ? 1u : 0u);
                     o_init[g] = true;
                 }
                 tc_commit(&p_free[g]);
@@ -384,24 +372,32 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     } else {
         // ------------------------------------------------------------ softmax groups
         const int g = (int)(warp - 2) >> 2;                   // 0: even pages, 1: odd pages
+        const int gt = (int)threadIdx.x - 64 - 128 * g;       // thread index within the group
         const uint32_t qd = warp & 3;                         // TMEM sub-partition
         const int r = (int)(32 * qd + lane);                  // MMA row
-        const int w = r >> 4, node = r & 15;
-        const bool row_ok = w < group;
-        const int hq = h * group + w;
+        const int w = r / p.rows_w, node = r % p.rows_w;      // query head within the CTA, node / query
+        const bool row_ok = w < p.nheads;
+        const int hq = hq0 + w;
         const int T = p.T;
         const int64_t L = p.ctx_len;
         const uint32_t row_t = tmem_base + ((32u * qd) << 16);
         const uint32_t s_t = row_t + (g ? ATT_TM_S1 : ATT_TM_S0);
         const uint32_t o_t = row_t + (g ? ATT_TM_O1 : ATT_TM_O0);
+        uint8_t *pb = smem + ATT_OFF_P + g * ATT_P16_BYTES;
+        uint8_t *vb = smem + ATT_OFF_V16 + g * ATT_V16_BYTES;
 
         // ---- Q -> two E4M3 terms, row scaled by a power of two into [128, 256);
-        //      group g converts dims 64g .. 64g+63 of row r
+        //      group g converts dims 64g .. 64g+63 of row r.  Every global
+        //      load of the prologue is issued first, in one round trip.
         float c_row;
         uint32_t anc = 0;
+        int32_t pid = -1, pid_next = -1;
         {
             const bool has_q = row_ok && node < T;
-            const int par_l = (int)lane < T ? p.parent[lane] : -1;
+            const int par_l = (!p.causal && (int)lane < T) ? p.parent[lane] : -1;
+            const float k_sc = p.k_scale[h];
+            if (g < n_pages) pid = p.page_table[pg0 + g];
+            if (g + 2 < n_pages) pid_next = p.page_table[pg0 + g + 2];
             uint4 qraw[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
@@ -417,19 +413,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                              fabsf(__uint_as_float(wd[j] & 0xFFFF0000u))));
             }
             xch[g * 128 + r] = amax;
-            // the ones block of every stage: operand row 128 (16 bytes per 16-token chunk) = 1.0, rest 0
-            for (int idx = (int)threadIdx.x - 64; idx < ATT_STAGES * (int)(ATT_ONES_BYTES / 16); idx += 256) {
-                const uint32_t off = (uint32_t)(idx % (ATT_ONES_BYTES / 16)) * 16u;
-                const uint32_t v = (off < 512u && (off & 127u) == 0u) ? 0x38383838u : 0u;
-                *reinterpret_cast<uint4 *>(smem + (idx / (ATT_ONES_BYTES / 16)) * ATT_STAGE_BYTES + ATT_K_BYTES +
-                                           ATT_V_BYTES + off) = make_uint4(v, v, v, v);
+            // the ones block of this group's widened-V buffer: operand rows
+            // 128..143 (dims 128..143), row 128 = 1.0 for every token, the rest 0
+            for (int idx = gt; idx < 2 * 8 * 8; idx += 128) {          // 2 row groups x 8 column groups x 8 rows
+                const uint32_t rr = 128u + (uint32_t)(idx >> 6) * 8u + (uint32_t)(idx & 7);
+                const uint32_t kc = (uint32_t)((idx >> 3) & 7) * 8u;
+                const uint32_t v = rr == 128u ? 0x3C003C00u : 0u;
+                *reinterpret_cast<uint4 *>(vb + f16_core_offset(rr, kc)) = make_uint4(v, v, v, v);
             }
             named_bar_sync(1, 256);
             amax = fmaxf(xch[r], xch[128 + r]);
             int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 0;
             e = max(-120, min(127, e));
             const float qs = amax > 0.f ? __uint_as_float((uint32_t)(127 + 7 - e) << 23) : 1.f;
-            c_row = __fdiv_rn(p.k_scale[h] * p.sm_scale * LOG2E, qs);
+            c_row = __fdiv_rn(k_sc * p.sm_scale * LOG2E, qs);
             // A operand of S = Q K^T in tensor memory: row r in lane r, dims 4c .. 4c+3
             // in column c; this group writes columns 16g .. 16g+15 of each term
             uint32_t hw[16], lw[16];
@@ -451,7 +448,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             tmem_st_x16(row_t + ATT_TM_Q + 32u + 16u * (uint32_t)g, lw);
             tmem_wait_st();
             // ancestors of this node: walk the parent array held one entry per lane
-            {
+            if (!p.causal) {
                 int a = has_q ? node : -1;
                 bool bad = false;
 #pragma unroll 1
@@ -473,10 +470,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
         float m_ref = -INFINITY;
         bool ok = true;
-        int32_t pid = g < n_pages ? p.page_table[pg0 + g] : -1;
         for (int i = g; i < n_pages; i += 2) {
             const bool vpage = pid >= 0 && pid < p.n_pool_pages;
-            if (i + 2 < n_pages) pid = p.page_table[pg0 + i + 2];
+            pid = pid_next;
+            if (i + 4 < n_pages) pid_next = p.page_table[pg0 + i + 4];
             bool w_ok = true;
             if (lane == 0) w_ok = mbar_wait(&s_full[g], (uint32_t)((i >> 1) & 1), 320, s_abort);
             if (!__shfl_sync(0xFFFFFFFFu, w_ok ? 1 : 0, 0)) { ok = false; break; }
@@ -503,7 +500,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const int tj = t0 + j;                     // negative: context position
-                    const bool vis = tj < 0 || (tj < T && ((anc >> (tj & 31)) & 1u));
+                    const bool vis = tj < 0 || (tj < T && (p.causal ? tj <= node : ((anc >> (tj & 31)) & 1u) != 0));
                     if (!vis) s[j] = 0xFF800000u;             // -inf
                 }
             }
@@ -534,35 +531,56 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tmem_wait_st();
             }
             if (need) m_ref = mx;
-            const float nb = m_ref > -INFINITY ? ATT_PSHIFT - m_ref : 0.f;
-            uint32_t ph[16], pl[16];
+            const float nb = m_ref > -INFINITY ? -m_ref : 0.f;
+            // P' = 2^(s c - m) in f16: the exponent is rounded to f16, then ex2 on pairs
+            uint32_t ph[32];
 #pragma unroll
-            for (int j = 0; j < 64; j += 4)
-                split4_f16(fast_exp2(fmaf(__uint_as_float(s[j]), c_row, nb)),
-                           fast_exp2(fmaf(__uint_as_float(s[j + 1]), c_row, nb)),
-                           fast_exp2(fmaf(__uint_as_float(s[j + 2]), c_row, nb)),
-                           fast_exp2(fmaf(__uint_as_float(s[j + 3]), c_row, nb)), ph[j >> 2], pl[j >> 2]);
-            if (pos0 + ATT_P > L + T) {
-                // slots past the last written token may hold any byte (NaN codes
-                // included); zero their V so that 0 * V stays 0 in the product
-                const bool k_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
-                if (!__all_sync(0xFFFFFFFFu, k_ok)) { ok = false; break; }
-                uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
-                for (int t = (int)(L + T - pos0); t < ATT_P; ++t) vs[v_offset((uint32_t)r, (uint32_t)t)] = 0;
-            }
-            // the P buffer of this group's previous page must have been consumed
+            for (int j = 0; j < 32; ++j)
+                ph[j] = ex2_f16x2(f32x2_to_f16x2(fmaf(__uint_as_float(s[2 * j]), c_row, nb),
+                                                 fmaf(__uint_as_float(s[2 * j + 1]), c_row, nb)));
+            // the P and widened-V buffers of this group's previous page must have been consumed
             if (!waited && i >= 2) {
                 bool f_ok = true;
                 if (lane == 0) f_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 322, s_abort);
                 if (!__shfl_sync(0xFFFFFFFFu, f_ok ? 1 : 0, 0)) { ok = false; break; }
             }
-            uint8_t *pb = smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {                      // tokens 16c .. 16c+15
-                const uint32_t off = (((uint32_t)r >> 3) * 4u + (uint32_t)c) * 128u + ((uint32_t)r & 7u) * 16u;
-                *reinterpret_cast<uint4 *>(pb + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-                *reinterpret_cast<uint4 *>(pb + ATT_PB_BYTES + off) =
-                    make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+            for (int c = 0; c < 8; ++c)                        // tokens 8c .. 8c+7 of row r
+                *reinterpret_cast<uint4 *>(pb + f16_core_offset((uint32_t)r, 8u * c)) =
+                    make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+            // V of this page, E4M3 -> f16 (exact), into the operand image: each
+            // thread widens 4 of the page's 512 tiled rows (dim d, tokens
+            // 16j .. 16j+15); slots past the last written position may hold any
+            // byte and are written as zeros, so that 0 * V stays 0
+            {
+                const bool v_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
+                if (!__all_sync(0xFFFFFFFFu, v_ok)) { ok = false; break; }
+                const uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
+                const int valid = (int)(L + T - pos0 < ATT_P ? L + T - pos0 : ATT_P);   // slots holding written positions
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t x = (uint32_t)gt + 128u * m;                 // tiled row: tile x/8, line x%8
+                    const uint32_t tile = x >> 3, dgrp = tile >> 2, jt = tile & 3;
+                    const uint32_t d = dgrp * 8u + (x & 7u);
+                    uint4 b = *reinterpret_cast<const uint4 *>(vs + 16u * x);
+                    if ((int)(16 * jt + 16) > valid) {
+                        uint32_t wv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            if ((int)(16 * jt) + k >= valid) wv[k >> 2] &= ~(0xFFu << (8 * (k & 3)));
+                        b = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    }
+                    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+                    uint32_t hv[8];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        hv[2 * k] = e4m3x2_to_f16x2(bw[k] & 0xFFFFu);
+                        hv[2 * k + 1] = e4m3x2_to_f16x2(bw[k] >> 16);
+                    }
+                    *reinterpret_cast<uint4 *>(vb + f16_core_offset(d, 16u * jt)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    *reinterpret_cast<uint4 *>(vb + f16_core_offset(d, 16u * jt + 8u)) =
+                        make_uint4(hv[4], hv[5], hv[6], hv[7]);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -578,7 +596,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         xch[256 + g * 128 + r] = m_ref;
         named_bar_sync(1, 256);
         const float mA = xch[256 + r], mB = xch[384 + r];
-        const int64_t prow = (((int64_t)h * p.S + split) * group) * 16 + r;
+        const int64_t prow = ((int64_t)ch * p.S + split) * rows_cta + r;
         if (d_ok) {
             tc_fence_after();
             const float M = fmaxf(mA, mB);
@@ -612,9 +630,69 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     }
                 }
             }
-            if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M - ATT_PSHIFT, l));
+            if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M, l));
         } else if (n_pages == 0 && row_ok && g == 0) {
             __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(0.f, 0.f));
+        }
+
+        if (p.fuse) {
+            // ---- fused combine: publish, meet the head's other splits, then
+            //      merge rows r0 .. r1-1 of this KV head (row = w*T + node)
+            __threadfence();
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 64) {
+                red_release_gpu_add(p.cnt + ch, 1);
+                if (!poll_counter_ge(p.cnt + ch, p.S, 325, s_abort)) *s_abort = 1;
+            }
+            named_bar_sync(1, 256);
+            __threadfence();
+            const bool merge = !*s_abort;                          // one decision for the whole group
+            const int nr = p.nheads * T;
+            const int r0 = (int)((int64_t)split * nr / p.S), r1 = (int)((int64_t)(split + 1) * nr / p.S);
+            const int d = gt;                                      // dimension of this thread
+            float *crow = reinterpret_cast<float *>(smem + ATT_OFF_C) + 128 * g;
+            const float vsc = p.v_scale[h];
+            for (int row = r0 + g; merge && row < r1; row += 2) {
+                const int ww = row / T, nd = row % T;
+                const int64_t base = (int64_t)ch * p.S * rows_cta + ww * p.rows_w + nd;   // + s * rows_cta
+                const int64_t sstride = rows_cta;
+                float M = -INFINITY;
+                for (int sp = 0; sp < p.S; ++sp) {
+                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * (base + sp * sstride)));
+                    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+                }
+                float num = 0.f, den = 0.f;
+                for (int sp = 0; sp < p.S; ++sp) {
+                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * (base + sp * sstride)));
+                    if (ml.y > 0.f) {
+                        const float ws = ml.y * fast_exp2(ml.x - M);
+                        num += ws * __ldcg(p.part_o + (base + sp * sstride) * ATT_D + d);
+                        den += ws;
+                    }
+                }
+                const float o = den > 0.f ? num / den * vsc : 0.f;
+                const __nv_bfloat16 obf = __float2bfloat16_rn(o);
+                const int hq2 = hq0 + ww;
+                p.out[((int64_t)nd * p.Hq + hq2) * ATT_D + d] = obf;
+                if (p.act) {
+                    crow[d] = __bfloat162float(obf);
+                    named_bar_sync(2 + g, 128);
+                    if (d < ATT_D / 16) {
+                        float v[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) v[k] = crow[16 * d + k];
+                        uint2 pk;
+                        const uint32_t sc = quant_block16(v, *p.g_act, pk);
+                        store_prepared(p.act, nd, (int64_t)hq2 * (ATT_D / 16) + d, pk, sc);
+                    }
+                    named_bar_sync(2 + g, 128);
+                }
+            }
+            // the last CTA of the head through here resets its counter for the next call
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 64 && merge) {
+                if (atomicAdd(p.cnt + ch, 1) == 2 * p.S - 1) atomicExch(p.cnt + ch, 0);
+            }
         }
     }
 
@@ -642,9 +720,11 @@ __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnPara
     pdl_launch_dependents();
     const int i = blockIdx.x, hq = blockIdx.y, tid = threadIdx.x;
     const int wp = tid >> 5, lane = tid & 31;
-    const int h = hq / p.group, w = hq % p.group;
+    const int h = hq / p.group;                                   // KV head
+    const int ch = p.causal ? hq : h, w = p.causal ? 0 : hq % p.group;
     const int S = p.S;
-    auto row = [&](int s) { return (((int64_t)h * S + s) * p.group + w) * 16 + i; };
+    const int64_t rows_cta = (int64_t)p.nheads * p.rows_w;
+    auto row = [&](int s) { return ((int64_t)ch * S + s) * rows_cta + (int64_t)w * p.rows_w + i; };
     float4 pv[CMB_PF];
 #pragma unroll
     for (int k = 0; k < CMB_PF; ++k) {

@@ -33,10 +33,17 @@
 //   warp 0   producer: weight units of the first stages are requested before
 //            griddepcontrol.wait (weights never depend on the previous
 //            kernel); activation chunks after it.
-//   warp 1   allocates TMEM; lane 0 copies scales smem->TMEM (tcgen05.cp) and
-//            issues the MMAs, releasing stages with tcgen05.commit.
-//   warps 2-5 epilogue: tcgen05.ld of the 128x16 accumulator, scale by
-//            g_a*g_w, optional residual, bf16 store or split-K fix-up.
+//   warp 1   allocates TMEM; lane 0 issues the MMAs, releasing stages with
+//            tcgen05.commit.
+//   warps 2-5 stage the scale factors of every unit into tensor memory with
+//            tcgen05.st (one warp per TMEM sub-partition), a few units ahead of
+//            the MMAs; and the epilogue: tcgen05.ld of the 128x16 accumulator,
+//            scale by g_a*g_w, optional residual, bf16 store or split-K fix-up.
+// (Measured on B200: a tcgen05.cp of one scale block takes ~47 cycles of the
+// tensor pipe and an N = 16 block-scaled MMA ~52, and the two serialise: the
+// 16 copies + 8 MMAs of a unit held the pipe ~1,165 cycles, 70% of the
+// unit's HBM time.  Staging the scales through the idle epilogue warps leaves
+// only the MMAs on the pipe.)
 #pragma once
 #include "common.cuh"
 
@@ -61,12 +68,14 @@ constexpr int LIN_SFB_SLOTS = 11;                 // activation-scale chunks kep
 // TMEM columns: accumulator a of buffer b at 16*(LIN_NACC*b + a) (16 fp32
 // columns = 16 tokens; the MMAs of a tile rotate over the LIN_NACC
 // accumulators so that consecutive products do not wait on each other, and
-// the epilogue adds them in a fixed order); weight scales SFA[r] and
-// activation scales SFB[r] 32 columns each (4 per MMA step), resident
-// activation scales of up to LIN_SFB_SLOTS K chunks after them.  Scale-factor
-// column addresses handed to the MMA stay multiples of 4.
-constexpr uint32_t TM_ACC = 0, TM_SFA = 32 * LIN_NACC, TM_SFB = TM_SFA + 64, TM_SFB_RES = TM_SFB + 64;
-static_assert(TM_SFB_RES + 32 * LIN_SFB_SLOTS <= LIN_TMEM_COLS, "tensor memory budget");
+// the epilogue adds them in a fixed order); the weight scales SFA and the
+// activation scales SFB of the unit in pipeline stage s, 32 columns each per
+// stage (4 per MMA step), or, when the activation scales stay resident, up to
+// LIN_SFB_SLOTS K chunks of SFB in place of the per-stage SFB buffers.
+// Scale-factor column addresses handed to the MMA stay multiples of 4.
+constexpr uint32_t TM_ACC = 0, TM_SFA = 32 * LIN_NACC, TM_SFB = TM_SFA + 32 * LIN_STAGES, TM_SFB_RES = TM_SFB;
+static_assert(TM_SFB + 32 * LIN_STAGES <= LIN_TMEM_COLS && TM_SFB_RES + 32 * LIN_SFB_SLOTS <= LIN_TMEM_COLS,
+              "tensor memory budget");
 
 // Instruction descriptor (kind::mxf4nvf4): A/B format E2M1 (1) in bits 7-9 and
 // 10-12, K-major A and B, N>>3 in bits 17-22, scale format UE4M3 (0) in
@@ -118,8 +127,34 @@ __device__ __forceinline__ bool poll_counter(const int *p, int want, uint32_t si
     }
 }
 
+// Wait (bounded) until *p >= want; returns false and records a timeout otherwise.
+__device__ __forceinline__ bool poll_counter_ge(const int *p, int want, uint32_t site, volatile int *abort)
+{
+    if (ld_acquire_gpu(p) >= want) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 8; ++i)
+            if (ld_acquire_gpu(p) >= want) return true;
+        if (abort && *abort) return false;
+        if (globaltimer() - t0 > g_timeout_ns) {
+            report_error(ERRBIT_TIMEOUT, site);
+            if (abort) *abort = 1;
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ int64_t lin_start(int64_t c, int64_t U, int64_t G) { return c * U / G; }
 __device__ __forceinline__ int64_t lin_cta_of(int64_t u, int64_t U, int64_t G) { return ((u + 1) * G + U - 1) / U - 1; }
+
+// The activation scales of K chunk kc are the same for every weight tile:
+// when a CTA sweeps all K chunks at least four times (an LM-head-like shape:
+// many tiles, short K), each chunk's scales are staged into tensor memory
+// once (slot kc - kc0 mod KC) and reused by every later tile.
+__device__ __forceinline__ bool lin_sfb_resident(int64_t n_units, int64_t KC)
+{
+    return n_units >= 4 * KC && KC <= LIN_SFB_SLOTS;
+}
 
 __global__ void __launch_bounds__(LIN_THREADS, 1)
     nvfp4_linear_kernel(const LinearParams p)
@@ -131,7 +166,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     uint64_t *accf = empty + LIN_STAGES;
     uint64_t *acce = accf + 2;
     uint64_t *drain = acce + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *sf_ready = drain + 1;                 // [LIN_STAGES]: scales of the stage's unit are in TMEM
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sf_ready + LIN_STAGES);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const uint32_t warp = warp_id(), lane = lane_id();
@@ -150,6 +186,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             mbar_init(&acce[b], 4);
         }
         mbar_init(drain, 1);
+        for (int st = 0; st < LIN_STAGES; ++st) mbar_init(&sf_ready[st], 4);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -200,20 +237,15 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         } else {
             pdl_wait();
         }
+        __syncwarp();          // reconverge before the CTA-wide barrier below
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = lin_idesc(128, 16);
             int64_t i = 0, seg = 0;
             bool ok = true;
-            // The activation scales of K chunk kc are the same for every weight tile:
-            // when this CTA sweeps all K chunks at least four times (an LM-head-like
-            // shape: many tiles, short K), each chunk's scales are copied into tensor
-            // memory once (slot kc - kc0 mod KC) and reused by every later tile.
-            // (Measured: with less reuse the per-unit copies are as fast.)
-            const bool sfb_resident = n_units >= 4 * (int64_t)KC && KC <= LIN_SFB_SLOTS;
+            const bool sfb_resident = lin_sfb_resident(n_units, KC);
             const int64_t kc0 = u0 % KC;
-            uint32_t sfb_loaded = 0;
             for (int64_t u = u0; u < u1 && ok; ++seg) {
                 const int64_t ka = u % KC;
                 const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
@@ -223,29 +255,17 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 const uint32_t d_tmem = tmem_base + TM_ACC + 16 * LIN_NACC * b;
                 for (int64_t kc = ka; kc < kend; ++kc, ++i) {
                     const int s = (int)(i % LIN_STAGES);
-                    if (!mbar_wait(&full[s], (uint32_t)((i / LIN_STAGES) & 1), 104, s_abort)) { ok = false; break; }
+                    const uint32_t par = (uint32_t)((i / LIN_STAGES) & 1);
+                    if (!mbar_wait(&full[s], par, 104, s_abort) || !mbar_wait(&sf_ready[s], par, 109, s_abort)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t r = (uint32_t)(i & 1);
                     const uint32_t w_s = smem_u32(smem + s * LIN_STAGE_BYTES);
                     const uint32_t a_s = w_s + LIN_W_UNIT;
-                    const uint32_t sfa_s = w_s + 2 * LIN_W_ATOM, sfb_s = a_s + 2 * LIN_A_ATOM;
-                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * r;
-                    uint32_t sfb_t = tmem_base + TM_SFB + 32 * r;
-                    bool copy_sfb = true;
-                    if (sfb_resident) {
-                        const uint32_t slot = (uint32_t)((kc - kc0 + KC) % KC);
-                        sfb_t = tmem_base + TM_SFB_RES + 32 * slot;
-                        copy_sfb = !((sfb_loaded >> slot) & 1u);
-                        sfb_loaded |= 1u << slot;
-                    }
-#pragma unroll
-                    for (int j = 0; j < LIN_KSTEPS; ++j)
-                        tmem_cp_32x128b_warpx4(sfa_t + 4 * j, smem_desc(sfa_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
-                    if (copy_sfb) {
-#pragma unroll
-                        for (int j = 0; j < LIN_KSTEPS; ++j)
-                            tmem_cp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + LIN_SF_IMG * j, 512, 128, SWZ_NONE));
-                    }
+                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * (uint32_t)s;
+                    const uint32_t sfb_t = sfb_resident ? tmem_base + TM_SFB_RES + 32 * (uint32_t)((kc - kc0 + KC) % KC)
+                                                        : tmem_base + TM_SFB + 32 * (uint32_t)s;
 #pragma unroll
                     for (int j = 0; j < LIN_KSTEPS; ++j) {
                         const uint32_t atom = (uint32_t)(j >> 2), ko = 32u * (uint32_t)(j & 3);
@@ -275,11 +295,66 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         const float gs = __fmul_rn(*p.g_a, *p.g_w);
         const int M = p.M;
         const int64_t first_tile_of_me = u0 / KC;
+        // Scale staging: the weight and activation scale images of unit i (each
+        // 8 blocks of 32 lines x 16 bytes, line l = rows l, l+32, l+64, l+96)
+        // go to every TMEM sub-partition (this warp writes its own), the layout
+        // the block-scaled MMA reads; then one arrive on sf_ready of the stage.
+        // The per-stage buffers of unit i are free again once unit i has landed:
+        // the producer refilled its stage only after the MMAs of unit i-STAGES
+        // had completed.
+        const bool sfb_resident = lin_sfb_resident(n_units, KC);
+        const int64_t kc0 = u0 % KC;
+        const uint32_t lane_base = tmem_base + ((32u * q) << 16);
+        uint32_t sfb_loaded = 0;
+        int64_t next_sf = 0;
+        bool sf_ok = true;
+        auto stage_scales = [&](int64_t i) -> bool {
+            const int s = (int)(i % LIN_STAGES);
+            const bool landed = mbar_wait(&full[s], (uint32_t)((i / LIN_STAGES) & 1), 108, s_abort);
+            if (!__all_sync(0xFFFFFFFFu, landed)) return false;
+            const uint8_t *st = smem + s * LIN_STAGE_BYTES;
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < LIN_KSTEPS; ++j) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(st + 2 * LIN_W_ATOM + LIN_SF_IMG * j + 16 * lane);
+                v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+            }
+            tmem_st_x32(lane_base + TM_SFA + 32 * (uint32_t)s, v);
+            uint32_t sfb_col = TM_SFB + 32 * (uint32_t)s;
+            bool copy_sfb = true;
+            if (sfb_resident) {
+                const uint32_t slot = (uint32_t)((((u0 + i) % KC) - kc0 + KC) % KC);
+                sfb_col = TM_SFB_RES + 32 * slot;
+                copy_sfb = !((sfb_loaded >> slot) & 1u);
+                sfb_loaded |= 1u << slot;
+            }
+            if (copy_sfb) {
+#pragma unroll
+                for (int j = 0; j < LIN_KSTEPS; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(st + LIN_W_UNIT + 2 * LIN_A_ATOM + LIN_SF_IMG * j +
+                                                                     16 * lane);
+                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                }
+                tmem_st_x32(lane_base + sfb_col, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sf_ready[s]);
+            return true;
+        };
+        auto stage_scales_until = [&](int64_t last) {
+            while (sf_ok && next_sf <= last && next_sf < n_units) sf_ok = stage_scales(next_sf++);
+            return sf_ok;
+        };
         int64_t seg = 0;
         for (int64_t u = u0; u < u1; ++seg) {
             const int64_t t = u / KC, ka = u % KC;
             const int64_t kend = (ka + (u1 - u)) < KC ? ka + (u1 - u) : KC;
             const uint32_t b = (uint32_t)(seg & 1);
+            // stage the scales of this tile's units and of up to STAGES-1 later
+            // ones, so that the MMAs keep going while this tile is written out
+            if (!stage_scales_until((u - u0) + (kend - ka) - 1 + (LIN_STAGES - 1))) break;
             const bool whole = ka == 0 && kend == KC;
             const int64_t first = whole ? c : lin_cta_of(t * KC, U, G);
             const int64_t last = whole ? c : lin_cta_of(t * KC + KC - 1, U, G);

@@ -19,6 +19,7 @@
 #include "linear.cuh"
 #include "quant.cuh"
 #include "restore.cuh"
+#include "wide.cuh"
 
 using namespace nvfp4sk;
 
@@ -86,6 +87,7 @@ int device_info(DevInfo **out)
                 set_smem(nvfp4_linear_kernel, LIN_SMEM_BYTES),
                 set_smem(tree_attn_split_kernel, ATT_SMEM_BYTES),
                 set_smem(kv_page_restore_kernel, RST_SMEM_BUDGET + 1024),
+                set_smem(nvfp4_linear_wide_kernel, WD_SMEM_BYTES),
                 allow_big_cluster(quant_fused_kernel<__nv_bfloat16, 0>),
                 allow_big_cluster(quant_fused_kernel<float, 0>),
                 allow_big_cluster(quant_fused_kernel<__nv_bfloat16, 1>),
@@ -195,13 +197,76 @@ int attn_splits(const DevInfo &d, int Hkv, int64_t n_log)
     int64_t S = g_opt_attn_splits > 0 ? g_opt_attn_splits : std::max<int64_t>(1, d.sms / std::max(1, Hkv));
     return (int)std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(S, ATT_MAX_SPLITS), n_log));
 }
-size_t attn_ws(int Hkv, int S, int group)
+// Attention workspace: per-CTA-head arrival counters of the fused combine at
+// offset 0 (ATT_CNT_BYTES), then the split results: o fp32
+// [heads][S][rows_cta][128] and (m, l) fp32 [heads][S][rows_cta][2].  Tree
+// mode: heads = Hkv, rows_cta = group*16; causal mode: heads = Hq, rows_cta = 128.
+size_t attn_ws(int heads, int S, int rows_cta)
 {
-    const size_t rows = (size_t)Hkv * S * group * 16;
-    return up256(rows * ATT_D * 4) + up256(rows * 2 * 4);
+    const size_t rows = (size_t)heads * S * rows_cta;
+    return ATT_CNT_BYTES + up256(rows * ATT_D * 4) + up256(rows * 2 * 4);
 }
 
 int argmax_chunks(int64_t n) { return (int)std::max<int64_t>(1, std::min<int64_t>(64, n / 4096)); }
+
+// Shared launch of the attention kernel (tree or causal mode, see attn.cuh)
+// after the entry points' argument checks.
+int attn_launch(const void *q, int64_t ld_q, int T, int Hq, int Hkv, const uint8_t *k_pool, const uint8_t *v_pool,
+                int64_t n_pool_pages, const int32_t *page_table, int64_t ctx_len, const int32_t *parent,
+                const float *k_scale, const float *v_scale, float sm_scale, void *out, const float *g_act,
+                uint8_t *act_prepared, void *ws, size_t ws_bytes, nvfp4sk_stream_t stream, int causal)
+{
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    const int64_t n_log = cdiv(ctx_len + T, ATT_P);
+    const int group = Hq / Hkv;
+    const int heads = causal ? Hq : Hkv;                      // grid.y
+    const int rows_w = causal ? ATT_ROWS : 16, nheads = causal ? 1 : group;
+    const int S = attn_splits(*d, heads, n_log);
+    const size_t need = attn_ws(heads, S, nheads * rows_w);
+    if (!ws || ws_bytes < need || !al16(ws))
+        return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
+    CUtensorMap tk;
+    if (int rc = make_map_u8(&tk, k_pool, ATT_D, (uint64_t)n_pool_pages * Hkv * ATT_P, ATT_D, ATT_D, ATT_P,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    AttnParams p;
+    p.q = (const __nv_bfloat16 *)q;
+    p.ld_q = ld_q;
+    p.v_pool = v_pool;
+    p.page_table = page_table;
+    p.parent = parent;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.cnt = (int *)ws;
+    p.part_o = (float *)((uint8_t *)ws + ATT_CNT_BYTES);
+    p.part_ml = (float *)((uint8_t *)ws + ATT_CNT_BYTES + up256((size_t)heads * S * nheads * rows_w * ATT_D * 4));
+    p.out = (__nv_bfloat16 *)out;
+    p.g_act = g_act;
+    p.act = act_prepared;
+    p.ctx_len = ctx_len;
+    p.n_pool_pages = n_pool_pages;
+    p.sm_scale = sm_scale;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.group = group;
+    p.S = S;
+    p.n_log_pages = (int)n_log;
+    p.causal = causal;
+    p.rows_w = rows_w;
+    p.nheads = nheads;
+    // fused combine when every CTA of the grid can be resident at once (one
+    // CTA per SM): the CTAs of a head wait for each other before merging
+    p.fuse = (int64_t)S * heads <= d->sms ? 1 : 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, heads), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, 1, tk, p);
+    if (e != cudaSuccess) return cuda_fail(e, "tree_attn_split_kernel");
+    if (p.fuse) return NVFP4SK_OK;
+    return launched(launch(tree_attn_combine_kernel, dim3(T, Hq), dim3(ATT_D), 0, st, 1, p),
+                    "tree_attn_combine_kernel");
+}
+
 
 }  // namespace
 
@@ -397,6 +462,38 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t
                     "nvfp4_linear_kernel");
 }
 
+nvfp4sk_status nvfp4_linear_wide(const uint8_t *a_prepared, const float *g_a, int64_t S, const uint8_t *w_prepared,
+                                 const float *g_w, int64_t N, int64_t K, const void *residual, void *y, int64_t ldy,
+                                 nvfp4sk_stream_t stream)
+{
+    if (!a_prepared || !g_a || !w_prepared || !g_w || !y) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (S < 1 || S > INT32_MAX / 2 || N < 1 || N > INT32_MAX / 2 || K < 64 || K % 64 != 0 || ldy < N)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need S >= 1, N >= 1, K %% 64 == 0, ldy >= N");
+    if (!al16(a_prepared) || !al16(w_prepared))
+        return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    WideParams p;
+    p.w = w_prepared;
+    p.a = a_prepared;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.residual = (const __nv_bfloat16 *)residual;
+    p.y = (__nv_bfloat16 *)y;
+    p.ldy = ldy;
+    p.S = S;
+    p.N = N;
+    p.NT = (int)cdiv(N, 128);
+    p.ST = (int)cdiv(S, 128);
+    p.KC = (int)cdiv(K, LIN_KC);
+    const int64_t tiles = (int64_t)p.NT * ((p.ST + 1) / 2);
+    if (tiles > INT32_MAX) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "too many output tiles");
+    p.n_tiles = (int)tiles;
+    const int G = (int)std::min<int64_t>(d->sms, tiles);
+    return launched(launch(nvfp4_linear_wide_kernel, dim3(G), dim3(WD_THREADS), WD_SMEM_BYTES, (cudaStream_t)stream, 1, p),
+                    "nvfp4_linear_wide_kernel");
+}
+
 // ---------------------------------------------------------------- attention
 size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len)
 {
@@ -404,7 +501,16 @@ size_t tree_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, i
     DevInfo *d;
     if (device_info(&d) || Hkv <= 0 || page_size <= 0 || Hq % Hkv) return 0;
     const int64_t n_log = cdiv(ctx_len + T, page_size);
-    return attn_ws(Hkv, attn_splits(*d, Hkv, n_log), Hq / Hkv);
+    return attn_ws(Hkv, attn_splits(*d, Hkv, n_log), Hq / Hkv * 16);
+}
+
+size_t causal_attn_workspace_bytes(int T, int Hq, int Hkv, int D, int page_size, int64_t ctx_len)
+{
+    (void)D; (void)Hkv;
+    DevInfo *d;
+    if (device_info(&d) || Hq <= 0 || page_size <= 0) return 0;
+    const int64_t n_log = cdiv(ctx_len + T, page_size);
+    return attn_ws(Hq, attn_splits(*d, Hq, n_log), ATT_ROWS);
 }
 
 nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D, const uint8_t *k_pool,
@@ -423,45 +529,27 @@ nvfp4sk_status tree_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int H
     if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool) || !al16(act_prepared))
         return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes), the pools and act_prepared must be 16-byte aligned");
     if (act_prepared && !g_act) return fail(NVFP4SK_ERR_INVALID_ARG, "act_prepared needs the static scale g_act");
-    DevInfo *d;
-    if (int rc = device_info(&d)) return rc;
-    const int64_t n_log = cdiv(ctx_len + T, ATT_P);
-    const int group = Hq / Hkv;
-    const int S = attn_splits(*d, Hkv, n_log);
-    const size_t need = attn_ws(Hkv, S, group);
-    if (!ws || ws_bytes < need || !al16(ws))
-        return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
-    CUtensorMap tk;
-    if (int rc = make_map_u8(&tk, k_pool, ATT_D, (uint64_t)n_pool_pages * Hkv * ATT_P, ATT_D, ATT_D, ATT_P,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
-        return rc;
-    AttnParams p;
-    p.q = (const __nv_bfloat16 *)q;
-    p.ld_q = ld_q;
-    p.v_pool = v_pool;
-    p.page_table = page_table;
-    p.parent = parent;
-    p.k_scale = k_scale;
-    p.v_scale = v_scale;
-    p.part_o = (float *)ws;
-    p.part_ml = (float *)((uint8_t *)ws + up256((size_t)Hkv * S * group * 16 * ATT_D * 4));
-    p.out = (__nv_bfloat16 *)out;
-    p.g_act = g_act;
-    p.act = act_prepared;
-    p.ctx_len = ctx_len;
-    p.n_pool_pages = n_pool_pages;
-    p.sm_scale = sm_scale;
-    p.T = T;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.group = group;
-    p.S = S;
-    p.n_log_pages = (int)n_log;
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, Hkv), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, 1, tk, p);
-    if (e != cudaSuccess) return cuda_fail(e, "tree_attn_split_kernel");
-    return launched(launch(tree_attn_combine_kernel, dim3(T, Hq), dim3(ATT_D), 0, st, 1, p),
-                    "tree_attn_combine_kernel");
+    return attn_launch(q, ld_q, T, Hq, Hkv, k_pool, v_pool, n_pool_pages, page_table, ctx_len, parent, k_scale,
+                       v_scale, sm_scale, out, g_act, act_prepared, ws, ws_bytes, stream, 0);
+}
+
+nvfp4sk_status causal_attn_fp8kv(const void *q, int64_t ld_q, int T, int Hq, int Hkv, int D, const uint8_t *k_pool,
+                                 const uint8_t *v_pool, int64_t n_pool_pages, int page_size,
+                                 const int32_t *page_table, int64_t ctx_len, const float *k_scale,
+                                 const float *v_scale, float sm_scale, void *out, void *ws, size_t ws_bytes,
+                                 nvfp4sk_stream_t stream)
+{
+    if (!q || !k_pool || !v_pool || !page_table || !k_scale || !v_scale || !out)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (D != ATT_D || page_size != ATT_P || T < 1 || T > ATT_ROWS || Hkv < 1 || Hq % Hkv != 0 ||
+        Hq * 4 > (int)ATT_CNT_BYTES || ctx_len < 0 || n_pool_pages < 1 || ld_q < (int64_t)Hq * D ||
+        n_pool_pages * Hkv * ATT_P > INT32_MAX)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "need D == 128, page_size == 64, 1 <= T <= 128, Hq %% Hkv == 0, Hq <= 64, ld_q >= Hq*D");
+    if (!al16(q) || ld_q % 8 != 0 || !al16(k_pool) || !al16(v_pool))
+        return fail(NVFP4SK_ERR_MISALIGNED, "q (and ld_q*2 bytes) and the pools must be 16-byte aligned");
+    return attn_launch(q, ld_q, T, Hq, Hkv, k_pool, v_pool, n_pool_pages, page_table, ctx_len, nullptr, k_scale,
+                       v_scale, sm_scale, out, nullptr, nullptr, ws, ws_bytes, stream, 1);
 }
 
 // ---------------------------------------------------------------- restore
@@ -502,8 +590,12 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
     (void)ws; (void)ws_bytes;
     if (!x || !w || !g_out || (!act_prepared && (!codes || !scales)))
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (rows < 1 || rows > 16 || n < 64 || n % 64 != 0 || n > (int64_t)RTHREADS * RNB * 16)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, n %% 64 == 0, n <= 8192");
+    // the static-scale path with canonical outputs takes any row count (the
+    // suffix prefill); the dynamic path and the 16-row prepared image do not
+    const int64_t max_rows = (g_in && !act_prepared) ? (int64_t)INT32_MAX : 16;
+    if (rows < 1 || rows > max_rows || n < 64 || n % 64 != 0 || n > (int64_t)RTHREADS * RNB * 16)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "need 1 <= rows <= 16 (any with g_in and no act_prepared), n %% 64 == 0, n <= 8192");
     if (!al16(x) || !al16(w) || (reinterpret_cast<uintptr_t>(codes) & 7u) ||
         (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "x, w, act_prepared must be 16-byte aligned, codes 8-byte aligned");
@@ -528,8 +620,11 @@ nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, co
     (void)ws; (void)ws_bytes;
     if (!gu || !g_out || (!act_prepared && (!codes || !scales)))
         return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
-    if (rows < 1 || rows > 16 || F < 64 || F % 64 != 0 || rows * (F / 16) > QSMALL_MAX_BLOCKS)
-        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= rows <= 16, F %% 64 == 0, rows*F <= 524288");
+    const bool any_rows = g_in && !act_prepared;        // static scale, canonical outputs: any row count
+    if (rows < 1 || (!any_rows && (rows > 16 || rows * (F / 16) > QSMALL_MAX_BLOCKS)) || rows > INT32_MAX || F < 64 ||
+        F % 64 != 0)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE,
+                    "need 1 <= rows <= 16 (any with g_in and no act_prepared), F %% 64 == 0, rows*F <= 524288");
     if (!al16(gu) || (reinterpret_cast<uintptr_t>(codes) & 7u) || (reinterpret_cast<uintptr_t>(act_prepared) & 15u))
         return fail(NVFP4SK_ERR_MISALIGNED, "gu, act_prepared must be 16-byte aligned, codes 8-byte aligned");
     DevInfo *d;

@@ -455,6 +455,7 @@ __global__ void debug_wait_timeout_kernel()
     }
     __syncthreads();
     if (threadIdx.x == 0) mbar_wait(&bar, 0, 900);
+    __syncwarp();
     __syncthreads();
 }
 

@@ -42,11 +42,15 @@ _SIGS = {
     "nvfp4_prepare_weight": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
+    "nvfp4_linear_wide": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
     "nvfp4_linear_noalloc_scratch_bytes": (_sz, []),
     "nvfp4_linear_noalloc": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
     "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
     "tree_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
                                _vp, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "causal_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
+    "causal_attn_fp8kv": (_int, [_vp, _i64, _int, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp,
+                                 _f32, _vp, _vp, _sz, _vp]),
     "kv_page_restore": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
     "kv_v_pages_to_tiled": (_int, [_vp, _vp, _i64, _int, _int, _vp]),
     "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -152,11 +156,11 @@ def get_option(opt):
 
 
 # default workspaces whose arrival counters must read zero when a call starts
-_COUNTER_KINDS = ("linear", "argmax")
+_COUNTER_KINDS = ("linear", "argmax", "attn")
 
 
 def _rezero_counter_workspaces():
-    """Zero the default linear / argmax workspaces of every device: a call whose
+    """Zero the default linear / argmax / attention workspaces of every device: a call whose
     device wait ran out can leave their arrival counters non-zero, and the next
     call on the same workspace would count stale arrivals."""
     for (dev, kind), ws in _default_ws.items():
@@ -166,7 +170,7 @@ def _rezero_counter_workspaces():
 
 def device_status(stream=None):
     """(status code, site): synchronises the stream, reads and clears the error
-    word.  On a non-zero status the default linear and argmax workspaces are
+    word.  On a non-zero status the default linear, argmax and attention workspaces are
     zeroed again (stream-ordered on the current stream), as the C ABI's
     workspace rule asks of every caller-owned workspace after a failure."""
     site = _int(0)
@@ -210,8 +214,18 @@ def prepare_act(codes: torch.Tensor, scales: torch.Tensor, K: int, act=None, str
     return act
 
 
-def prepare_weight(codes: torch.Tensor, scales: torch.Tensor, N: int, K: int, stream=None):
-    out = torch.empty(load().nvfp4_prepared_weight_bytes(N, K), dtype=torch.uint8, device=codes.device)
+def prepared_weight_bytes(N: int, K: int) -> int:
+    return load().nvfp4_prepared_weight_bytes(N, K)
+
+
+def prepare_weight(codes: torch.Tensor, scales: torch.Tensor, N: int, K: int, out=None, stream=None):
+    """Tile image of an NVFP4 matrix (a weight, or an activation of many tokens
+    for nvfp4_linear_wide); out: a device buffer of at least
+    prepared_weight_bytes(N, K) bytes, or None to allocate one."""
+    if out is None:
+        out = torch.empty(load().nvfp4_prepared_weight_bytes(N, K), dtype=torch.uint8, device=codes.device)
+    elif out.numel() < load().nvfp4_prepared_weight_bytes(N, K):
+        raise ValueError("prepare_weight: out is too small")
     _call("nvfp4_prepare_weight", _d(codes), _d(scales), N, K, _d(out), _stream(stream))
     return out
 
@@ -223,6 +237,16 @@ def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, str
     wp, wn = _ws(ws, load().nvfp4_linear_workspace_bytes(M, N, K), "linear")
     _call("nvfp4_linear", _d(a_act), _d(g_a), M, _d(w_prep), _d(g_w), N, K,
           _p(residual), _d(y), y.stride(0), wp, wn, _stream(stream))
+    return y
+
+
+def linear_wide(a_prep, g_a, S, w_prep, g_w, N, K, y=None, residual=None, stream=None):
+    """Y [S, N] bf16 = NVFP4 linear (+ residual) for S tokens; a_prep is the
+    activation in the weight tile image (prepare_weight of its codes/scales)."""
+    if y is None:
+        y = torch.empty(S, N, dtype=torch.bfloat16, device=a_prep.device)
+    _call("nvfp4_linear_wide", _d(a_prep), _d(g_a), S, _d(w_prep), _d(g_w), N, K,
+          _p(residual), _d(y), y.stride(0), _stream(stream))
     return y
 
 
@@ -245,6 +269,27 @@ def tree_attn(q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, 
     _call("tree_attn_fp8kv", _d(q), ld_q, T, Hq, Hkv, D, _d(k_pool), _d(v_pool), n_pages, P,
           _d(page_table), int(ctx_len), _d(parent), _d(k_scale), _d(v_scale),
           float(sm_scale), _d(out), _p(g_act), _p(act), wp, wn, _stream(stream))
+    return out
+
+
+def causal_attn(q, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, sm_scale=None, out=None, ld_q=None,
+                T=None, Hq=None, ws=None, stream=None):
+    """Causal attention of T <= 128 new tokens (positions ctx_len ..) over the
+    FP8 paged cache; q bf16 [T, Hq, D] or a strided view with ld_q; returns
+    bf16 [T, Hq, D]."""
+    n_pages, Hkv, P, D = k_pool.shape
+    if T is None:
+        T, Hq = q.shape[0], q.shape[1]
+    if ld_q is None:
+        ld_q = q.stride(0)
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty(T, Hq, D, dtype=torch.bfloat16, device=q.device)
+    wp, wn = _ws(ws, load().causal_attn_workspace_bytes(T, Hq, Hkv, D, P, int(ctx_len)), "attn")
+    _call("causal_attn_fp8kv", _d(q), ld_q, T, Hq, Hkv, D, _d(k_pool), _d(v_pool), n_pages, P,
+          _d(page_table), int(ctx_len), _d(k_scale), _d(v_scale), float(sm_scale), _d(out), wp, wn,
+          _stream(stream))
     return out
 
 

@@ -15,9 +15,10 @@ NVFP4 and the cache is FP8 ("NVFP4 and FP8").
 
 Suffix prefill (VerifyModel.prefill) writes the K/V of the prompt tokens that
 the prefix cache does not hold ("KV-cache reuse between agent steps": only the
-new suffix is prefilled) through the same kernels, 16 tokens at a time: each
-group of 16 is a chain (causal) tree over everything before it, which is
-causal attention over the whole suffix split at group boundaries.
+new suffix is prefilled) with the many-token kernels: every glue op over all S
+rows in one launch, the NVFP4 linears as tiles of 128 weight rows x 256 tokens
+(nvfp4_linear_wide), and causal attention in blocks of 128 queries, block b
+attending to everything before it plus its own causal chain.
 
 All buffers are allocated once, so a step can be captured in a CUDA graph.
 """
@@ -32,13 +33,13 @@ from . import inputs as I
 from . import lib as nv
 
 PAGE_BYTES = I.N_KV_HEADS * I.PAGE * I.HEAD_DIM      # one (layer, K|V, page) plane: 32 KB
-PREFILL_CHUNK = 16                                   # rows per skinny launch (linear M, attention T)
+PREFILL_CHUNK = 128                                  # queries per causal-attention launch
 
 
 def prefill_chunks(start: int, S: int, C: int = PREFILL_CHUNK):
-    """Row groups of a suffix prefill: (row0, rows, ctx_len) for rows
-    row0 .. row0+rows-1 of the S suffix tokens, which sit at positions
-    start+row0 ..; ctx_len = start+row0 is the context each group attends to
+    """Query blocks of a suffix prefill's attention: (row0, rows, ctx_len) for
+    rows row0 .. row0+rows-1 of the S suffix tokens, which sit at positions
+    start+row0 ..; ctx_len = start+row0 is the context each block attends to
     in full before its own causal chain."""
     if start < 0 or S < 0 or C < 1:
         raise ValueError("need start >= 0, S >= 0, C >= 1")
@@ -280,28 +281,43 @@ class VerifyModel:
 
     # ------------------------------------------------------------------ prefill
     def _prefill_buffers(self, S):
-        """Per-suffix buffers, kept for later calls of up to the same length."""
+        """Per-suffix buffers, kept for later calls of up to the same length:
+        the bf16 activations of all S rows, one canonical NVFP4 code / scale
+        buffer and one tile-image buffer for the widest K (reused by every
+        quantisation site), and the head's one-row operands."""
         pf = getattr(self, "_pf", None)
         if pf is not None and pf["cap"] >= S:
             return pf
-        H, F, Hq, Hkv, D, C = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM, PREFILL_CHUNK
-        cap = -(-S // C) * C
-        n = cap // C
+        H, F, Hq, Hkv, D = I.HIDDEN, I.FFN, I.N_Q_HEADS, I.N_KV_HEADS, I.HEAD_DIM
+        cap = max(S, 1)
+        kmax = max(H, F, Hq * D)
         dev = self.dev
         pf = {
             "cap": cap,
             "qkv": torch.empty(cap, (Hq + 2 * Hkv) * D, dtype=torch.bfloat16, device=dev),
             "attn": torch.empty(cap, Hq * D, dtype=torch.bfloat16, device=dev),
-            "gu": torch.empty(C, 2 * F, dtype=torch.bfloat16, device=dev),
-            "q_h": [Act(H, dev) for _ in range(n)],
-            "q_a": [Act(Hq * D, dev) for _ in range(n)],
-            "q_f": [Act(F, dev) for _ in range(n)],
-            "parent": torch.from_numpy(I.chain_parent(C)).to(dev),
+            "gu": torch.empty(cap, 2 * F, dtype=torch.bfloat16, device=dev),
+            "codes": torch.empty(cap * kmax // 2, dtype=torch.uint8, device=dev),
+            "scales": torch.empty(cap * kmax // 16, dtype=torch.uint8, device=dev),
+            "g": torch.empty(1, dtype=torch.float32, device=dev),
+            "wide": torch.empty(nv.prepared_weight_bytes(cap, kmax), dtype=torch.uint8, device=dev),
+            "q_h": Act(H, dev),
             "logits": torch.empty(1, I.VOCAB, dtype=torch.bfloat16, device=dev),
             "ids": torch.empty(1, dtype=torch.int32, device=dev),
         }
         self._pf = pf
         return pf
+
+    @staticmethod
+    def _canon(pf, S, K):
+        """(codes [S, K/2], scales [S, K/16], g): the canonical NVFP4 outputs of
+        a quantisation site over S rows of width K."""
+        return (pf["codes"][:S * K // 2].view(S, K // 2), pf["scales"][:S * K // 16].view(S, K // 16), pf["g"])
+
+    @staticmethod
+    def _wide_act(pf, S, K, out):
+        """The tile image the wide linear streams, from canonical codes / scales."""
+        return nv.prepare_weight(out[0], out[1], S, K, out=pf["wide"])
 
     def prefill(self, h: torch.Tensor, start: int, layers=None):
         """Prefill the S = h.shape[0] suffix tokens at positions start .. start+S-1.
@@ -318,15 +334,15 @@ class VerifyModel:
         when they end with the last layer.  Running range(0, k) and then
         range(k, n_layers) gives the same result as one call.
 
-        Needs static activation scales (calibrate()): with them, quantising a
-        row does not depend on the other rows, so 16-row groups give the
-        result of one pass over all S rows.
+        Needs static activation scales (calibrate()): one calibrated tensor
+        scale per quantisation site, as in the verify step.
 
-        Order inside a layer: each op runs over all row groups before the
-        next op starts, so a linear's weights can stay in L2 for the later
-        groups; all groups' K/V are appended before any
-        group attends, and group c attends to the context (start + 16c
-        tokens, the earlier groups included) plus its own chain."""
+        Per layer: RMSNorm + NVFP4 over all S rows, the QKV linear over all
+        rows, the FP8 append of all S tokens' K/V, then causal attention in
+        blocks of 128 queries (block b attends to the context, start + 128 b
+        tokens, the earlier blocks included, plus its own causal chain), the
+        attention output quantised with its site scale, the O linear (+h),
+        RMSNorm + NVFP4, gate+up, SwiGLU + NVFP4, down (+h)."""
         if not self.static:
             raise RuntimeError("prefill needs static activation scales: call calibrate() first")
         S = h.shape[0]
@@ -343,44 +359,41 @@ class VerifyModel:
         if S == 0:
             return None
         pf = self._prefill_buffers(S)
-        groups = prefill_chunks(start, S)
+        H, F = I.HIDDEN, I.FFN
         qd = I.N_Q_HEADS * I.HEAD_DIM
         kd = I.N_KV_HEADS * I.HEAD_DIM
-        qkv, attn, gu = pf["qkv"], pf["attn"], pf["gu"]
+        qkv, attn, gu = pf["qkv"][:S], pf["attn"][:S], pf["gu"][:S]
         for l in layers:
             lay, s0 = self.layers[l], l * self.SITES
             kp, vp = self.k_pool(l), self.v_pool(l)
-            for c, (r, t, _) in enumerate(groups):
-                a = pf["q_h"][c]
-                nv.rmsnorm_quantize(h[r:r + t], self.norm_w[2 * l], self.eps, a.out, act=a.buf,
-                                    g_in=self._site(s0))
-                self._linear(a.buf, a.g, lay["qkv"], qkv[r:r + t], M=t)
-            nv.kv_append(qkv[:S, qd:], qkv[:S, qd + kd:], qkv.stride(0), S, kp, vp, self.page_table, start,
+            out = self._canon(pf, S, H)
+            nv.rmsnorm_quantize(h, self.norm_w[2 * l], self.eps, out, g_in=self._site(s0))
+            self._wide(self._wide_act(pf, S, H, out), out[2], lay["qkv"], qkv)
+            nv.kv_append(qkv[:, qd:], qkv[:, qd + kd:], qkv.stride(0), S, kp, vp, self.page_table, start,
                          self.k_scale[l], self.v_scale[l])
-            for c, (r, t, ctx) in enumerate(groups):
-                a = pf["q_a"][c]
-                nv.tree_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, pf["parent"], self.k_scale[l],
-                             self.v_scale[l], out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS,
-                             g_act=self._site(s0 + 1), act=a.buf)
-                self._linear(a.buf, self._site(s0 + 1), lay["o"], h[r:r + t], residual=h[r:r + t], M=t)
-                a = pf["q_h"][c]
-                nv.rmsnorm_quantize(h[r:r + t], self.norm_w[2 * l + 1], self.eps, a.out, act=a.buf,
-                                    g_in=self._site(s0 + 2))
-            for c, (r, t, _) in enumerate(groups):
-                a, f = pf["q_h"][c], pf["q_f"][c]
-                self._linear(a.buf, a.g, lay["gate_up"], gu[:t], M=t)
-                nv.swiglu_quantize(gu[:t], f.out, act=f.buf, g_in=self._site(s0 + 3))
-            for c, (r, t, _) in enumerate(groups):
-                f = pf["q_f"][c]
-                self._linear(f.buf, f.g, lay["down"], h[r:r + t], residual=h[r:r + t], M=t)
+            for r, t, ctx in prefill_chunks(start, S):
+                nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
+                               out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS)
+            out = self._canon(pf, S, qd)
+            nv.quantize(attn, g_in=self._site(s0 + 1), out=out)
+            self._wide(self._wide_act(pf, S, qd, out), out[2], lay["o"], h, residual=h)
+            out = self._canon(pf, S, H)
+            nv.rmsnorm_quantize(h, self.norm_w[2 * l + 1], self.eps, out, g_in=self._site(s0 + 2))
+            self._wide(self._wide_act(pf, S, H, out), out[2], lay["gate_up"], gu)
+            out = self._canon(pf, S, F)
+            nv.swiglu_quantize(gu, out, g_in=self._site(s0 + 3))
+            self._wide(self._wide_act(pf, S, F, out), out[2], lay["down"], h, residual=h)
         if self.lm_head is None or len(layers) == 0 or layers[-1] != self.n_layers - 1:
             return None
         i = self.n_layers * self.SITES
-        a = pf["q_h"][0]
+        a = pf["q_h"]
         nv.rmsnorm_quantize(h[S - 1:S], self.norm_w[-1], self.eps, a.out, act=a.buf, g_in=self._site(i))
         self._linear(a.buf, a.g, self.lm_head, pf["logits"], M=1)
         nv.argmax(pf["logits"], pf["ids"])
         return pf["ids"]
+
+    def _wide(self, act, g, lin, y, residual=None):
+        nv.linear_wide(act, g, y.shape[0], lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
 
     def turn(self, h_suffix: torch.Tensor, draft_tokens: torch.Tensor | None = None):
         """One agent turn's forward work: restore the reused prefix pages,
@@ -401,11 +414,12 @@ class VerifyModel:
         return nxt, self.ids, acc
 
     def prefill_launches(self, S):
-        """Kernel launches of prefill(S rows): per layer and row group norm-q,
-        qkv, attention split + combine, o, norm-q, gate_up, swiglu-q, down,
-        plus one K/V append per layer; then the head on the last row."""
+        """Kernel launches of prefill(S rows): per layer norm-q, tile image,
+        qkv, K/V append, one causal attention per block of 128 queries,
+        quantise, tile image, o, norm-q, tile image, gate_up, swiglu-q, tile
+        image, down; then the head on the last row."""
         n = len(prefill_chunks(0, S))
-        return 0 if S == 0 else self.n_layers * (9 * n + 1) + (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
+        return 0 if S == 0 else self.n_layers * (13 + n) + (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     def step(self, restore=True):
         """One verify step on the current self.h / self.parent; result in self.ids."""
@@ -420,10 +434,10 @@ class VerifyModel:
 
     @property
     def launches_per_layer(self):
-        """norm-q, qkv, kv-append, attention split + combine, [quantise], o,
+        """norm-q, qkv, kv-append, attention (split with fused combine), [quantise], o,
         norm-q, gate_up, swiglu-q, down (the attention output is quantised in
         the combine launch when the scales are static)."""
-        return 10 if self.static else 11
+        return 9 if self.static else 10
 
     def launches_per_step(self, restore=True):
         return (1 if restore else 0) + self.n_layers * self.launches_per_layer + \

@@ -10,7 +10,8 @@ Labels are hash-consed: a label is the integer id of a flat tuple whose parts
 are strings, numbers or the ids of other labels, so deep layer stacks compare
 in constant time.
 No kernel and no oracle runs; launches are counted as the library would
-launch kernels (the attention is a split and a combine launch).
+launch kernels (the attention is one launch: its combine is fused when the
+split grid fits on the GPU at once, as it does at the verify step's shapes).
 """
 import numpy as np
 import torch
@@ -106,28 +107,73 @@ class FakeLib:
         self.launches += 1
         assert (path, n) == ("path", "n") and ctx_len == self.m.L and n_layers == self.m.n_layers
 
+    def _quant_out(self, out, act, labels):
+        """A quantiser writes the 16-row prepared image (act) or, for any row
+        count with a static scale, the canonical codes (out[0])."""
+        if act is not None:
+            assert len(labels) <= 16
+            self.put(act, labels)
+        else:
+            assert out[0] is not None and out[0].shape[0] == len(labels)
+            self.put(out[0], labels)
+
     def quantize(self, x, g_in=None, out=None, act=None, canonical=True, ws=None, stream=None):
         self.launches += 1
-        assert x.shape[0] <= 16 and act is not None
+        assert act is not None or g_in is not None
         src = self.get(x)
         lab = self.scale(g_in, out[2], src)
-        self.put(act, [self.L("quant", lab, v) for v in src])
+        self._quant_out(out, act, [self.L("quant", lab, v) for v in src])
         return out
 
     def rmsnorm_quantize(self, x, w, eps, out, act=None, stream=None, g_in=None):
         self.launches += 1
-        assert x.shape[0] <= 16
+        assert x.shape[0] <= 16 or (g_in is not None and act is None)
         src = self.get(x)
         widx = (w.data_ptr() - self.m.norm_w.data_ptr()) // (I.HIDDEN * 2)
         lab = self.scale(g_in, out[2], src)
-        self.put(act, [self.L("norm", widx, lab, v) for v in src])
+        self._quant_out(out, act, [self.L("norm", widx, lab, v) for v in src])
 
     def swiglu_quantize(self, gu, out, act=None, stream=None, g_in=None):
         self.launches += 1
-        assert gu.shape[0] <= 16
+        assert gu.shape[0] <= 16 or (g_in is not None and act is None)
         src = self.get(gu)
         lab = self.scale(g_in, out[2], src)
-        self.put(act, [self.L("swiglu", lab, v) for v in src])
+        self._quant_out(out, act, [self.L("swiglu", lab, v) for v in src])
+
+    def prepared_weight_bytes(self, N, K):
+        return N * K
+
+    def prepare_weight(self, codes, scales, N, K, out=None, stream=None):
+        """Tile image of canonical codes: moves row labels (rows 0 .. N-1 of out)."""
+        self.launches += 1
+        assert codes.shape[0] == N and out is not None
+        self.put(out[:N], self.get(codes))
+        return out
+
+    def linear_wide(self, a_prep, g_a, S, w_prep, g_w, N, K, y=None, residual=None, stream=None):
+        self.launches += 1
+        assert y.shape[0] == S
+        l, name = self.wmap[id(w_prep)]
+        a = self.get(a_prep[:S])
+        res = None
+        if residual is not None:
+            assert residual.data_ptr() == y.data_ptr()
+            res = self.get(residual)
+        self.put(y, [self.L("linear", l, name, self.gl[g_a.data_ptr()], v, None if res is None else res[i])
+                     for i, v in enumerate(a)])
+
+    def causal_attn(self, q, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, sm_scale=None, out=None,
+                    ld_q=None, T=None, Hq=None, ws=None, stream=None):
+        """Query i (position ctx_len + i) attends to every labelled context
+        position and to the new positions ctx_len .. ctx_len + i."""
+        self.launches += 1
+        l = self.layer_of_pool(k_pool)
+        assert 1 <= T <= 128 and Hq == I.N_Q_HEADS and ld_q == q.stride(0)
+        assert (ctx_len + T + I.PAGE - 1) // I.PAGE <= self.m.n_log
+        qs = self.get(q, T)
+        ctx = [self.kv.get((l, p)) for p in range(self.start, ctx_len)]
+        self.put(out, [self.L("attn", qs[i], *ctx, *[self.kv.get((l, ctx_len + j)) for j in range(i + 1)])
+                       for i in range(T)])
 
     def linear(self, a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, stream=None):
         self.launches += 1
@@ -159,7 +205,7 @@ class FakeLib:
 
     def tree_attn(self, q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None,
                   out=None, ld_q=None, T=None, Hq=None, ws=None, stream=None, g_act=None, act=None):
-        self.launches += 2
+        self.launches += 1
         l = self.layer_of_pool(k_pool)
         assert 1 <= T <= 16 and Hq == I.N_Q_HEADS and ld_q == q.stride(0)
         assert (ctx_len + T + I.PAGE - 1) // I.PAGE <= self.m.n_log

@@ -97,6 +97,12 @@ def test_host_checks_reject_bad_arguments_before_the_device():
         (E_SHAPE, "nvfp4_linear", A, A, 16, A, A, 524289, 128, None, A, 524289, A, 1 << 20, None),
         (E_SHAPE, "nvfp4_linear", A, A, 16, A, A, 128, 96, None, A, 128, A, 1 << 20, None),
         (E_ALIGN, "nvfp4_linear", MIS, A, 16, A, A, 128, 128, None, A, 128, A, 1 << 20, None),
+        # nvfp4_linear_wide(a, g_a, S, w, g_w, N, K, residual, y, ldy, stream)
+        (E_ARG, "nvfp4_linear_wide", None, A, 100, A, A, 128, 128, None, A, 128, None),
+        (E_SHAPE, "nvfp4_linear_wide", A, A, 0, A, A, 128, 128, None, A, 128, None),
+        (E_SHAPE, "nvfp4_linear_wide", A, A, 100, A, A, 128, 96, None, A, 128, None),
+        (E_SHAPE, "nvfp4_linear_wide", A, A, 100, A, A, 128, 128, None, A, 64, None),
+        (E_ALIGN, "nvfp4_linear_wide", MIS, A, 100, A, A, 128, 128, None, A, 128, None),
         # nvfp4_linear_noalloc(a, g_a, M, w, g_w, N, K, residual, y, ldy, stream)
         (E_SHAPE, "nvfp4_linear_noalloc", A, A, 16, A, A, 524289, 128, None, A, 524289, None),
         # tree_attn_fp8kv(q, ld_q, T, Hq, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, parent,
@@ -111,13 +117,27 @@ def test_host_checks_reject_bad_arguments_before_the_device():
          None, A, 1 << 20, None),
         (E_ARG, "tree_attn_fp8kv", A, 3072, 16, 24, 4, 128, A, A, 8, 64, A, 100, A, A, A, 0.088, A, None,
          A, A, 1 << 20, None),
+        # causal_attn_fp8kv(q, ld_q, T, Hq, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len,
+        #                   k_scale, v_scale, sm_scale, out, ws, ws_bytes, stream)
+        (E_ARG, "causal_attn_fp8kv", None, 3072, 128, 24, 4, 128, A, A, 8, 64, A, 100, A, A, 0.088, A, A, 1 << 20,
+         None),
+        (E_SHAPE, "causal_attn_fp8kv", A, 3072, 129, 24, 4, 128, A, A, 8, 64, A, 100, A, A, 0.088, A, A, 1 << 20,
+         None),
+        (E_SHAPE, "causal_attn_fp8kv", A, 3072, 64, 24, 5, 128, A, A, 8, 64, A, 100, A, A, 0.088, A, A, 1 << 20,
+         None),
+        (E_ALIGN, "causal_attn_fp8kv", MIS, 3072, 64, 24, 4, 128, A, A, 8, 64, A, 100, A, A, 0.088, A, A, 1 << 20,
+         None),
         # kv_page_restore(src, src_ids, dst, dst_ids, n, page_bytes, n_src, n_dst, stream)
         (E_SHAPE, "kv_page_restore", A, A, A, A, 4, 15, 8, 8, None),
         (E_ALIGN, "kv_page_restore", MIS, A, A, A, 4, 32768, 8, 8, None),
         # nvfp4_rmsnorm_quantize(x, w, eps, rows, n, g_in, codes, scales, g_out, act, ws, ws_bytes, stream)
         (E_SHAPE, "nvfp4_rmsnorm_quantize", A, A, 1e-6, 16, 8256, None, A, A, A, None, None, 0, None),
+        (E_SHAPE, "nvfp4_rmsnorm_quantize", A, A, 1e-6, 17, 5120, None, A, A, A, None, None, 0, None),
+        (E_SHAPE, "nvfp4_rmsnorm_quantize", A, A, 1e-6, 17, 5120, A, A, A, A, A, None, 0, None),
         # nvfp4_swiglu_quantize(gu, rows, F, g_in, codes, scales, g_out, act, ws, ws_bytes, stream)
         (E_SHAPE, "nvfp4_swiglu_quantize", A, 0, 17408, None, A, A, A, None, None, 0, None),
+        (E_SHAPE, "nvfp4_swiglu_quantize", A, 17, 17408, None, A, A, A, None, None, 0, None),
+        (E_SHAPE, "nvfp4_swiglu_quantize", A, 17, 17408, A, A, A, A, A, None, 0, None),
         # kv_append_fp8(k, v, ld, T, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, k_s, v_s, stream)
         (E_SHAPE, "kv_append_fp8", A, A, 4096, 16, 4, 12, A, A, 8, 64, A, 100, A, A, None),
         # argmax_rows_bf16(x, rows, n, ld, idx, ws, ws_bytes, stream)
@@ -184,6 +204,9 @@ def test_binding_rejects_host_tensors():
                               h(16, dt=torch.int32), g, g, out=bf(16, 24, 128), ws=HostWs()),
         lambda: lib.argmax(bf(16, 4096), idx=h(16, dt=torch.int32), ws=HostWs()),
         lambda: lib.v_pages_to_tiled(h(2, 64, 128), h(2, 8192)),
+        lambda: lib.linear_wide(h(36864), g, 20, h(36864), g, 128, 512, y=bf(20, 128)),
+        lambda: lib.causal_attn(bf(32, 24, 128), h(2, 4, 64, 128), h(2, 4, 8192), h(2, dt=torch.int32), 10,
+                                g, g, out=bf(32, 24, 128), ws=HostWs()),
     ]
     for i, call in enumerate(calls):
         with pytest.raises(ValueError, match="device tensor"):
@@ -191,9 +214,9 @@ def test_binding_rejects_host_tensors():
 
 
 def test_failing_status_rezeroes_counter_workspaces(monkeypatch):
-    """After a failing device status the binding zeroes its default linear and
-    argmax workspaces (their arrival counters may be stale after a wait ran
-    out) and leaves the others alone; a clean status touches nothing."""
+    """After a failing device status the binding zeroes its default linear,
+    argmax and attention workspaces (their arrival counters may be stale after
+    a wait ran out) and leaves the others alone; a clean status touches nothing."""
     import torch
 
     class FakeWs:
@@ -215,5 +238,5 @@ def test_failing_status_rezeroes_counter_workspaces(monkeypatch):
     state["rc"] = -6
     assert lib.device_status()[0] == -6
     for (_, kind), w in spaces.items():
-        want = 0 if kind in ("linear", "argmax") else 7
+        want = 0 if kind in ("linear", "argmax", "attn") else 7
         assert int(w.buf.min()) == want and int(w.buf.max()) == want, kind

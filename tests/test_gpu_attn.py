@@ -180,3 +180,67 @@ def test_fused_nvfp4_output_matches_separate_quantisation():
     nv.quantize(out.view(T, Hq * 128), g_in=g, act=ref_act, canonical=False)
     assert torch.equal(act, ref_act)
     assert nv.device_status()[0] == 0
+
+
+def test_fused_combine_leaves_counters_zero_and_is_repeatable():
+    """The fused combine's per-head arrival counters sit at the start of the
+    workspace: after each call they read zero again, and a second call on the
+    same workspace gives bit-identical outputs."""
+    cuda()
+    L = 5000
+    cache = inputs.kv_cache(81, L)
+    parent = inputs.tree_parent(81)
+    q = to_dev(inputs.query_bf16(81))
+    kp, vp, pt, ks, vs = _dev_cache(cache)
+    ws = nv.Workspace()
+    a = nv.tree_attn(q, kp, vp, pt, L, to_dev(parent), ks, vs, ws=ws).clone()
+    torch.cuda.synchronize()
+    assert int(ws.buf[:64].count_nonzero()) == 0
+    b = nv.tree_attn(q, kp, vp, pt, L, to_dev(parent), ks, vs, ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws.buf[:64].count_nonzero()) == 0
+    assert torch.equal(a, b)
+    assert nv.device_status()[0] == 0
+
+
+def _run_causal(q, cache, ctx, T, rows=None, dev=None):
+    kp, vp, pt, ks, vs = dev if dev is not None else _dev_cache(cache)
+    qd = to_dev(q)
+    out = nv.causal_attn(qd, kp, vp, pt, ctx, ks, vs, T=T, Hq=q.shape[1], ld_q=qd.stride(0))
+    return host(out)
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,L", [(1, 24, 4, 0), (17, 24, 4, 300), (100, 8, 2, 1000), (128, 24, 4, 37),
+                                        (128, 6, 1, 4096), (64, 24, 4, 0)])
+def test_causal_attention(oracle, T, Hq, Hkv, L):
+    """Causal attention of T new tokens over the context (the suffix prefill's
+    attention) against the oracle's attention with a chain parent array (a
+    chain tree is causal attention over context + chain)."""
+    cuda()
+    seed = 82 + T + L % 7
+    cache = inputs.kv_cache(seed, L, T=T, Hkv=Hkv, extra_pages=2)
+    q = inputs.query_bf16(seed, T, Hq)
+    got = _run_causal(q, cache, L, T)
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, L, inputs.chain_parent(T),
+                            cache.k_scale, cache.v_scale)
+    err = np.abs(got - want)
+    assert np.all(err <= ATTN_ABS_TOL + 2.0 ** -8 * np.abs(want)), err.max()
+
+
+def test_causal_attention_prefill_blocks(oracle):
+    """A 300-token suffix after 22,000 cached tokens, run as blocks of 128, 128
+    and 44 queries (block b at ctx = start + 128 b): together they equal one
+    causal pass over the whole suffix, within the stated 2e-3 bar."""
+    cuda()
+    start, S, Hq = 22000, 300, 24
+    cache = inputs.kv_cache(85, start, T=S)
+    q = inputs.query_bf16(85, S, Hq)
+    dev = _dev_cache(cache)
+    got = np.concatenate([_run_causal(q[b:b + 128], cache, start + b, min(128, S - b), dev=dev)
+                          for b in range(0, S, 128)])
+    want = oracle.tree_attn(q.float().numpy(), cache.k_pool, cache.v_pool, cache.page_table, start,
+                            inputs.chain_parent(S), cache.k_scale, cache.v_scale)
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    print(f"causal prefill blocks: max abs err {err.max():.3e}, rel-Frobenius {rel:.3e}")
+    assert err.max() <= ATTN_ABS_TOL

@@ -2,10 +2,10 @@
 the label-moving fake of the library (tests/fake_lib.py): the final labels of
 the hidden rows, of every layer's cache positions and of the returned token
 must be those of the layer definition applied to all suffix rows at once, as
-one causal chain.  So the test fails if a row group reads a buffer that
-another group has overwritten, attends before the K/V it needs is written or
-to K/V it must not see, reads another layer's pool or weights, or quantises
-with another site's scale.
+one causal chain.  So the test fails if an attention block attends before
+the K/V it needs is written or to K/V it must not see, a linear reads another
+site's activation, another layer's pool or weights, or a quantiser uses
+another site's scale.
 """
 import pytest
 import torch
@@ -27,7 +27,7 @@ def _expected(fake, n_layers, start, S):
     return expected_layers(fake.L, n_layers, start, S, I.chain_parent(S), _inputs(fake, S))
 
 
-@pytest.mark.parametrize("S", [1, 16, 37, 48])
+@pytest.mark.parametrize("S", [1, 16, 37, 130, 300])
 def test_prefill_dataflow(monkeypatch, S):
     L = 1040
     start = L - S
@@ -52,7 +52,7 @@ def test_prefill_dataflow(monkeypatch, S):
 def test_prefill_groups():
     assert step.prefill_chunks(100, 0) == []
     assert step.prefill_chunks(100, 5) == [(0, 5, 100)]
-    assert step.prefill_chunks(7, 40) == [(0, 16, 7), (16, 16, 23), (32, 8, 39)]
+    assert step.prefill_chunks(7, 300) == [(0, 128, 7), (128, 128, 135), (256, 44, 263)]
     for start, S in [(0, 1), (3, 16), (998, 42), (0, 1000)]:
         g = step.prefill_chunks(start, S)
         assert sum(t for _, t, _ in g) == S
@@ -82,7 +82,7 @@ def test_prefill_arguments(monkeypatch):
 def test_prefill_layer_ranges(monkeypatch):
     """Layers 0..k-1 and then k..n-1 in two calls give the labels of one call;
     the head runs only in the call that ends with the last layer."""
-    L, S = 1040, 21
+    L, S = 1040, 150
     start = L - S
     m, fake = _model(monkeypatch, 3, L)
     fake.start = start
