@@ -169,18 +169,24 @@ def test_suffix_groups_equal_whole_causal(oracle):
     """Row group (r, t) of a causal suffix sees positions < start + r + i for
     its row i, which is a chain of t tokens after a context of start + r: the
     oracle visits the same positions in the same order, so the results match
-    exactly.  S = 37 gives two full groups and a ragged one."""
-    from nvfp4_skinny_gemm_b200.step import prefill_chunks
-    S, Hq, Hkv, D, P, start = 37, 4, 2, 16, 16, 29
+    exactly.  Groups of 16 (S = 37: two full groups and a ragged one) and the
+    prefill's blocks of 128 queries (S = 150: one full block and a ragged one)."""
+    from nvfp4_skinny_gemm_b200.step import PREFILL_CHUNK, prefill_chunks
+    Hq, Hkv, D, P, start = 4, 2, 16, 16, 29
+    for S, C, sizes in [(37, 16, [16, 16, 5]), (150, PREFILL_CHUNK, [128, 22])]:
+        cache = inputs.kv_cache(104, start, T=S, Hkv=Hkv, D=D, P=P, extra_pages=2)
+        q = inputs.query_bf16(104, S, Hq, D).float().numpy()
+        whole = _run(oracle, q, cache, inputs.chain_parent(S))
+        groups = prefill_chunks(start, S, C)
+        assert [t for _, t, _ in groups] == sizes
+        for r, t, ctx in groups:
+            part = oracle.tree_attn(q[r:r + t], cache.k_pool, cache.v_pool, cache.page_table, ctx,
+                                    inputs.chain_parent(t), cache.k_scale, cache.v_scale)
+            assert np.array_equal(part, whole[r:r + t]), (S, r, t)
+    S = 37
     cache = inputs.kv_cache(104, start, T=S, Hkv=Hkv, D=D, P=P, extra_pages=2)
     q = inputs.query_bf16(104, S, Hq, D).float().numpy()
     whole = _run(oracle, q, cache, inputs.chain_parent(S))
-    groups = prefill_chunks(start, S)
-    assert [t for _, t, _ in groups] == [16, 16, 5]
-    for r, t, ctx in groups:
-        part = oracle.tree_attn(q[r:r + t], cache.k_pool, cache.v_pool, cache.page_table, ctx,
-                                inputs.chain_parent(t), cache.k_scale, cache.v_scale)
-        assert np.array_equal(part, whole[r:r + t]), (r, t)
     # the check has teeth: rows that skip the earlier rows of their own group differ
     wrong = oracle.tree_attn(q[16:32], cache.k_pool, cache.v_pool, cache.page_table, start + 16,
                              np.full(16, -1, np.int32), cache.k_scale, cache.v_scale)
