@@ -642,11 +642,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             named_bar_sync(1, 256);
             if (threadIdx.x == 64) {
                 red_release_gpu_add(p.cnt + ch, 1);
-                if (!poll_counter_ge(p.cnt + ch, p.S, 325, s_abort)) *s_abort = 1;
+                const bool all_in = poll_counter_ge(p.cnt + ch, p.S, 325, s_abort);
+                if (!all_in) *s_abort = 1;
+                xch[0] = (all_in && !*s_abort) ? 1.f : 0.f;        // one decision for every thread
             }
             named_bar_sync(1, 256);
             __threadfence();
-            const bool merge = !*s_abort;                          // one decision for the whole group
+            const bool merge = xch[0] != 0.f;
             const int nr = p.nheads * T;
             const int r0 = (int)((int64_t)split * nr / p.S), r1 = (int)((int64_t)(split + 1) * nr / p.S);
             const int d = gt;                                      // dimension of this thread
