@@ -56,7 +56,8 @@ def parse():
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--kernel-case", default=None,
                     choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "linear_o", "linear_down",
-                             "linear_m1_2048", "attn", "restore", "quantize"],
+                             "linear_m1_2048", "wide_gate_up", "wide_down", "causal_attn", "attn", "restore",
+                             "quantize"],
                     help="run one kernel on a small case (for ncu captures) instead of the step")
     return ap.parse_args()
 
@@ -550,6 +551,34 @@ def run_prefill(args):
         assert rc == 0, f"device status {rc} at site {site}"
         assert ids is not None and 0 <= int(ids.cpu()[0]) < I.VOCAB
 
+        # ---- breakdown: the prefill's wide linears alone, then its causal
+        #      attention calls alone (same shapes, same buffers, back to back)
+        pf = model._pf
+        scratch_h = torch.empty_like(h)
+
+        def wide_linears():
+            for lay in model.layers:
+                for name, y in (("qkv", pf["qkv"][:S]), ("o", scratch_h), ("gate_up", pf["gu"][:S]),
+                                ("down", scratch_h)):
+                    lin = lay[name]
+                    nv.linear_wide(pf["wide"], pf["g"], S, lin.prep, lin.g, lin.N, lin.K, y=y)
+
+        def causal_attention():
+            from nvfp4_skinny_gemm_b200.step import prefill_chunks
+            for l in range(model.n_layers):
+                for r, t, ctx in prefill_chunks(start, S):
+                    nv.causal_attn(pf["qkv"][r:r + t], model.k_pool(l), model.v_pool(l), model.page_table, ctx,
+                                   model.k_scale[l], model.v_scale[l], out=pf["attn"][r:r + t],
+                                   ld_q=pf["qkv"].stride(0), T=t, Hq=I.N_Q_HEADS)
+
+        g_lin = capture(stream, wide_linears)
+        g_att = capture(stream, causal_attention)
+        t_lin = time_graph(g_lin, stream, max(2, args.steps))
+        t_att = time_graph(g_att, stream, max(2, args.steps))
+        rc, site = nv.device_status(stream)
+        assert rc == 0, f"device status {rc} at site {site}"
+        del g_lin, g_att
+
     lin_flops, attn_flops = prefill_flops(S, start, args.layers)
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
@@ -563,7 +592,8 @@ def run_prefill(args):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate); fp8 e4m3 KV", "data": "synthetic",
         "config": {"workload": f"{args.layers}-layer suffix prefill of {S} tokens after {start} cached tokens, "
-                               f"16-row groups through the skinny kernels, LM head on the last token",
+                               f"wide NVFP4 linears and causal attention in 128-query blocks, LM head on the "
+                               f"last token",
                    "layers": args.layers, "ctx": L, "suffix": S, "parallelism": "single GPU",
                    "l2": "inputs larger than L2 (11.4 GB of weights)"},
         "roofline": {"bound": "tensor", "achieved": round(flops / t / 1e12, 1),
@@ -572,6 +602,16 @@ def run_prefill(args):
                                     f"weighted by their FLOPs",
                      "linear_tflop": round(lin_flops / 1e12, 2), "attention_tflop": round(attn_flops / 1e12, 2),
                      "traffic": None},
+        "breakdown": {
+            "wide_linears": {"ms": round(t_lin * 1e3, 3), "tflops": round(lin_flops / t_lin / 1e12, 1),
+                             "frac": round(lin_flops / t_lin / (4 * bf16 * 1e12), 4),
+                             "note": "all nvfp4_linear_wide launches of one prefill, back to back; frac of the "
+                                     "FP4 peak (sustained bf16 x 4)"},
+            "causal_attention": {"ms": round(t_att * 1e3, 3), "tflops": round(attn_flops / t_att / 1e12, 1),
+                                 "frac": round(attn_flops / t_att / (2 * bf16 * 1e12), 4),
+                                 "note": "all causal_attn_fp8kv launches of one prefill, back to back; frac of "
+                                         "the FP8 peak (sustained bf16 x 2)"},
+            "rest_ms": round((t - t_lin - t_att) * 1e3, 3)},
         "clocks": clk,
         "gpu_launches": model.prefill_launches(S) * args.steps,
     }
@@ -607,6 +647,28 @@ def run_kernel_case(args):
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         fn = lambda i: nv.linear(act, ga, M, ws[i % ncopy][0], ws[i % ncopy][1], N, K, y=y)
         nbytes = N * K * 9 // 16
+    elif case.startswith("wide"):
+        K, N = I.LAYER_LINEARS[case[5:]]
+        S = 942
+        wc = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        wsc = torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g)
+        w_p = nv.prepare_weight(wc, wsc, N, K)
+        ac = torch.randint(0, 256, (S, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        asc = torch.randint(0x30, 0x40, (S, K // 16), dtype=torch.uint8, device=dev, generator=g)
+        a_p = nv.prepare_weight(ac, asc, S, K)
+        one = torch.full((1,), 0.01, device=dev)
+        y = torch.empty(S, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: nv.linear_wide(a_p, one, S, w_p, one, N, K, y=y)
+        nbytes = N * K * 9 // 16
+    elif case == "causal_attn":
+        start, T = 22610, 128
+        cache = I.kv_cache(3, start, T=T)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+        kp, vp, pt, ks, vs = t(cache.k_pool), t(cache.v_pool), t(cache.page_table), t(cache.k_scale), t(cache.v_scale)
+        q = I.query_bf16(3, T).to(dev)
+        out = torch.empty(T, 24, 128, dtype=torch.bfloat16, device=dev)
+        fn = lambda i: nv.causal_attn(q, kp, vp, pt, start, ks, vs, out=out)
+        nbytes = (start + T) * 4 * 128 * 2
     elif case == "attn":
         cache = I.kv_cache(3, I.CTX_MAX)
         t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)

@@ -122,6 +122,8 @@ NVFP4SK_API nvfp4sk_status nvfp4_prepare_act(const uint8_t *codes, const uint8_t
  * step for the NVFP4 weights of section "NVFP4 and FP8" (calibrated once,
  * then served).  prepared: nvfp4_prepared_weight_bytes(N, K) bytes, 16-byte
  * aligned (opaque).  K % 64 == 0; rows/columns beyond N/K are zero-padded.
+ * codes must be 16-byte aligned and scales 4-byte aligned.  Also the tile
+ * image of a many-token activation for nvfp4_linear_wide (tokens as rows).
  * ---------------------------------------------------------------------- */
 NVFP4SK_API size_t nvfp4_prepared_weight_bytes(int64_t N, int64_t K);
 NVFP4SK_API nvfp4sk_status nvfp4_prepare_weight(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K,
@@ -383,7 +385,10 @@ enum {
     NVFP4SK_OPT_PDL = 0,          /* 1: launch with programmatic dependent launch (default 1) */
     NVFP4SK_OPT_TIMEOUT_NS = 1,   /* per-wait limit of device spin-waits (default 1e9)        */
     NVFP4SK_OPT_ATTN_SPLITS = 2,  /* 0: automatic; else KV splits per KV head                 */
-    NVFP4SK_OPT_LINEAR_CTAS = 3   /* 0: one CTA per SM; else the split-K grid size            */
+    NVFP4SK_OPT_LINEAR_CTAS = 3,  /* 0: one CTA per SM; else the split-K grid size            */
+    NVFP4SK_OPT_ATTN_FUSED_COMBINE = 4 /* 1: the attention's CTAs merge their split results
+                                        themselves (needs splits x heads <= #SMs); 0 (default):
+                                        a second launch merges them (measured faster on B200) */
 };
 NVFP4SK_API nvfp4sk_status nvfp4sk_set_option(int option, int64_t value);
 NVFP4SK_API int64_t nvfp4sk_get_option(int option);

@@ -14,22 +14,25 @@
 //               query, K as the cached E4M3 codes (128-byte-swizzled TMA
 //               tile); fp32 S in tensor memory.
 //   softmax     one thread per row: S row -> registers (tcgen05.ld), ancestor
-//               mask on the page that holds the tree, running max in the
-//               log2 domain, P' = 2^(s - m) in f16 (ex2.approx.f16x2 on the
-//               f16-rounded exponent), stored to shared memory in the MMA's
+//               (or causal) mask on the pages that hold the new positions,
+//               running max in the log2 domain, P' = 2^(s - m + 6) as two
+//               E4M3 terms (hi + lo) stored to shared memory in the MMA's
 //               core-matrix layout.  O is rescaled in tensor memory only when
-//               a row max grows by more than 2^2.
-//   O += P V    tcgen05.mma kind::f16, M=128, N=144, K=16: the page's V codes
-//               (kept in HBM in a tiled core-matrix layout, one bulk copy per
-//               page) are widened E4M3 -> f16 (exact) into the operand image
-//               by the softmax threads; 16 extra operand rows (one of them all
-//               ones) make column 128 of O the row sum of P', accumulated in
-//               fp32 by the tensor core.
+//               a row max grows by more than 2^2.  Warps whose 32 rows are all
+//               padding skip this work and only keep the barriers in step.
+//   O += P V    M=128, N=144, K=32: the V pages are kept in HBM in the
+//               core-matrix layout, so one bulk copy lands the operand; 16
+//               extra operand rows (one of them all ones) make column 128 of
+//               O the row sum of P', accumulated in fp32 by the tensor core.
+// (Measured: an f16 P with V widened to f16 in shared memory gains nothing --
+// ex2.approx.f16x2 runs at the f32 rate, 16 values per SM per clock -- and its
+// operand buffers cost two of the ten ring stages, which made the last pages
+// of each CTA arrive late.)
 // Two softmax warpgroups take alternate pages, each with its own S and O
 // accumulators in tensor memory and its own running max, so that two pages
 // are in the exponent stage at once; their results are merged in the
 // epilogue.
-// Warp roles: 0 producer (lane s feeds stage s of an 8-stage ring: TMA K page
+// Warp roles: 0 producer (lane s feeds stage s of a 10-stage ring: TMA K page
 // + bulk V page; context pages are requested before the wait on the
 // preceding kernel), 1 TMEM allocation + QK issue (one thread), 10 PV issue
 // (one thread), 2-5 and 6-9 softmax.  The two issuers run independently, so
@@ -49,18 +52,17 @@ constexpr int ATT_D = 128;
 constexpr int ATT_P = 64;
 constexpr int ATT_T = 16;
 constexpr int ATT_ROWS = 128;
-constexpr int ATT_STAGES = 8;
+constexpr int ATT_STAGES = 10;
 constexpr int ATT_THREADS = 352;
 constexpr int ATT_MAX_SPLITS = 1024;
 constexpr uint32_t ATT_K_BYTES = ATT_P * ATT_D;                 // 8 KB token-major page
 constexpr uint32_t ATT_V_BYTES = ATT_D * ATT_P;                 // 8 KB tiled page
-constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES; // 16 KB
+constexpr uint32_t ATT_ONES_BYTES = 16 * ATT_P;                 // 16 operand rows: ones, then zeros
+constexpr uint32_t ATT_STAGE_BYTES = ATT_K_BYTES + ATT_V_BYTES + ATT_ONES_BYTES;   // 17 KB
 constexpr uint32_t ATT_NO = ATT_D + 16;                         // O columns: 128 dims + row sum block
-constexpr uint32_t ATT_P16_BYTES = ATT_ROWS * ATT_P * 2;        // P of one page in f16: 16 KB
-constexpr uint32_t ATT_V16_BYTES = ATT_NO * ATT_P * 2;          // V of one page in f16 + ones block: 18 KB
-constexpr uint32_t ATT_OFF_P = ATT_STAGES * ATT_STAGE_BYTES;    // P[2 groups]
-constexpr uint32_t ATT_OFF_V16 = ATT_OFF_P + 2 * ATT_P16_BYTES; // V16[2 groups]
-constexpr uint32_t ATT_OFF_X = ATT_OFF_V16 + 2 * ATT_V16_BYTES; // float exchange [2][2][128]
+constexpr uint32_t ATT_PB_BYTES = ATT_ROWS * ATT_P;             // one E4M3 term of P
+constexpr uint32_t ATT_OFF_P = ATT_STAGES * ATT_STAGE_BYTES;    // P[2 groups] x (hi | lo)
+constexpr uint32_t ATT_OFF_X = ATT_OFF_P + 4 * ATT_PB_BYTES;    // float exchange [2][2][128]
 constexpr uint32_t ATT_OFF_C = ATT_OFF_X + 2048;                // combine: bf16 rows as float [2][128]
 constexpr uint32_t ATT_OFF_BAR = ATT_OFF_C + 1024;
 constexpr uint32_t ATT_SMEM_BYTES = ATT_OFF_BAR + 512 + 1024;
@@ -69,6 +71,7 @@ constexpr uint32_t ATT_TM_S0 = 0, ATT_TM_S1 = 64;
 constexpr uint32_t ATT_TM_O0 = 128, ATT_TM_O1 = 288;
 constexpr uint32_t ATT_TM_Q = 448;                              // Q hi 448..479, Q lo 480..511 (A operand)
 constexpr float ATT_TAU = 2.0f;       // log2 growth of a row max that triggers an O rescale
+constexpr float ATT_PSHIFT = 6.0f;    // P' = 2^(s - m + 6) <= 2^(6 + TAU) = 256 < 448
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint32_t ATT_CNT_BYTES = 256;                         // per-head arrival counters (fused combine)
 static_assert(ATT_STAGE_BYTES % 1024 == 0, "K tiles need 1024-byte alignment (128-byte swizzle atoms)");
@@ -83,9 +86,8 @@ __host__ __device__ __forceinline__ uint32_t v_offset(uint32_t d, uint32_t t)
     return ((d >> 3) * (ATT_P / 16) + (t >> 4)) * 128u + (d & 7u) * 16u + (t & 15u);
 }
 
-// Instruction descriptor: fp32 accumulate (bits 4-5 = 1), A and B format 0
-// (E4M3 under kind::f8f6f4, f16 under kind::f16), K-major, N>>3 in bits
-// 17-22, M>>4 in bits 24-28.
+// Instruction descriptor, kind::f8f6f4: fp32 accumulate (bits 4-5 = 1), A and
+// B E4M3 (format 0), K-major, N>>3 in bits 17-22, M>>4 in bits 24-28.
 constexpr uint32_t att_idesc(uint32_t M, uint32_t N) { return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24); }
 
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -142,32 +144,23 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c)
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)c));
     return d;
 }
-__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t h)
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b)
 {
     uint32_t d;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(d) : "r"(h));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
-// D[tmem] (+)= A x B^T, A and B f16 in shared memory (K-major), fp32 accumulate.
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate)
+// Four non-negative values -> E4M3 codes hi (bytes 0..3) and lo with x ~= hi + lo:
+// x is rounded to f16 (11 bits), hi = E4M3(x), lo = E4M3(x - hi) (exact f16 difference).
+__device__ __forceinline__ void split4_f16(float x0, float x1, float x2, float x3, uint32_t &hi, uint32_t &lo)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Byte offset of (row r, column k) in a K-major f16 operand image without
-// swizzle: core matrices of 8 rows x 8 columns (16-byte rows), 8 core
-// matrices along K per 64 columns (leading byte offset 128), row groups 1 KB
-// apart (stride byte offset 1024).
-__device__ __forceinline__ uint32_t f16_core_offset(uint32_t r, uint32_t k)
-{
-    return ((r >> 3) * 8u + (k >> 3)) * 128u + (r & 7u) * 16u + (k & 7u) * 2u;
+    const uint32_t a = f32x2_to_f16x2(x0, x1), b = f32x2_to_f16x2(x2, x3);
+    const uint32_t ha = f16x2_to_e4m3x2(a), hb = f16x2_to_e4m3x2(b);
+    const uint32_t la = f16x2_to_e4m3x2(hsub2_u32(a, e4m3x2_to_f16x2(ha)));
+    const uint32_t lb = f16x2_to_e4m3x2(hsub2_u32(b, e4m3x2_to_f16x2(hb)));
+    hi = ha | (hb << 16);
+    lo = la | (lb << 16);
 }
 
 // x0, x1 -> (hi, lo) E4M3 pairs (byte 0 = x0, byte 1 = x1) with x ~= hi + lo, in fp32.
@@ -339,7 +332,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         __syncwarp();
     } else if (warp == 10) {
         // ------------------------------------------------------------ PV issuer
-        // O_g += P V of page j once group g has written P and the widened V
+        // O_g += P V of page j once group g has written P (hi, lo) for it
         if (lane == 0) {
             constexpr uint32_t idesc_o = att_idesc(128, ATT_NO);
             bool o_init[2] = {false, false};
@@ -349,13 +342,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if (!mbar_wait(&p_full[g], (uint32_t)((j >> 1) & 1), 311, s_abort)) { ok = false; break; }
                 tc_fence_after();
                 if (s_page_ok[j % ATT_STAGES]) {
-                    const uint32_t p_s = smem_u32(smem + ATT_OFF_P + g * ATT_P16_BYTES);
-                    const uint32_t v_s = smem_u32(smem + ATT_OFF_V16 + g * ATT_V16_BYTES);
+                    const uint32_t v_s = smem_u32(smem + (j % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES);
+                    const uint32_t p_hi = smem_u32(smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES), p_lo = p_hi + ATT_PB_BYTES;
                     const uint32_t o_t = tmem_base + (g ? ATT_TM_O1 : ATT_TM_O0);
 #pragma unroll
-                    for (int t = 0; t < ATT_P / 16; ++t)
-                        mma_f16(o_t, smem_desc(p_s + 256 * t, 128, 1024, SWZ_NONE),
-                                smem_desc(v_s + 256 * t, 128, 1024, SWZ_NONE), idesc_o, (o_init[g] || t > 0) ? 1u : 0u);
+                    for (int t = 0; t < ATT_P / 32; ++t) {
+                        const uint64_t vd = smem_desc(v_s + 256 * t, 128, 512, SWZ_NONE);
+                        mma_f8f6f4(o_t, smem_desc(p_hi + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o,
+                                   (o_init[g] || t > 0) ? 1u : 0u);
+                        mma_f8f6f4(o_t, smem_desc(p_lo + 256 * t, 128, 512, SWZ_NONE), vd, idesc_o, 1u);
+                    }
                     o_init[g] = true;
                 }
                 tc_commit(&p_free[g]);
@@ -383,8 +379,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t row_t = tmem_base + ((32u * qd) << 16);
         const uint32_t s_t = row_t + (g ? ATT_TM_S1 : ATT_TM_S0);
         const uint32_t o_t = row_t + (g ? ATT_TM_O1 : ATT_TM_O0);
-        uint8_t *pb = smem + ATT_OFF_P + g * ATT_P16_BYTES;
-        uint8_t *vb = smem + ATT_OFF_V16 + g * ATT_V16_BYTES;
+        uint8_t *pb = smem + ATT_OFF_P + g * 2 * ATT_PB_BYTES;
+        // a warp whose 32 rows are all padding does no softmax work (the
+        // products of its rows are never read) and only keeps the barriers in step
+        const bool pad_warp = !__any_sync(0xFFFFFFFFu, row_ok && node < p.T);
 
         // ---- Q -> two E4M3 terms, row scaled by a power of two into [128, 256);
         //      group g converts dims 64g .. 64g+63 of row r.  Every global
@@ -413,13 +411,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                              fabsf(__uint_as_float(wd[j] & 0xFFFF0000u))));
             }
             xch[g * 128 + r] = amax;
-            // the ones block of this group's widened-V buffer: operand rows
-            // 128..143 (dims 128..143), row 128 = 1.0 for every token, the rest 0
-            for (int idx = gt; idx < 2 * 8 * 8; idx += 128) {          // 2 row groups x 8 column groups x 8 rows
-                const uint32_t rr = 128u + (uint32_t)(idx >> 6) * 8u + (uint32_t)(idx & 7);
-                const uint32_t kc = (uint32_t)((idx >> 3) & 7) * 8u;
-                const uint32_t v = rr == 128u ? 0x3C003C00u : 0u;
-                *reinterpret_cast<uint4 *>(vb + f16_core_offset(rr, kc)) = make_uint4(v, v, v, v);
+            // the ones block of every stage: operand row 128 (16 bytes per 16-token chunk) = 1.0, rest 0
+            for (int idx = (int)threadIdx.x - 64; idx < ATT_STAGES * (int)(ATT_ONES_BYTES / 16); idx += 256) {
+                const uint32_t off = (uint32_t)(idx % (ATT_ONES_BYTES / 16)) * 16u;
+                const uint32_t v = (off < 512u && (off & 127u) == 0u) ? 0x38383838u : 0u;
+                *reinterpret_cast<uint4 *>(smem + (idx / (ATT_ONES_BYTES / 16)) * ATT_STAGE_BYTES + ATT_K_BYTES +
+                                           ATT_V_BYTES + off) = make_uint4(v, v, v, v);
             }
             named_bar_sync(1, 256);
             amax = fmaxf(xch[r], xch[128 + r]);
@@ -495,91 +492,81 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 continue;
             }
             const int64_t pos0 = (int64_t)(pg0 + i) * ATT_P;
-            if (pos0 + ATT_P > L) {
-                const int t0 = (int)(pos0 - L);                // tree slot of column 0 (> -64)
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const int tj = t0 + j;                     // negative: context position
-                    const bool vis = tj < 0 || (tj < T && (p.causal ? tj <= node : ((anc >> (tj & 31)) & 1u) != 0));
-                    if (!vis) s[j] = 0xFF800000u;             // -inf
-                }
-            }
-            float mr = __uint_as_float(s[0]);
-#pragma unroll
-            for (int j = 1; j < 64; ++j) mr = fmaxf(mr, __uint_as_float(s[j]));
-            const float mx = mr * c_row;
-            const bool need = mx > m_ref + ATT_TAU;
-            const bool resc = need && m_ref > -INFINITY;
             bool waited = false;
-            if (__any_sync(0xFFFFFFFFu, resc)) {
-                // every product of this group so far must be in O before it is rescaled
-                bool r_ok = true;
-                if (lane == 0) r_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 321, s_abort);
-                if (!__shfl_sync(0xFFFFFFFFu, r_ok ? 1 : 0, 0)) { ok = false; break; }
-                waited = true;
-                tc_fence_after();
-                const float alpha = resc ? fast_exp2(m_ref - mx) : 1.f;
-#pragma unroll 1
-                for (uint32_t col = 0; col < ATT_NO; col += 16) {
-                    uint32_t o[16];
-                    tmem_ld_32x32b_x16(o_t + col, o);
-                    tmem_wait_ld();
+            if (!pad_warp) {
+                if (pos0 + ATT_P > L) {
+                    const int t0 = (int)(pos0 - L);            // new-position slot of column 0 (> -64)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                    tmem_st_x16(o_t + col, o);
+                    for (int j = 0; j < 64; ++j) {
+                        const int tj = t0 + j;                 // negative: context position
+                        const bool vis = tj < 0 || (tj < T && (p.causal ? tj <= node : ((anc >> (tj & 31)) & 1u) != 0));
+                        if (!vis) s[j] = 0xFF800000u;         // -inf
+                    }
                 }
-                tmem_wait_st();
-            }
-            if (need) m_ref = mx;
-            const float nb = m_ref > -INFINITY ? -m_ref : 0.f;
-            // P' = 2^(s c - m) in f16: the exponent is rounded to f16, then ex2 on pairs
-            uint32_t ph[32];
+                // row max as a tree (8 independent chains, then 3 levels): a
+                // 63-deep chain of dependent maxes is on every page's critical path
+                float m8[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                ph[j] = ex2_f16x2(f32x2_to_f16x2(fmaf(__uint_as_float(s[2 * j]), c_row, nb),
-                                                 fmaf(__uint_as_float(s[2 * j + 1]), c_row, nb)));
-            // the P and widened-V buffers of this group's previous page must have been consumed
+                for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(s[k]);
+#pragma unroll
+                for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], __uint_as_float(s[j]));
+                const float mr = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                const float mx = mr * c_row;
+                const bool need = mx > m_ref + ATT_TAU;
+                const bool resc = need && m_ref > -INFINITY;
+                if (__any_sync(0xFFFFFFFFu, resc)) {
+                    // every product of this group so far must be in O before it is rescaled
+                    bool r_ok = true;
+                    if (lane == 0) r_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 321, s_abort);
+                    if (!__shfl_sync(0xFFFFFFFFu, r_ok ? 1 : 0, 0)) { ok = false; break; }
+                    waited = true;
+                    tc_fence_after();
+                    const float alpha = resc ? fast_exp2(m_ref - mx) : 1.f;
+#pragma unroll 1
+                    for (uint32_t col = 0; col < ATT_NO; col += 16) {
+                        uint32_t o[16];
+                        tmem_ld_32x32b_x16(o_t + col, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st_x16(o_t + col, o);
+                    }
+                    tmem_wait_st();
+                }
+                if (need) m_ref = mx;
+            }
+            uint32_t ph[16], pl[16];
+            if (!pad_warp) {
+                const float nb = m_ref > -INFINITY ? ATT_PSHIFT - m_ref : 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; j += 4)
+                    split4_f16(fast_exp2(fmaf(__uint_as_float(s[j]), c_row, nb)),
+                               fast_exp2(fmaf(__uint_as_float(s[j + 1]), c_row, nb)),
+                               fast_exp2(fmaf(__uint_as_float(s[j + 2]), c_row, nb)),
+                               fast_exp2(fmaf(__uint_as_float(s[j + 3]), c_row, nb)), ph[j >> 2], pl[j >> 2]);
+            }
+            if (pos0 + ATT_P > L + T) {
+                // slots past the last written position may hold any byte (NaN codes
+                // included); zero their V (this thread: dimension r) so 0 * V stays 0
+                const bool k_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
+                if (!__all_sync(0xFFFFFFFFu, k_ok)) { ok = false; break; }
+                uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
+                for (int t = (int)(L + T - pos0); t < ATT_P; ++t) vs[v_offset((uint32_t)r, (uint32_t)t)] = 0;
+            }
+            // the P buffer of this group's previous page must have been consumed
             if (!waited && i >= 2) {
                 bool f_ok = true;
                 if (lane == 0) f_ok = mbar_wait(&p_free[g], (uint32_t)(((i - 2) >> 1) & 1), 322, s_abort);
                 if (!__shfl_sync(0xFFFFFFFFu, f_ok ? 1 : 0, 0)) { ok = false; break; }
             }
+            if (!pad_warp) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c)                        // tokens 8c .. 8c+7 of row r
-                *reinterpret_cast<uint4 *>(pb + f16_core_offset((uint32_t)r, 8u * c)) =
-                    make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-            // V of this page, E4M3 -> f16 (exact), into the operand image: each
-            // thread widens 4 of the page's 512 tiled rows (dim d, tokens
-            // 16j .. 16j+15); slots past the last written position may hold any
-            // byte and are written as zeros, so that 0 * V stays 0
-            {
-                const bool v_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
-                if (!__all_sync(0xFFFFFFFFu, v_ok)) { ok = false; break; }
-                const uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
-                const int valid = (int)(L + T - pos0 < ATT_P ? L + T - pos0 : ATT_P);   // slots holding written positions
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const uint32_t x = (uint32_t)gt + 128u * m;                 // tiled row: tile x/8, line x%8
-                    const uint32_t tile = x >> 3, dgrp = tile >> 2, jt = tile & 3;
-                    const uint32_t d = dgrp * 8u + (x & 7u);
-                    uint4 b = *reinterpret_cast<const uint4 *>(vs + 16u * x);
-                    if ((int)(16 * jt + 16) > valid) {
-                        uint32_t wv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            if ((int)(16 * jt) + k >= valid) wv[k >> 2] &= ~(0xFFu << (8 * (k & 3)));
-                        b = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    }
-                    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-                    uint32_t hv[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        hv[2 * k] = e4m3x2_to_f16x2(bw[k] & 0xFFFFu);
-                        hv[2 * k + 1] = e4m3x2_to_f16x2(bw[k] >> 16);
-                    }
-                    *reinterpret_cast<uint4 *>(vb + f16_core_offset(d, 16u * jt)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                    *reinterpret_cast<uint4 *>(vb + f16_core_offset(d, 16u * jt + 8u)) =
-                        make_uint4(hv[4], hv[5], hv[6], hv[7]);
+                for (int c = 0; c < 4; ++c) {                  // tokens 16c .. 16c+15
+                    const uint32_t off = (((uint32_t)r >> 3) * 4u + (uint32_t)c) * 128u + ((uint32_t)r & 7u) * 16u;
+                    *reinterpret_cast<uint4 *>(pb + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(pb + ATT_PB_BYTES + off) =
+                        make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
                 }
             }
             fence_proxy_async_smem();
@@ -630,15 +617,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     }
                 }
             }
-            if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M, l));
+            if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M - ATT_PSHIFT, l));
         } else if (n_pages == 0 && row_ok && g == 0) {
             __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(0.f, 0.f));
         }
 
         if (p.fuse) {
             // ---- fused combine: publish, meet the head's other splits, then
-            //      merge rows r0 .. r1-1 of this KV head (row = w*T + node)
-            __threadfence();
+            //      merge rows r0 .. r1-1 of this KV head (row = w*T + node).
+            //      The barrier orders every thread's partial stores before the
+            //      one release-add (a release is cumulative over what its thread
+            //      has synchronised with); likewise the acquiring poll, then the
+            //      barrier, before any thread reads the other splits' results.
             named_bar_sync(1, 256);
             if (threadIdx.x == 64) {
                 red_release_gpu_add(p.cnt + ch, 1);
@@ -647,48 +637,103 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 xch[0] = (all_in && !*s_abort) ? 1.f : 0.f;        // one decision for every thread
             }
             named_bar_sync(1, 256);
-            __threadfence();
             const bool merge = xch[0] != 0.f;
             const int nr = p.nheads * T;
             const int r0 = (int)((int64_t)split * nr / p.S), r1 = (int)((int64_t)(split + 1) * nr / p.S);
-            const int d = gt;                                      // dimension of this thread
+            const int nrow = r1 - r0;
+            // warps = R row slots x Q split slices: rows go in parallel when the
+            // CTA has many (causal mode), splits when it has few (tree mode)
+            const int sw = (int)warp - 2;                          // softmax warp 0..7
+            const int R = nrow < 8 ? (nrow > 0 ? nrow : 1) : 8, Q = 8 / R;
+            const int rs = sw % R, qs = sw / R;
+            const bool worker = qs < Q;
+            float *accs = reinterpret_cast<float *>(smem + ATT_OFF_P);   // [8 warps][128], the idle P buffer
             float *crow = reinterpret_cast<float *>(smem + ATT_OFF_C) + 128 * g;
             const float vsc = p.v_scale[h];
-            for (int row = r0 + g; merge && row < r1; row += 2) {
-                const int ww = row / T, nd = row % T;
-                const int64_t base = (int64_t)ch * p.S * rows_cta + ww * p.rows_w + nd;   // + s * rows_cta
-                const int64_t sstride = rows_cta;
-                float M = -INFINITY;
-                for (int sp = 0; sp < p.S; ++sp) {
-                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * (base + sp * sstride)));
-                    if (ml.y > 0.f) M = fmaxf(M, ml.x);
-                }
-                float num = 0.f, den = 0.f;
-                for (int sp = 0; sp < p.S; ++sp) {
-                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * (base + sp * sstride)));
-                    if (ml.y > 0.f) {
-                        const float ws = ml.y * fast_exp2(ml.x - M);
-                        num += ws * __ldcg(p.part_o + (base + sp * sstride) * ATT_D + d);
-                        den += ws;
-                    }
-                }
-                const float o = den > 0.f ? num / den * vsc : 0.f;
-                const __nv_bfloat16 obf = __float2bfloat16_rn(o);
-                const int hq2 = hq0 + ww;
-                p.out[((int64_t)nd * p.Hq + hq2) * ATT_D + d] = obf;
-                if (p.act) {
-                    crow[d] = __bfloat162float(obf);
-                    named_bar_sync(2 + g, 128);
-                    if (d < ATT_D / 16) {
-                        float v[16];
+            for (int k0 = 0; merge && k0 < nrow; k0 += R) {
+                const int j = k0 + rs;                             // this warp's row of the round
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (worker && j < nrow) {
+                    const int row = r0 + j, ww = row / T, nd = row % T;
+                    const int64_t base = (int64_t)ch * p.S * rows_cta + ww * p.rows_w + nd;   // + s * rows_cta
+                    // one round trip: the (m, l) of every split (lane holds splits
+                    // lane, lane+32, ...) and this warp's partial rows (splits qs,
+                    // qs+Q, ..., up to 24 per lane) are requested together
+                    float2 ml[5];
+                    float4 v[24];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) v[k] = crow[16 * d + k];
-                        uint2 pk;
-                        const uint32_t sc = quant_block16(v, *p.g_act, pk);
-                        store_prepared(p.act, nd, (int64_t)hq2 * (ATT_D / 16) + d, pk, sc);
+                    for (int i = 0; i < 5; ++i) {
+                        const int sp = (int)lane + 32 * i;
+                        ml[i] = sp < p.S ? __ldcg(reinterpret_cast<const float2 *>(p.part_ml + 2 * (base + sp * rows_cta)))
+                                         : make_float2(0.f, 0.f);
                     }
-                    named_bar_sync(2 + g, 128);
+#pragma unroll
+                    for (int k = 0; k < 24; ++k) {
+                        const int sp = qs + k * Q;
+                        v[k] = sp < p.S ? __ldcg(reinterpret_cast<const float4 *>(p.part_o + (base + sp * rows_cta) * ATT_D) + lane)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    float mloc = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 5; ++i)
+                        if (ml[i].y > 0.f) mloc = fmaxf(mloc, ml[i].x);
+                    const float M = warp_max(mloc);
+                    float wv[5], dloc = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 5; ++i) {
+                        wv[i] = ml[i].y > 0.f ? ml[i].y * fast_exp2(ml[i].x - M) : 0.f;
+                        dloc += wv[i];
+                    }
+                    const float den = warp_sum(dloc);
+                    const float inv = den > 0.f ? 1.f / den : 0.f;
+                    auto weight = [&](int sp) {                        // sp warp-uniform
+                        float wsel = wv[0];
+#pragma unroll
+                        for (int i = 1; i < 5; ++i)
+                            if ((sp >> 5) == i) wsel = wv[i];
+                        return __shfl_sync(0xFFFFFFFFu, wsel, sp & 31) * inv;
+                    };
+#pragma unroll
+                    for (int k = 0; k < 24; ++k) {
+                        const int sp = qs + k * Q;
+                        if (sp < p.S) {
+                            const float w = weight(sp);
+                            acc.x += w * v[k].x; acc.y += w * v[k].y; acc.z += w * v[k].z; acc.w += w * v[k].w;
+                        }
+                    }
+                    // splits beyond the first 24 of this warp (many splits, few rows)
+                    for (int sp = qs + 24 * Q; sp < p.S; sp += Q) {
+                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(p.part_o + (base + sp * rows_cta) * ATT_D) + lane);
+                        const float w = weight(sp);
+                        acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+                    }
                 }
+                reinterpret_cast<float4 *>(accs + 128 * sw)[lane] = acc;
+                named_bar_sync(1, 256);
+                // outputs of the round's rows: group g takes row slots g, g+2, ...
+                for (int rr = g; rr < R && k0 + rr < nrow; rr += 2) {
+                    const int row = r0 + k0 + rr, ww = row / T, nd = row % T;
+                    const int d = gt;
+                    float o = 0.f;
+                    for (int qq = 0; qq < Q; ++qq) o += accs[128 * (qq * R + rr) + d];
+                    const __nv_bfloat16 obf = __float2bfloat16_rn(o * vsc);
+                    const int hq2 = hq0 + ww;
+                    p.out[((int64_t)nd * p.Hq + hq2) * ATT_D + d] = obf;
+                    if (p.act) {
+                        crow[d] = __bfloat162float(obf);
+                        named_bar_sync(2 + g, 128);
+                        if (d < ATT_D / 16) {
+                            float v[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) v[k] = crow[16 * d + k];
+                            uint2 pk;
+                            const uint32_t sc = quant_block16(v, *p.g_act, pk);
+                            store_prepared(p.act, nd, (int64_t)hq2 * (ATT_D / 16) + d, pk, sc);
+                        }
+                        named_bar_sync(2 + g, 128);
+                    }
+                }
+                named_bar_sync(1, 256);                            // accs reused by the next round
             }
             // the last CTA of the head through here resets its counter for the next call
             named_bar_sync(1, 256);

@@ -128,12 +128,16 @@ __device__ __forceinline__ bool poll_counter(const int *p, int want, uint32_t si
 }
 
 // Wait (bounded) until *p >= want; returns false and records a timeout otherwise.
+// Polls with a short sleep in between: many CTAs may wait on one counter, and
+// back-to-back polls of one L2 line slow the memory traffic of the CTAs that
+// are still working.
 __device__ __forceinline__ bool poll_counter_ge(const int *p, int want, uint32_t site, volatile int *abort)
 {
     if (ld_acquire_gpu(p) >= want) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
-        for (int i = 0; i < 8; ++i)
+        __nanosleep(64);
+        for (int i = 0; i < 2; ++i)
             if (ld_acquire_gpu(p) >= want) return true;
         if (abort && *abort) return false;
         if (globaltimer() - t0 > g_timeout_ns) {
@@ -485,31 +489,40 @@ __host__ __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t b)
 // Weight units: for tile t, chunk c:
 //   atom a, row r, byte b   <- codes[t*128 + r][c*256 + a*128 + b]
 //   scale image j, line l, byte 4*cc + kb <- scales[t*128 + l + 32*cc][c*32 + 4*j + kb]
-// zero outside the matrix.
-__global__ void prepare_weight_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
-                                      int64_t N, int64_t K, int64_t KC, uint8_t *__restrict__ out, int64_t total)
+// zero outside the matrix.  One CTA per unit; each thread writes whole
+// 16-byte chunks: the 128-byte swizzle permutes whole 16-byte chunks of a
+// code row, so a code chunk is one 16-byte source load, and a scale chunk
+// gathers four 4-byte pieces (rows l, l+32, l+64, l+96).  Needs codes
+// 16-byte and scales 4-byte aligned (checked by the caller).
+__global__ void __launch_bounds__(256) prepare_weight_kernel(const uint8_t *__restrict__ codes,
+                                                             const uint8_t *__restrict__ scales, int64_t N, int64_t K,
+                                                             int64_t KC, uint8_t *__restrict__ out)
 {
     pdl_wait();
     pdl_launch_dependents();
+    const int64_t unit = blockIdx.x;
+    const int64_t t = unit / KC, c = unit % KC;
     const int64_t kbytes = K / 2, kb = K / 16;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t unit = i / LIN_W_UNIT, o = i % LIN_W_UNIT;
-        const int64_t t = unit / KC, cidx = unit % KC;
-        uint8_t v = 0;
-        if (o < 2 * LIN_W_ATOM) {
-            const uint32_t a = (uint32_t)(o / LIN_W_ATOM), o2 = (uint32_t)(o % LIN_W_ATOM);
-            const uint32_t r = o2 / 128u, pos = o2 % 128u;
-            const uint32_t b = (((pos >> 4) ^ (r & 7u)) << 4) | (pos & 15u);     // inverse of swz128
-            const int64_t row = t * 128 + r, col = cidx * 256 + a * 128 + b;
-            if (row < N && col < kbytes) v = codes[row * kbytes + col];
+    uint8_t *u = out + unit * (int64_t)LIN_W_UNIT;
+    for (int k = threadIdx.x; k < (int)(LIN_W_UNIT / 16); k += blockDim.x) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (k < (int)(2 * LIN_W_ATOM / 16)) {
+            const int a = k >> 10, r = (k >> 3) & 127, j = k & 7;       // atom, row, stored chunk
+            const int64_t row = t * 128 + r;
+            const int64_t col = c * 256 + a * 128 + (int64_t)((j ^ (r & 7)) << 4);
+            if (row < N && col < kbytes) v = *reinterpret_cast<const uint4 *>(codes + row * kbytes + col);
         } else {
-            const uint32_t o2 = (uint32_t)(o - 2 * LIN_W_ATOM);
-            const uint32_t j = o2 / 512u, l = (o2 % 512u) / 16u, cc = (o2 % 16u) / 4u, kbi = o2 % 4u;
-            const int64_t row = t * 128 + l + 32 * cc, blk = cidx * 32 + 4 * j + kbi;
-            if (row < N && blk < kb) v = scales[row * kb + blk];
+            const int k2 = k - (int)(2 * LIN_W_ATOM / 16), jimg = k2 >> 5, l = k2 & 31;
+            const int64_t blk = c * 32 + 4 * jimg;
+            uint32_t w[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int64_t row = t * 128 + l + 32 * cc;
+                w[cc] = (row < N && blk < kb) ? *reinterpret_cast<const uint32_t *>(scales + row * kb + blk) : 0u;
+            }
+            v = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        out[i] = v;
+        *reinterpret_cast<uint4 *>(u + 16 * (int64_t)k) = v;
     }
 }
 

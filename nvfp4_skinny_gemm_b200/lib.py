@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libnvfp4sk.so")
 HEADER = os.path.join(ROOT, "include", "nvfp4sk.h")
 
 BF16, FP32 = 0, 1
-OPT_PDL, OPT_TIMEOUT_NS, OPT_ATTN_SPLITS, OPT_LINEAR_CTAS = 0, 1, 2, 3
+OPT_PDL, OPT_TIMEOUT_NS, OPT_ATTN_SPLITS, OPT_LINEAR_CTAS, OPT_ATTN_FUSED_COMBINE = 0, 1, 2, 3, 4
 STATUS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED_SHAPE", -3: "MISALIGNED", -4: "WORKSPACE",
           -5: "CUDA", -6: "TIMEOUT", -7: "OUT_OF_RANGE", -8: "DEVICE"}
 

@@ -91,6 +91,8 @@ def test_host_checks_reject_bad_arguments_before_the_device():
         # nvfp4_prepare_weight(codes, scales, N, K, prepared, stream)
         (E_SHAPE, "nvfp4_prepare_weight", A, A, 128, 100, A, None),
         (E_ALIGN, "nvfp4_prepare_weight", A, A, 128, 128, MIS, None),
+        (E_ALIGN, "nvfp4_prepare_weight", MIS, A, 128, 128, A, None),
+        (E_ALIGN, "nvfp4_prepare_weight", A, A + 2, 128, 128, A, None),
         # nvfp4_linear(a, g_a, M, w, g_w, N, K, residual, y, ldy, ws, ws_bytes, stream)
         (E_ARG, "nvfp4_linear", None, A, 16, A, A, 128, 128, None, A, 128, A, 1 << 20, None),
         (E_SHAPE, "nvfp4_linear", A, A, 17, A, A, 128, 128, None, A, 128, A, 1 << 20, None),

@@ -58,7 +58,16 @@ def test_attention_small(oracle, T, Hq, Hkv, L, kind):
     assert np.all(err <= bound), f"max err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
 
 
-def test_attention_full_context(oracle):
+@pytest.fixture(params=[0, 1], ids=["separate_combine", "fused_combine"])
+def combine_mode(request):
+    """Both ways the split results are merged: a second launch (default), and
+    the CTAs of a head merging them themselves."""
+    nv.set_option(nv.OPT_ATTN_FUSED_COMBINE, request.param)
+    yield request.param
+    nv.set_option(nv.OPT_ATTN_FUSED_COMBINE, 0)
+
+
+def test_attention_full_context(oracle, combine_mode):
     """The 23,552-token workload: 16-node tree, 24 query / 4 KV heads, FP8 pages."""
     cuda()
     L = inputs.CTX_MAX
@@ -163,7 +172,7 @@ def test_bad_page_id_and_parent_are_flagged():
     assert nv.device_status()[0] == 0
 
 
-def test_fused_nvfp4_output_matches_separate_quantisation():
+def test_fused_nvfp4_output_matches_separate_quantisation(combine_mode):
     """With a static tensor scale the combine launch also writes the NVFP4
     prepared activation of its bf16 output: byte-identical to quantising the
     bf16 output in a separate call (same recipe, same values)."""
@@ -182,7 +191,7 @@ def test_fused_nvfp4_output_matches_separate_quantisation():
     assert nv.device_status()[0] == 0
 
 
-def test_fused_combine_leaves_counters_zero_and_is_repeatable():
+def test_fused_combine_leaves_counters_zero_and_is_repeatable(combine_mode):
     """The fused combine's per-head arrival counters sit at the start of the
     workspace: after each call they read zero again, and a second call on the
     same workspace gives bit-identical outputs."""
@@ -212,7 +221,7 @@ def _run_causal(q, cache, ctx, T, rows=None, dev=None):
 
 @pytest.mark.parametrize("T,Hq,Hkv,L", [(1, 24, 4, 0), (17, 24, 4, 300), (100, 8, 2, 1000), (128, 24, 4, 37),
                                         (128, 6, 1, 4096), (64, 24, 4, 0)])
-def test_causal_attention(oracle, T, Hq, Hkv, L):
+def test_causal_attention(oracle, T, Hq, Hkv, L, combine_mode):
     """Causal attention of T new tokens over the context (the suffix prefill's
     attention) against the oracle's attention with a chain parent array (a
     chain tree is causal attention over context + chain)."""
