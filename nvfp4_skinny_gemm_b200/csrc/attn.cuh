@@ -32,8 +32,8 @@
 // accumulators in tensor memory and its own running max, so that two pages
 // are in the exponent stage at once; their results are merged in the
 // epilogue.
-// Warp roles: 0 producer (lane s feeds stage s of a 10-stage ring: TMA K page
-// + bulk V page; context pages are requested before the wait on the
+// Warp roles: 0 producer (one thread feeds a 10-stage ring: TMA K page + bulk
+// V page; context pages are requested before the wait on the
 // preceding kernel), 1 TMEM allocation + QK issue (one thread), 10 PV issue
 // (one thread), 2-5 and 6-9 softmax.  The two issuers run independently, so
 // a group's next scores never wait behind the other group's product.
@@ -262,25 +262,37 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        // lane st feeds stage st (pages st, st + 8, ...): the copies of
-        // different stages are issued by different threads, which keeps
-        // several page loads in flight per SM.  Context pages of the first
-        // round are requested before the wait on the preceding kernel (the
-        // context and the page table are not written by it; the tree slots,
-        // which the K/V append of the same step writes, are loaded after it).
-        if (lane < ATT_STAGES) {
-            const int st = (int)lane;
-            int last = -1;
-            bool waited = false;
-            for (int i = st; i < n_pages; i += ATT_STAGES) {
-                if (!waited && (i >= ATT_STAGES || (int64_t)(pg0 + i + 1) * ATT_P > p.ctx_len)) {
-                    pdl_wait();
-                    waited = true;
-                }
-                if (i >= ATT_STAGES &&
-                    !mbar_wait(&kv_empty[st], (uint32_t)(((i / ATT_STAGES) - 1) & 1), 301, s_abort))
-                    break;
-                const int32_t pg = p.page_table[pg0 + i];
+        // One converged warp; lane 0 waits and issues, in page order (stages
+        // free in that order).  (Measured: one issuing thread keeps as many
+        // bytes in flight as twenty; lanes that each wait on their own stage
+        // diverge, and a suspended wait of one lane holds back the refills
+        // of the others by microseconds.)  Page ids are read 32 at a time,
+        // the next block's while the current one is issued.  Context pages of
+        // the first round are requested before the wait on the preceding
+        // kernel (the context and the page table are not written by it; the
+        // tree slots, which the K/V append of the same step writes, are
+        // loaded after it).
+        auto pid_at = [&](int i) -> int32_t { return i < n_pages ? p.page_table[pg0 + i] : -1; };
+        int32_t ids_cur = pid_at((int)lane), ids_nxt = pid_at(32 + (int)lane);
+        int last = -1;
+        bool waited = false;
+        for (int i = 0; i < n_pages; ++i) {
+            if (i > 0 && (i & 31) == 0) {
+                ids_cur = ids_nxt;
+                ids_nxt = pid_at(i + 32 + (int)lane);
+            }
+            const int st = i % ATT_STAGES;
+            if (!waited && (i >= ATT_STAGES || (int64_t)(pg0 + i + 1) * ATT_P > p.ctx_len)) {
+                pdl_wait();
+                waited = true;
+            }
+            if (i >= ATT_STAGES) {
+                bool e_ok = true;
+                if (lane == 0) e_ok = mbar_wait(&kv_empty[st], (uint32_t)(((i / ATT_STAGES) - 1) & 1), 301, s_abort);
+                if (!__shfl_sync(0xFFFFFFFFu, e_ok ? 1 : 0, 0)) break;
+            }
+            const int32_t pg = __shfl_sync(0xFFFFFFFFu, ids_cur, i & 31);
+            if (lane == 0) {
                 uint8_t *dst = smem + st * ATT_STAGE_BYTES;
                 const bool ok = pg >= 0 && pg < p.n_pool_pages;
                 s_page_ok[st] = ok ? 1 : 0;
@@ -293,13 +305,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     report_error(ERRBIT_RANGE, 302);
                     mbar_arrive(&kv_full[st]);        // page skipped: its scores are masked out
                 }
-                last = i;
             }
-            if (!waited) pdl_wait();
-            // on abort, let this stage's last copy land before the CTA exits
-            if (*s_abort && last >= 0) mbar_wait_drain(&kv_full[st], (uint32_t)((last / ATT_STAGES) & 1), 303);
-        } else {
-            pdl_wait();
+            last = i;
+        }
+        if (!waited) pdl_wait();
+        // on abort, let the copies still in flight land before the CTA exits
+        if (lane == 0 && *s_abort) {
+            for (int i = last >= ATT_STAGES ? last - ATT_STAGES + 1 : 0; i <= last; ++i)
+                mbar_wait_drain(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 303);
         }
         __syncwarp();          // reconverge before the CTA-wide barrier below
     } else if (warp == 1) {
@@ -444,20 +457,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             tmem_st_x16(row_t + ATT_TM_Q + 16u * (uint32_t)g, hw);
             tmem_st_x16(row_t + ATT_TM_Q + 32u + 16u * (uint32_t)g, lw);
             tmem_wait_st();
-            // ancestors of this node: walk the parent array held one entry per lane
+            // ancestors (and self) of every node by pointer doubling: lane t holds
+            // node t's set and a jump pointer; each round joins the set of the
+            // node the pointer names and doubles the pointer's reach, so
+            // log2(ATT_T) rounds cover any chain of ATT_T nodes
             if (!p.causal) {
-                int a = has_q ? node : -1;
-                bool bad = false;
-#pragma unroll 1
-                for (int it = 0; it < ATT_T; ++it) {
-                    const bool act = a >= 0 && !bad;
-                    if (act && a >= T) bad = true;             // malformed tree: parent id out of range
-                    const bool take = act && !bad;
-                    if (take) anc |= 1u << a;
-                    const int nxt = __shfl_sync(0xFFFFFFFFu, par_l, take ? a : 0);
-                    a = take ? nxt : -1;
+                int jmp = par_l;
+                const bool bad = (int)lane < T && jmp >= T;  // malformed tree: parent id out of range
+                if (bad || jmp < 0) jmp = -1;
+                uint32_t set = (int)lane < T ? 1u << lane : 0u;
+#pragma unroll
+                for (int k = 0; (1 << k) < ATT_T; ++k) {
+                    const int src = jmp >= 0 ? jmp : (int)lane;
+                    const uint32_t set2 = __shfl_sync(0xFFFFFFFFu, set, src);
+                    const int jmp2 = __shfl_sync(0xFFFFFFFFu, jmp, src);
+                    if (jmp >= 0) {
+                        set |= set2;
+                        jmp = jmp2;
+                    }
                 }
-                if (bad) report_error(ERRBIT_RANGE, 305);
+                anc = __shfl_sync(0xFFFFFFFFu, set, has_q ? node : 0);
+                if (!has_q) anc = 0;
+                if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report_error(ERRBIT_RANGE, 305);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -495,12 +516,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             bool waited = false;
             if (!pad_warp) {
                 if (pos0 + ATT_P > L) {
-                    const int t0 = (int)(pos0 - L);            // new-position slot of column 0 (> -64)
+                    // column j holds new-position slot t0 + j (negative: context);
+                    // bit j of vis = column j visible to this row
+                    const int t0 = (int)(pos0 - L);            // > -64
+                    uint64_t vis;
+                    if (p.causal) {                            // slots 0 .. node (node < T)
+                        const int lim = min(node, T - 1) - t0;
+                        vis = lim >= 63 ? ~0ull : lim < 0 ? 0ull : ((2ull << lim) - 1ull);
+                    } else {                                   // context, then the ancestor slots
+                        const uint64_t ctx = t0 >= 0 ? 0ull : ((1ull << (-t0)) - 1ull);
+                        vis = ctx | (t0 >= 0 ? ((uint64_t)anc >> t0) : ((uint64_t)anc << (-t0)));
+                    }
+                    const uint32_t v_lo = (uint32_t)vis, v_hi = (uint32_t)(vis >> 32);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int tj = t0 + j;                 // negative: context position
-                        const bool vis = tj < 0 || (tj < T && (p.causal ? tj <= node : ((anc >> (tj & 31)) & 1u) != 0));
-                        if (!vis) s[j] = 0xFF800000u;         // -inf
+                    for (int j = 0; j < 32; ++j) {
+                        if (!((v_lo >> j) & 1u)) s[j] = 0xFF800000u;          // -inf
+                        if (!((v_hi >> j) & 1u)) s[32 + j] = 0xFF800000u;
                     }
                 }
                 // row max as a tree (8 independent chains, then 3 levels): a
@@ -551,8 +582,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 // included); zero their V (this thread: dimension r) so 0 * V stays 0
                 const bool k_ok = mbar_wait(&kv_full[i % ATT_STAGES], (uint32_t)((i / ATT_STAGES) & 1), 324, s_abort);
                 if (!__all_sync(0xFFFFFFFFu, k_ok)) { ok = false; break; }
-                uint8_t *vs = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES;
-                for (int t = (int)(L + T - pos0); t < ATT_P; ++t) vs[v_offset((uint32_t)r, (uint32_t)t)] = 0;
+                // slots tz .. 63 of dimension r: 16 contiguous bytes per 16-slot chunk
+                uint8_t *vd = smem + (i % ATT_STAGES) * ATT_STAGE_BYTES + ATT_K_BYTES + v_offset((uint32_t)r, 0);
+                const int tz = (int)(L + T - pos0);           // 1 .. 63: the last page holds position L+T-1
+                int c = tz >> 4;
+                if (tz & 15) {
+                    for (int t = tz & 15; t < 16; ++t) vd[c * 128 + t] = 0;
+                    ++c;
+                }
+                for (; c < ATT_P / 16; ++c) *reinterpret_cast<uint4 *>(vd + c * 128) = make_uint4(0, 0, 0, 0);
             }
             // the P buffer of this group's previous page must have been consumed
             if (!waited && i >= 2) {

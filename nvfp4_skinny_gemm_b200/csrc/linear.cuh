@@ -443,14 +443,21 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     if (lane == 0) p.counters[t * 4 + q] = 0;
                 }
                 if (n < p.N) {
+                    // y may alias the residual (y = h + linear(h)): every residual
+                    // load goes out before the first store
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        if (m < M) {
-                            float o = __fmul_rn(acc[m], gs);
-                            if (p.residual) o = __fadd_rn(o, __bfloat162float(p.residual[m * p.ldy + n]));
-                            p.y[m * p.ldy + n] = __float2bfloat16_rn(o);
-                        }
+                    for (int m = 0; m < 16; ++m) acc[m] = __fmul_rn(acc[m], gs);
+                    if (p.residual) {
+                        __nv_bfloat16 res[16];
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            res[m] = m < M ? p.residual[m * p.ldy + n] : __float2bfloat16_rn(0.f);
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) acc[m] = __fadd_rn(acc[m], __bfloat162float(res[m]));
                     }
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        if (m < M) p.y[m * p.ldy + n] = __float2bfloat16_rn(acc[m]);
                 }
             } else {
                 // contributor: publish the partial sum, then one release add on the

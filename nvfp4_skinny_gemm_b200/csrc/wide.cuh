@@ -8,10 +8,12 @@
 // (nvfp4_prepare_weight applied to the S x K activation).
 //
 // Tile = 128 weight rows x 256 tokens, the whole K range in one CTA (no
-// split-K: a prefill has hundreds of such tiles).  Per 256-K stage: half a
-// weight unit (16 KB codes + 2 KB scales) and half a unit of each of the two
-// 128-token activation tiles (2 x 18 KB), 54 KB in all, four stages.  Per
-// 64-K step two tcgen05.mma.kind::mxf4nvf4.block_scale.block16 with
+// split-K: a prefill has hundreds of such tiles).  Per 512-K stage: one
+// weight unit and the units of the two 128-token activation tiles, three
+// 36 KB bulk copies (108 KB), two stages.  (Measured: shared memory fills
+// from L2 at ~150 GB/s per SM with few large copies and ~85 GB/s with six
+// copies of 16 KB and 2 KB per stage; the products of a stage need ~0.5 us.)
+// Per 64-K step two tcgen05.mma.kind::mxf4nvf4.block_scale.block16 with
 // M = 128 weight rows, N = 128 tokens each, into two fp32 accumulators of
 // 128 columns in tensor memory.  The scale factors go to tensor memory with
 // tcgen05.st from the epilogue warps (one warp per TMEM sub-partition), which
@@ -29,20 +31,18 @@
 
 namespace nvfp4sk {
 
-constexpr int WD_STAGES = 4;
+constexpr int WD_STAGES = 2;
 constexpr int WD_THREADS = 192;
-constexpr uint32_t WD_HALF_CODES = LIN_W_ATOM;                     // 16 KB: 128 rows x 256 K
-constexpr uint32_t WD_HALF_SF = 4 * LIN_SF_IMG;                    // 2 KB: four 64-K scale images
-constexpr uint32_t WD_HALF = WD_HALF_CODES + WD_HALF_SF;           // 18 KB per 128-row tile and 256 K
-constexpr uint32_t WD_STAGE_BYTES = 3 * WD_HALF;                   // weights + two token tiles: 54 KB
+constexpr uint32_t WD_STAGE_BYTES = 3 * LIN_W_UNIT;                // weights + two token tiles: 108 KB
 constexpr uint32_t WD_OFF_BAR = WD_STAGES * WD_STAGE_BYTES;
 constexpr uint32_t WD_SMEM_BYTES = WD_OFF_BAR + 256 + 1024;
 constexpr uint32_t WD_TMEM_COLS = 512;
 // TMEM columns: accumulators of token tiles 0 and 1 at 0 and 128; per stage s
-// the weight scales (4 steps x 4 columns) at 256 + 16 s and the two token
-// tiles' scales at 320 + 32 s (+16 for the second).
+// the weight scales (8 steps x 4 columns) at 256 + 32 s and the two token
+// tiles' scales at 320 + 64 s (+32 for the second).
 constexpr uint32_t WD_TM_ACC = 0, WD_TM_SFA = 256, WD_TM_SFB = 320;
-static_assert(WD_TM_SFB + 32 * WD_STAGES <= WD_TMEM_COLS, "tensor memory budget");
+static_assert(WD_TM_SFA + 32 * WD_STAGES <= WD_TM_SFB && WD_TM_SFB + 64 * WD_STAGES <= WD_TMEM_COLS,
+              "tensor memory budget");
 static_assert(WD_STAGE_BYTES % 1024 == 0, "swizzled code atoms need 1024-byte alignment");
 static_assert(WD_SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const uint32_t warp = warp_id(), lane = lane_id();
-    const int KH = 2 * p.KC;                       // 256-K steps per tile
+    const int KH = p.KC;                           // 512-K steps per tile
     const int n_st2 = (p.ST + 1) / 2;              // 256-token tiles
     // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
     const int my_tiles = p.n_tiles > (int)blockIdx.x ? (p.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -119,18 +119,13 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
                 int tw, ts0;
                 bool two;
                 tile_of(i / KH, tw, ts0, two);
-                const int kh = (int)(i % KH), c = kh >> 1, hf = kh & 1;
+                const int c = (int)(i % KH);
                 uint8_t *dst = smem + s * WD_STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], (two ? 3u : 2u) * WD_HALF);
-                const uint8_t *wu = p.w + ((int64_t)tw * p.KC + c) * LIN_W_UNIT;
-                bulk_load_hint(dst, wu + hf * LIN_W_ATOM, WD_HALF_CODES, &full[s], pol_w);
-                bulk_load_hint(dst + WD_HALF_CODES, wu + 2 * LIN_W_ATOM + hf * WD_HALF_SF, WD_HALF_SF, &full[s], pol_w);
-                for (int tt = 0; tt < (two ? 2 : 1); ++tt) {
-                    const uint8_t *au = p.a + ((int64_t)(ts0 + tt) * p.KC + c) * LIN_W_UNIT;
-                    uint8_t *ad = dst + (1 + tt) * WD_HALF;
-                    bulk_load_hint(ad, au + hf * LIN_W_ATOM, WD_HALF_CODES, &full[s], pol_a);
-                    bulk_load_hint(ad + WD_HALF_CODES, au + 2 * LIN_W_ATOM + hf * WD_HALF_SF, WD_HALF_SF, &full[s], pol_a);
-                }
+                mbar_arrive_expect_tx(&full[s], (two ? 3u : 2u) * LIN_W_UNIT);
+                bulk_load_hint(dst, p.w + ((int64_t)tw * p.KC + c) * LIN_W_UNIT, LIN_W_UNIT, &full[s], pol_w);
+                for (int tt = 0; tt < (two ? 2 : 1); ++tt)
+                    bulk_load_hint(dst + (1 + tt) * LIN_W_UNIT, p.a + ((int64_t)(ts0 + tt) * p.KC + c) * LIN_W_UNIT,
+                                   LIN_W_UNIT, &full[s], pol_a);
             };
             pdl_wait();
             int64_t issued = 0;
@@ -170,17 +165,18 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * WD_STAGE_BYTES);
-                    const uint32_t sfa_t = tmem_base + WD_TM_SFA + 16 * (uint32_t)s;
-                    const uint32_t sfb_t = tmem_base + WD_TM_SFB + 32 * (uint32_t)s;
+                    const uint32_t sfa_t = tmem_base + WD_TM_SFA + 32 * (uint32_t)s;
+                    const uint32_t sfb_t = tmem_base + WD_TM_SFB + 64 * (uint32_t)s;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint64_t adesc = smem_desc(st + 32u * j, 16, 1024, SWZ_128B);
+                    for (int j = 0; j < LIN_KSTEPS; ++j) {
+                        const uint32_t ko = (uint32_t)(j >> 2) * LIN_W_ATOM + 32u * (uint32_t)(j & 3);
+                        const uint64_t adesc = smem_desc(st + ko, 16, 1024, SWZ_128B);
 #pragma unroll
                         for (int tt = 0; tt < 2; ++tt) {
                             if (tt == 1 && !two) break;
-                            const uint64_t bdesc = smem_desc(st + (1 + tt) * WD_HALF + 32u * j, 16, 1024, SWZ_128B);
+                            const uint64_t bdesc = smem_desc(st + (1 + tt) * LIN_W_UNIT + ko, 16, 1024, SWZ_128B);
                             mma_mxf4nvf4(tmem_base + WD_TM_ACC + 128 * tt, adesc, bdesc, idesc, sfa_t + 4 * j,
-                                         sfb_t + 16 * tt + 4 * j, (kh > 0 || j > 0) ? 1u : 0u);
+                                         sfb_t + 32 * tt + 4 * j, (kh > 0 || j > 0) ? 1u : 0u);
                         }
                     }
                     tc_commit(&empty[s]);
@@ -202,8 +198,8 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
         const float gs = __fmul_rn(*p.g_a, *p.g_w);
         int64_t next_sf = 0;
         bool sf_ok = true;
-        // the scale images of step i (four 64-K images per 128-row tile, line l =
-        // rows l, l+32, l+64, l+96) to every TMEM sub-partition, then one arrive
+        // the scale images of step i (eight 64-K images per 128-row tile, line l
+        // = rows l, l+32, l+64, l+96) to every TMEM sub-partition, then one arrive
         auto stage_scales = [&](int64_t i) -> bool {
             const int s = (int)(i % WD_STAGES);
             const bool landed = mbar_wait(&full[s], (uint32_t)((i / WD_STAGES) & 1), 607, s_abort);
@@ -211,15 +207,15 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
             const uint8_t *st = smem + s * WD_STAGE_BYTES;
 #pragma unroll
             for (int part = 0; part < 3; ++part) {
-                const uint8_t *img = st + part * WD_HALF + WD_HALF_CODES;
-                uint32_t v[16];
+                const uint8_t *img = st + part * LIN_W_UNIT + 2 * LIN_W_ATOM;
+                uint32_t v[32];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < LIN_KSTEPS; ++j) {
                     const uint4 x = *reinterpret_cast<const uint4 *>(img + LIN_SF_IMG * j + 16 * lane);
                     v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
-                const uint32_t col = part == 0 ? WD_TM_SFA + 16 * (uint32_t)s : WD_TM_SFB + 32 * (uint32_t)s + 16 * (part - 1);
-                tmem_st_x16(lane_base + col, v);
+                const uint32_t col = part == 0 ? WD_TM_SFA + 32 * (uint32_t)s : WD_TM_SFB + 64 * (uint32_t)s + 32 * (part - 1);
+                tmem_st_x32(lane_base + col, v);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -248,15 +244,24 @@ __global__ void __launch_bounds__(WD_THREADS, 1) nvfp4_linear_wide_kernel(const 
                     tmem_wait_ld();
                     const int64_t s0 = (int64_t)(ts0 + tt) * 128 + cb;
                     if (n < p.N) {
-#pragma unroll 4
-                        for (int m = 0; m < 32; ++m) {
-                            const int64_t s = s0 + m;
-                            if (s < p.S) {
-                                float o = __fmul_rn(__uint_as_float(r[m]), gs);
-                                if (p.residual) o = __fadd_rn(o, __bfloat162float(p.residual[s * p.ldy + n]));
-                                p.y[s * p.ldy + n] = __float2bfloat16_rn(o);
-                            }
+                        // y may alias the residual (y = h + linear(h)): all 32
+                        // residual loads go out before the first store
+                        if (p.residual) {
+                            __nv_bfloat16 res[32];
+#pragma unroll
+                            for (int m = 0; m < 32; ++m)
+                                res[m] = s0 + m < p.S ? p.residual[(s0 + m) * p.ldy + n] : __float2bfloat16_rn(0.f);
+#pragma unroll
+                            for (int m = 0; m < 32; ++m)
+                                r[m] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(r[m]), gs),
+                                                                 __bfloat162float(res[m])));
+                        } else {
+#pragma unroll
+                            for (int m = 0; m < 32; ++m) r[m] = __float_as_uint(__fmul_rn(__uint_as_float(r[m]), gs));
                         }
+#pragma unroll
+                        for (int m = 0; m < 32; ++m)
+                            if (s0 + m < p.S) p.y[(s0 + m) * p.ldy + n] = __float2bfloat16_rn(__uint_as_float(r[m]));
                     }
                 }
             }
