@@ -371,10 +371,12 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             float part[LIN_PF][16];
             bool ok = true;
             if (owner) {
+                // lane 0's acquire, then the warp barrier (which orders memory
+                // among the warp's threads), before any lane reads a partial sum
                 if (lane == 0) ok = poll_counter(p.counters + t * 4 + q, (int)(last - first), 107, s_abort);
+                __syncwarp();
                 ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                __threadfence();
 #pragma unroll
                 for (int k = 0; k < LIN_PF; ++k) {
                     const int64_t cc = first + 1 + k;
@@ -468,7 +470,9 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 for (int v = 0; v < 4; ++v)
                     __stcg(P + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
-                __threadfence();
+                // the warp barrier orders every lane's stores before lane 0's
+                // release add (a release is cumulative over what its thread has
+                // synchronised with), so no separate fence is needed
                 __syncwarp();
                 if (lane == 0) red_release_gpu_add(p.counters + t * 4 + q, 1);
             }
