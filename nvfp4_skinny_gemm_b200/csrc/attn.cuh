@@ -199,7 +199,8 @@ struct AttnParams {
 };
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-    tree_attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const AttnParams p)
+    tree_attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_o,
+                           const AttnParams p)
 {
     extern __shared__ uint8_t att_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(att_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -641,6 +642,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tmem_ld_x32(row_t + ATT_TM_O0 + col, oa);
                 tmem_ld_x32(row_t + ATT_TM_O1 + col, ob);
                 tmem_wait_ld();
+                // without the fused combine: dims col .. col+31 of the CTA's rows
+                // form box 2g+cc of the tensor store below, staged in the ring
+                // (free after o_done) as 128-byte rows, 16-byte chunk j of row r
+                // at chunk j ^ (r % 8)
+                uint8_t *box = smem + (2u * (uint32_t)g + (uint32_t)cc) * (uint32_t)rows_cta * 128u + (uint32_t)r * 128u;
                 if (row_ok) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
@@ -651,13 +657,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                             const float b = cb > 0.f ? cb * __uint_as_float(ob[j + k]) : 0.f;
                             v[k] = a + b;
                         }
-                        __stcg(reinterpret_cast<float4 *>(dst + col + j), make_float4(v[0], v[1], v[2], v[3]));
+                        if (p.fuse)
+                            __stcg(reinterpret_cast<float4 *>(dst + col + j), make_float4(v[0], v[1], v[2], v[3]));
+                        else
+                            *reinterpret_cast<float4 *>(box + ((((uint32_t)j >> 2) ^ ((uint32_t)r & 7u)) << 4)) =
+                                make_float4(v[0], v[1], v[2], v[3]);
                     }
                 }
             }
             if (row_ok && g == 0) __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(M - ATT_PSHIFT, l));
         } else if (n_pages == 0 && row_ok && g == 0) {
             __stcg(reinterpret_cast<float2 *>(p.part_ml + prow * 2), make_float2(0.f, 0.f));
+        }
+        if (!p.fuse) {
+            // four TMA tensor stores (32 dims x rows_cta rows each) of the staged
+            // split result; the store is complete before the CTA exits
+            fence_proxy_async_smem();
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 64 && n_pages > 0 && !*s_abort) {
+                const int32_t row0 = (int32_t)(((int64_t)ch * p.S + split) * rows_cta);
+#pragma unroll
+                for (int b = 0; b < 4; ++b) tma_store_2d(&tm_o, smem + b * rows_cta * 128, 128 * b, row0);
+                bulk_commit();
+                bulk_wait<0>();
+            }
         }
 
         if (p.fuse) {

@@ -165,6 +165,16 @@ __device__ __forceinline__ void bulk_load_hint(void *dst, const void *src, uint3
         : "memory");
 }
 
+// shared -> global tiled TMA store (tracked by bulk groups); x: innermost
+// coordinate in elements, its byte offset a multiple of 16; never negative
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x, int32_t y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
 // shared -> global bulk store, tracked by bulk groups
 __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes)
 {

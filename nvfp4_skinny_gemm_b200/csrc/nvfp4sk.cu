@@ -263,7 +263,12 @@ int attn_launch(const void *q, int64_t ld_q, int T, int Hq, int Hkv, const uint8
     // fused against 24.6 us with the separate combine launch, so off by default.
     p.fuse = (g_opt_attn_fused && (int64_t)S * heads <= d->sms) ? 1 : 0;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, heads), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, 1, tk, p);
+    // split results: fp32 rows of 512 bytes, one TMA box = 128 bytes (32 dims) x the CTA's rows
+    CUtensorMap to;
+    if (int rc = make_map_u8(&to, p.part_o, ATT_D * 4, (uint64_t)heads * S * nheads * rows_w, ATT_D * 4, 128,
+                             (uint32_t)(nheads * rows_w), CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    cudaError_t e = launch(tree_attn_split_kernel, dim3(S, heads), dim3(ATT_THREADS), ATT_SMEM_BYTES, st, 1, tk, to, p);
     if (e != cudaSuccess) return cuda_fail(e, "tree_attn_split_kernel");
     if (p.fuse) return NVFP4SK_OK;
     return launched(launch(tree_attn_combine_kernel, dim3(T, Hq), dim3(ATT_D), 0, st, 1, p),
