@@ -292,7 +292,7 @@ def linear_launches(model):
 
 
 def attention_launches(model):
-    """The step's attention calls (split with the fused combine, and the static NVFP4
+    """The step's attention calls (split and combine, with the static NVFP4
     output), one per layer over that layer's pools, back to back."""
     from nvfp4_skinny_gemm_b200 import inputs as I
     from nvfp4_skinny_gemm_b200 import lib as nv
@@ -430,8 +430,8 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_step": lin_bytes, "launches": n_lin,
                      "us_per_step_of_linears": round(t_lin * 1e6, 1),
                      "traffic": traffic},
-        "roofline_attn": {"kernel": f"tree_attn_split_kernel with the fused combine ({model.n_layers} calls of "
-                                    f"one step, back to back)",
+        "roofline_attn": {"kernel": f"tree_attn_split_kernel + tree_attn_combine_kernel ({model.n_layers} calls "
+                                    f"of one step, back to back)",
                           "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
                           "frac": round(attn_gbs / peak, 4),
                           "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",

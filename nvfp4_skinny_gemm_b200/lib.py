@@ -151,6 +151,13 @@ def set_option(opt, value):
     _call("nvfp4sk_set_option", opt, int(value))
 
 
+def attn_launches():
+    """Kernel launches per tree_attn / causal_attn call at the library's own
+    split counts: 1 with the fused combine (OPT_ATTN_FUSED_COMBINE on; those
+    split grids always fit on the GPU at once), else 2 (split, then combine)."""
+    return 1 if get_option(OPT_ATTN_FUSED_COMBINE) and get_option(OPT_ATTN_SPLITS) <= 0 else 2
+
+
 def get_option(opt):
     return load().nvfp4sk_get_option(opt)
 

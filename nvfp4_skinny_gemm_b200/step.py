@@ -415,11 +415,13 @@ class VerifyModel:
 
     def prefill_launches(self, S):
         """Kernel launches of prefill(S rows): per layer norm-q, tile image,
-        qkv, K/V append, one causal attention per block of 128 queries,
-        quantise, tile image, o, norm-q, tile image, gate_up, swiglu-q, tile
-        image, down; then the head on the last row."""
+        qkv, K/V append, one causal attention call per block of 128 queries
+        (nv.attn_launches() launches each), quantise, tile image, o, norm-q,
+        tile image, gate_up, swiglu-q, tile image, down; then the head on the
+        last row."""
         n = len(prefill_chunks(0, S))
-        return 0 if S == 0 else self.n_layers * (13 + n) + (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
+        return 0 if S == 0 else self.n_layers * (13 + n * nv.attn_launches()) + \
+            (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     def step(self, restore=True):
         """One verify step on the current self.h / self.parent; result in self.ids."""
@@ -434,10 +436,11 @@ class VerifyModel:
 
     @property
     def launches_per_layer(self):
-        """norm-q, qkv, kv-append, attention (split with fused combine), [quantise], o,
-        norm-q, gate_up, swiglu-q, down (the attention output is quantised in
-        the combine launch when the scales are static)."""
-        return 9 if self.static else 10
+        """norm-q, qkv, kv-append, attention (nv.attn_launches(): split and
+        combine, or one with the fused combine), [quantise], o, norm-q,
+        gate_up, swiglu-q, down (the attention output is quantised in the
+        combine when the scales are static)."""
+        return (8 if self.static else 9) + nv.attn_launches()
 
     def launches_per_step(self, restore=True):
         return (1 if restore else 0) + self.n_layers * self.launches_per_layer + \

@@ -10,8 +10,8 @@ Labels are hash-consed: a label is the integer id of a flat tuple whose parts
 are strings, numbers or the ids of other labels, so deep layer stacks compare
 in constant time.
 No kernel and no oracle runs; launches are counted as the library would
-launch kernels (the attention is one launch: its combine is fused when the
-split grid fits on the GPU at once, as it does at the verify step's shapes).
+launch kernels (an attention call is two launches, split and combine: the
+library's default, which attn_launches() reports).
 """
 import numpy as np
 import torch
@@ -166,7 +166,7 @@ class FakeLib:
                     ld_q=None, T=None, Hq=None, ws=None, stream=None):
         """Query i (position ctx_len + i) attends to every labelled context
         position and to the new positions ctx_len .. ctx_len + i."""
-        self.launches += 1
+        self.launches += self.attn_launches()
         l = self.layer_of_pool(k_pool)
         assert 1 <= T <= 128 and Hq == I.N_Q_HEADS and ld_q == q.stride(0)
         assert (ctx_len + T + I.PAGE - 1) // I.PAGE <= self.m.n_log
@@ -203,9 +203,13 @@ class FakeLib:
             assert 0 <= pt[(ctx_len + i) // I.PAGE] < self.m.n_pool
             self.kv[(l, ctx_len + i)] = self.L("kv", src[i])
 
+    @staticmethod
+    def attn_launches():
+        return 2
+
     def tree_attn(self, q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None,
                   out=None, ld_q=None, T=None, Hq=None, ws=None, stream=None, g_act=None, act=None):
-        self.launches += 1
+        self.launches += self.attn_launches()
         l = self.layer_of_pool(k_pool)
         assert 1 <= T <= 16 and Hq == I.N_Q_HEADS and ld_q == q.stride(0)
         assert (ctx_len + T + I.PAGE - 1) // I.PAGE <= self.m.n_log

@@ -81,7 +81,10 @@ def test_attention_full_context(oracle, combine_mode):
     rel = np.linalg.norm(got - want) / np.linalg.norm(want)
     print(f"config3: max abs err {err.max():.3e}, rel-Frobenius {rel:.3e}, max |o| {np.abs(want).max():.3e}")
     assert err.max() <= ATTN_ABS_TOL
-    assert rel <= 2e-2
+    # measured on B200: max abs 1.25e-4, rel-Frobenius 1.77e-3 (bf16 output rounding
+    # dominates: |o| <= 0.057 here); gated at about twice that
+    assert err.max() <= 3e-4
+    assert rel <= 4e-3
 
 
 @pytest.mark.parametrize("L", [1000, 1008, 4080])
