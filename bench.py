@@ -56,7 +56,8 @@ def parse():
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--kernel-case", default=None,
                     choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "linear_o", "linear_down",
-                             "linear_m1_2048", "wide_gate_up", "wide_down", "causal_attn", "attn", "restore",
+                             "linear_m1_2048", "wide_qkv", "wide_o", "wide_gate_up", "wide_down", "causal_attn", "attn",
+                             "restore",
                              "quantize"],
                     help="run one kernel on a small case (for ncu captures) instead of the step")
     return ap.parse_args()
@@ -134,11 +135,13 @@ class Clocks:
 
 # ------------------------------------------------------------------ peaks / traffic
 def measured_peak():
+    """HBM copy bandwidth (GB/s) and where it comes from: MEASURED_PEAKS.json's
+    hbm_gbs when the file is there, else the profiling recipe's fallback figure."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return 6650.0, "fallback 6,650 GB/s (no MEASURED_PEAKS.json)"
 
 
 def kernel_source_hash():
@@ -426,7 +429,7 @@ def run_ours(args, world, rank, local):
         "step_pct_of_peak": round(100 * step_bytes / (t_dev / args.steps) / 1e9 / peak, 1),
         "roofline": {"kernel": "nvfp4_linear_kernel (all 257 linear launches of one step, back to back)",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                      "algorithmic_bytes_per_step": lin_bytes, "launches": n_lin,
                      "us_per_step_of_linears": round(t_lin * 1e6, 1),
                      "traffic": traffic},
@@ -434,7 +437,7 @@ def run_ours(args, world, rank, local):
                                     f"of one step, back to back)",
                           "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
                           "frac": round(attn_gbs / peak, 4),
-                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                          "peak_source": peak_kind,
                           "algorithmic_bytes_per_step": attn_bytes,
                           "algorithmic_bytes_per_call": attn_bytes // model.n_layers,
                           "us_per_call": round(t_attn / model.n_layers * 1e6, 2), "traffic": None},
@@ -653,12 +656,14 @@ def run_kernel_case(args):
         wc = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
         wsc = torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g)
         w_p = nv.prepare_weight(wc, wsc, N, K)
+        ncopy = max(1, math.ceil(250e6 / w_p.numel()))          # rotate copies: > L2 per sweep
+        w_ps = [w_p] + [w_p.clone() for _ in range(ncopy - 1)]
         ac = torch.randint(0, 256, (S, K // 2), dtype=torch.uint8, device=dev, generator=g)
         asc = torch.randint(0x30, 0x40, (S, K // 16), dtype=torch.uint8, device=dev, generator=g)
         a_p = nv.prepare_weight(ac, asc, S, K)
         one = torch.full((1,), 0.01, device=dev)
         y = torch.empty(S, N, dtype=torch.bfloat16, device=dev)
-        fn = lambda i: nv.linear_wide(a_p, one, S, w_p, one, N, K, y=y)
+        fn = lambda i: nv.linear_wide(a_p, one, S, w_ps[i % ncopy], one, N, K, y=y)
         nbytes = N * K * 9 // 16
     elif case == "causal_attn":
         start, T = 22610, 128
@@ -667,7 +672,8 @@ def run_kernel_case(args):
         kp, vp, pt, ks, vs = t(cache.k_pool), t(cache.v_pool), t(cache.page_table), t(cache.k_scale), t(cache.v_scale)
         q = I.query_bf16(3, T).to(dev)
         out = torch.empty(T, 24, 128, dtype=torch.bfloat16, device=dev)
-        fn = lambda i: nv.causal_attn(q, kp, vp, pt, start, ks, vs, out=out)
+        pools = [(kp, vp)] + [(kp.clone(), vp.clone()) for _ in range(7)]   # > L2 per sweep
+        fn = lambda i: nv.causal_attn(q, pools[i % 8][0], pools[i % 8][1], pt, start, ks, vs, out=out)
         nbytes = (start + T) * 4 * 128 * 2
     elif case == "attn":
         cache = I.kv_cache(3, I.CTX_MAX)
@@ -675,7 +681,8 @@ def run_kernel_case(args):
         kp, vp, pt, ks, vs = t(cache.k_pool), t(cache.v_pool), t(cache.page_table), t(cache.k_scale), t(cache.v_scale)
         par, q = t(I.tree_parent(3)), I.query_bf16(3).to(dev)
         out = torch.empty(16, 24, 128, dtype=torch.bfloat16, device=dev)
-        fn = lambda i: nv.tree_attn(q, kp, vp, pt, I.CTX_MAX, par, ks, vs, out=out)
+        pools = [(kp, vp)] + [(kp.clone(), vp.clone()) for _ in range(7)]   # > L2 per sweep
+        fn = lambda i: nv.tree_attn(q, pools[i % 8][0], pools[i % 8][1], pt, I.CTX_MAX, par, ks, vs, out=out)
         nbytes = (I.CTX_MAX + 16) * 4 * 128 * 2
     elif case == "restore":
         pb, n = 32768, 354 * 128
@@ -699,8 +706,16 @@ def run_kernel_case(args):
     e1.record()
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) * 1e-3 / 3
+    # the same calls back to back in one CUDA graph (dependent launch between
+    # them, as inside the step), operands rotated so that each sweep exceeds L2
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        graph = capture(stream, lambda: [fn(6 + i) for i in range(20)])
+        t_graph = time_graph(graph, stream, 5) / 20
+    del graph
     print(json.dumps({"kernel_case": case, "us_per_call_incl_launch": round(t * 1e6, 2),
-                      "algorithmic_bytes": nbytes, "status": nv.device_status()[0]}), flush=True)
+                      "us_per_call_graph": round(t_graph * 1e6, 2), "algorithmic_bytes": nbytes,
+                      "gbs_graph": round(nbytes / t_graph / 1e9, 1), "status": nv.device_status()[0]}), flush=True)
 
 
 def main():
