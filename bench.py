@@ -285,12 +285,20 @@ def time_graph(graph, stream, reps, warm=3):
 
 
 def linear_launches(model):
-    """The step's 257 linear launches (same operands, shapes and order)."""
-    for lay in model.layers:
+    """The step's 257 linear launches (same operands, shapes and order; with
+    static scales gate+up is the launch that also does SwiGLU + NVFP4)."""
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    for l, lay in enumerate(model.layers):
         model._linear(model.q_h.buf, model.q_h.g, lay["qkv"], model.qkv)
         model._linear(model.q_a.buf, model.q_a.g, lay["o"], model.h, residual=model.h)
-        model._linear(model.q_h.buf, model.q_h.g, lay["gate_up"], model.gu)
-        model._linear(model.q_f.buf, model.q_f.g, lay["down"], model.h, residual=model.h)
+        gu = lay["gate_up"]
+        if model.static:
+            g_f = model._site(l * model.SITES + 3)
+            nv.linear_swiglu(model.q_h.buf, model.q_h.g, model.T, gu.prep, gu.g, gu.N // 2, gu.K, g_f, model.q_f.buf)
+        else:
+            g_f = model.q_f.g
+            model._linear(model.q_h.buf, model.q_h.g, gu, model.gu)
+        model._linear(model.q_f.buf, g_f, lay["down"], model.h, residual=model.h)
     model._linear(model.q_h.buf, model.q_h.g, model.lm_head, model.logits)
 
 

@@ -158,6 +158,34 @@ NVFP4SK_API nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *
                                         nvfp4sk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_linear_swiglu -- the gate+up linear of the verify step with the
+ * SwiGLU and its NVFP4 quantisation in the epilogue (the down linear's input;
+ * section "NVFP4 and FP8": activations are NVFP4, here with a calibrated
+ * static tensor scale).  For f < F and m < M, with gate = row f and up = row
+ * F + f of the [2F, K] weight:
+ *   gu[m][f]  = bf16( g_a*g_w * sum ... )      (what nvfp4_linear would store)
+ *   s[m][f]   = bf16( silu(gu_gate) * gu_up )   (silu(x) = x / (1 + exp(-x)))
+ *   act_out   = NVFP4 of s with tensor scale *g_out, in the prepared image
+ * -- byte for byte what nvfp4_linear followed by nvfp4_swiglu_quantize with
+ * g_in = g_out write, in one launch.
+ * a_prepared, g_a: the M-row activation (as nvfp4_linear), 1 <= M <= 16.
+ * w_prepared, g_w: nvfp4_prepare_weight of the [2F, K] gate+up weight (gate
+ *   rows first); F % 128 == 0, K % 64 == 0.
+ * g_out: device fp32, the static scale of the SwiGLU output (pass it as g_a
+ *   of the down linear).  act_out: nvfp4_prepared_act_bytes(F) bytes;
+ *   rows m < M are written.
+ * ws: nvfp4_linear_swiglu_workspace_bytes(M, F, K) bytes, zero-filled at
+ *   allocation and again after a failing device status (the workspace rule).
+ * Dynamic activation scales need a grid-wide amax of s: use nvfp4_linear and
+ * nvfp4_swiglu_quantize instead.
+ * ---------------------------------------------------------------------- */
+NVFP4SK_API size_t nvfp4_linear_swiglu_workspace_bytes(int64_t M, int64_t F, int64_t K);
+NVFP4SK_API nvfp4sk_status nvfp4_linear_swiglu(const uint8_t *a_prepared, const float *g_a, int64_t M,
+                                               const uint8_t *w_prepared, const float *g_w, int64_t F, int64_t K,
+                                               const float *g_out, uint8_t *act_out, void *ws, size_t ws_bytes,
+                                               nvfp4sk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_linear_wide -- the same NVFP4 linear for many tokens at once: the
  * linears of the suffix prefill (section "KV-cache reuse between agent
  * steps": after the reused prefix is restored only the new suffix of the

@@ -62,6 +62,11 @@ constexpr uint32_t LIN_A_UNIT = 2 * LIN_A_ATOM + LIN_KSTEPS * LIN_SF_IMG;    // 
 constexpr uint32_t LIN_STAGE_BYTES = LIN_W_UNIT + LIN_A_UNIT;                // 45056 = 44 * 1024
 constexpr uint32_t LIN_OFF_BAR = LIN_STAGES * LIN_STAGE_BYTES;
 constexpr uint32_t LIN_SMEM_BYTES = LIN_OFF_BAR + 256 + 1024;
+// gate+up with SwiGLU: two stages of (gate unit, up unit, activation chunk),
+// then per epilogue warp a 16 x 33 float transpose buffer
+constexpr uint32_t LIN_SW_X_BYTES = 4 * 16 * 33 * 4;
+constexpr uint32_t LIN_SMEM_BYTES_SW = 2 * (2 * LIN_W_UNIT + LIN_A_UNIT) + 256 + LIN_SW_X_BYTES + 1024;
+static_assert(LIN_SMEM_BYTES_SW <= 227 * 1024, "shared memory budget");
 constexpr uint32_t LIN_TMEM_COLS = 512;
 constexpr int LIN_NACC = 1;                       // independent accumulators per tile (MMA j -> j % LIN_NACC)
 constexpr int LIN_SFB_SLOTS = 11;                 // activation-scale chunks kept resident in TMEM
@@ -95,9 +100,16 @@ struct LinearParams {
     float *partial;                // [G][2][128 rows][16 tokens]
     int *counters;                 // [NT][4] (one per TMEM sub-partition)
     int64_t ldy;
-    int64_t U;                     // NT * KC
-    int M, N, NT, KC;
+    int64_t U;                     // NT * KC (gate+up with SwiGLU: gate tiles x KC)
+    int M, N, NT, KC;              // (gate+up with SwiGLU: N = F features, NT = F / 128)
+    uint8_t *sw_act;               // gate+up with SwiGLU: prepared NVFP4 activation [M] x F
+    const float *sw_g;             //   and its static tensor scale
 };
+
+// defined in quant.cuh (the SwiGLU epilogue quantises like the SwiGLU quantiser)
+__device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float g, uint2 &packed);
+__device__ __forceinline__ void store_prepared(uint8_t *act, int64_t r, int64_t blk, uint2 pk, uint32_t sc);
+__device__ __forceinline__ float swiglu_bf16(float gate, float up);
 
 __device__ __forceinline__ int ld_acquire_gpu(const int *p)
 {
@@ -160,18 +172,33 @@ __device__ __forceinline__ bool lin_sfb_resident(int64_t n_units, int64_t KC)
     return n_units >= 4 * KC && KC <= LIN_SFB_SLOTS;
 }
 
+template <bool SW>
 __global__ void __launch_bounds__(LIN_THREADS, 1)
     nvfp4_linear_kernel(const LinearParams p)
 {
+    // SW (gate+up with SwiGLU): a unit is the gate unit u and the up unit
+    // U + u of the same K chunk (the up rows follow the gate rows in the
+    // weight), two accumulators per tile, two stages of 80 KB.
+    constexpr int NH = SW ? 2 : 1;                        // weight units per stage
+    constexpr int STG = SW ? 2 : LIN_STAGES;
+    constexpr uint32_t STB = NH * LIN_W_UNIT + LIN_A_UNIT;
+    constexpr uint32_t OFF_BAR = STG * STB;
+    constexpr int PF = SW ? 2 : LIN_PF;
+    constexpr int PW = 16 * NH;                           // partial-sum floats per row
+    constexpr uint32_t T_SFA = TM_ACC + 2 * 16 * NH;      // after 2 buffers x NH accumulators
+    constexpr uint32_t T_SFB = T_SFA + 32 * NH * STG;
+    static_assert(LIN_NACC == 1, "one accumulator per tile and half");
+    static_assert(T_SFB + 32 * STG <= LIN_TMEM_COLS, "tensor memory budget");
+    static_assert(!SW || OFF_BAR + 256 + LIN_SW_X_BYTES + 1024 <= LIN_SMEM_BYTES_SW, "shared memory budget");
     extern __shared__ uint8_t lin_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lin_smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + LIN_OFF_BAR);
-    uint64_t *empty = full + LIN_STAGES;
-    uint64_t *accf = empty + LIN_STAGES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *empty = full + STG;
+    uint64_t *accf = empty + STG;
     uint64_t *acce = accf + 2;
     uint64_t *drain = acce + 2;
-    uint64_t *sf_ready = drain + 1;                 // [LIN_STAGES]: scales of the stage's unit are in TMEM
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sf_ready + LIN_STAGES);
+    uint64_t *sf_ready = drain + 1;                 // [STG]: scales of the stage's unit are in TMEM
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(sf_ready + STG);
     volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const uint32_t warp = warp_id(), lane = lane_id();
@@ -181,7 +208,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     const int64_t n_units = u1 - u0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < LIN_STAGES; ++s) {
+        for (int s = 0; s < STG; ++s) {
             mbar_init(&full[s], 2);          // weight-unit arrive.expect_tx + activation arrive.expect_tx
             mbar_init(&empty[s], 1);
         }
@@ -190,7 +217,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             mbar_init(&acce[b], 4);
         }
         mbar_init(drain, 1);
-        for (int st = 0; st < LIN_STAGES; ++st) mbar_init(&sf_ready[st], 4);
+        for (int st = 0; st < STG; ++st) mbar_init(&sf_ready[st], 4);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -209,34 +236,36 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
-            const int64_t n_pre = n_units < LIN_STAGES ? n_units : LIN_STAGES;
+            const int64_t n_pre = n_units < STG ? n_units : STG;
             auto issue_w = [&](int64_t i) {
-                const int s = (int)(i % LIN_STAGES);
-                mbar_arrive_expect_tx(&full[s], LIN_W_UNIT);
-                bulk_load_hint(smem + s * LIN_STAGE_BYTES, p.w + (u0 + i) * (int64_t)LIN_W_UNIT, LIN_W_UNIT,
-                               &full[s], pol_w);
+                const int s = (int)(i % STG);
+                mbar_arrive_expect_tx(&full[s], NH * LIN_W_UNIT);
+                bulk_load_hint(smem + s * STB, p.w + (u0 + i) * (int64_t)LIN_W_UNIT, LIN_W_UNIT, &full[s], pol_w);
+                if (SW)
+                    bulk_load_hint(smem + s * STB + LIN_W_UNIT, p.w + (U + u0 + i) * (int64_t)LIN_W_UNIT, LIN_W_UNIT,
+                                   &full[s], pol_w);
             };
             auto issue_a = [&](int64_t i) {
-                const int s = (int)(i % LIN_STAGES);
+                const int s = (int)(i % STG);
                 const int64_t kc = (u0 + i) % KC;
                 mbar_arrive_expect_tx(&full[s], LIN_A_UNIT);
-                bulk_load_hint(smem + s * LIN_STAGE_BYTES + LIN_W_UNIT, p.a + kc * (int64_t)LIN_A_UNIT, LIN_A_UNIT,
-                               &full[s], pol_a);
+                bulk_load_hint(smem + s * STB + NH * LIN_W_UNIT, p.a + kc * (int64_t)LIN_A_UNIT, LIN_A_UNIT, &full[s],
+                               pol_a);
             };
             for (int64_t i = 0; i < n_pre; ++i) issue_w(i);
             pdl_wait();
             for (int64_t i = 0; i < n_pre; ++i) issue_a(i);
             int64_t issued = n_pre;
             for (int64_t i = n_pre; i < n_units; ++i) {
-                if (!mbar_wait(&empty[i % LIN_STAGES], (uint32_t)(((i / LIN_STAGES) & 1) ^ 1), 101, s_abort)) break;
+                if (!mbar_wait(&empty[i % STG], (uint32_t)(((i / STG) & 1) ^ 1), 101, s_abort)) break;
                 issue_w(i);
                 issue_a(i);
                 issued = i + 1;
             }
             if (*s_abort) {
                 // let every copy still in flight land before the CTA exits
-                for (int64_t i = issued > LIN_STAGES ? issued - LIN_STAGES : 0; i < issued; ++i)
-                    mbar_wait_drain(&full[i % LIN_STAGES], (uint32_t)((i / LIN_STAGES) & 1), 102);
+                for (int64_t i = issued > STG ? issued - STG : 0; i < issued; ++i)
+                    mbar_wait_drain(&full[i % STG], (uint32_t)((i / STG) & 1), 102);
             }
         } else {
             pdl_wait();
@@ -248,7 +277,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             constexpr uint32_t idesc = lin_idesc(128, 16);
             int64_t i = 0, seg = 0;
             bool ok = true;
-            const bool sfb_resident = lin_sfb_resident(n_units, KC);
+            const bool sfb_resident = !SW && lin_sfb_resident(n_units, KC);
             const int64_t kc0 = u0 % KC;
             for (int64_t u = u0; u < u1 && ok; ++seg) {
                 const int64_t ka = u % KC;
@@ -256,27 +285,31 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 const uint32_t b = (uint32_t)(seg & 1);
                 if (!mbar_wait(&acce[b], (uint32_t)(((seg >> 1) & 1) ^ 1), 103, s_abort)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + TM_ACC + 16 * LIN_NACC * b;
+                const uint32_t d_tmem = tmem_base + TM_ACC + 16 * NH * b;
                 for (int64_t kc = ka; kc < kend; ++kc, ++i) {
-                    const int s = (int)(i % LIN_STAGES);
-                    const uint32_t par = (uint32_t)((i / LIN_STAGES) & 1);
+                    const int s = (int)(i % STG);
+                    const uint32_t par = (uint32_t)((i / STG) & 1);
                     if (!mbar_wait(&full[s], par, 104, s_abort) || !mbar_wait(&sf_ready[s], par, 109, s_abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t w_s = smem_u32(smem + s * LIN_STAGE_BYTES);
-                    const uint32_t a_s = w_s + LIN_W_UNIT;
-                    const uint32_t sfa_t = tmem_base + TM_SFA + 32 * (uint32_t)s;
+                    const uint32_t w_s = smem_u32(smem + s * STB);
+                    const uint32_t a_s = w_s + NH * LIN_W_UNIT;
                     const uint32_t sfb_t = sfb_resident ? tmem_base + TM_SFB_RES + 32 * (uint32_t)((kc - kc0 + KC) % KC)
-                                                        : tmem_base + TM_SFB + 32 * (uint32_t)s;
+                                                        : tmem_base + T_SFB + 32 * (uint32_t)s;
 #pragma unroll
-                    for (int j = 0; j < LIN_KSTEPS; ++j) {
-                        const uint32_t atom = (uint32_t)(j >> 2), ko = 32u * (uint32_t)(j & 3);
-                        const uint64_t adesc = smem_desc(w_s + atom * LIN_W_ATOM + ko, 16, 1024, SWZ_128B);
-                        const uint64_t bdesc = smem_desc(a_s + atom * LIN_A_ATOM + ko, 16, 1024, SWZ_128B);
-                        mma_mxf4nvf4(d_tmem + 16 * (j % LIN_NACC), adesc, bdesc, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
-                                     (kc > ka || j >= LIN_NACC) ? 1u : 0u);
+                    for (int h = 0; h < NH; ++h) {
+                        const uint32_t sfa_t = tmem_base + T_SFA + 32 * (uint32_t)(NH * s + h);
+#pragma unroll
+                        for (int j = 0; j < LIN_KSTEPS; ++j) {
+                            const uint32_t atom = (uint32_t)(j >> 2), ko = 32u * (uint32_t)(j & 3);
+                            const uint64_t adesc =
+                                smem_desc(w_s + h * LIN_W_UNIT + atom * LIN_W_ATOM + ko, 16, 1024, SWZ_128B);
+                            const uint64_t bdesc = smem_desc(a_s + atom * LIN_A_ATOM + ko, 16, 1024, SWZ_128B);
+                            mma_mxf4nvf4(d_tmem + 16 * h, adesc, bdesc, idesc, sfa_t + 4 * j, sfb_t + 4 * j,
+                                         (kc > ka || j > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit(&empty[s]);
                 }
@@ -313,18 +346,22 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         int64_t next_sf = 0;
         bool sf_ok = true;
         auto stage_scales = [&](int64_t i) -> bool {
-            const int s = (int)(i % LIN_STAGES);
-            const bool landed = mbar_wait(&full[s], (uint32_t)((i / LIN_STAGES) & 1), 108, s_abort);
+            const int s = (int)(i % STG);
+            const bool landed = mbar_wait(&full[s], (uint32_t)((i / STG) & 1), 108, s_abort);
             if (!__all_sync(0xFFFFFFFFu, landed)) return false;
-            const uint8_t *st = smem + s * LIN_STAGE_BYTES;
+            const uint8_t *st = smem + s * STB;
             uint32_t v[32];
 #pragma unroll
-            for (int j = 0; j < LIN_KSTEPS; ++j) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(st + 2 * LIN_W_ATOM + LIN_SF_IMG * j + 16 * lane);
-                v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+            for (int h = 0; h < NH; ++h) {
+#pragma unroll
+                for (int j = 0; j < LIN_KSTEPS; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(st + h * LIN_W_UNIT + 2 * LIN_W_ATOM +
+                                                                     LIN_SF_IMG * j + 16 * lane);
+                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                }
+                tmem_st_x32(lane_base + T_SFA + 32 * (uint32_t)(NH * s + h), v);
             }
-            tmem_st_x32(lane_base + TM_SFA + 32 * (uint32_t)s, v);
-            uint32_t sfb_col = TM_SFB + 32 * (uint32_t)s;
+            uint32_t sfb_col = T_SFB + 32 * (uint32_t)s;
             bool copy_sfb = true;
             if (sfb_resident) {
                 const uint32_t slot = (uint32_t)((((u0 + i) % KC) - kc0 + KC) % KC);
@@ -335,8 +372,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             if (copy_sfb) {
 #pragma unroll
                 for (int j = 0; j < LIN_KSTEPS; ++j) {
-                    const uint4 x = *reinterpret_cast<const uint4 *>(st + LIN_W_UNIT + 2 * LIN_A_ATOM + LIN_SF_IMG * j +
-                                                                     16 * lane);
+                    const uint4 x = *reinterpret_cast<const uint4 *>(st + NH * LIN_W_UNIT + 2 * LIN_A_ATOM +
+                                                                     LIN_SF_IMG * j + 16 * lane);
                     v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
                 tmem_st_x32(lane_base + sfb_col, v);
@@ -358,7 +395,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             const uint32_t b = (uint32_t)(seg & 1);
             // stage the scales of this tile's units and of up to STAGES-1 later
             // ones, so that the MMAs keep going while this tile is written out
-            if (!stage_scales_until((u - u0) + (kend - ka) - 1 + (LIN_STAGES - 1))) break;
+            if (!stage_scales_until((u - u0) + (kend - ka) - 1 + (STG - 1))) break;
             const bool whole = ka == 0 && kend == KC;
             const int64_t first = whole ? c : lin_cta_of(t * KC, U, G);
             const int64_t last = whole ? c : lin_cta_of(t * KC + KC - 1, U, G);
@@ -368,7 +405,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             // partial sums while its own products are still in flight, then adds
             // them to its accumulator in contributor order.
             const bool owner = !whole && c == first;
-            float part[LIN_PF][16];
+            float part[PF][PW];
             bool ok = true;
             if (owner) {
                 // lane 0's acquire, then the warp barrier (which orders memory
@@ -378,13 +415,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
 #pragma unroll
-                for (int k = 0; k < LIN_PF; ++k) {
+                for (int k = 0; k < PF; ++k) {
                     const int64_t cc = first + 1 + k;
                     if (cc <= last) {
                         const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
-                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
+                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * PW);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
+                        for (int v = 0; v < PW / 4; ++v) {
                             const float4 f = __ldcg(Q + v);
                             part[k][4 * v] = f.x; part[k][4 * v + 1] = f.y; part[k][4 * v + 2] = f.z; part[k][4 * v + 3] = f.w;
                         }
@@ -395,23 +432,11 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[16];
+            uint32_t r[PW];                               // [half][token]
             {
-                const uint32_t acc_t = tmem_base + ((32u * q) << 16) + TM_ACC + 16 * LIN_NACC * b;
-                tmem_ld_32x32b_x16(acc_t, r);
-                if (LIN_NACC > 1) {
-                    uint32_t r2[LIN_NACC > 1 ? LIN_NACC - 1 : 1][16];
-#pragma unroll
-                    for (int a = 1; a < LIN_NACC; ++a) tmem_ld_32x32b_x16(acc_t + 16 * a, r2[a - 1]);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        float v = __uint_as_float(r[m]);
-#pragma unroll
-                        for (int a = 1; a < LIN_NACC; ++a) v = __fadd_rn(v, __uint_as_float(r2[a - 1][m]));
-                        r[m] = __float_as_uint(v);
-                    }
-                }
+                const uint32_t acc_t = tmem_base + ((32u * q) << 16) + TM_ACC + 16 * NH * b;
+                tmem_ld_32x32b_x16(acc_t, *reinterpret_cast<uint32_t (*)[16]>(&r[0]));
+                if constexpr (SW) tmem_ld_32x32b_x16(acc_t + 16, *reinterpret_cast<uint32_t (*)[16]>(&r[16]));
             }
             tmem_wait_ld();
             tc_fence_before();
@@ -419,22 +444,22 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             if (lane == 0) mbar_arrive(&acce[b]);
             const int64_t n = t * 128 + row;
             if (whole || owner) {
-                float acc[16];
+                float acc[PW];
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc[m] = __uint_as_float(r[m]);
+                for (int m = 0; m < PW; ++m) acc[m] = __uint_as_float(r[m]);
                 if (owner) {
 #pragma unroll
-                    for (int k = 0; k < LIN_PF; ++k)
+                    for (int k = 0; k < PF; ++k)
                         if (first + 1 + k <= last) {
 #pragma unroll
-                            for (int m = 0; m < 16; ++m) acc[m] = __fadd_rn(acc[m], part[k][m]);
+                            for (int m = 0; m < PW; ++m) acc[m] = __fadd_rn(acc[m], part[k][m]);
                         }
-                    // tiles split over more than LIN_PF + 1 CTAs: the rest, in order
-                    for (int64_t cc = first + 1 + LIN_PF; cc <= last; ++cc) {
+                    // tiles split over more than PF + 1 CTAs: the rest, in order
+                    for (int64_t cc = first + 1 + PF; cc <= last; ++cc) {
                         const int sl = ((lin_start(cc, U, G) / KC) == t) ? 0 : 1;
-                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * 16);
+                        const float4 *Q = reinterpret_cast<const float4 *>(p.partial + ((cc * 2 + sl) * 128 + row) * PW);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
+                        for (int v = 0; v < PW / 4; ++v) {
                             const float4 f = __ldcg(Q + v);
                             acc[4 * v] = __fadd_rn(acc[4 * v], f.x);
                             acc[4 * v + 1] = __fadd_rn(acc[4 * v + 1], f.y);
@@ -444,7 +469,30 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     }
                     if (lane == 0) p.counters[t * 4 + q] = 0;
                 }
-                if (n < p.N) {
+                if constexpr (SW) {
+                    // gate and up of feature n for the 16 tokens, rounded to bf16 as a
+                    // stored linear output would be, then SwiGLU rounded to bf16 (the
+                    // arithmetic of the SwiGLU quantiser); a per-warp transpose through
+                    // shared memory gives each lane one NVFP4 block (token, 16 features)
+                    float *xs = reinterpret_cast<float *>(smem + OFF_BAR + 256) + q * (16 * 33);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float gt = __bfloat162float(__float2bfloat16_rn(__fmul_rn(acc[m], gs)));
+                        const float up = __bfloat162float(__float2bfloat16_rn(__fmul_rn(acc[16 + m], gs)));
+                        xs[m * 33 + lane] = swiglu_bf16(gt, up);
+                    }
+                    __syncwarp();
+                    const int tok = (int)(lane & 15u), hb = (int)(lane >> 4);
+                    float v[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) v[k] = xs[tok * 33 + 16 * hb + k];
+                    __syncwarp();
+                    if (tok < M) {
+                        uint2 pk;
+                        const uint32_t sc = quant_block16(v, *p.sw_g, pk);
+                        store_prepared(p.sw_act, tok, (t * 128 + 32 * q + 16 * hb) / 16, pk, sc);
+                    }
+                } else if (n < p.N) {
                     // y may alias the residual (y = h + linear(h)): every residual
                     // load goes out before the first store
 #pragma unroll
@@ -465,9 +513,9 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 // contributor: publish the partial sum, then one release add on the
                 // tile's arrival counter (per warp: each warp owns rows 32q..32q+31)
                 const int slot = (t == first_tile_of_me) ? 0 : 1;
-                float4 *P = reinterpret_cast<float4 *>(p.partial + ((c * 2 + slot) * 128 + row) * 16);
+                float4 *P = reinterpret_cast<float4 *>(p.partial + ((c * 2 + slot) * 128 + row) * PW);
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
+                for (int v = 0; v < PW / 4; ++v)
                     __stcg(P + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                 // the warp barrier orders every lane's stores before lane 0's

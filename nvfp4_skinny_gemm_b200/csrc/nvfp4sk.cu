@@ -85,7 +85,8 @@ int device_info(DevInfo **out)
                 return fail(NVFP4SK_ERR_DEVICE, "libnvfp4sk is built for sm_100a; device %d is sm_%d%d", dev,
                             d.major, d.minor);
             cudaError_t es[] = {
-                set_smem(nvfp4_linear_kernel, LIN_SMEM_BYTES),
+                set_smem(nvfp4_linear_kernel<false>, LIN_SMEM_BYTES),
+                set_smem(nvfp4_linear_kernel<true>, LIN_SMEM_BYTES_SW),
                 set_smem(tree_attn_split_kernel, ATT_SMEM_BYTES),
                 set_smem(kv_page_restore_kernel, RST_SMEM_BUDGET + 1024),
                 set_smem(nvfp4_linear_wide_kernel, WD_SMEM_BYTES),
@@ -192,6 +193,8 @@ int linear_grid(const DevInfo &d, int64_t U)
 constexpr int64_t LIN_MAX_NT = 4096;
 constexpr size_t LIN_COUNTER_BYTES = LIN_MAX_NT * 4 * 4;
 size_t linear_ws(int64_t G, int64_t NT) { (void)NT; return LIN_COUNTER_BYTES + up256((size_t)G * 2 * 16 * 128 * 4); }
+// gate+up with SwiGLU: the same counters, partial tiles of gate and up, fp32 [G][2][128][32]
+size_t linear_sw_ws(int64_t G) { return LIN_COUNTER_BYTES + up256((size_t)G * 2 * 32 * 128 * 4); }
 
 int attn_splits(const DevInfo &d, int Hkv, int64_t n_log)
 {
@@ -468,9 +471,60 @@ nvfp4sk_status nvfp4_linear(const uint8_t *a_prepared, const float *g_a, int64_t
     p.N = (int)N;
     p.NT = (int)NT;
     p.KC = (int)KC;
-    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, (cudaStream_t)stream, 1,
+    p.sw_act = nullptr;
+    p.sw_g = nullptr;
+    return launched(launch(nvfp4_linear_kernel<false>, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, (cudaStream_t)stream, 1,
                            p),
                     "nvfp4_linear_kernel");
+}
+
+size_t nvfp4_linear_swiglu_workspace_bytes(int64_t M, int64_t F, int64_t K)
+{
+    (void)M;
+    DevInfo *d;
+    if (device_info(&d)) return 0;
+    const int64_t NT = cdiv(F, 128), KC = cdiv(K, LIN_KC);
+    const int64_t G = std::max<int64_t>(d->sms, g_opt_linear_ctas);
+    return linear_sw_ws(std::max<int64_t>(1, std::min<int64_t>(G, NT * KC)));
+}
+
+nvfp4sk_status nvfp4_linear_swiglu(const uint8_t *a_prepared, const float *g_a, int64_t M, const uint8_t *w_prepared,
+                                   const float *g_w, int64_t F, int64_t K, const float *g_out, uint8_t *act_out,
+                                   void *ws, size_t ws_bytes, nvfp4sk_stream_t stream)
+{
+    if (!a_prepared || !g_a || !w_prepared || !g_w || !g_out || !act_out)
+        return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (M < 1 || M > 16 || F < 128 || F % 128 != 0 || F > LIN_MAX_NT * 128 || K < 64 || K % 64 != 0)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need 1 <= M <= 16, F %% 128 == 0 (128 <= F <= 524288), K %% 64 == 0");
+    if (!al16(a_prepared) || !al16(w_prepared) || !al16(act_out))
+        return fail(NVFP4SK_ERR_MISALIGNED, "prepared operands and act_out must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    const int64_t NT = F / 128, KC = cdiv(K, LIN_KC), U = NT * KC;
+    const int G = linear_grid(*d, U);
+    const size_t need = linear_sw_ws(G);
+    if (!ws || ws_bytes < need || !al16(ws))
+        return fail(NVFP4SK_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
+    LinearParams p;
+    p.w = w_prepared;
+    p.a = a_prepared;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.residual = nullptr;
+    p.y = nullptr;
+    p.counters = (int *)ws;
+    p.partial = (float *)((uint8_t *)ws + LIN_COUNTER_BYTES);
+    p.ldy = 0;
+    p.U = U;
+    p.M = (int)M;
+    p.N = (int)F;
+    p.NT = (int)NT;
+    p.KC = (int)KC;
+    p.sw_act = act_out;
+    p.sw_g = g_out;
+    return launched(launch(nvfp4_linear_kernel<true>, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES_SW,
+                           (cudaStream_t)stream, 1, p),
+                    "nvfp4_linear_kernel (gate+up, SwiGLU)");
 }
 
 nvfp4sk_status nvfp4_linear_wide(const uint8_t *a_prepared, const float *g_a, int64_t S, const uint8_t *w_prepared,
@@ -865,7 +919,9 @@ nvfp4sk_status nvfp4_linear_noalloc(const uint8_t *a_prepared, const float *g_a,
     p.N = (int)N;
     p.NT = (int)NT;
     p.KC = (int)KC;
-    return launched(launch(nvfp4_linear_kernel, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, st, 1, p),
+    p.sw_act = nullptr;
+    p.sw_g = nullptr;
+    return launched(launch(nvfp4_linear_kernel<false>, dim3(G), dim3(LIN_THREADS), LIN_SMEM_BYTES, st, 1, p),
                     "nvfp4_linear_kernel (no-alloc)");
 }
 

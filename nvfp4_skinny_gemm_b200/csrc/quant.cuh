@@ -100,16 +100,20 @@ template <> __device__ __forceinline__ void load16<float>(const float *p, float 
 __device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 // SwiGLU block: h_k = bf16(silu(g_k) * u_k), silu(x) = x / (1 + e^-x)
+// silu(gate) * up of bf16 inputs, rounded to bf16 (reading 10)
+__device__ __forceinline__ float swiglu_bf16(float gate, float up)
+{
+    const float sg = __fdiv_rn(gate, 1.0f + expf(-gate));
+    return round_bf16(sg * up);
+}
+
 __device__ __forceinline__ void load16_swiglu(const __nv_bfloat16 *gp, const __nv_bfloat16 *up, float (&v)[16])
 {
     float g[16], u[16];
     load16<__nv_bfloat16>(gp, g);
     load16<__nv_bfloat16>(up, u);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const float sg = __fdiv_rn(g[k], 1.0f + expf(-g[k]));
-        v[k] = round_bf16(sg * u[k]);
-    }
+    for (int k = 0; k < 16; ++k) v[k] = swiglu_bf16(g[k], u[k]);
 }
 
 // ---- cluster-wide amax via distributed shared memory ----------------------

@@ -43,6 +43,8 @@ _SIGS = {
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _sz, _vp]),
     "nvfp4_linear_wide": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
+    "nvfp4_linear_swiglu_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "nvfp4_linear_swiglu": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_noalloc_scratch_bytes": (_sz, []),
     "nvfp4_linear_noalloc": (_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp]),
     "tree_attn_workspace_bytes": (_sz, [_int, _int, _int, _int, _int, _i64]),
@@ -163,7 +165,7 @@ def get_option(opt):
 
 
 # default workspaces whose arrival counters must read zero when a call starts
-_COUNTER_KINDS = ("linear", "argmax", "attn")
+_COUNTER_KINDS = ("linear", "linear_swiglu", "argmax", "attn")
 
 
 def _rezero_counter_workspaces():
@@ -245,6 +247,16 @@ def linear(a_act, g_a, M, w_prep, g_w, N, K, y=None, residual=None, ws=None, str
     _call("nvfp4_linear", _d(a_act), _d(g_a), M, _d(w_prep), _d(g_w), N, K,
           _p(residual), _d(y), y.stride(0), wp, wn, _stream(stream))
     return y
+
+
+def linear_swiglu(a_act, g_a, M, w_prep, g_w, F, K, g_out, act, ws=None, stream=None):
+    """gate+up linear ([2F, K] weight, gate rows first) with SwiGLU and its NVFP4
+    quantisation (static scale g_out) in the epilogue: writes the prepared
+    F-wide activation of the down linear into act (rows < M)."""
+    wp, wn = _ws(ws, load().nvfp4_linear_swiglu_workspace_bytes(M, F, K), "linear_swiglu")
+    _call("nvfp4_linear_swiglu", _d(a_act), _d(g_a), M, _d(w_prep), _d(g_w), F, K, _d(g_out), _d(act), wp, wn,
+          _stream(stream))
+    return act
 
 
 def linear_wide(a_prep, g_a, S, w_prep, g_w, N, K, y=None, residual=None, stream=None):

@@ -254,10 +254,17 @@ class VerifyModel:
         nv.rmsnorm_quantize(self.h, self.norm_w[2 * l + 1], self.eps, self.q_h.out, act=self.q_h.buf,
                             g_in=self._site(s0 + 2))
         self._note(s0 + 2, self.q_h)
-        self._linear(self.q_h.buf, self.q_h.g, lay["gate_up"], self.gu)
-        nv.swiglu_quantize(self.gu, self.q_f.out, act=self.q_f.buf, g_in=self._site(s0 + 3))
-        self._note(s0 + 3, self.q_f)
-        self._linear(self.q_f.buf, self.q_f.g, lay["down"], self.h, residual=self.h)
+        if self.static:
+            # gate+up, SwiGLU and its NVFP4 with the site's static scale in one launch
+            gu = lay["gate_up"]
+            g_f = self._site(s0 + 3)
+            nv.linear_swiglu(self.q_h.buf, self.q_h.g, T, gu.prep, gu.g, gu.N // 2, gu.K, g_f, self.q_f.buf)
+        else:
+            self._linear(self.q_h.buf, self.q_h.g, lay["gate_up"], self.gu)
+            nv.swiglu_quantize(self.gu, self.q_f.out, act=self.q_f.buf)
+            self._note(s0 + 3, self.q_f)
+            g_f = self.q_f.g
+        self._linear(self.q_f.buf, g_f, lay["down"], self.h, residual=self.h)
 
     def head(self):
         i = self.n_layers * self.SITES
@@ -438,9 +445,9 @@ class VerifyModel:
     def launches_per_layer(self):
         """norm-q, qkv, kv-append, attention (nv.attn_launches(): split and
         combine, or one with the fused combine), [quantise], o, norm-q,
-        gate_up, swiglu-q, down (the attention output is quantised in the
-        combine when the scales are static)."""
-        return (8 if self.static else 9) + nv.attn_launches()
+        gate_up, [swiglu-q], down (with static scales the attention output is
+        quantised in the combine and the SwiGLU in the gate+up launch)."""
+        return (7 if self.static else 9) + nv.attn_launches()
 
     def launches_per_step(self, restore=True):
         return (1 if restore else 0) + self.n_layers * self.launches_per_layer + \
@@ -449,11 +456,14 @@ class VerifyModel:
     # ------------------------------------------------------------------ bytes
     def linear_bytes(self):
         """Algorithmic HBM bytes of all linear launches in one step: weight codes
-        + scales, activation codes + scales, bf16 outputs (+ residual reads)."""
+        + scales, activation codes + scales, bf16 outputs (+ residual reads);
+        with static scales the gate+up launch writes the NVFP4 SwiGLU output
+        (N/2 features) instead of the bf16 gate and up."""
         T, tot = self.T, 0
         for lay in self.layers:
             for name, lin in lay.items():
-                tot += lin.nbytes + T * lin.K * 9 // 16 + T * lin.N * 2 * (2 if name in ("o", "down") else 1)
+                out = T * (lin.N // 2) * 9 // 16 if (name == "gate_up" and self.static) else T * lin.N * 2
+                tot += lin.nbytes + T * lin.K * 9 // 16 + out * (2 if name in ("o", "down") else 1)
         if self.lm_head is not None:
             lin = self.lm_head
             tot += lin.nbytes + T * lin.K * 9 // 16 + T * lin.N * 2

@@ -187,6 +187,18 @@ class FakeLib:
         self.put(y, [self.L("linear", l, name, self.gl[g_a.data_ptr()], v, None if res is None else res[i])
                      for i, v in enumerate(a)])
 
+    def linear_swiglu(self, a_act, g_a, M, w_prep, g_w, F, K, g_out, act, ws=None, stream=None):
+        """gate+up linear, SwiGLU and its quantisation with the static scale
+        g_out, in one launch: the labels the two-launch sequence gives."""
+        self.launches += 1
+        assert 1 <= M <= 16
+        l, name = self.wmap[id(w_prep)]
+        assert name == "gate_up" and 2 * F == I.LAYER_LINEARS[name][1]
+        gu = [self.L("linear", l, name, self.gl[g_a.data_ptr()], v, None) for v in self.get(a_act, M)]
+        lab = self.scale(g_out, g_out, gu)
+        self.put(act, [self.L("swiglu", lab, v) for v in gu])
+        return act
+
     def kv_append(self, k_new, v_new, ld_new, T, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale,
                   stream=None):
         self.launches += 1

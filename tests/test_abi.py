@@ -105,6 +105,12 @@ def test_host_checks_reject_bad_arguments_before_the_device():
         (E_SHAPE, "nvfp4_linear_wide", A, A, 100, A, A, 128, 96, None, A, 128, None),
         (E_SHAPE, "nvfp4_linear_wide", A, A, 100, A, A, 128, 128, None, A, 64, None),
         (E_ALIGN, "nvfp4_linear_wide", MIS, A, 100, A, A, 128, 128, None, A, 128, None),
+        # nvfp4_linear_swiglu(a, g_a, M, w, g_w, F, K, g_out, act_out, ws, ws_bytes, stream)
+        (E_ARG, "nvfp4_linear_swiglu", A, A, 16, A, A, 256, 128, None, A, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear_swiglu", A, A, 0, A, A, 256, 128, A, A, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear_swiglu", A, A, 16, A, A, 192, 128, A, A, A, 1 << 20, None),
+        (E_SHAPE, "nvfp4_linear_swiglu", A, A, 16, A, A, 256, 96, A, A, A, 1 << 20, None),
+        (E_ALIGN, "nvfp4_linear_swiglu", A, A, 16, A, A, 256, 128, A, MIS, A, 1 << 20, None),
         # nvfp4_linear_noalloc(a, g_a, M, w, g_w, N, K, residual, y, ldy, stream)
         (E_SHAPE, "nvfp4_linear_noalloc", A, A, 16, A, A, 524289, 128, None, A, 524289, None),
         # tree_attn_fp8kv(q, ld_q, T, Hq, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, parent,

@@ -54,18 +54,23 @@ def test_prefill_flops_brute_force():
 
 def test_verify_step_algorithmic_linear_bytes(monkeypatch):
     """The bytes the bench divides by for the linears' roofline: per launch the
-    weight codes + E4M3 scales, the activation codes + scales, the bf16 output
-    (and the residual read of O and down), 64 layers + LM head at 16 rows."""
+    weight codes + E4M3 scales, the activation codes + scales, the output (and
+    the residual read of O and down), 64 layers + LM head at 16 rows.  The
+    output is bf16, except gate+up with static scales, whose launch writes the
+    NVFP4 codes + E4M3 scales of SwiGLU's N/2 features."""
     from fake_lib import fake_model
     from nvfp4_skinny_gemm_b200 import inputs as I
     m, _ = fake_model(monkeypatch, 64, 1024)
     T, tot = 16, 0
     for name, (K, N) in list(I.LAYER_LINEARS.items()) * 64:
         res = 2 if name in ("o", "down") else 1
-        tot += N * K // 2 + N * K // 16 + T * K // 2 + T * K // 16 + res * T * N * 2
+        out = T * (N // 2) // 2 + T * (N // 2) // 16 if name == "gate_up" else res * T * N * 2
+        tot += N * K // 2 + N * K // 16 + T * K // 2 + T * K // 16 + out
     K, N = I.HIDDEN, I.VOCAB
     tot += N * K // 2 + N * K // 16 + T * K // 2 + T * K // 16 + T * N * 2
-    assert m.linear_bytes() == tot == 11_528_946_688
+    assert m.static and m.linear_bytes() == tot == 11_467_670_528
+    m.static = False        # dynamic scales: gate+up writes bf16 gate and up
+    assert m.linear_bytes() == 11_528_946_688
 
 
 def test_verify_step_attention_and_restore_bytes(monkeypatch):

@@ -34,16 +34,16 @@ def test_step_dataflow_and_launch_count(monkeypatch, static, T, chain):
     assert fake.get(m.ids.view(-1, 1)) == [
         Lb("argmax", Lb("linear", None, "lm_head", sc, Lb("norm", 2 * n_layers, sc, v), None)) for v in h_exp]
     assert fake.launches == m.launches_per_step(restore=True)
-    assert m.launches_per_layer == (10 if static else 11)
+    assert m.launches_per_layer == (9 if static else 11)
 
 
 def test_launch_count_of_the_benchmarked_step(monkeypatch):
-    """64 layers, static scales: 1 restore + 64 x 10 + 3 = 644 launches."""
+    """64 layers, static scales: 1 restore + 64 x 9 + 3 = 580 launches."""
     m, fake = fake_model(monkeypatch, 64, 1024)
     fake.start = 1024
     m.parent.copy_(torch.from_numpy(I.tree_parent(4)))
     m.step()
-    assert fake.launches == m.launches_per_step() == 644
+    assert fake.launches == m.launches_per_step() == 580
 
 
 def test_agent_turn_restore_prefill_verify_accept(monkeypatch):
