@@ -55,7 +55,8 @@ def parse():
     ap.add_argument("--profile-range", action="store_true",
                     help="bracket one untimed step replay with cudaProfilerStart/Stop (for ncu --profile-from-start off)")
     ap.add_argument("--kernel-case", default=None,
-                    choices=["linear_lmhead", "linear_gate_up", "linear_qkv", "linear_o", "linear_down",
+                    choices=["linear_lmhead", "linear_gate_up", "linear_gate_up_swiglu", "linear_qkv", "linear_o",
+                             "linear_down",
                              "linear_m1_2048", "wide_qkv", "wide_o", "wide_gate_up", "wide_down", "causal_attn", "attn",
                              "restore",
                              "quantize"],
@@ -642,6 +643,7 @@ def run_kernel_case(args):
     case = args.kernel_case
     if case.startswith("linear"):
         K, N = {"linear_lmhead": (I.HIDDEN, I.VOCAB), "linear_gate_up": I.LAYER_LINEARS["gate_up"],
+                "linear_gate_up_swiglu": I.LAYER_LINEARS["gate_up"],
                 "linear_qkv": I.LAYER_LINEARS["qkv"], "linear_o": I.LAYER_LINEARS["o"],
                 "linear_down": I.LAYER_LINEARS["down"], "linear_m1_2048": (2048, 2048)}[case]
         M = 1 if case == "linear_m1_2048" else 16
@@ -657,6 +659,9 @@ def run_kernel_case(args):
         _, _, ga = nv.quantize(a, act=act)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         fn = lambda i: nv.linear(act, ga, M, ws[i % ncopy][0], ws[i % ncopy][1], N, K, y=y)
+        if case == "linear_gate_up_swiglu":                       # + SwiGLU + NVFP4 in the epilogue
+            act_f, g_f = nv.act_buffer(N // 2), torch.full((1,), 0.01, device=dev)
+            fn = lambda i: nv.linear_swiglu(act, ga, M, ws[i % ncopy][0], ws[i % ncopy][1], N // 2, K, g_f, act_f)
         nbytes = N * K * 9 // 16
     elif case.startswith("wide"):
         K, N = I.LAYER_LINEARS[case[5:]]
