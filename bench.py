@@ -59,7 +59,7 @@ def parse():
                              "linear_down",
                              "linear_m1_2048", "wide_qkv", "wide_o", "wide_gate_up", "wide_down", "causal_attn", "attn",
                              "restore",
-                             "quantize"],
+                             "quantize", "rmsnorm_quantize"],
                     help="run one kernel on a small case (for ncu captures) instead of the step")
     return ap.parse_args()
 
@@ -705,6 +705,14 @@ def run_kernel_case(args):
         did = torch.randperm(n + 64, device=dev, generator=g)[:n].to(torch.int32)
         fn = lambda i: nv.kv_page_restore(src, sid, dst, did, pb)
         nbytes = 2 * n * pb
+    elif case == "rmsnorm_quantize":                      # the step's RMSNorm + NVFP4, static scale
+        x = torch.randn(16, I.HIDDEN, device=dev, generator=g).to(torch.bfloat16)
+        nw = torch.ones(I.HIDDEN, dtype=torch.bfloat16, device=dev)
+        act = nv.act_buffer(I.HIDDEN)
+        out = (None, None, torch.empty(1, dtype=torch.float32, device=dev))
+        g_in = torch.full((1,), 0.002, dtype=torch.float32, device=dev)
+        fn = lambda i: nv.rmsnorm_quantize(x, nw, 1e-6, out, act=act, g_in=g_in)
+        nbytes = x.numel() * 2 + act.numel()
     else:
         x = torch.randn(16, I.FFN, device=dev, generator=g).to(torch.bfloat16)
         fn = lambda i: nv.quantize(x)

@@ -167,9 +167,11 @@ __device__ __forceinline__ int64_t lin_cta_of(int64_t u, int64_t U, int64_t G) {
 // when a CTA sweeps all K chunks at least four times (an LM-head-like shape:
 // many tiles, short K), each chunk's scales are staged into tensor memory
 // once (slot kc - kc0 mod KC) and reused by every later tile.
+// (Not with SwiGLU: its TMEM columns past the per-stage scales are taken.)
+template <bool SW>
 __device__ __forceinline__ bool lin_sfb_resident(int64_t n_units, int64_t KC)
 {
-    return n_units >= 4 * KC && KC <= LIN_SFB_SLOTS;
+    return !SW && n_units >= 4 * KC && KC <= LIN_SFB_SLOTS;
 }
 
 template <bool SW>
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             constexpr uint32_t idesc = lin_idesc(128, 16);
             int64_t i = 0, seg = 0;
             bool ok = true;
-            const bool sfb_resident = !SW && lin_sfb_resident(n_units, KC);
+            const bool sfb_resident = lin_sfb_resident<SW>(n_units, KC);
             const int64_t kc0 = u0 % KC;
             for (int64_t u = u0; u < u1 && ok; ++seg) {
                 const int64_t ka = u % KC;
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         // The per-stage buffers of unit i are free again once unit i has landed:
         // the producer refilled its stage only after the MMAs of unit i-STAGES
         // had completed.
-        const bool sfb_resident = lin_sfb_resident(n_units, KC);
+        const bool sfb_resident = lin_sfb_resident<SW>(n_units, KC);
         const int64_t kc0 = u0 % KC;
         const uint32_t lane_base = tmem_base + ((32u * q) << 16);
         uint32_t sfb_loaded = 0;

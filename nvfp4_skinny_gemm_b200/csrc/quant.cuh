@@ -23,8 +23,26 @@ __device__ __forceinline__ float tensor_scale_from_amax(float amax)
     return amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
 }
 
+// x / s rounded to nearest even, given y = RN(1/s): Markstein's correction
+// of the product by the correctly rounded reciprocal (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990):
+//   q = RN(x y),  e = RN(x - s q) (exact, one fma),  RN(q + e y) = RN(x / s),
+// valid while nothing over- or underflows (the caller's range guard).  A zero
+// quotient takes the sign of x, as the division gives it.
+__device__ __forceinline__ float div_rn_by(float x, float s, float y)
+{
+    const float q = __fmul_rn(x, y);
+    const float e = __fmaf_rn(-q, s, x);
+    return copysignf(__fmaf_rn(e, y, q), x);
+}
+
 // Quantise one 16-element block held in registers; returns the scale code
 // and writes the 8 code bytes (two per byte, even element in the low nibble).
+// The element divisions x / s are correctly rounded: by the reciprocal and
+// Markstein's correction while 2^-100 <= s <= 2^100 and amax <= 2^100 s
+// (every quotient and remainder then stays normal or exact), else by the
+// IEEE division itself.
 __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float g, uint2 &packed)
 {
     float amax_b = 0.f;
@@ -36,16 +54,19 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float g,
     const float s = __fmul_rn(e4m3_to_float(sc), g);
     uint32_t w0 = 0, w1 = 0;
     if (s != 0.f) {
+        float q[16];
+        if (s >= 0x1p-100f && s <= 0x1p100f && amax_b <= __fmul_rn(s, 0x1p100f)) {
+            const float y = __frcp_rn(s);
 #pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-            uint32_t b0 = cvt_e2m1x2(__fdiv_rn(v[k], s), __fdiv_rn(v[k + 1], s));
-            w0 |= b0 << (k * 4);
+            for (int k = 0; k < 16; ++k) q[k] = div_rn_by(v[k], s, y);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) q[k] = __fdiv_rn(v[k], s);
         }
 #pragma unroll
-        for (int k = 8; k < 16; k += 2) {
-            uint32_t b1 = cvt_e2m1x2(__fdiv_rn(v[k], s), __fdiv_rn(v[k + 1], s));
-            w1 |= b1 << ((k - 8) * 4);
-        }
+        for (int k = 0; k < 8; k += 2) w0 |= cvt_e2m1x2(q[k], q[k + 1]) << (k * 4);
+#pragma unroll
+        for (int k = 8; k < 16; k += 2) w1 |= cvt_e2m1x2(q[k], q[k + 1]) << ((k - 8) * 4);
     }
     packed = make_uint2(w0, w1);
     return sc;

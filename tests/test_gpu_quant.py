@@ -54,6 +54,52 @@ def test_conversion_sweep_matches_oracle(oracle):
     assert bad4.size == 0, f"E4M3: {bad4.size} mismatches, e.g. x={x[bad4[:4]]} gpu={ge4[bad4[:4]]} oracle={oe4[bad4[:4]]}"
 
 
+def _bf16_values(bits):
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32)
+
+
+@pytest.mark.parametrize("g", [1e-3, 0.0037913, 3.7, 1e-30, 2.0 ** -120])
+def test_division_every_bf16_dividend_every_scale(oracle, g):
+    """The quantiser's element division x / s, exhaustively over bf16
+    dividends: for every positive finite E4M3 scale code (and a few amax
+    values that saturate the scale), blocks whose first element A sets the
+    block scale and whose other 15 elements run through every bf16 value of
+    magnitude <= A, both signs.  Codes and scales must equal the oracle's
+    (correctly rounded fp32 division) bit for bit.  Covers the reciprocal +
+    correction path and, with the tiny tensor scales, its exact-division
+    fallback (scales below 2^-100)."""
+    cuda()
+    e4 = oracle.e4m3_table()[1:0x7F].astype(np.float64)
+    amaxes = list(e4 * 6.0 * g) + [448.0 * 6.0 * g * 2.0 ** k for k in (1, 10, 60, 110)]
+    blocks = []
+    for A in amaxes:
+        A32 = np.float32(A)
+        if not np.isfinite(A32) or A32 == 0:
+            continue
+        a_bits = int(np.float32(A32).view(np.uint32)) >> 16          # bf16 at or below A
+        vals = _bf16_values(np.arange(0, a_bits + 1))
+        vals = np.stack([vals, -vals], 1).ravel()
+        n = -(-vals.size // 15) * 15
+        vals = np.concatenate([vals, np.zeros(n - vals.size, np.float32)]).reshape(-1, 15)
+        head = np.full((vals.shape[0], 1), _bf16_values([a_bits])[0], np.float32)
+        blocks.append(np.concatenate([head, vals], 1))
+    x = np.concatenate(blocks).ravel()
+    K = 16384
+    x = np.concatenate([x, np.zeros(-x.size % K, np.float32)]).reshape(-1, K)
+    xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    assert np.array_equal(xd.float().cpu().numpy(), x)               # every value is a bf16
+    codes, scales, _ = nv.quantize(xd, g_in=to_dev(np.array([g], np.float32)))
+    torch.cuda.synchronize()
+    oc, osc, _ = oracle.quantize(x, g_in=g)
+    gs, gc = scales.cpu().numpy(), codes.cpu().numpy()
+    bad_s = np.argwhere(gs != osc)
+    assert bad_s.size == 0, f"{len(bad_s)} scale mismatches, first {bad_s[:5].tolist()}"
+    bad_c = np.argwhere(gc != oc)
+    assert bad_c.size == 0, f"{len(bad_c)} code-byte mismatches, first {bad_c[:5].tolist()}"
+    assert len(np.unique(osc)) >= 100                                 # the sweep reaches the scale codes
+    print(f"g={g}: {x.size} elements, {len(np.unique(osc))} scale codes")
+
+
 @pytest.mark.parametrize("M,K,outliers", [(1, 2048, 0.0), (16, 5120, 0.01), (16, 3072, 0.01),
                                           (16, 17408, 0.01), (3, 80, 0.0), (16, 34816, 0.0)])
 def test_activation_bf16_bitexact(oracle, M, K, outliers):
