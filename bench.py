@@ -147,7 +147,7 @@ def measured_peak():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("linear.cuh", "common.cuh"):
+    for f in ("linear.cuh", "common.cuh", "quant.cuh"):          # the linear kernels and their epilogues
         h.update(open(os.path.join(ROOT, "nvfp4_skinny_gemm_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -490,8 +490,8 @@ def run_ours(args, world, rank, local):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         runs = [oracle_sample(args.ctx, args.layers) for _ in range(3)]
-        v = float(np.median([r[0] for r in runs]))
-        threads, desc = runs[0][1], runs[0][2]
+        med = sorted(runs, key=lambda r: r[0])[1]             # the median run, with its own description
+        v, threads, desc = float(med[0]), med[1], med[2]
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc + "; median of 3 runs",
                                 "runs": [r[0] for r in runs],
