@@ -565,7 +565,8 @@ __global__ void __launch_bounds__(256) prepare_weight_kernel(const uint8_t *__re
     const int64_t t = unit / KC, c = unit % KC;
     const int64_t kbytes = K / 2, kb = K / 16;
     uint8_t *u = out + unit * (int64_t)LIN_W_UNIT;
-    for (int k = threadIdx.x; k < (int)(LIN_W_UNIT / 16); k += blockDim.x) {
+#pragma unroll
+    for (int k = threadIdx.x; k < (int)(LIN_W_UNIT / 16); k += 256) {             // 9 chunks per thread, all in flight
         uint4 v = make_uint4(0, 0, 0, 0);
         if (k < (int)(2 * LIN_W_ATOM / 16)) {
             const int a = k >> 10, r = (k >> 3) & 127, j = k & 7;       // atom, row, stored chunk

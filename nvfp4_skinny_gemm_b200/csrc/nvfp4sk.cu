@@ -373,8 +373,11 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
     }
     if (!g_in && (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(rows, K)))
         return fail(NVFP4SK_ERR_WORKSPACE, "workspace too small");
-    const int grid = (int)std::min<int64_t>(std::min<int64_t>(QBIG_MAX_PARTIALS, 4 * d->sms),
-                                            cdiv(nblk, QBIG_THREADS));
+    // one thread per 16-block with a static scale; with a dynamic one the grid
+    // is capped by the amax partials it leaves
+    const int grid = g_in ? (int)std::min<int64_t>(INT32_MAX, cdiv(nblk, QBIG_THREADS))
+                          : (int)std::min<int64_t>(std::min<int64_t>(QBIG_MAX_PARTIALS, 4 * d->sms),
+                                                   cdiv(nblk, QBIG_THREADS));
     float *partial = (float *)ws;
     cudaError_t e = cudaSuccess;
     if (!g_in) {
@@ -667,7 +670,9 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
     DevInfo *d;
     if (int rc = device_info(&d)) return rc;
     if (g_in)
-        return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, RS_SPLIT), dim3(RS_THREADS), 0,
+        // RS_SPLIT CTAs per row while there are few rows; one per row once they fill the GPU
+        return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, rows >= d->sms ? 1 : RS_SPLIT),
+                               dim3(RS_THREADS), 0,
                                (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, n,
                                g_in, codes, scales, g_out, act_prepared),
                         "rmsnorm_quant_static_kernel");
@@ -697,7 +702,7 @@ nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, co
     const int64_t nblk = rows * (F / 16);
     if (g_in)
         return launched(launch(swiglu_quant_static_kernel,
-                               dim3((unsigned)std::min<int64_t>(4 * d->sms, cdiv(nblk, QBIG_THREADS_STATIC))),
+                               dim3((unsigned)std::min<int64_t>(INT32_MAX, cdiv(nblk, QBIG_THREADS_STATIC))),
                                dim3(QBIG_THREADS_STATIC), 0, (cudaStream_t)stream, 1, (const __nv_bfloat16 *)gu, rows,
                                F, g_in, codes, scales, g_out, act_prepared),
                         "swiglu_quant_static_kernel");

@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(RS_THREADS)
     const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
     const float g = *g_in;
     if (r == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
-    const int64_t b0 = blockIdx.y * kb / RS_SPLIT, b1 = (blockIdx.y + 1) * kb / RS_SPLIT;
+    const int64_t b0 = blockIdx.y * kb / gridDim.y, b1 = (blockIdx.y + 1) * kb / gridDim.y;
     for (int64_t c = b0 + threadIdx.x; c < b1; c += RS_THREADS) {
         float v[16], wv[16];
         load16<__nv_bfloat16>(xr + c * 16, v);
