@@ -355,6 +355,24 @@ NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, 
 NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, const float *g_in,
                                                  uint8_t *codes, uint8_t *scales, float *g_out, uint8_t *act_prepared,
                                                  void *ws, size_t ws_bytes, nvfp4sk_stream_t stream);
+/* The static-scale quantisers of nvfp4_quantize_act, nvfp4_rmsnorm_quantize
+ * and nvfp4_swiglu_quantize writing, instead of the canonical codes and
+ * scales, the tile image that nvfp4_linear_wide streams for a many-token
+ * activation: byte for byte what nvfp4_prepare_weight(codes, scales, rows, K)
+ * writes for their canonical outputs, in one launch (the suffix prefill's
+ * quantisation sites).  g_in: the static tensor scale (required); g_out
+ * receives it.  tiles: nvfp4_prepared_weight_bytes(rows, K) bytes, 16-byte
+ * aligned; the bytes of rows past `rows` in the last 128-row tile are not
+ * written (only those tokens' outputs read them).  K (n, F) % 512 == 0;
+ * rows >= 1; nvfp4_rmsnorm_quantize_tiles needs n <= 8192. */
+NVFP4SK_API nvfp4sk_status nvfp4_quantize_act_tiles(const void *x, int x_dtype, int64_t rows, int64_t K,
+                                                    int64_t ld_x, const float *g_in, float *g_out, uint8_t *tiles,
+                                                    nvfp4sk_stream_t stream);
+NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize_tiles(const void *x, const void *w, float eps, int64_t rows,
+                                                        int64_t n, const float *g_in, float *g_out, uint8_t *tiles,
+                                                        nvfp4sk_stream_t stream);
+NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize_tiles(const void *gu, int64_t rows, int64_t F, const float *g_in,
+                                                       float *g_out, uint8_t *tiles, nvfp4sk_stream_t stream);
 /* Append T new tokens' K and V (bf16, token i head h at k_new[i*ld_new +
  * h*D + d]) to the cache at positions ctx_len .. ctx_len+T-1 as
  * E4M3(fp32(x / scale[h])) (round-to-nearest-even, saturating); the FP8 KV

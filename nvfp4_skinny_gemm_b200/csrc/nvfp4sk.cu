@@ -391,10 +391,77 @@ nvfp4sk_status nvfp4_quantize_act(const void *x, int x_dtype, int64_t rows, int6
     e = x_dtype == NVFP4SK_BF16
             ? launch(quant_blocks_kernel<__nv_bfloat16>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1,
                      (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, (const float *)partial, grid, codes, scales,
-                     g_out, act_prepared)
+                     g_out, act_prepared, (uint8_t *)nullptr)
             : launch(quant_blocks_kernel<float>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1, (const float *)x, rows,
-                     K, ld_x, g_in, (const float *)partial, grid, codes, scales, g_out, act_prepared);
+                     K, ld_x, g_in, (const float *)partial, grid, codes, scales, g_out, act_prepared,
+                     (uint8_t *)nullptr);
     return launched(e, "quant_blocks_kernel");
+}
+
+// ---- quantisers writing the wide linear's tile image (static scale) --------
+static nvfp4sk_status tiles_check(const float *g_in, const float *g_out, const uint8_t *tiles, int64_t rows,
+                                  int64_t K)
+{
+    if (!g_in || !g_out || !tiles) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer (the tile image needs g_in)");
+    if (rows < 1 || rows > INT32_MAX || K < LIN_KC || K % LIN_KC != 0)
+        return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need rows >= 1, K %% 512 == 0");
+    if (!al16(tiles)) return fail(NVFP4SK_ERR_MISALIGNED, "tiles must be 16-byte aligned");
+    return NVFP4SK_OK;
+}
+
+nvfp4sk_status nvfp4_quantize_act_tiles(const void *x, int x_dtype, int64_t rows, int64_t K, int64_t ld_x,
+                                        const float *g_in, float *g_out, uint8_t *tiles, nvfp4sk_stream_t stream)
+{
+    if (!x) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (x_dtype != NVFP4SK_BF16 && x_dtype != NVFP4SK_FP32) return fail(NVFP4SK_ERR_INVALID_ARG, "bad dtype");
+    if (int rc = tiles_check(g_in, g_out, tiles, rows, K)) return rc;
+    if (ld_x < K) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need ld_x >= K");
+    const int64_t esz = x_dtype == NVFP4SK_BF16 ? 2 : 4;
+    if (!al16(x) || (ld_x * esz) % 16 != 0) return fail(NVFP4SK_ERR_MISALIGNED, "x and its row stride must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int grid = (int)std::min<int64_t>(INT32_MAX, cdiv(rows * (K / 16), QBIG_THREADS));
+    uint8_t *none = nullptr;
+    cudaError_t e = x_dtype == NVFP4SK_BF16
+                        ? launch(quant_blocks_kernel<__nv_bfloat16>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1,
+                                 (const __nv_bfloat16 *)x, rows, K, ld_x, g_in, (const float *)nullptr, 0, none, none,
+                                 g_out, none, tiles)
+                        : launch(quant_blocks_kernel<float>, dim3(grid), dim3(QBIG_THREADS), 0, st, 1, (const float *)x,
+                                 rows, K, ld_x, g_in, (const float *)nullptr, 0, none, none, g_out, none, tiles);
+    return launched(e, "quant_blocks_kernel (tile image)");
+}
+
+nvfp4sk_status nvfp4_rmsnorm_quantize_tiles(const void *x, const void *w, float eps, int64_t rows, int64_t n,
+                                            const float *g_in, float *g_out, uint8_t *tiles, nvfp4sk_stream_t stream)
+{
+    if (!x || !w) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (int rc = tiles_check(g_in, g_out, tiles, rows, n)) return rc;
+    if (n > (int64_t)RTHREADS * RNB * 16) return fail(NVFP4SK_ERR_UNSUPPORTED_SHAPE, "need n <= 8192");
+    if (!al16(x) || !al16(w)) return fail(NVFP4SK_ERR_MISALIGNED, "x and w must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    uint8_t *none = nullptr;
+    return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, rows >= d->sms ? 1 : RS_SPLIT),
+                           dim3(RS_THREADS), 0, (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x,
+                           (const __nv_bfloat16 *)w, eps, n, g_in, none, none, g_out, none, tiles),
+                    "rmsnorm_quant_static_kernel (tile image)");
+}
+
+nvfp4sk_status nvfp4_swiglu_quantize_tiles(const void *gu, int64_t rows, int64_t F, const float *g_in, float *g_out,
+                                           uint8_t *tiles, nvfp4sk_stream_t stream)
+{
+    if (!gu) return fail(NVFP4SK_ERR_INVALID_ARG, "null pointer");
+    if (int rc = tiles_check(g_in, g_out, tiles, rows, F)) return rc;
+    if (!al16(gu)) return fail(NVFP4SK_ERR_MISALIGNED, "gu must be 16-byte aligned");
+    DevInfo *d;
+    if (int rc = device_info(&d)) return rc;
+    uint8_t *none = nullptr;
+    return launched(launch(swiglu_quant_static_kernel,
+                           dim3((unsigned)std::min<int64_t>(INT32_MAX, cdiv(rows * (F / 16), QBIG_THREADS_STATIC))),
+                           dim3(QBIG_THREADS_STATIC), 0, (cudaStream_t)stream, 1, (const __nv_bfloat16 *)gu, rows, F,
+                           g_in, none, none, g_out, none, tiles),
+                    "swiglu_quant_static_kernel (tile image)");
 }
 
 nvfp4sk_status nvfp4_prepare_act(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,
@@ -674,7 +741,7 @@ nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, i
         return launched(launch(rmsnorm_quant_static_kernel, dim3((unsigned)rows, rows >= d->sms ? 1 : RS_SPLIT),
                                dim3(RS_THREADS), 0,
                                (cudaStream_t)stream, 1, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, eps, n,
-                               g_in, codes, scales, g_out, act_prepared),
+                               g_in, codes, scales, g_out, act_prepared, (uint8_t *)nullptr),
                         "rmsnorm_quant_static_kernel");
     const int cs = rows <= 8 ? 8 : 16;
     return launched(launch(rmsnorm_quant_kernel, dim3(cs), dim3(RTHREADS), 0, (cudaStream_t)stream, cs,
@@ -704,7 +771,7 @@ nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, int64_t F, co
         return launched(launch(swiglu_quant_static_kernel,
                                dim3((unsigned)std::min<int64_t>(INT32_MAX, cdiv(nblk, QBIG_THREADS_STATIC))),
                                dim3(QBIG_THREADS_STATIC), 0, (cudaStream_t)stream, 1, (const __nv_bfloat16 *)gu, rows,
-                               F, g_in, codes, scales, g_out, act_prepared),
+                               F, g_in, codes, scales, g_out, act_prepared, (uint8_t *)nullptr),
                         "swiglu_quant_static_kernel");
     const int cs = nblk <= (int64_t)8 * QTHREADS * QNB ? 8 : 16;
     return launched(launch(quant_fused_kernel<__nv_bfloat16, 1>, dim3(cs), dim3(QTHREADS), 0, (cudaStream_t)stream,

@@ -85,12 +85,27 @@ __device__ __forceinline__ void store_prepared(uint8_t *act, int64_t r, int64_t 
     base[2 * LIN_A_ATOM + (bi / 4) * LIN_SF_IMG + r * 16 + (bi % 4)] = (uint8_t)sc;
 }
 
-__device__ __forceinline__ void store_block(uint8_t *codes, uint8_t *scales, uint8_t *act, int64_t r, int64_t c,
-                                            int64_t K, uint2 pk, uint32_t sc)
+// Store one quantised 16-block (row r, block index blk along K) into the tile
+// image nvfp4_linear_wide streams for a many-token activation, byte for byte
+// what nvfp4_prepare_weight writes for the canonical codes and scales with
+// tokens as rows: unit (r / 128, blk / 32) of 36 KB; codes in atom
+// (blk % 32) / 16, row r % 128 (128-byte swizzled); the scale in image
+// (blk % 32) / 4, line r % 32, byte 4 ((r % 128) / 32) + blk % 4.
+__device__ __forceinline__ void store_tiles(uint8_t *tiles, int64_t KC, int64_t r, int64_t blk, uint2 pk, uint32_t sc)
+{
+    const uint32_t rr = (uint32_t)(r % 128), bi = (uint32_t)(blk % 32);
+    uint8_t *u = tiles + ((r / 128) * KC + blk / 32) * (int64_t)LIN_W_UNIT;
+    *reinterpret_cast<uint2 *>(u + (bi / 16) * LIN_W_ATOM + swz128(rr, (bi % 16) * 8)) = pk;
+    u[2 * LIN_W_ATOM + (bi / 4) * LIN_SF_IMG + (rr % 32) * 16 + 4 * (rr / 32) + (bi % 4)] = (uint8_t)sc;
+}
+
+__device__ __forceinline__ void store_block(uint8_t *codes, uint8_t *scales, uint8_t *act, uint8_t *tiles, int64_t r,
+                                            int64_t c, int64_t K, uint2 pk, uint32_t sc)
 {
     if (codes) *reinterpret_cast<uint2 *>(codes + r * (K / 2) + c * 8) = pk;
     if (scales) scales[r * (K / 16) + c] = (uint8_t)sc;
     if (act) store_prepared(act, r, c, pk, sc);
+    if (tiles) store_tiles(tiles, (K + LIN_KC - 1) / LIN_KC, r, c, pk, sc);
 }
 
 // ---- element loaders ------------------------------------------------------
@@ -257,7 +272,7 @@ __global__ void __launch_bounds__(QTHREADS, 1)
             const int64_t r = b / kb, c = b % kb;
             uint2 pk;
             const uint32_t sc = quant_block16(v[j], g, pk);
-            store_block(codes, scales, act, r, c, K, pk, sc);
+            store_block(codes, scales, act, nullptr, r, c, K, pk, sc);
         }
     }
     cluster_sync_all();   // keep this CTA's shared memory alive until peers have read it
@@ -310,7 +325,7 @@ __global__ void __launch_bounds__(RTHREADS, 1)
         if (r < rows && c < kb) {
             uint2 pk;
             const uint32_t sc = quant_block16(v[j], g, pk);
-            store_block(codes, scales, act, r, c, n, pk, sc);
+            store_block(codes, scales, act, nullptr, r, c, n, pk, sc);
         }
     }
     cluster_sync_all();
@@ -326,7 +341,8 @@ constexpr int RS_THREADS = 128;
 __global__ void __launch_bounds__(RS_THREADS)
     rmsnorm_quant_static_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
                                 int64_t n, const float *__restrict__ g_in, uint8_t *__restrict__ codes,
-                                uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
+                                uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act,
+                                uint8_t *__restrict__ tiles)
 {
     __shared__ float s_red[RS_THREADS / 32];
     pdl_launch_dependents();
@@ -357,7 +373,7 @@ __global__ void __launch_bounds__(RS_THREADS)
         for (int k = 0; k < 16; ++k) v[k] = round_bf16(__fmul_rn(__fmul_rn(v[k], inv), wv[k]));
         uint2 pk;
         const uint32_t sc = quant_block16(v, g, pk);
-        store_block(codes, scales, act, r, c, n, pk, sc);
+        store_block(codes, scales, act, tiles, r, c, n, pk, sc);
     }
 }
 
@@ -365,7 +381,8 @@ __global__ void __launch_bounds__(RS_THREADS)
 __global__ void __launch_bounds__(QBIG_THREADS_STATIC)
     swiglu_quant_static_kernel(const __nv_bfloat16 *__restrict__ gu, int64_t rows, int64_t F,
                                const float *__restrict__ g_in, uint8_t *__restrict__ codes,
-                               uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act)
+                               uint8_t *__restrict__ scales, float *__restrict__ g_out, uint8_t *__restrict__ act,
+                               uint8_t *__restrict__ tiles)
 {
     pdl_launch_dependents();
     pdl_wait();
@@ -378,7 +395,7 @@ __global__ void __launch_bounds__(QBIG_THREADS_STATIC)
         load16_swiglu(gu + r * 2 * F + c * 16, gu + r * 2 * F + F + c * 16, v);
         uint2 pk;
         const uint32_t sc = quant_block16(v, g, pk);
-        store_block(codes, scales, act, r, c, F, pk, sc);
+        store_block(codes, scales, act, tiles, r, c, F, pk, sc);
     }
 }
 
@@ -415,7 +432,8 @@ __global__ void __launch_bounds__(QBIG_THREADS) quant_blocks_kernel(const T *__r
                                                                      int n_partial, uint8_t *__restrict__ codes,
                                                                      uint8_t *__restrict__ scales,
                                                                      float *__restrict__ g_out,
-                                                                     uint8_t *__restrict__ act)
+                                                                     uint8_t *__restrict__ act,
+                                                                     uint8_t *__restrict__ tiles)
 {
     __shared__ float s_red[33];
     pdl_wait();
@@ -437,7 +455,7 @@ __global__ void __launch_bounds__(QBIG_THREADS) quant_blocks_kernel(const T *__r
         load16<T>(x + r * ld_x + c * 16, v);
         uint2 pk;
         const uint32_t sc = quant_block16(v, g, pk);
-        store_block(codes, scales, act, r, c, K, pk, sc);
+        store_block(codes, scales, act, tiles, r, c, K, pk, sc);
     }
 }
 

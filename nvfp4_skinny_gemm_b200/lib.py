@@ -57,6 +57,9 @@ _SIGS = {
     "kv_v_pages_to_tiled": (_int, [_vp, _vp, _i64, _int, _int, _vp]),
     "nvfp4_rmsnorm_quantize": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_swiglu_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_quantize_act_tiles": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "nvfp4_rmsnorm_quantize_tiles": (_int, [_vp, _vp, _f32, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "nvfp4_swiglu_quantize_tiles": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "kv_append_fp8": (_int, [_vp, _vp, _i64, _int, _int, _int, _vp, _vp, _i64, _int, _vp, _i64, _vp, _vp, _vp]),
     "argmax_workspace_bytes": (_sz, [_i64, _i64]),
     "argmax_rows_bf16": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
@@ -344,6 +347,32 @@ def swiglu_quantize(gu, out, act=None, stream=None, g_in=None):
     _call("nvfp4_swiglu_quantize", _d(gu), rows, F2 // 2, _p(g_in), _p(codes), _p(scales), _d(g),
           _p(act), None, 0, _stream(stream))
     return out
+
+
+def quantize_tiles(x, g_in, tiles, g_out, stream=None):
+    """NVFP4 of x [rows, K] with the static scale g_in straight into the tile
+    image nvfp4_linear_wide streams (tokens as rows); g_out receives g_in."""
+    rows, K = x.shape
+    assert x.stride(1) == 1
+    dt = BF16 if x.dtype == torch.bfloat16 else FP32
+    _call("nvfp4_quantize_act_tiles", _d(x), dt, rows, K, x.stride(0), _d(g_in), _d(g_out), _d(tiles),
+          _stream(stream))
+    return tiles
+
+
+def rmsnorm_quantize_tiles(x, w, eps, g_in, tiles, g_out, stream=None):
+    """rmsnorm_quantize with a static scale into the wide tile image."""
+    rows, n = x.shape
+    _call("nvfp4_rmsnorm_quantize_tiles", _d(x), _d(w), float(eps), rows, n, _d(g_in), _d(g_out), _d(tiles),
+          _stream(stream))
+    return tiles
+
+
+def swiglu_quantize_tiles(gu, g_in, tiles, g_out, stream=None):
+    """swiglu_quantize with a static scale into the wide tile image."""
+    rows, F2 = gu.shape
+    _call("nvfp4_swiglu_quantize_tiles", _d(gu), rows, F2 // 2, _d(g_in), _d(g_out), _d(tiles), _stream(stream))
+    return tiles
 
 
 def kv_append(k_new, v_new, ld_new, T, k_pool, v_pool, page_table, ctx_len, k_scale, v_scale, stream=None):

@@ -289,9 +289,9 @@ class VerifyModel:
     # ------------------------------------------------------------------ prefill
     def _prefill_buffers(self, S):
         """Per-suffix buffers, kept for later calls of up to the same length:
-        the bf16 activations of all S rows, one canonical NVFP4 code / scale
-        buffer and one tile-image buffer for the widest K (reused by every
-        quantisation site), and the head's one-row operands."""
+        the bf16 activations of all S rows, one tile-image buffer for the
+        widest K (reused by every quantisation site, whose quantiser writes it
+        directly), and the head's one-row operands."""
         pf = getattr(self, "_pf", None)
         if pf is not None and pf["cap"] >= S:
             return pf
@@ -304,8 +304,6 @@ class VerifyModel:
             "qkv": torch.empty(cap, (Hq + 2 * Hkv) * D, dtype=torch.bfloat16, device=dev),
             "attn": torch.empty(cap, Hq * D, dtype=torch.bfloat16, device=dev),
             "gu": torch.empty(cap, 2 * F, dtype=torch.bfloat16, device=dev),
-            "codes": torch.empty(cap * kmax // 2, dtype=torch.uint8, device=dev),
-            "scales": torch.empty(cap * kmax // 16, dtype=torch.uint8, device=dev),
             "g": torch.empty(1, dtype=torch.float32, device=dev),
             "wide": torch.empty(nv.prepared_weight_bytes(cap, kmax), dtype=torch.uint8, device=dev),
             "q_h": Act(H, dev),
@@ -314,17 +312,6 @@ class VerifyModel:
         }
         self._pf = pf
         return pf
-
-    @staticmethod
-    def _canon(pf, S, K):
-        """(codes [S, K/2], scales [S, K/16], g): the canonical NVFP4 outputs of
-        a quantisation site over S rows of width K."""
-        return (pf["codes"][:S * K // 2].view(S, K // 2), pf["scales"][:S * K // 16].view(S, K // 16), pf["g"])
-
-    @staticmethod
-    def _wide_act(pf, S, K, out):
-        """The tile image the wide linear streams, from canonical codes / scales."""
-        return nv.prepare_weight(out[0], out[1], S, K, out=pf["wide"])
 
     def prefill(self, h: torch.Tensor, start: int, layers=None):
         """Prefill the S = h.shape[0] suffix tokens at positions start .. start+S-1.
@@ -366,30 +353,27 @@ class VerifyModel:
         if S == 0:
             return None
         pf = self._prefill_buffers(S)
-        H, F = I.HIDDEN, I.FFN
         qd = I.N_Q_HEADS * I.HEAD_DIM
         kd = I.N_KV_HEADS * I.HEAD_DIM
         qkv, attn, gu = pf["qkv"][:S], pf["attn"][:S], pf["gu"][:S]
+        wide, g = pf["wide"], pf["g"]
         for l in layers:
             lay, s0 = self.layers[l], l * self.SITES
             kp, vp = self.k_pool(l), self.v_pool(l)
-            out = self._canon(pf, S, H)
-            nv.rmsnorm_quantize(h, self.norm_w[2 * l], self.eps, out, g_in=self._site(s0))
-            self._wide(self._wide_act(pf, S, H, out), out[2], lay["qkv"], qkv)
+            # each quantiser writes the tile image the wide linear streams
+            nv.rmsnorm_quantize_tiles(h, self.norm_w[2 * l], self.eps, self._site(s0), wide, g)
+            self._wide(wide, g, lay["qkv"], qkv)
             nv.kv_append(qkv[:, qd:], qkv[:, qd + kd:], qkv.stride(0), S, kp, vp, self.page_table, start,
                          self.k_scale[l], self.v_scale[l])
             for r, t, ctx in prefill_chunks(start, S):
                 nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
                                out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS)
-            out = self._canon(pf, S, qd)
-            nv.quantize(attn, g_in=self._site(s0 + 1), out=out)
-            self._wide(self._wide_act(pf, S, qd, out), out[2], lay["o"], h, residual=h)
-            out = self._canon(pf, S, H)
-            nv.rmsnorm_quantize(h, self.norm_w[2 * l + 1], self.eps, out, g_in=self._site(s0 + 2))
-            self._wide(self._wide_act(pf, S, H, out), out[2], lay["gate_up"], gu)
-            out = self._canon(pf, S, F)
-            nv.swiglu_quantize(gu, out, g_in=self._site(s0 + 3))
-            self._wide(self._wide_act(pf, S, F, out), out[2], lay["down"], h, residual=h)
+            nv.quantize_tiles(attn, self._site(s0 + 1), wide, g)
+            self._wide(wide, g, lay["o"], h, residual=h)
+            nv.rmsnorm_quantize_tiles(h, self.norm_w[2 * l + 1], self.eps, self._site(s0 + 2), wide, g)
+            self._wide(wide, g, lay["gate_up"], gu)
+            nv.swiglu_quantize_tiles(gu, self._site(s0 + 3), wide, g)
+            self._wide(wide, g, lay["down"], h, residual=h)
         if self.lm_head is None or len(layers) == 0 or layers[-1] != self.n_layers - 1:
             return None
         i = self.n_layers * self.SITES
@@ -421,13 +405,13 @@ class VerifyModel:
         return nxt, self.ids, acc
 
     def prefill_launches(self, S):
-        """Kernel launches of prefill(S rows): per layer norm-q, tile image,
-        qkv, K/V append, one causal attention call per block of 128 queries
-        (nv.attn_launches() launches each), quantise, tile image, o, norm-q,
-        tile image, gate_up, swiglu-q, tile image, down; then the head on the
-        last row."""
+        """Kernel launches of prefill(S rows): per layer norm-q, qkv, K/V
+        append, one causal attention call per block of 128 queries
+        (nv.attn_launches() launches each), quantise, o, norm-q, gate_up,
+        swiglu-q, down (each quantiser writes the wide linear's tile image);
+        then the head on the last row."""
         n = len(prefill_chunks(0, S))
-        return 0 if S == 0 else self.n_layers * (13 + n * nv.attn_launches()) + \
+        return 0 if S == 0 else self.n_layers * (9 + n * nv.attn_launches()) + \
             (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     def step(self, restore=True):

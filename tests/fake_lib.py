@@ -140,6 +140,30 @@ class FakeLib:
         lab = self.scale(g_in, out[2], src)
         self._quant_out(out, act, [self.L("swiglu", lab, v) for v in src])
 
+    def _tiles_out(self, tiles, labels):
+        """A quantiser writing the wide tile image: rows 0 .. S-1 of tiles."""
+        self.put(tiles[:len(labels)], labels)
+        return tiles
+
+    def quantize_tiles(self, x, g_in, tiles, g_out, stream=None):
+        self.launches += 1
+        src = self.get(x)
+        lab = self.scale(g_in, g_out, src)
+        return self._tiles_out(tiles, [self.L("quant", lab, v) for v in src])
+
+    def rmsnorm_quantize_tiles(self, x, w, eps, g_in, tiles, g_out, stream=None):
+        self.launches += 1
+        src = self.get(x)
+        widx = (w.data_ptr() - self.m.norm_w.data_ptr()) // (I.HIDDEN * 2)
+        lab = self.scale(g_in, g_out, src)
+        return self._tiles_out(tiles, [self.L("norm", widx, lab, v) for v in src])
+
+    def swiglu_quantize_tiles(self, gu, g_in, tiles, g_out, stream=None):
+        self.launches += 1
+        src = self.get(gu)
+        lab = self.scale(g_in, g_out, src)
+        return self._tiles_out(tiles, [self.L("swiglu", lab, v) for v in src])
+
     def prepared_weight_bytes(self, N, K):
         return N * K
 

@@ -111,6 +111,18 @@ def test_host_checks_reject_bad_arguments_before_the_device():
         (E_SHAPE, "nvfp4_linear_swiglu", A, A, 16, A, A, 192, 128, A, A, A, 1 << 20, None),
         (E_SHAPE, "nvfp4_linear_swiglu", A, A, 16, A, A, 256, 96, A, A, A, 1 << 20, None),
         (E_ALIGN, "nvfp4_linear_swiglu", A, A, 16, A, A, 256, 128, A, MIS, A, 1 << 20, None),
+        # nvfp4_quantize_act_tiles(x, dtype, rows, K, ld_x, g_in, g_out, tiles, stream)
+        (E_ARG, "nvfp4_quantize_act_tiles", A, 0, 942, 3072, 3072, None, A, A, None),
+        (E_SHAPE, "nvfp4_quantize_act_tiles", A, 0, 942, 3008, 3072, A, A, A, None),
+        (E_ALIGN, "nvfp4_quantize_act_tiles", A, 0, 942, 3072, 3072, A, A, MIS, None),
+        # nvfp4_rmsnorm_quantize_tiles(x, w, eps, rows, n, g_in, g_out, tiles, stream)
+        (E_ARG, "nvfp4_rmsnorm_quantize_tiles", A, None, 1e-6, 942, 5120, A, A, A, None),
+        (E_SHAPE, "nvfp4_rmsnorm_quantize_tiles", A, A, 1e-6, 942, 8704, A, A, A, None),
+        (E_SHAPE, "nvfp4_rmsnorm_quantize_tiles", A, A, 1e-6, 0, 5120, A, A, A, None),
+        # nvfp4_swiglu_quantize_tiles(gu, rows, F, g_in, g_out, tiles, stream)
+        (E_ARG, "nvfp4_swiglu_quantize_tiles", A, 942, 17408, A, None, A, None),
+        (E_SHAPE, "nvfp4_swiglu_quantize_tiles", A, 942, 17344, A, A, A, None),
+        (E_ALIGN, "nvfp4_swiglu_quantize_tiles", MIS, 942, 17408, A, A, A, None),
         # nvfp4_linear_noalloc(a, g_a, M, w, g_w, N, K, residual, y, ldy, stream)
         (E_SHAPE, "nvfp4_linear_noalloc", A, A, 16, A, A, 524289, 128, None, A, 524289, None),
         # tree_attn_fp8kv(q, ld_q, T, Hq, Hkv, D, k_pool, v_pool, n_pool, P, page_table, ctx_len, parent,

@@ -121,3 +121,51 @@ def test_prefill_head_ranges_determinism():
     assert changed[:, :, sorted(pages)].any(axis=(2, 3)).all()
     others = [pg for pg in range(m.n_pool) if pg not in pages]
     assert not changed[:, :, others].any()
+
+
+@pytest.mark.parametrize("rows", [942, 130, 1, 256])
+def test_quantisers_write_the_wide_tile_image(rows):
+    """The prefill's quantisation sites write the wide linear's tile image
+    directly: byte for byte what nvfp4_prepare_weight makes of the same
+    quantiser's canonical codes and scales (rows past `rows` in the last
+    128-row tile are left as they were: zero here, as prepare_weight pads)."""
+    cuda()
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    dev = torch.device("cuda")
+    g_in = torch.full((1,), 0.0023, dtype=torch.float32, device=dev)
+    g_out = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def check(K, canon, tiles_call):
+        ref = nv.prepare_weight(*canon, rows, K)
+        tiles = torch.zeros(nv.prepared_weight_bytes(rows, K), dtype=torch.uint8, device=dev)
+        tiles_call(tiles)
+        torch.cuda.synchronize()
+        assert nv.device_status() == (0, 0)
+        assert float(g_out.cpu()[0]) == float(g_in.cpu()[0])
+        assert torch.equal(tiles.cpu(), ref.cpu())
+
+    def canon_out(K):
+        return (torch.empty(rows, K // 2, dtype=torch.uint8, device=dev),
+                torch.empty(rows, K // 16, dtype=torch.uint8, device=dev),
+                torch.empty(1, dtype=torch.float32, device=dev))
+
+    H, F, QD = I.HIDDEN, I.FFN, I.N_Q_HEADS * I.HEAD_DIM
+    x = (I.bf16_normal(95, 0, (rows, H)) * 2).to(dev)
+    w = (I.bf16_normal(95, 1, (H,)) * 0.1 + 1).to(dev)
+    out = canon_out(H)
+    nv.rmsnorm_quantize(x, w, 1e-6, out, g_in=g_in)
+    check(H, out[:2], lambda t: nv.rmsnorm_quantize_tiles(x, w, 1e-6, g_in, t, g_out))
+
+    a = I.bf16_normal(95, 2, (rows, QD)).to(dev)
+    out = canon_out(QD)
+    nv.quantize(a, g_in=g_in, out=out)
+    check(QD, out[:2], lambda t: nv.quantize_tiles(a, g_in, t, g_out))
+    a32 = a.float()
+    out = canon_out(QD)
+    nv.quantize(a32, g_in=g_in, out=out)
+    check(QD, out[:2], lambda t: nv.quantize_tiles(a32, g_in, t, g_out))
+
+    gu = (I.bf16_normal(95, 3, (rows, 2 * F)) * 2).to(dev)
+    out = canon_out(F)
+    nv.swiglu_quantize(gu, out, g_in=g_in)
+    check(F, out[:2], lambda t: nv.swiglu_quantize_tiles(gu, g_in, t, g_out))
