@@ -332,12 +332,16 @@ __global__ void __launch_bounds__(RTHREADS, 1)
 }
 
 // ---- static tensor scale: no grid-wide reduction, one launch --------------
-// RMSNorm + quantise with a given g: RSPLIT CTAs per row; each CTA reduces
-// the whole row's sum of squares (the row is 10 KB, read from L2 by every
-// CTA of the row) and encodes its share of the row's 16-blocks, one block per
-// thread.
+// RMSNorm + quantise with a given g: gridDim.y CTAs per row, CTA y encoding
+// the row's 16-blocks [b0, b1) = [y kb / gridDim.y, (y + 1) kb / gridDim.y).
+// Each CTA loads the whole row once (16-block i of the rotation starting at
+// b0 goes to thread i % RS_THREADS, all of a thread's loads in flight at
+// once), sums its squares (per thread, then a warp tree and the four warps in
+// order), and encodes its own blocks from the same registers: block b0 + i is
+// thread i's for i < b1 - b0.
 constexpr int RS_SPLIT = 4;
 constexpr int RS_THREADS = 128;
+constexpr int RS_MAXJ = RTHREADS * RNB / RS_THREADS;   // 16-blocks per thread of an 8192-wide row
 __global__ void __launch_bounds__(RS_THREADS)
     rmsnorm_quant_static_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w, float eps,
                                 int64_t n, const float *__restrict__ g_in, uint8_t *__restrict__ codes,
@@ -349,13 +353,27 @@ __global__ void __launch_bounds__(RS_THREADS)
     pdl_wait();
     const int64_t r = blockIdx.x;
     const int64_t kb = n / 16;
+    const int64_t b0 = blockIdx.y * kb / gridDim.y, b1 = (blockIdx.y + 1) * kb / gridDim.y;
     const __nv_bfloat16 *xr = x + r * n;
-    float ss = 0.f;
-    for (int64_t c = threadIdx.x; c < kb; c += RS_THREADS) {
-        float v[16];
-        load16<__nv_bfloat16>(xr + c * 16, v);
+    uint4 xb[RS_MAXJ][2];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
+    for (int j = 0; j < RS_MAXJ; ++j) {
+        const int64_t i = threadIdx.x + RS_THREADS * j;
+        if (i < kb) {
+            const uint4 *q = reinterpret_cast<const uint4 *>(xr + ((b0 + i) % kb) * 16);
+            xb[j][0] = q[0];
+            xb[j][1] = q[1];
+        }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < RS_MAXJ; ++j) {
+        if (threadIdx.x + RS_THREADS * j < kb) {
+            float v[16];
+            load16<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16 *>(xb[j]), v);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
+        }
     }
     ss = warp_sum(ss);
     if (lane_id() == 0) s_red[warp_id()] = ss;
@@ -364,16 +382,20 @@ __global__ void __launch_bounds__(RS_THREADS)
     const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
     const float g = *g_in;
     if (r == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
-    const int64_t b0 = blockIdx.y * kb / gridDim.y, b1 = (blockIdx.y + 1) * kb / gridDim.y;
-    for (int64_t c = b0 + threadIdx.x; c < b1; c += RS_THREADS) {
-        float v[16], wv[16];
-        load16<__nv_bfloat16>(xr + c * 16, v);
-        load16<__nv_bfloat16>(w + c * 16, wv);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = round_bf16(__fmul_rn(__fmul_rn(v[k], inv), wv[k]));
-        uint2 pk;
-        const uint32_t sc = quant_block16(v, g, pk);
-        store_block(codes, scales, act, tiles, r, c, n, pk, sc);
+    for (int j = 0; j < RS_MAXJ; ++j) {
+        const int64_t i = threadIdx.x + RS_THREADS * j;
+        if (i < b1 - b0) {
+            const int64_t c = b0 + i;
+            float v[16], wv[16];
+            load16<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16 *>(xb[j]), v);
+            load16<__nv_bfloat16>(w + c * 16, wv);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = round_bf16(__fmul_rn(__fmul_rn(v[k], inv), wv[k]));
+            uint2 pk;
+            const uint32_t sc = quant_block16(v, g, pk);
+            store_block(codes, scales, act, tiles, r, c, n, pk, sc);
+        }
     }
 }
 
