@@ -576,12 +576,9 @@ def run_prefill(args):
                     nv.linear_wide(pf["wide"], pf["g"], S, lin.prep, lin.g, lin.N, lin.K, y=y)
 
         def causal_attention():
-            from nvfp4_skinny_gemm_b200.step import prefill_chunks
+            # the blocks of each layer as the prefill launches them (round its streams)
             for l in range(model.n_layers):
-                for r, t, ctx in prefill_chunks(start, S):
-                    nv.causal_attn(pf["qkv"][r:r + t], model.k_pool(l), model.v_pool(l), model.page_table, ctx,
-                                   model.k_scale[l], model.v_scale[l], out=pf["attn"][r:r + t],
-                                   ld_q=pf["qkv"].stride(0), T=t, Hq=I.N_Q_HEADS)
+                model._causal_blocks(pf, l, pf["qkv"][:S], pf["attn"][:S], start, S)
 
         g_lin = capture(stream, wide_linears)
         g_att = capture(stream, causal_attention)
@@ -621,8 +618,9 @@ def run_prefill(args):
                                      "FP4 peak (sustained bf16 x 4)"},
             "causal_attention": {"ms": round(t_att * 1e3, 3), "tflops": round(attn_flops / t_att / 1e12, 1),
                                  "frac": round(attn_flops / t_att / (2 * bf16 * 1e12), 4),
-                                 "note": "all causal_attn_fp8kv launches of one prefill, back to back; frac of "
-                                         "the FP8 peak (sustained bf16 x 2)"},
+                                 "note": "all causal_attn_fp8kv launches of one prefill, back to back (each "
+                                         "layer's blocks round the prefill's streams); frac of the FP8 peak "
+                                         "(sustained bf16 x 2)"},
             "rest_ms": round((t - t_lin - t_att) * 1e3, 3)},
         "clocks": clk,
         "gpu_launches": model.prefill_launches(S) * args.steps,

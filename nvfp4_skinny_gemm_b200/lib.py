@@ -140,13 +140,22 @@ class Workspace:
 _default_ws = {}
 
 
+def default_workspace(kind, slot=0):
+    """The library's default workspace of an op kind on the current device;
+    slot > 0: another one of the same kind (for calls of that kind that run
+    at the same time on other streams), zeroed like the default after a
+    failing device status."""
+    dev = torch.cuda.current_device()
+    key = kind if slot == 0 else f"{kind}#{slot}"
+    return _default_ws.setdefault((dev, key), Workspace(f"cuda:{dev}"))
+
+
 def _ws(ws, nbytes, kind):
     """Workspace pointer and size; by default one zero-filled buffer per
     (device, op kind): the linear and argmax workspaces hold arrival counters
     that must read zero at call start, which another op's partials would break."""
     if ws is None:
-        dev = torch.cuda.current_device()
-        ws = _default_ws.setdefault((dev, kind), Workspace(f"cuda:{dev}"))
+        ws = default_workspace(kind)
     buf = ws.get(nbytes)
     return buf.data_ptr(), buf.numel()
 
@@ -176,7 +185,7 @@ def _rezero_counter_workspaces():
     device wait ran out can leave their arrival counters non-zero, and the next
     call on the same workspace would count stale arrivals."""
     for (dev, kind), ws in _default_ws.items():
-        if kind in _COUNTER_KINDS and ws.buf is not None:
+        if kind.split("#")[0] in _COUNTER_KINDS and ws.buf is not None:
             ws.buf.zero_()
 
 

@@ -34,6 +34,7 @@ from . import lib as nv
 
 PAGE_BYTES = I.N_KV_HEADS * I.PAGE * I.HEAD_DIM      # one (layer, K|V, page) plane: 32 KB
 PREFILL_CHUNK = 128                                  # queries per causal-attention launch
+PREFILL_STREAMS = 4                                  # streams the blocks of a layer's attention share
 
 
 def prefill_chunks(start: int, S: int, C: int = PREFILL_CHUNK):
@@ -307,6 +308,8 @@ class VerifyModel:
             "g": torch.empty(1, dtype=torch.float32, device=dev),
             "wide": torch.empty(nv.prepared_weight_bytes(cap, kmax), dtype=torch.uint8, device=dev),
             "q_h": Act(H, dev),
+            "streams": [torch.cuda.Stream(device=dev) for _ in range(PREFILL_STREAMS)]
+            if dev.type == "cuda" else [],
             "logits": torch.empty(1, I.VOCAB, dtype=torch.bfloat16, device=dev),
             "ids": torch.empty(1, dtype=torch.int32, device=dev),
         }
@@ -365,9 +368,7 @@ class VerifyModel:
             self._wide(wide, g, lay["qkv"], qkv)
             nv.kv_append(qkv[:, qd:], qkv[:, qd + kd:], qkv.stride(0), S, kp, vp, self.page_table, start,
                          self.k_scale[l], self.v_scale[l])
-            for r, t, ctx in prefill_chunks(start, S):
-                nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
-                               out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS)
+            self._causal_blocks(pf, l, qkv, attn, start, S)
             nv.quantize_tiles(attn, self._site(s0 + 1), wide, g)
             self._wide(wide, g, lay["o"], h, residual=h)
             nv.rmsnorm_quantize_tiles(h, self.norm_w[2 * l + 1], self.eps, self._site(s0 + 2), wide, g)
@@ -382,6 +383,36 @@ class VerifyModel:
         self._linear(a.buf, a.g, self.lm_head, pf["logits"], M=1)
         nv.argmax(pf["logits"], pf["ids"])
         return pf["ids"]
+
+    def _causal_blocks(self, pf, l, qkv, attn, start, S):
+        """The layer's causal attention, one call per block of 128 queries.  The
+        blocks are independent once every suffix token's K/V is appended, so on
+        the GPU they go round PREFILL_STREAMS streams (each with its own
+        workspace), forked from and joined back into the current stream: one
+        block's start overlaps another's tail."""
+        kp, vp = self.k_pool(l), self.v_pool(l)
+        chunks = prefill_chunks(start, S)
+        k = min(len(pf["streams"]), len(chunks))
+        if k < 2:
+            for r, t, ctx in chunks:
+                nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
+                               out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS)
+            return
+        main = torch.cuda.current_stream(self.dev)
+        fork = torch.cuda.Event()
+        fork.record(main)
+        for i, (r, t, ctx) in enumerate(chunks):
+            s = pf["streams"][i % k]
+            if i < k:
+                s.wait_event(fork)
+            with torch.cuda.stream(s):
+                nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
+                               out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS,
+                               ws=nv.default_workspace("attn", i % k))
+        for s in pf["streams"][:k]:
+            join = torch.cuda.Event()
+            join.record(s)
+            main.wait_event(join)
 
     def _wide(self, act, g, lin, y, residual=None):
         nv.linear_wide(act, g, y.shape[0], lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
