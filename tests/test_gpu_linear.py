@@ -221,3 +221,13 @@ def test_prepared_activation_layout(M, K):
             want[off:off + 8] = c[m, blk * 8:blk * 8 + 8]
             want[base + 4096 + (bi // 4) * 512 + m * 16 + bi % 4] = sc[m, blk]
     assert np.array_equal(act.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("M", list(range(1, 17)))
+def test_linear_every_row_count(oracle, M):
+    """Every token count 1..16 (rows past M of the prepared activation are
+    zero; outputs past M are never written), whole outputs on a ragged shape."""
+    cuda()
+    y, want, _ = _case(oracle, M, 384, 1088, 0.01, seed=100 + M)
+    err = rel_fro(y, bf16_round(want))
+    assert err <= REL_FRO_TOL, f"M={M}: rel err {err:.3e}"

@@ -78,3 +78,21 @@ def test_fused_repeatable_and_rows_independent():
     torch.cuda.synchronize()
     assert torch.equal(one.cpu(), ref.cpu())
     assert nv.device_status() == (0, 0)
+
+
+def test_fused_many_tiles_short_k():
+    """Many gate tiles over a short K (F = 131,072, K = 512: each CTA sweeps
+    the single K chunk several times), the shape where an activation-scale
+    layout for repeated chunks would apply to a plain linear: the fused launch
+    must stage every unit's scales and still equal the two-launch sequence
+    (M = 4 keeps the reference quantiser's prepared image within its limit)."""
+    cuda()
+    M, F, K = 4, 131072, 512
+    w_p, g_w, act, g_a = _operands(M, F, K, 11)
+    g_out = torch.full((1,), 0.02, dtype=torch.float32, device="cuda")
+    _, ref = _two_launches(act, g_a, M, w_p, g_w, F, K, g_out)
+    fused = nv.act_buffer(F)
+    nv.linear_swiglu(act, g_a, M, w_p, g_w, F, K, g_out, fused)
+    torch.cuda.synchronize()
+    assert nv.device_status() == (0, 0)
+    assert torch.equal(fused.cpu(), ref.cpu())
