@@ -152,6 +152,25 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+def attn_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn.cuh", "common.cuh"):                          # the attention kernels' memory traffic
+        h.update(open(os.path.join(ROOT, "nvfp4_skinny_gemm_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_attn_traffic():
+    """DRAM bytes per tree-attention call (the split kernel), from the committed
+    ncu summary, if it was taken on the current attention source (else None)."""
+    p = os.path.join(ROOT, "profiles", "tree_attn_fp8kv_ctx23552_t16.md")
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"traffic_bytes_per_call_of_split:\s*([0-9.eE+]+)\s+source:\s*([0-9a-f]+)", open(p).read())
+    if m and m.group(2) == attn_source_hash():
+        return float(m.group(1))
+    return None
+
+
 def recorded_traffic():
     """DRAM bytes per linear launch of the step, from the committed ncu summary,
     if it was taken on the current kernel source (else None)."""
@@ -449,7 +468,10 @@ def run_ours(args, world, rank, local):
                           "peak_source": peak_kind,
                           "algorithmic_bytes_per_step": attn_bytes,
                           "algorithmic_bytes_per_call": attn_bytes // model.n_layers,
-                          "us_per_call": round(t_attn / model.n_layers * 1e6, 2), "traffic": None},
+                          "us_per_call": round(t_attn / model.n_layers * 1e6, 2),
+                          "traffic": recorded_attn_traffic() if args.ctx == 23552 else None,
+                          "traffic_note": "DRAM bytes per call of the split kernel (ncu, 23,552-token "
+                                          "context); the combine was not captured"},
         "no_restore": {"value": world / t_nr, "unit": UNIT, "ms_per_step": round(t_nr * 1e3, 3),
                        "note": "the same step without the per-step kv_page_restore of the prefix "
                                "(the pages restore once per agent turn)"},

@@ -96,3 +96,24 @@ def test_oracle_sample_on_one_thread():
     v1 = bench.oracle_sample_one_thread(1024, 2)
     assert v1 is not None and v1 > 0
     assert bench.oracle_sample_one_thread(1024, 2, timeout=0.01) is None
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """The DRAM traffic the bench reports next to each roofline comes from the
+    committed ncu summary only while the summary's source hash matches the
+    current kernel source; any other hash (an edited kernel) gives None."""
+    import bench
+    lin = bench.recorded_traffic()
+    att = bench.recorded_attn_traffic()
+    # when present (the kernels unchanged since the capture), close to the algorithmic bytes
+    assert lin is None or 0.99 < lin / 11_468_270_000 < 1.01
+    assert att is None or 0.99 < att / 24_133_632 < 1.02
+    (tmp_path / "profiles").mkdir()
+    for name, key in (("nvfp4_linear_verify_step.md", "traffic_bytes_per_step_of_linears"),
+                      ("tree_attn_fp8kv_ctx23552_t16.md", "traffic_bytes_per_call_of_split")):
+        (tmp_path / "profiles" / name).write_text(f"{key}: 1.0e+07 source: 0123456789abcdef\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0123456789abcdef")
+    monkeypatch.setattr(bench, "attn_source_hash", lambda: "fedcba9876543210")
+    assert bench.recorded_traffic() == 1.0e7
+    assert bench.recorded_attn_traffic() is None
