@@ -7,6 +7,7 @@ is missing, the first call raises -- there is no CPU fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import re
@@ -165,11 +166,30 @@ def set_option(opt, value):
     _call("nvfp4sk_set_option", opt, int(value))
 
 
-def attn_launches():
-    """Kernel launches per tree_attn / causal_attn call at the library's own
-    split counts: 1 with the fused combine (OPT_ATTN_FUSED_COMBINE on; those
-    split grids always fit on the GPU at once), else 2 (split, then combine)."""
-    return 1 if get_option(OPT_ATTN_FUSED_COMBINE) and get_option(OPT_ATTN_SPLITS) <= 0 else 2
+def attn_launches(ctas=None, sms=None):
+    """Kernel launches per tree_attn / causal_attn call: 1 with the fused
+    combine (OPT_ATTN_FUSED_COMBINE on and the whole split grid resident at
+    once, one CTA per SM), else 2 (split, then combine).  The library's own
+    split counts always give a grid that fits; for a call made at an explicit
+    OPT_ATTN_SPLITS, pass its grid size (ctas = splits x heads) and the
+    device's SM count (sms), else 2 is assumed."""
+    if not get_option(OPT_ATTN_FUSED_COMBINE):
+        return 2
+    if get_option(OPT_ATTN_SPLITS) <= 0:
+        return 1
+    return 1 if ctas is not None and sms is not None and ctas <= sms else 2
+
+
+@contextlib.contextmanager
+def option(opt, value):
+    """Set a library option for the calls made inside the block, then put its
+    previous value back."""
+    old = get_option(opt)
+    set_option(opt, value)
+    try:
+        yield
+    finally:
+        set_option(opt, old)
 
 
 def get_option(opt):

@@ -24,6 +24,7 @@ All buffers are allocated once, so a step can be captured in a CUDA graph.
 """
 from __future__ import annotations
 
+import contextlib
 import math
 
 import numpy as np
@@ -34,7 +35,8 @@ from . import lib as nv
 
 PAGE_BYTES = I.N_KV_HEADS * I.PAGE * I.HEAD_DIM      # one (layer, K|V, page) plane: 32 KB
 PREFILL_CHUNK = 128                                  # queries per causal-attention launch
-PREFILL_STREAMS = 4                                  # streams the blocks of a layer's attention share
+PREFILL_STREAMS = 8                                  # streams the blocks of a layer's attention share
+PREFILL_ATTN_SPLITS = 3                              # context splits per query head of a block while >= 4 overlap
 
 
 def prefill_chunks(start: int, S: int, C: int = PREFILL_CHUNK):
@@ -401,18 +403,34 @@ class VerifyModel:
         main = torch.cuda.current_stream(self.dev)
         fork = torch.cuda.Event()
         fork.record(main)
-        for i, (r, t, ctx) in enumerate(chunks):
-            s = pf["streams"][i % k]
-            if i < k:
-                s.wait_event(fork)
-            with torch.cuda.stream(s):
-                nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
-                               out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS,
-                               ws=nv.default_workspace("attn", i % k))
+        splits = self._causal_splits(len(chunks))
+        with nv.option(nv.OPT_ATTN_SPLITS, splits) if splits else contextlib.nullcontext():
+            for i, (r, t, ctx) in enumerate(chunks):
+                s = pf["streams"][i % k]
+                if i < k:
+                    s.wait_event(fork)
+                with torch.cuda.stream(s):
+                    nv.causal_attn(qkv[r:r + t], kp, vp, self.page_table, ctx, self.k_scale[l], self.v_scale[l],
+                                   out=attn[r:r + t], ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS,
+                                   ws=nv.default_workspace("attn", i % k))
         for s in pf["streams"][:k]:
             join = torch.cuda.Event()
             join.record(s)
             main.wait_event(join)
+
+    def _causal_splits(self, n_blocks):
+        """Context splits per query head that the prefill gives each causal
+        call: PREFILL_ATTN_SPLITS while at least 4 blocks run at once on the
+        streams, else 0 (the library's own count, which fills the GPU with one
+        call).  With several calls in flight, fewer and longer CTAs pay the
+        per-CTA query setup, split write-out and combine fewer times (on B200,
+        8 blocks of a 942-token suffix: 471 us per layer at 3 splits on 8
+        streams against 517 us at the library's 6).  A split count the caller
+        set through OPT_ATTN_SPLITS stands."""
+        k = min(PREFILL_STREAMS, n_blocks) if self.dev.type == "cuda" else 1
+        if k < 4 or nv.get_option(nv.OPT_ATTN_SPLITS) > 0:
+            return 0
+        return PREFILL_ATTN_SPLITS
 
     def _wide(self, act, g, lin, y, residual=None):
         nv.linear_wide(act, g, y.shape[0], lin.prep, lin.g, lin.N, lin.K, y=y, residual=residual)
@@ -438,11 +456,18 @@ class VerifyModel:
     def prefill_launches(self, S):
         """Kernel launches of prefill(S rows): per layer norm-q, qkv, K/V
         append, one causal attention call per block of 128 queries
-        (nv.attn_launches() launches each), quantise, o, norm-q, gate_up,
+        (nv.attn_launches() launches each, at the split count the blocks
+        run at), quantise, o, norm-q, gate_up,
         swiglu-q, down (each quantiser writes the wide linear's tile image);
         then the head on the last row."""
         n = len(prefill_chunks(0, S))
-        return 0 if S == 0 else self.n_layers * (9 + n * nv.attn_launches()) + \
+        splits = self._causal_splits(n)
+        if splits:
+            sms = torch.cuda.get_device_properties(self.dev).multi_processor_count
+            per_call = nv.attn_launches(splits * I.N_Q_HEADS, sms)
+        else:
+            per_call = nv.attn_launches()
+        return 0 if S == 0 else self.n_layers * (9 + n * per_call) + \
             (self.LAUNCHES_HEAD if self.lm_head is not None else 0)
 
     def step(self, restore=True):

@@ -240,7 +240,7 @@ class FakeLib:
             self.kv[(l, ctx_len + i)] = self.L("kv", src[i])
 
     @staticmethod
-    def attn_launches():
+    def attn_launches(ctas=None, sms=None):
         return 2
 
     def tree_attn(self, q, k_pool, v_pool, page_table, ctx_len, parent, k_scale, v_scale, sm_scale=None,

@@ -1,7 +1,7 @@
 """Suffix prefill on the GPU (VerifyModel.prefill): S prompt tokens that the
-prefix cache does not hold go through every layer 16 rows at a time, each
-group attending to the context before it (earlier groups included) plus its
-own causal chain.
+prefix cache does not hold go through every layer, all rows at once in the
+linears; the attention runs in blocks of 128 queries, each block attending to
+the context before it (earlier blocks included) plus its own causal chain.
 
 (1) Per layer, teacher-forced against the oracle run over all S rows at once
     (no groups): RMSNorm + NVFP4 with the static site scales, the NVFP4
@@ -10,6 +10,9 @@ own causal chain.
     bars are those of the one-layer verify test (rel-Frobenius 1e-2 on the
     composed outputs; attention 2e-3 + 2^-8 |o| against the oracle fed the
     GPU's own Q and cache).  S = 20 spans a full group and a ragged one.
+(1b) The attention blocks of a 5-block suffix as prefill() runs them (spread
+    over streams at the prefill's split count): against the oracle's one
+    causal chain, and bit-identical to the same calls made one after another.
 (2) The whole call with the LM head: the returned token is the first argmax
     of the last row's logits; two calls over layer ranges [0, 1) and [1, 2)
     give the bits of one call; a second run gives the same bits.
@@ -18,7 +21,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import cuda, rel_fro
+from gpu_helpers import ATTN_ABS_TOL, cuda, rel_fro
 from nvfp4_skinny_gemm_b200 import inputs as I
 
 pytestmark = pytest.mark.gpu
@@ -88,6 +91,42 @@ def test_prefill_layers_teacher_forced(oracle):
         err = rel_fro(h2_gpu, h2)
         print(f"prefill layer {l}: rel-Frobenius {err:.2e}")
         assert err <= 1e-2 and np.isfinite(h2_gpu).all()
+
+
+def test_prefill_attention_blocks_on_streams(oracle):
+    """A 520-token suffix after 4,000 cached tokens: 5 blocks, which prefill()
+    spreads over its streams at PREFILL_ATTN_SPLITS splits per query head."""
+    cuda()
+    from nvfp4_skinny_gemm_b200 import lib as nv
+    from nvfp4_skinny_gemm_b200.step import PREFILL_ATTN_SPLITS, VerifyModel, prefill_chunks
+    start, S = 4000, 520
+    L = start + S
+    m = VerifyModel(n_layers=1, ctx_len=L, T=I.TREE_NODES, weights="device", lm_head=False)
+    m.restore()
+    qd, kd = I.N_Q_HEADS * I.HEAD_DIM, I.N_KV_HEADS * I.HEAD_DIM
+    pf = m._prefill_buffers(S)
+    qkv, attn = pf["qkv"][:S], pf["attn"][:S]
+    qkv.copy_(I.bf16_normal(4, 303, (S, qkv.shape[1])) * 0.5)
+    kp_d, vp_d, ks, vs = m.k_pool(0), m.v_pool(0), m.k_scale[0], m.v_scale[0]
+    nv.kv_append(qkv[:, qd:], qkv[:, qd + kd:], qkv.stride(0), S, kp_d, vp_d, m.page_table, start, ks, vs)
+    chunks = prefill_chunks(start, S)
+    assert len(chunks) == 5 and m._causal_splits(len(chunks)) == PREFILL_ATTN_SPLITS
+    m._causal_blocks(pf, 0, qkv, attn, start, S)
+    seq = torch.empty_like(attn)
+    with nv.option(nv.OPT_ATTN_SPLITS, PREFILL_ATTN_SPLITS):
+        for r, t, ctx in chunks:
+            nv.causal_attn(qkv[r:r + t], kp_d, vp_d, m.page_table, ctx, ks, vs, out=seq[r:r + t],
+                           ld_q=qkv.stride(0), T=t, Hq=I.N_Q_HEADS)
+    torch.cuda.synchronize()
+    assert nv.get_option(nv.OPT_ATTN_SPLITS) == 0
+    assert torch.equal(attn, seq)
+    got = attn.float().cpu().numpy()
+    a = oracle.tree_attn(qkv[:, :qd].float().cpu().numpy().reshape(S, I.N_Q_HEADS, I.HEAD_DIM),
+                         kp_d.cpu().numpy(), vp_d.cpu().numpy(), m.page_table_h, start, I.chain_parent(S),
+                         ks.cpu().numpy(), vs.cpu().numpy())
+    assert np.isfinite(got).all()
+    err = np.abs(got.reshape(a.shape) - a)
+    assert np.all(err <= ATTN_ABS_TOL + 2.0 ** -8 * np.abs(a)), err.max()
 
 
 def test_prefill_head_ranges_determinism():
