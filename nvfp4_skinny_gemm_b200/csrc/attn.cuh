@@ -15,10 +15,10 @@
 //               tile); fp32 S in tensor memory.
 //   softmax     one thread per row: S row -> registers (tcgen05.ld), ancestor
 //               (or causal) mask on the pages that hold the new positions,
-//               running max in the log2 domain, P' = 2^(s - m + 6) as two
+//               running max in the log2 domain, P' = 2^(s - m + 4) as two
 //               E4M3 terms (hi + lo) stored to shared memory in the MMA's
 //               core-matrix layout.  O is rescaled in tensor memory only when
-//               a row max grows by more than 2^2.  Warps whose 32 rows are all
+//               a row max grows by more than 2^4.  Warps whose 32 rows are all
 //               padding skip this work and only keep the barriers in step.
 //   O += P V    M=128, N=144, K=32: the V pages are kept in HBM in the
 //               core-matrix layout, so one bulk copy lands the operand; 16
@@ -70,8 +70,14 @@ constexpr uint32_t ATT_TMEM_COLS = 512;
 constexpr uint32_t ATT_TM_S0 = 0, ATT_TM_S1 = 64;
 constexpr uint32_t ATT_TM_O0 = 128, ATT_TM_O1 = 288;
 constexpr uint32_t ATT_TM_Q = 448;                              // Q hi 448..479, Q lo 480..511 (A operand)
-constexpr float ATT_TAU = 2.0f;       // log2 growth of a row max that triggers an O rescale
-constexpr float ATT_PSHIFT = 6.0f;    // P' = 2^(s - m + 6) <= 2^(6 + TAU) = 256 < 448
+// A rescale costs a wait for the group's previous product plus a pass over O,
+// and gates the whole page (the PV product waits for all four warps): with
+// a threshold of 2^2, Gaussian scores, whose row max still grows by ~1.7 in
+// log2 over a CTA's pages, made some row of most warps rescale on most pages.
+// 2^4 leaves P' <= 2^(4 + 4) = 256 < 448 (E4M3 max) and the largest P' of a
+// row >= 2^4, so a P' below the E4M3 normal range (2^-6) is < 2^-10 of it.
+constexpr float ATT_TAU = 4.0f;       // log2 growth of a row max that triggers an O rescale
+constexpr float ATT_PSHIFT = 4.0f;    // P' = 2^(s - m + 4) <= 2^(4 + TAU) = 256 < 448
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint32_t ATT_CNT_BYTES = 256;                         // per-head arrival counters (fused combine)
 static_assert(ATT_STAGE_BYTES % 1024 == 0, "K tiles need 1024-byte alignment (128-byte swizzle atoms)");
