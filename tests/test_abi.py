@@ -260,3 +260,52 @@ def test_failing_status_rezeroes_counter_workspaces(monkeypatch):
     for (_, kind), w in spaces.items():
         want = 0 if kind in ("linear", "argmax", "attn") else 7
         assert int(w.buf.min()) == want and int(w.buf.max()) == want, kind
+
+
+def test_option_block_restores_the_previous_value():
+    """lib.option sets a library option for the calls inside the block and
+    puts the previous value back, on an exception too."""
+    lib.load()
+    assert lib.get_option(lib.OPT_ATTN_SPLITS) == 0
+    with lib.option(lib.OPT_ATTN_SPLITS, 3):
+        assert lib.get_option(lib.OPT_ATTN_SPLITS) == 3
+    assert lib.get_option(lib.OPT_ATTN_SPLITS) == 0
+    try:
+        with lib.option(lib.OPT_ATTN_SPLITS, 5):
+            raise KeyError("inside")
+    except KeyError:
+        pass
+    assert lib.get_option(lib.OPT_ATTN_SPLITS) == 0
+
+
+def test_attention_launch_count_follows_the_split_grid():
+    """One launch (split kernel with the combine fused) only when the fused
+    combine is on and the split grid fits on the GPU at once; an explicit
+    split count whose grid is not given counts two."""
+    lib.load()
+    assert lib.attn_launches() == 2
+    with lib.option(lib.OPT_ATTN_FUSED_COMBINE, 1):
+        assert lib.attn_launches() == 1
+        with lib.option(lib.OPT_ATTN_SPLITS, 3):
+            assert lib.attn_launches() == 2
+            assert lib.attn_launches(3 * 24, 148) == 1
+            assert lib.attn_launches(7 * 24, 148) == 2
+    assert lib.attn_launches(3 * 24, 148) == 2
+
+
+def test_prefill_split_count_rule():
+    """The prefill gives its causal calls PREFILL_ATTN_SPLITS splits only on
+    the GPU with at least four blocks in flight, and leaves a split count the
+    caller set alone."""
+    import types
+    import torch
+    from nvfp4_skinny_gemm_b200 import step
+    lib.load()
+    gpu = types.SimpleNamespace(dev=torch.device("cuda", 0))
+    cpu = types.SimpleNamespace(dev=torch.device("cpu"))
+    f = step.VerifyModel._causal_splits
+    assert f(gpu, 8) == f(gpu, 4) == step.PREFILL_ATTN_SPLITS
+    assert f(gpu, 3) == f(gpu, 1) == 0
+    assert f(cpu, 8) == 0
+    with lib.option(lib.OPT_ATTN_SPLITS, 5):
+        assert f(gpu, 8) == 0
