@@ -343,7 +343,10 @@ NVFP4SK_API nvfp4sk_status kv_page_restore(const uint8_t *src_pool, const int32_
  * calibrated checkpoint's; one launch with no grid-wide reduction).  x bf16
  * [rows][n] (row stride n), w bf16 [n].  rows <= 16, n % 64 == 0, n <= 8192;
  * with a static g_in and only the canonical outputs (act_prepared NULL) any
- * number of rows (the suffix prefill). */
+ * number of rows (the suffix prefill).  With a static g_in and programmatic
+ * dependent launch on, w is read before the preceding kernel on the stream
+ * has finished, as nvfp4_linear reads its weights: no kernel that may still
+ * run may write it (see tree_attn_fp8kv for the rule). */
 NVFP4SK_API nvfp4sk_status nvfp4_rmsnorm_quantize(const void *x, const void *w, float eps, int64_t rows,
                                                   int64_t n, const float *g_in, uint8_t *codes, uint8_t *scales,
                                                   float *g_out, uint8_t *act_prepared, void *ws, size_t ws_bytes,
@@ -364,7 +367,8 @@ NVFP4SK_API nvfp4sk_status nvfp4_swiglu_quantize(const void *gu, int64_t rows, i
  * receives it.  tiles: nvfp4_prepared_weight_bytes(rows, K) bytes, 16-byte
  * aligned; the bytes of rows past `rows` in the last 128-row tile are not
  * written (only those tokens' outputs read them).  K (n, F) % 512 == 0;
- * rows >= 1; nvfp4_rmsnorm_quantize_tiles needs n <= 8192. */
+ * rows >= 1; nvfp4_rmsnorm_quantize_tiles needs n <= 8192 and reads w before
+ * the preceding kernel has finished, as nvfp4_rmsnorm_quantize does. */
 NVFP4SK_API nvfp4sk_status nvfp4_quantize_act_tiles(const void *x, int x_dtype, int64_t rows, int64_t K,
                                                     int64_t ld_x, const float *g_in, float *g_out, uint8_t *tiles,
                                                     nvfp4sk_stream_t stream);

@@ -350,10 +350,24 @@ __global__ void __launch_bounds__(RS_THREADS)
 {
     __shared__ float s_red[RS_THREADS / 32];
     pdl_launch_dependents();
-    pdl_wait();
     const int64_t r = blockIdx.x;
     const int64_t kb = n / 16;
     const int64_t b0 = blockIdx.y * kb / gridDim.y, b1 = (blockIdx.y + 1) * kb / gridDim.y;
+    // the norm weight is not written by a kernel that may still run (a rule
+    // of the call, as for a linear's weights): the blocks this thread scales
+    // are requested before the wait on the preceding kernel
+    uint4 wb[RS_MAXJ][2];
+#pragma unroll
+    for (int j = 0; j < RS_MAXJ; ++j) {
+        const int64_t i = threadIdx.x + RS_THREADS * j;
+        if (i < b1 - b0) {
+            const uint4 *q = reinterpret_cast<const uint4 *>(w + (b0 + i) * 16);
+            wb[j][0] = q[0];
+            wb[j][1] = q[1];
+        }
+    }
+    pdl_wait();
+    const float g = *g_in;
     const __nv_bfloat16 *xr = x + r * n;
     uint4 xb[RS_MAXJ][2];
 #pragma unroll
@@ -380,7 +394,6 @@ __global__ void __launch_bounds__(RS_THREADS)
     __syncthreads();
     const float tot = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
     const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)n), eps));
-    const float g = *g_in;
     if (r == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
 #pragma unroll
     for (int j = 0; j < RS_MAXJ; ++j) {
@@ -389,7 +402,7 @@ __global__ void __launch_bounds__(RS_THREADS)
             const int64_t c = b0 + i;
             float v[16], wv[16];
             load16<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16 *>(xb[j]), v);
-            load16<__nv_bfloat16>(w + c * 16, wv);
+            load16<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16 *>(wb[j]), wv);
 #pragma unroll
             for (int k = 0; k < 16; ++k) v[k] = round_bf16(__fmul_rn(__fmul_rn(v[k], inv), wv[k]));
             uint2 pk;
