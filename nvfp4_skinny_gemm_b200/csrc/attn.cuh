@@ -839,6 +839,10 @@ __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnPara
     const int S = p.S;
     const int64_t rows_cta = (int64_t)p.nheads * p.rows_w;
     auto row = [&](int s) { return ((int64_t)ch * S + s) * rows_cta + (int64_t)w * p.rows_w + i; };
+    // the scales the tail needs go out with the split results, not after
+    // the reductions (two round trips off the end of the call)
+    const float vsc = p.v_scale[h];
+    const float g_act = p.act ? *p.g_act : 0.f;
     float4 pv[CMB_PF];
 #pragma unroll
     for (int k = 0; k < CMB_PF; ++k) {
@@ -889,7 +893,7 @@ __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnPara
     __syncthreads();
     const float *xf = reinterpret_cast<const float *>(xs);
     const float num = (xf[tid] + xf[ATT_D + tid]) + (xf[2 * ATT_D + tid] + xf[3 * ATT_D + tid]);
-    const float o = den > 0.f ? num / den * p.v_scale[h] : 0.f;
+    const float o = den > 0.f ? num / den * vsc : 0.f;
     const __nv_bfloat16 ob = __float2bfloat16_rn(o);
     p.out[((int64_t)i * p.Hq + hq) * ATT_D + tid] = ob;
     if (p.act) {
@@ -903,7 +907,7 @@ __global__ void __launch_bounds__(ATT_D) tree_attn_combine_kernel(const AttnPara
 #pragma unroll
             for (int k = 0; k < 16; ++k) v[k] = orow[16 * tid + k];
             uint2 pk;
-            const uint32_t sc = quant_block16(v, *p.g_act, pk);
+            const uint32_t sc = quant_block16(v, g_act, pk);
             store_prepared(p.act, i, (int64_t)hq * (ATT_D / 16) + tid, pk, sc);
         }
     }
